@@ -1,0 +1,481 @@
+"""Benchmark of the LittleBit factored layer's forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {lb,reference}]
+                    [--config NAME] [--tokens M]
+
+One step is one ``lb_linear_forward`` call (both contractions, both paths)
+over one batch of synthetic input.  Default workload: the Llama-2-7B q_proj
+shape (4096 -> 4096, eff_bit 1.0, residual on: two paths of rank 1024) at
+batch 1.  Steps rotate over enough copies of the weights that the set is
+larger than twice the L2 cache, so every call streams its sign bits from HBM;
+the calls run back to back from CUDA graphs (the chained, per-layer number).
+
+Printed on rank 0, one JSON line:
+  value       whole-job algorithmic HBM GB/s (prefill workloads: TFLOP/s),
+              device-timed with CUDA events, max over ranks
+  e2e         the same metric through the public Python API with pinned host
+              x copied in and y copied out every step
+  roofline    achieved GB/s of the forward call against the measured HBM peak
+  cpu_baseline the fp64 oracle on this host's cores (bounded sample)
+  clocks      SM clocks and throttle reasons sampled during the timed region
+With ``--impl reference`` the fp64 CPU oracle is timed instead (rank 0 only).
+Multi-GPU runs are independent replicas (the layer needs no exchange at this
+scale): every rank runs the same workload on its own GPU.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from binarized_rank_linear_b200 import synth  # noqa: E402
+
+METRIC = "LittleBitLinear µs/call & HBM GB/s (batch 1); prefill TFLOP/s; % of roofline"
+DECODE_MAX_TOKENS = 32
+L2_BYTES = 126 * 1024 * 1024
+KERNEL_SOURCES = ["lb_common.cuh", "lb_decode.cu", "lb_internal.h", "lb_api.cu"]
+
+
+# ---------------------------------------------------------------- workload arithmetic
+
+def algorithmic_bytes(n_in, n_out, ranks, tokens):
+    """Packed sign bits + fp16 scales + bf16 x and y, per call."""
+    bits = sum(r * (n_in + n_out) for r in ranks) // 8
+    scales = sum(2 * (n_in + n_out + r) for r in ranks)
+    return bits + scales + 2 * tokens * n_in + 2 * tokens * n_out
+
+
+def algorithmic_flops(n_in, n_out, ranks, tokens):
+    """The two sign contractions: 2 * M * sum_p r_p (n_in + n_out)."""
+    return 2 * tokens * sum(r * (n_in + n_out) for r in ranks)
+
+
+def workload_name(c, tokens):
+    return (f"{c.name}: {c.n_in}->{c.n_out}, eff_bit {c.eff_num}/{c.eff_den}, "
+            f"{c.paths} path(s) x rank {c.rank}, {tokens} token(s)")
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "binarized_rank_linear_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sustained=d["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def load_traffic(config, tokens):
+    """dram bytes per call from a committed ncu summary, only if it was taken
+    on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{config}/M{tokens}")
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e.get("dram_bytes_per_call")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML in a thread."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index, interval=0.005):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self.interval = interval
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                self.h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + uuid if not uuid.startswith("GPU-") else uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        r = [name for bit, name in self.REASONS.items() if self.reasons & bit and name != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": r, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_setup(gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value, world, device="cpu"):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(per_rank_units, seconds_max, world):
+    """Whole-job throughput: every rank processes the same units; the job takes
+    the slowest rank's time."""
+    return per_rank_units * world / seconds_max
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+def oracle_sample(layer, budget_s, min_runs=2):
+    """Time the oracle on a bounded sample of the workload: a contiguous block
+    of latent indices k of every path (the layer is a sum over k, so this is an
+    exact sub-problem), sized so one run takes about budget_s / min_runs.
+    Returns (seconds per run, algorithmic bytes per run, flops per run,
+    description)."""
+    import oracle
+    x = oracle.bf16_bits_to_f64(layer["x"])
+    full = [dict(su=p["su"], sv=p["sv"], h=oracle.f16_to_f64(p["h"]), g=oracle.f16_to_f64(p["g"]),
+                 l=oracle.f16_to_f64(p["l"])) for p in layer["paths"]]
+    n_in, n_out, M = layer["n_in"], layer["n_out"], x.shape[0]
+    rank = full[0]["su"].shape[1]
+
+    def sliced(kb):
+        return [dict(p, su=np.ascontiguousarray(p["su"][:, :kb]), sv=np.ascontiguousarray(p["sv"][:, :kb]),
+                     l=p["l"][:kb]) for p in full]
+
+    kb = min(rank, 32)
+    t0 = time.perf_counter()
+    oracle.forward(x, sliced(kb))
+    t1 = time.perf_counter() - t0
+    target = budget_s / min_runs
+    kb = int(max(1, min(rank, kb * target / max(t1, 1e-6))))
+    paths = sliced(kb)
+    runs, t_total = 0, 0.0
+    while runs < min_runs or t_total < budget_s * 0.5:
+        t0 = time.perf_counter()
+        oracle.forward(x, paths)
+        t_total += time.perf_counter() - t0
+        runs += 1
+        if t_total > budget_s * 2:
+            break
+    per = t_total / runs
+    nb = algorithmic_bytes(n_in, n_out, [kb] * len(paths), M)
+    nf = algorithmic_flops(n_in, n_out, [kb] * len(paths), M)
+    desc = (f"{M} token(s), latent indices 0..{kb - 1} of {rank} in each of {len(paths)} path(s) "
+            f"({runs} run(s), {t_total:.1f} s)")
+    return per, nb, nf, desc
+
+
+def run_reference(args, world, rank):
+    """--impl reference: the fp64 CPU oracle on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    c = synth.CONFIGS[args.config]
+    tokens = args.tokens or c.tokens[0]
+    decode = tokens <= DECODE_MAX_TOKENS
+    layer = synth.make_config(args.config, min(tokens, 64))
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    per, nb, nf, desc = oracle_sample(layer, max(budget, 0.05), min_runs=1)
+    for _ in range(args.warmup):
+        pass  # the sample run above is the warm-up
+    t_steps = per * args.steps
+    value = (nb / per / 1e9) if decode else (nf / per / 1e12)
+    unit = "GB/s" if decode else "TFLOP/s"
+    if tokens > 64:
+        desc += f" (first 64 of {tokens} tokens)"
+    out = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": workload_name(c, tokens), "tokens": tokens},
+           "impl": "reference",
+           "cpu_baseline": {"value": value, "unit": unit, "cores": oracle.num_threads(), "kind": "oracle",
+                            "sample": desc},
+           "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+           "timed_seconds": t_steps}
+    print(json.dumps(out), flush=True)
+
+
+# ---------------------------------------------------------------- the GPU arm
+
+def run_lb(args, world, rank, local):
+    import torch
+    import binarized_rank_linear_b200 as lb
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    c = synth.CONFIGS[args.config]
+    tokens = args.tokens or c.tokens[0]
+    ranks = [c.rank] * c.paths
+    decode = tokens <= DECODE_MAX_TOKENS
+    nbytes = algorithmic_bytes(c.n_in, c.n_out, ranks, tokens)
+    nflops = algorithmic_flops(c.n_in, c.n_out, ranks, tokens)
+    layer = synth.make_config(args.config, tokens)
+
+    # weights: one packed set through the C ABI, then copies so the rotation
+    # covers more than twice the L2 cache
+    base = []
+    for p in layer["paths"]:
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        base.append(lb.PackedPath.from_factors(dev(p["su"]), dev(p["sv"]), dev(p["h"]), dev(p["g"]), dev(p["l"])))
+    set_bytes = sum(p.u_bits.numel() * 4 + p.vt_bits.numel() * 4 for p in base)
+    io_bytes = 2 * tokens * (c.n_in + c.n_out)
+    nsets = 1 if io_bytes > 2 * L2_BYTES else max(1, min(512, -(-2 * L2_BYTES // set_bytes) + 1))
+
+    def clone(p):
+        return lb.PackedPath(p.u_bits.clone(), p.vt_bits.clone(), p.h.clone(), p.g.clone(), p.l.clone(), p.rank)
+
+    sets = [base] + [[clone(p) for p in base] for _ in range(nsets - 1)]
+    x = torch.from_numpy(layer["x"].view(np.int16)).to(device).view(torch.bfloat16)
+    y = torch.empty((tokens, c.n_out), dtype=torch.bfloat16, device=device)
+    ws = torch.empty(max(16, lb.forward_workspace_bytes(tokens, c.n_in, c.n_out, c.rank,
+                                                        c.rank if c.paths > 1 else 0)),
+                     dtype=torch.uint8, device=device)
+
+    def call(i, stream=None):
+        s = sets[i % nsets]
+        lb.linear_forward(x, s[0], s[1] if len(s) > 1 else None, y=y, workspace=ws, stream=stream)
+
+    # parity of the benchmarked configuration against the oracle (sampled rows)
+    call(0)
+    torch.cuda.synchronize()
+    assert lb.device_status() == lb.LB_OK
+    parity = None
+    if rank == 0 and not args.no_parity:
+        import oracle
+        rows = np.arange(tokens) if tokens <= 8 else np.linspace(0, tokens - 1, 8).astype(int)
+        ref = oracle.forward(oracle.bf16_bits_to_f64(layer["x"][rows]),
+                             [dict(su=p["su"], sv=p["sv"], h=oracle.f16_to_f64(p["h"]),
+                                   g=oracle.f16_to_f64(p["g"]), l=oracle.f16_to_f64(p["l"]))
+                              for p in layer["paths"]])
+        got = oracle.bf16_bits_to_f64(y[torch.from_numpy(rows).to(device)].view(torch.int16).cpu().numpy()
+                                      .view(np.uint16))
+        parity = {"rows": int(len(rows)),
+                  "rel_l2": float(np.linalg.norm(got - ref) / np.linalg.norm(ref)),
+                  "max_err_over_max_y": float(np.abs(got - ref).max() / np.abs(ref).max())}
+        assert parity["rel_l2"] <= 5e-3 and parity["max_err_over_max_y"] <= 1e-2, parity
+
+    # CUDA graphs of consecutive calls over the rotating weight sets
+    per_graph = max(1, min(nsets * (2 if nsets < 64 else 1), 512)) if decode else 1
+    cap_stream = torch.cuda.Stream(device)
+
+    def capture(n, start):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap_stream):
+            for i in range(n):
+                call(start + i)
+        return g
+
+    graph = capture(per_graph, 0)
+    tail_n = args.steps % per_graph
+    tail = capture(tail_n, 0) if tail_n else None
+    full_graphs = args.steps // per_graph
+
+    def run_steps(n_full, tail_graph):
+        for _ in range(n_full):
+            graph.replay()
+        if tail_graph is not None:
+            tail_graph.replay()
+
+    # warm-up
+    wf, wt = divmod(args.warmup, per_graph)
+    run_steps(wf, capture(wt, 0) if wt else None)
+    torch.cuda.synchronize()
+
+    # timed region
+    stream = torch.cuda.current_stream(device)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    with clk:
+        start.record(stream)
+        run_steps(full_graphs, tail)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = start.elapsed_time(stop)
+    ms_max = max_over_ranks(ms, world, device)
+    per_call_s = ms_max / 1e3 / args.steps
+    units = nbytes / 1e9 if decode else nflops / 1e12
+    value = aggregate(units * args.steps, ms_max / 1e3, world)
+    assert lb.device_status() == lb.LB_OK
+
+    # isolated calls: cold L2 before each
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
+    iso = []
+    for i in range(20):
+        flush.fill_(i & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        call(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        iso.append(e0.elapsed_time(e1) * 1e3)
+    iso_us = statistics.median(iso)
+    del flush
+
+    # end to end through the public API: pinned x in, y out, every step
+    x_host = torch.empty_like(x, device="cpu").pin_memory()
+    x_host.copy_(x.cpu())
+    y_host = torch.empty((tokens, c.n_out), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = min(args.steps, max(50, args.e2e_steps))
+    for i in range(min(20, e2e_steps)):
+        x.copy_(x_host, non_blocking=True)
+        call(i)
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        x.copy_(x_host, non_blocking=True)
+        call(i)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    e2e_value = aggregate(units * e2e_steps, e2e_ms / 1e3, world)
+
+    if rank != 0:
+        return
+    peaks = load_peaks()
+    if decode:
+        achieved = nbytes / per_call_s / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm"], "traffic": load_traffic(args.config, tokens),
+                "kernel": "lb_linear_forward call (latent_kernel + expand_kernel, PDL-chained)",
+                "peak_source": peaks["source"]}
+    else:
+        achieved = nflops / per_call_s / 1e12
+        pk = peaks["bf16_sustained"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
+                "frac": achieved / pk, "traffic": load_traffic(args.config, tokens),
+                "kernel": "lb_linear_forward call", "peak_source": peaks["source"] + " (sustained)"}
+    cpu = None
+    if world == 1 and not args.no_cpu:
+        import oracle
+        per, nb, nf, desc = oracle_sample(synth.make_config(args.config, min(tokens, 64)), args.cpu_seconds)
+        cpu = {"value": (nb / per / 1e9) if decode else (nf / per / 1e12), "unit": "GB/s" if decode else "TFLOP/s",
+               "cores": oracle.num_threads(), "kind": "oracle", "sample": desc}
+    out = {"metric": METRIC, "value": value, "unit": "GB/s" if decode else "TFLOP/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+           "data": "synthetic",
+           "config": {"workload": workload_name(c, tokens), "tokens": tokens, "weight_sets": nsets,
+                      "l2": ("weights rotated over %.0f MB > 2x L2" % (nsets * set_bytes / 1e6)) if nsets > 1
+                      else "inputs larger than L2",
+                      "launch": "CUDA graphs of %d back-to-back calls" % per_graph,
+                      "parallelism": "replicas" if world > 1 else "single GPU"},
+           "us_per_call": per_call_s * 1e6, "us_per_call_isolated_cold_l2": iso_us,
+           "algorithmic_bytes_per_call": nbytes, "algorithmic_flops_per_call": nflops,
+           "roofline": roof, "cpu_baseline": cpu, "parity": parity, "clocks": clk.summary(),
+           "e2e": {"value": e2e_value, "unit": "GB/s" if decode else "TFLOP/s",
+                   "h2d_bytes_per_step": 2 * tokens * c.n_in, "d2h_bytes_per_step": 2 * tokens * c.n_out,
+                   "steps": e2e_steps},
+           "gpu_launches": 2 * args.steps * -(-tokens // DECODE_MAX_TOKENS) if decode else None,
+           "impl": "lb"}
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=2000)
+    ap.add_argument("--impl", choices=["lb", "reference"], default="lb")
+    ap.add_argument("--config", default="llama2_7b_q", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--tokens", type=int, default=0, help="default: the config's first token count")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--e2e-steps", type=int, default=5000)
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-parity", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        # the oracle runs on rank 0's host cores; other ranks exit at once
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        run_lb(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

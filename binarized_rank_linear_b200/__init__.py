@@ -1,0 +1,256 @@
+"""LittleBit factored linear layer on NVIDIA B200: Python binding of ``liblb.so``.
+
+The layer (sesamedisk.com, "Samsung LittleBit 13B Model", section "What the
+method actually computes", Proposition 1) is
+``y = h (.) (sign(U) (l (.) (sign(V)^T (g (.) x))))`` per path, with an optional
+residual path added on top.  Every step runs in the library's CUDA kernels;
+this module only marshals arguments through the C ABI declared in
+``include/lb.h``.  PyTorch provides device memory and streams.  There is no
+CPU fallback: if ``liblb.so`` is missing or the device is not an sm_100 part,
+the calls raise.
+
+Build the library with ``python -m binarized_rank_linear_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblb.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "lb.h")
+
+# lb_status
+LB_OK = 0
+LB_ERR_INVALID_ARGUMENT = 1
+LB_ERR_UNSUPPORTED_SHAPE = 2
+LB_ERR_MISALIGNED = 3
+LB_ERR_CUDA = 4
+LB_ERR_DEVICE_TIMEOUT = 5
+LB_ERR_NOT_SUPPORTED_DEVICE = 6
+LB_ERR_WORKSPACE_TOO_SMALL = 7
+LB_ERR_RANGE = 8
+# lb_dtype
+LB_F32, LB_F16, LB_BF16, LB_I8 = 0, 1, 2, 3
+# lb_factor
+LB_FACTOR_U, LB_FACTOR_V = 0, 1
+
+
+class LbPath(ctypes.Structure):
+    """``lb_path`` of include/lb.h."""
+    _fields_ = [
+        ("u_bits", ctypes.c_void_p),
+        ("vt_bits", ctypes.c_void_p),
+        ("h", ctypes.c_void_p),
+        ("g", ctypes.c_void_p),
+        ("l", ctypes.c_void_p),
+        ("rank", ctypes.c_int64),
+        ("u_ld", ctypes.c_int64),
+        ("vt_ld", ctypes.c_int64),
+    ]
+
+
+class LbError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}" if what else status_string(status))
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``liblb.so`` (once).  Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with `python -m binarized_rank_linear_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            i64, vp, sz, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+            L.lb_status_string.restype = ctypes.c_char_p
+            L.lb_status_string.argtypes = [i32]
+            L.lb_packed_ld_words.restype = i64
+            L.lb_packed_ld_words.argtypes = [i64]
+            L.lb_packed_bytes.restype = sz
+            L.lb_packed_bytes.argtypes = [i32, i64, i64]
+            L.lb_rank_for_budget.restype = i32
+            L.lb_rank_for_budget.argtypes = [i64, i64, i64, i64, i32, i32, ctypes.POINTER(i64)]
+            L.lb_pack_signs.restype = i32
+            L.lb_pack_signs.argtypes = [vp, i32, i32, i64, i64, i64, vp, i64, vp]
+            L.lb_forward_workspace_bytes.restype = sz
+            L.lb_forward_workspace_bytes.argtypes = [i64, i64, i64, i64, i64]
+            L.lb_linear_forward.restype = i32
+            L.lb_linear_forward.argtypes = [vp, i64, i64, i64, i64, ctypes.POINTER(LbPath),
+                                            ctypes.POINTER(LbPath), vp, i64, vp, sz, vp]
+            L.lb_device_status.restype = i32
+            L.lb_device_status.argtypes = [vp, ctypes.POINTER(i32)]
+            _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().lb_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != LB_OK:
+        raise LbError(status, what)
+
+
+# ------------------------------------------------------------------ host-only queries
+
+def packed_ld_words(cols: int) -> int:
+    return int(lib().lb_packed_ld_words(cols))
+
+
+def packed_bytes(kind: int, n_in_or_out: int, rank: int) -> int:
+    return int(lib().lb_packed_bytes(kind, n_in_or_out, rank))
+
+
+def rank_for_budget(n_in: int, n_out: int, eff_num: int, eff_den: int, paths: int = 1,
+                    align: int = 32) -> int:
+    r = ctypes.c_int64(0)
+    _check(lib().lb_rank_for_budget(n_in, n_out, eff_num, eff_den, paths, align, ctypes.byref(r)),
+           "lb_rank_for_budget")
+    return int(r.value)
+
+
+def forward_workspace_bytes(tokens: int, n_in: int, n_out: int, rank_main: int,
+                            rank_residual: int = 0) -> int:
+    return int(lib().lb_forward_workspace_bytes(tokens, n_in, n_out, rank_main, rank_residual))
+
+
+# ------------------------------------------------------------------ device calls
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    codes = {torch.float32: LB_F32, torch.float16: LB_F16, torch.bfloat16: LB_BF16, torch.int8: LB_I8}
+    if t.dtype not in codes:
+        raise TypeError(f"unsupported factor dtype {t.dtype}")
+    return codes[t.dtype]
+
+
+def pack_signs(src, kind: str, ld_words: int | None = None, stream=None):
+    """Pack a device factor (f32 / f16 / bf16 / int8, 2-D, unit column stride)
+    with ``lb_pack_signs``.  ``kind`` is ``"U"`` (src = U [n_out, r]) or
+    ``"V"`` (src = V [n_in, r], packed as V^T).  Returns an int32 tensor of
+    packed words (bit patterns)."""
+    torch = _torch()
+    if src.dim() != 2 or src.stride(1) != 1 or not src.is_cuda:
+        raise ValueError("src must be a 2-D CUDA tensor with unit column stride")
+    rows, cols = src.shape
+    packed_rows, packed_cols = (rows, cols) if kind == "U" else (cols, rows)
+    ld = packed_ld_words(packed_cols) if ld_words is None else int(ld_words)
+    dst = torch.empty((packed_rows, ld), dtype=torch.int32, device=src.device)
+    code = LB_FACTOR_U if kind == "U" else LB_FACTOR_V
+    _check(lib().lb_pack_signs(src.data_ptr(), _dtype_code(src), code, rows, cols, src.stride(0),
+                               dst.data_ptr(), ld, _stream_handle(stream)), "lb_pack_signs")
+    return dst
+
+
+@dataclass
+class PackedPath:
+    """One binarized path on the device: packed sign(U) [n_out, u_ld] and
+    sign(V)^T [rank, vt_ld] (int32 words) and fp16 scales h [n_out], g [n_in],
+    l [rank]."""
+    u_bits: object
+    vt_bits: object
+    h: object
+    g: object
+    l: object
+    rank: int
+
+    @classmethod
+    def from_factors(cls, su, sv, h, g, l, stream=None) -> "PackedPath":
+        """Pack U [n_out, r] and V [n_in, r] (any supported dtype, on the
+        device) and keep the fp16 scales."""
+        torch = _torch()
+        f16 = lambda t: t.to(device=su.device, dtype=torch.float16).contiguous()
+        return cls(pack_signs(su, "U", stream=stream), pack_signs(sv, "V", stream=stream),
+                   f16(h), f16(g), f16(l), int(su.shape[1]))
+
+    def as_c(self) -> LbPath:
+        return LbPath(self.u_bits.data_ptr(), self.vt_bits.data_ptr(), self.h.data_ptr(),
+                      self.g.data_ptr(), self.l.data_ptr(), self.rank, self.u_bits.shape[1],
+                      self.vt_bits.shape[1])
+
+
+def linear_forward(x, main: PackedPath, residual: PackedPath | None = None, y=None,
+                   workspace=None, stream=None):
+    """``lb_linear_forward``: x bf16 [tokens, n_in] (row stride a multiple of 8)
+    -> y bf16 [tokens, n_out].  Allocates y and the workspace with torch when
+    not given."""
+    torch = _torch()
+    tokens, n_in = x.shape
+    n_out = main.h.shape[0]
+    if y is None:
+        y = torch.empty((tokens, n_out), dtype=torch.bfloat16, device=x.device)
+    need = forward_workspace_bytes(tokens, n_in, n_out, main.rank, residual.rank if residual else 0)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    cm = main.as_c()
+    cr = residual.as_c() if residual is not None else None
+    _check(lib().lb_linear_forward(
+        x.data_ptr(), tokens, n_in, n_out, x.stride(0), ctypes.byref(cm),
+        ctypes.byref(cr) if cr is not None else None, y.data_ptr(), y.stride(0),
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream)),
+        "lb_linear_forward")
+    return y
+
+
+def device_status(stream=None) -> int:
+    """``lb_device_status``: synchronise the stream, return and clear the
+    device status word (an lb_status code)."""
+    out = ctypes.c_int(0)
+    _check(lib().lb_device_status(_stream_handle(stream), ctypes.byref(out)), "lb_device_status")
+    return int(out.value)
+
+
+class LittleBitLinear:
+    """A deployed LittleBit layer: one or two packed paths on the device.
+
+    ``layer(x)`` runs ``lb_linear_forward`` on the current stream."""
+
+    def __init__(self, main: PackedPath, residual: PackedPath | None = None):
+        self.main, self.residual = main, residual
+        self.n_out = int(main.h.shape[0])
+        self.n_in = int(main.g.shape[0])
+        self._ws = None
+
+    @classmethod
+    def from_factors(cls, paths: list[dict], device="cuda") -> "LittleBitLinear":
+        """``paths``: one or two dicts of host or device arrays ``su`` [n_out, r],
+        ``sv`` [n_in, r] (+-1, any supported dtype) and fp16 ``h``, ``g``, ``l``."""
+        torch = _torch()
+        dev = lambda a: torch.as_tensor(a).to(device)
+        packed = [PackedPath.from_factors(dev(p["su"]), dev(p["sv"]), dev(p["h"]), dev(p["g"]),
+                                          dev(p["l"])) for p in paths]
+        return cls(packed[0], packed[1] if len(packed) > 1 else None)
+
+    def workspace(self, tokens: int, device):
+        torch = _torch()
+        need = forward_workspace_bytes(tokens, self.n_in, self.n_out, self.main.rank,
+                                       self.residual.rank if self.residual else 0)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(max(need, 16), dtype=torch.uint8, device=device)
+        return self._ws
+
+    def __call__(self, x, y=None, stream=None):
+        return linear_forward(x, self.main, self.residual, y=y,
+                              workspace=self.workspace(x.shape[0], x.device), stream=stream)

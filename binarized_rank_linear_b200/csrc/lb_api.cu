@@ -1,0 +1,266 @@
+// lb_api.cu - the C ABI (include/lb.h): argument checks, per-device set-up,
+// dispatch by token count, and the device status word.
+#include <array>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda_runtime.h>
+
+#include "lb.h"
+#include "lb_internal.h"
+
+// One status word per device (each device that loads the library has its own
+// copy of this variable).  Kernels set it with atomicCAS(0 -> code).
+__device__ int g_lb_status = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxDim = int64_t(1) << 20;     // n_in, n_out
+constexpr int64_t kMaxRank = 32768;
+constexpr int64_t kMaxTokens = int64_t(1) << 24;
+
+std::mutex g_mutex;
+std::array<lb::DeviceInfo, kMaxDevices> g_dev;
+std::array<bool, kMaxDevices> g_ready{};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t ceil_words(int64_t cols) { return (cols + 31) / 32; }
+
+// Set-up for the current device, once: check it is an sm_100 part, read its
+// SM count and shared-memory limit, resolve the status word's device address
+// and raise the kernels' dynamic shared-memory limits.
+lb_status device_info(lb::DeviceInfo *out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return LB_ERR_NOT_SUPPORTED_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_ready[dev]) {
+        *out = g_dev[dev];
+        return LB_OK;
+    }
+    int major = 0, minor = 0;
+    lb::DeviceInfo info;
+    info.device = dev;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&info.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&info.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    if (major != 10 || minor != 0) return LB_ERR_NOT_SUPPORTED_DEVICE;
+    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&info.status), g_lb_status) != cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    if (lb::decode_prepare_device(info) != cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    g_dev[dev] = info;
+    g_ready[dev] = true;
+    *out = info;
+    return LB_OK;
+}
+
+// Checks one path against the layer's sizes; fills `d` on success.
+lb_status check_path(const lb_path *p, int64_t n_in, int64_t n_out, lb::PathDesc *d)
+{
+    if (!p || !p->u_bits || !p->vt_bits || !p->h || !p->g || !p->l) return LB_ERR_INVALID_ARGUMENT;
+    if (p->rank <= 0 || p->u_ld < 0 || p->vt_ld < 0) return LB_ERR_INVALID_ARGUMENT;
+    if (p->rank % 32 != 0 || p->rank > kMaxRank) return LB_ERR_UNSUPPORTED_SHAPE;
+    const int64_t u_ld = p->u_ld ? p->u_ld : ceil_words(p->rank);
+    const int64_t vt_ld = p->vt_ld ? p->vt_ld : ceil_words(n_in);
+    if (u_ld < ceil_words(p->rank) || vt_ld < ceil_words(n_in)) return LB_ERR_INVALID_ARGUMENT;
+    if (!aligned16(p->u_bits) || !aligned16(p->vt_bits) || !aligned16(p->h) || !aligned16(p->g) ||
+        !aligned16(p->l))
+        return LB_ERR_MISALIGNED;
+    (void)n_out;
+    d->u_bits = p->u_bits;
+    d->vt_bits = p->vt_bits;
+    d->h = p->h;
+    d->g = p->g;
+    d->l = p->l;
+    d->rank = (int)p->rank;
+    d->u_ld = u_ld;
+    d->vt_ld = vt_ld;
+    return LB_OK;
+}
+
+size_t workspace_for(int64_t tokens, int64_t n_in, int64_t n_out, const int *ranks, int npaths)
+{
+    return lb::decode_workspace_bytes((int)tokens, (int)n_in, (int)n_out, ranks, npaths);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *lb_status_string(lb_status s)
+{
+    switch (s) {
+    case LB_OK: return "LB_OK";
+    case LB_ERR_INVALID_ARGUMENT: return "LB_ERR_INVALID_ARGUMENT";
+    case LB_ERR_UNSUPPORTED_SHAPE: return "LB_ERR_UNSUPPORTED_SHAPE";
+    case LB_ERR_MISALIGNED: return "LB_ERR_MISALIGNED";
+    case LB_ERR_CUDA: return "LB_ERR_CUDA";
+    case LB_ERR_DEVICE_TIMEOUT: return "LB_ERR_DEVICE_TIMEOUT";
+    case LB_ERR_NOT_SUPPORTED_DEVICE: return "LB_ERR_NOT_SUPPORTED_DEVICE";
+    case LB_ERR_WORKSPACE_TOO_SMALL: return "LB_ERR_WORKSPACE_TOO_SMALL";
+    case LB_ERR_RANGE: return "LB_ERR_RANGE";
+    }
+    return "LB_ERR_UNKNOWN";
+}
+
+int64_t lb_packed_ld_words(int64_t cols)
+{
+    return cols <= 0 ? -1 : ceil_words(cols);
+}
+
+size_t lb_packed_bytes(lb_factor kind, int64_t n_in_or_out, int64_t rank)
+{
+    if (n_in_or_out <= 0 || rank <= 0 || n_in_or_out > kMaxDim * 64 || rank > kMaxDim * 64) return 0;
+    if (kind == LB_FACTOR_U) return (size_t)n_in_or_out * (size_t)ceil_words(rank) * 4u;
+    if (kind == LB_FACTOR_V) return (size_t)rank * (size_t)ceil_words(n_in_or_out) * 4u;
+    return 0;
+}
+
+lb_status lb_rank_for_budget(int64_t n_in, int64_t n_out, int64_t eff_num, int64_t eff_den, int paths,
+                             int align, int64_t *rank)
+{
+    if (!rank) return LB_ERR_INVALID_ARGUMENT;
+    *rank = 0;
+    if (n_in <= 0 || n_out <= 0 || eff_num <= 0 || eff_den <= 0 || (paths != 1 && paths != 2) || align < 1)
+        return LB_ERR_INVALID_ARGUMENT;
+    // numerator eff_num * n_in * n_out and denominator eff_den * paths * (n_in + n_out)
+    // in unsigned 128-bit arithmetic: no overflow for any int64 inputs.
+    const unsigned __int128 num = (unsigned __int128)eff_num * (unsigned __int128)n_in * (unsigned __int128)n_out;
+    const unsigned __int128 den =
+        (unsigned __int128)eff_den * (unsigned __int128)paths * ((unsigned __int128)n_in + (unsigned __int128)n_out);
+    unsigned __int128 r = num / den;
+    r -= r % (unsigned __int128)align;
+    if (r > (unsigned __int128)INT64_MAX) return LB_ERR_INVALID_ARGUMENT;
+    *rank = (int64_t)r;
+    return r == 0 ? LB_ERR_UNSUPPORTED_SHAPE : LB_OK;
+}
+
+lb_status lb_pack_signs(const void *src, lb_dtype dtype, lb_factor kind, int64_t rows, int64_t cols,
+                        int64_t src_ld, uint32_t *dst, int64_t dst_ld_words, void *stream)
+{
+    if (!src || !dst) return LB_ERR_INVALID_ARGUMENT;
+    if (dtype != LB_F32 && dtype != LB_F16 && dtype != LB_BF16 && dtype != LB_I8) return LB_ERR_INVALID_ARGUMENT;
+    if (kind != LB_FACTOR_U && kind != LB_FACTOR_V) return LB_ERR_INVALID_ARGUMENT;
+    if (rows <= 0 || cols <= 0 || src_ld < cols) return LB_ERR_INVALID_ARGUMENT;
+    if (rows > kMaxDim * 64 || cols > kMaxDim * 64) return LB_ERR_UNSUPPORTED_SHAPE;
+    const int64_t packed_cols = kind == LB_FACTOR_U ? cols : rows;
+    if (dst_ld_words < ceil_words(packed_cols)) return LB_ERR_INVALID_ARGUMENT;
+    const size_t esize = dtype == LB_F32 ? 4 : (dtype == LB_I8 ? 1 : 2);
+    if ((reinterpret_cast<uintptr_t>(src) % esize) != 0 || (reinterpret_cast<uintptr_t>(dst) & 3u) != 0)
+        return LB_ERR_MISALIGNED;
+    lb::DeviceInfo dev;
+    const lb_status st = device_info(&dev);
+    if (st != LB_OK) return st;
+    const cudaError_t e = lb::pack_signs_launch(src, dtype, kind, rows, cols, src_ld, dst, dst_ld_words,
+                                                static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    return LB_OK;
+}
+
+size_t lb_forward_workspace_bytes(int64_t tokens, int64_t n_in, int64_t n_out, int64_t rank_main,
+                                  int64_t rank_residual)
+{
+    if (tokens < 0 || n_in <= 0 || n_out <= 0 || rank_main <= 0 || rank_residual < 0) return 0;
+    if (tokens > kMaxTokens || n_in > kMaxDim || n_out > kMaxDim || rank_main > kMaxRank ||
+        rank_residual > kMaxRank)
+        return 0;
+    if (tokens == 0) return 0;
+    const int ranks[2] = {(int)rank_main, (int)rank_residual};
+    return workspace_for(tokens, n_in, n_out, ranks, rank_residual > 0 ? 2 : 1);
+}
+
+lb_status lb_linear_forward(const uint16_t *x, int64_t tokens, int64_t n_in, int64_t n_out, int64_t ldx,
+                            const lb_path *main, const lb_path *residual, uint16_t *y, int64_t ldy,
+                            void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (tokens < 0 || n_in <= 0 || n_out <= 0) return LB_ERR_INVALID_ARGUMENT;
+    if (tokens == 0) return LB_OK;
+    if (!x || !y || !main) return LB_ERR_INVALID_ARGUMENT;
+    if (ldx < n_in || ldy < n_out) return LB_ERR_INVALID_ARGUMENT;
+    if (n_in % 32 != 0 || n_out % 32 != 0 || n_in > kMaxDim || n_out > kMaxDim || tokens > kMaxTokens)
+        return LB_ERR_UNSUPPORTED_SHAPE;
+    if (ldx % 8 != 0 || ldy % 8 != 0 || !aligned16(x) || !aligned16(y)) return LB_ERR_MISALIGNED;
+
+    lb::ForwardArgs a{};
+    a.npaths = residual ? 2 : 1;
+    lb_status st = check_path(main, n_in, n_out, &a.path[0]);
+    if (st != LB_OK) return st;
+    if (residual) {
+        st = check_path(residual, n_in, n_out, &a.path[1]);
+        if (st != LB_OK) return st;
+    }
+    const int ranks[2] = {a.path[0].rank, a.npaths > 1 ? a.path[1].rank : 0};
+    const size_t need = workspace_for(tokens, n_in, n_out, ranks, a.npaths);
+    if (need > 0 && !workspace) return LB_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes < need) return LB_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace && !aligned16(workspace)) return LB_ERR_MISALIGNED;
+
+    a.x = x;
+    a.ldx = ldx;
+    a.tokens = (int)tokens;
+    a.n_in = (int)n_in;
+    a.n_out = (int)n_out;
+    a.y = y;
+    a.ldy = ldy;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+
+    lb::DeviceInfo dev;
+    st = device_info(&dev);
+    if (st != LB_OK) return st;
+    const cudaError_t e = lb::decode_forward(a, dev, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    return LB_OK;
+}
+
+lb_status lb_device_status(void *stream, lb_status *out)
+{
+    if (!out) return LB_ERR_INVALID_ARGUMENT;
+    *out = LB_OK;
+    lb::DeviceInfo dev;
+    const lb_status st = device_info(&dev);
+    if (st != LB_OK) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_lb_status, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_lb_status, &zero, sizeof(int)) != cudaSuccess) {
+            cudaGetLastError();
+            return LB_ERR_CUDA;
+        }
+    }
+    *out = static_cast<lb_status>(v);
+    return LB_OK;
+}
+
+}  // extern "C"

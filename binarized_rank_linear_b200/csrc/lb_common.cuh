@@ -1,0 +1,120 @@
+// lb_common.cuh - device helpers shared by the library's kernels (sm_100a).
+//
+// Thin wrappers over PTX: asynchronous global->shared copies, the register
+// tensor-core MMA used by the decode kernels, programmatic dependent launch,
+// thread-block-cluster barriers and distributed shared memory, and the device
+// status word.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "lb.h"
+
+namespace lb {
+
+// ---------------------------------------------------------------- status word
+// Kernels record the first device-side failure here (see lb_device_status).
+__device__ __forceinline__ void set_status(int *status, int code)
+{
+    if (status) atomicCAS(status, 0, code);
+}
+
+// ---------------------------------------------------------------- cp.async
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte async copy global -> shared; bytes past `src_bytes` (0 or 16) are zero-filled.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t src_bytes = 16)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n"
+                 :: "r"(smem_u32(dst)), "l"(src), "r"(src_bytes) : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(void *dst, const void *src, uint32_t src_bytes = 4)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n"
+                 :: "r"(smem_u32(dst)), "l"(src), "r"(src_bytes) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+
+// ---------------------------------------------------------------- PDL
+// Wait until the grids this one depends on (programmatic stream
+// serialisation) have completed and their writes are visible.  A no-op when
+// the kernel was launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+// Let the next grid on the stream start its prologue early.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+// ---------------------------------------------------------------- clusters
+__device__ __forceinline__ uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;\n" : "=r"(r));
+    return r;
+}
+// Full cluster barrier with release/acquire semantics for shared::cluster memory.
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n"
+                 "barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+// Address of `p` (a shared-memory variable of this CTA) in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_shared_rank(const void *p, uint32_t rank)
+{
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
+    return out;
+}
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// ---------------------------------------------------------------- tensor cores
+// D = A * B + D, m16n8k16, A/B fp16, accumulate fp32 (register operands).
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------- numerics
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b16) { return __uint_as_float(b16 << 16); }
+
+// Two floats -> packed fp16x2 (round to nearest even); lo in bits 0..15.
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// float -> bf16 bits, round to nearest even.
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float v)
+{
+    uint16_t r;
+    asm("cvt.rn.bf16.f32 %0, %1;\n" : "=h"(r) : "f"(v));
+    return r;
+}
+
+// True if |v| would round to an fp16 infinity (or v is not finite).
+__device__ __forceinline__ bool beyond_f16(float v) { return !(fabsf(v) < 65520.0f); }
+
+}  // namespace lb

@@ -1,0 +1,54 @@
+// lb_internal.h - host-side interfaces between the C ABI (lb_api.cu) and the
+// kernel translation units.  Not installed; not part of the ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "lb.h"
+
+namespace lb {
+
+// Per-device facts the launchers need (cached by lb_api.cu).
+struct DeviceInfo {
+    int device = -1;
+    int sm_count = 0;
+    int max_smem_optin = 0;  // bytes of dynamic shared memory a block may opt into
+    int *status = nullptr;   // device address of this device's status word
+};
+
+// ----------------------------------------------------------------- packing
+cudaError_t pack_signs_launch(const void *src, lb_dtype dtype, lb_factor kind, int64_t rows, int64_t cols,
+                              int64_t src_ld, uint32_t *dst, int64_t dst_ld, cudaStream_t stream);
+
+// ----------------------------------------------------------------- forward
+// Up to two paths, already validated, with their strides resolved.
+struct PathDesc {
+    const uint32_t *u_bits;
+    const uint32_t *vt_bits;
+    const uint16_t *h, *g, *l;
+    int rank;
+    int64_t u_ld, vt_ld;
+};
+
+struct ForwardArgs {
+    const uint16_t *x;
+    int64_t ldx;
+    int tokens;
+    int n_in, n_out;
+    int npaths;
+    PathDesc path[2];
+    uint16_t *y;
+    int64_t ldy;
+    void *workspace;
+    size_t workspace_bytes;
+};
+
+// Decode path (1..32 tokens per launch pair; larger batches are sliced).
+constexpr int kDecodeMaxTokens = 32;
+size_t decode_workspace_bytes(int tokens, int n_in, int n_out, const int *ranks, int npaths);
+cudaError_t decode_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream);
+cudaError_t decode_prepare_device(const DeviceInfo &dev);
+
+}  // namespace lb

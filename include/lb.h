@@ -1,0 +1,188 @@
+/*
+ * lb.h - C ABI of the LittleBit factored linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer.  LittleBit replaces a dense weight W [n_out x n_in] by binarized
+ * low-rank factors and three scale vectors (sesamedisk.com, "Samsung LittleBit
+ * 13B Model", section "How low-rank binarization works"; littlebitllm.com,
+ * section "The method"):
+ *
+ *     W ~= diag(h) . sign(U) . diag(l) . sign(V)^T . diag(g)
+ *
+ * with U [n_out x r], V [n_in x r], h the row scale [n_out], g the column
+ * scale [n_in] and l the latent scale [r].  The forward pass is taken in the
+ * factored order of Proposition 1 (sesamedisk.com, section "What the method
+ * actually computes"), per token x [n_in]:
+ *
+ *     y = h (.) ( sign(U) . ( l (.) ( sign(V)^T . ( g (.) x ) ) ) )
+ *
+ * With residual compensation a second path (U2, V2, h2, g2, l2) of the same
+ * form is added to the first (sesamedisk.com, "How low-rank binarization
+ * works", last paragraph; littlebitllm.com, "Pipeline", step 04).  The rank
+ * per path follows from the bit budget (see lb_rank_for_budget).
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library never allocates, frees or synchronises inside lb_pack_signs or
+ *     lb_linear_forward; both only enqueue work on `stream`.
+ *   - `stream` is a cudaStream_t passed as a plain pointer (NULL = the legacy
+ *     default stream).  The current CUDA device must own every pointer.
+ *   - bf16 and fp16 values travel as their 16-bit patterns (uint16_t).
+ *   - Arguments are checked on the host before anything is enqueued.  On any
+ *     error nothing is launched and no output byte is written.
+ *   - Every call is thread-safe; the library keeps only per-device cached
+ *     attributes and one device status word per device (lb_device_status).
+ *   - There is no CPU fallback: without a usable sm_100 device the compute
+ *     calls return LB_ERR_NOT_SUPPORTED_DEVICE or LB_ERR_CUDA.
+ */
+#ifndef LB_H
+#define LB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+/* Symbols of the shared library are exported explicitly; everything else in
+ * it is hidden. */
+#if defined(LB_BUILDING) && defined(__GNUC__)
+#define LB_API __attribute__((visibility("default")))
+#else
+#define LB_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LB_OK = 0,
+    LB_ERR_INVALID_ARGUMENT = 1,   /* null pointer, negative size, bad enum   */
+    LB_ERR_UNSUPPORTED_SHAPE = 2,  /* a size outside what the kernels take    */
+    LB_ERR_MISALIGNED = 3,         /* a pointer or stride breaks an alignment */
+    LB_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed    */
+    LB_ERR_DEVICE_TIMEOUT = 5,     /* a device-side wait gave up (async)      */
+    LB_ERR_NOT_SUPPORTED_DEVICE = 6, /* the current device is not sm_100    */
+    LB_ERR_WORKSPACE_TOO_SMALL = 7,  /* workspace_bytes below the query    */
+    LB_ERR_RANGE = 8               /* an fp16 operand overflowed (async)      */
+} lb_status;
+
+typedef enum { LB_F32 = 0, LB_F16 = 1, LB_BF16 = 2, LB_I8 = 3 } lb_dtype;
+
+/* Which factor a packed matrix holds.
+ *   LB_FACTOR_U: source U [n_out x r]; packed rows are U's rows, packed along r.
+ *   LB_FACTOR_V: source V [n_in x r]; packed rows are V^T's rows (one per
+ *                latent index k), packed along n_in.                          */
+typedef enum { LB_FACTOR_U = 0, LB_FACTOR_V = 1 } lb_factor;
+
+/* One binarized path of the layer.  All pointers are device memory.
+ *   u_bits : packed sign(U),   [n_out x u_ld] uint32 words (LB_FACTOR_U)
+ *   vt_bits: packed sign(V)^T, [rank  x vt_ld] uint32 words (LB_FACTOR_V)
+ *   h, g, l: fp16 row scale [n_out], column scale [n_in], latent scale [rank]
+ *   rank   : r of this path
+ *   u_ld, vt_ld: words per packed row; 0 means lb_packed_ld_words(rank) and
+ *            lb_packed_ld_words(n_in).  Any value >= those is accepted.      */
+typedef struct lb_path {
+    const uint32_t *u_bits;
+    const uint32_t *vt_bits;
+    const uint16_t *h;
+    const uint16_t *g;
+    const uint16_t *l;
+    int64_t rank;
+    int64_t u_ld;
+    int64_t vt_ld;
+} lb_path;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+LB_API const char *lb_status_string(lb_status status);
+
+/* Packed layout.  Word w of a packed row holds columns 32w .. 32w+31; bit j
+ * (value 1u << j) is 1 iff column 32w + j is -1.  The pages fix one bit per
+ * factor entry, each entry +1 or -1 (sesamedisk.com, "How low-rank
+ * binarization works"); the word layout is this library's own.  Unused bits
+ * of the last word of a row, and any words past it up to the row's stride,
+ * are written as 0.
+ *
+ * Returns ceil(cols / 32), the smallest legal stride in words (rows are
+ * dense, 4-byte aligned), or -1 if cols <= 0. */
+LB_API int64_t lb_packed_ld_words(int64_t cols);
+
+/* Bytes of a packed factor at the smallest stride:
+ *   LB_FACTOR_U: n_out rows x lb_packed_ld_words(rank) words x 4
+ *   LB_FACTOR_V: rank rows  x lb_packed_ld_words(n_in) words x 4
+ * `n_in_or_out` is n_out for U and n_in for V.  Returns 0 on a bad argument. */
+LB_API size_t lb_packed_bytes(lb_factor kind, int64_t n_in_or_out, int64_t rank);
+
+/* Rank per path from the bit budget.  The budget is eff * n_in * n_out sign
+ * bits (linear layers only, scale vectors not counted: littlebitllm.com,
+ * section "How small"); a path of rank r stores r * (n_in + n_out) of them
+ * ("the rank sets the bit budget", sesamedisk.com, "How low-rank binarization
+ * works"), and the residual path shares the same budget (same section).  So
+ *     *rank = floor(eff_num * n_in * n_out / (eff_den * paths * (n_in + n_out)))
+ * rounded down to a multiple of `align`, in exact integer arithmetic
+ * (eff = eff_num / eff_den as a fraction, never a float).
+ * Host only.  Errors: LB_ERR_INVALID_ARGUMENT for non-positive sizes, paths
+ * outside {1, 2}, align < 1, a null `rank`, or products that overflow int64;
+ * LB_ERR_UNSUPPORTED_SHAPE when the result would be 0 (*rank is then 0). */
+LB_API lb_status lb_rank_for_budget(int64_t n_in, int64_t n_out, int64_t eff_num, int64_t eff_den,
+                             int paths, int align, int64_t *rank);
+
+/* Pack a factor's signs into the layout above, on `stream`.
+ *   src      : device, `rows` rows of `cols` elements, row stride `src_ld`
+ *              elements (>= cols), element type `dtype`.
+ *              LB_FACTOR_U: src is U, rows = n_out, cols = r.
+ *              LB_FACTOR_V: src is V, rows = n_in,  cols = r.
+ *   dst      : device, LB_FACTOR_U: [rows x dst_ld_words]; LB_FACTOR_V:
+ *              [cols x dst_ld_words] (V^T).  dst_ld_words >=
+ *              lb_packed_ld_words(packed row length).  Every word of every
+ *              destination row is written.
+ * An element is -1 (bit 1) iff it is strictly negative: +0, -0 and NaN give
+ * bit 0, -inf and negative subnormals bit 1 (the pages only say each entry is
+ * +1 or -1; this is the library's reading, tested bit-exactly).
+ * Alignment: src 4-byte aligned for f32, 2 for f16/bf16; dst 4-byte aligned.
+ * One-off weight preparation, not on the forward path. */
+LB_API lb_status lb_pack_signs(const void *src, lb_dtype dtype, lb_factor kind, int64_t rows,
+                        int64_t cols, int64_t src_ld, uint32_t *dst, int64_t dst_ld_words,
+                        void *stream);
+
+/* Workspace that lb_linear_forward needs for these sizes (rank_residual = 0
+ * without the residual path).  Holds the latent between the two contractions.
+ * Returns 0 on a bad argument; a valid call may also need 0 bytes. */
+LB_API size_t lb_forward_workspace_bytes(int64_t tokens, int64_t n_in, int64_t n_out,
+                                  int64_t rank_main, int64_t rank_residual);
+
+/* The layer's forward pass (Proposition 1, both paths fused), on `stream`.
+ *   x        : device bf16 [tokens x n_in], row stride ldx elements
+ *   main     : the primary path (required)
+ *   residual : the residual path, or NULL for none
+ *   y        : device bf16 [tokens x n_out], row stride ldy elements; written,
+ *              never read.  y = sum over paths of h (.) sign(U)(l (.) sign(V)^T (g (.) x)),
+ *              computed with fp32 accumulation and rounded to bf16 (nearest even).
+ *   workspace: device scratch of at least lb_forward_workspace_bytes(...) bytes,
+ *              16-byte aligned; its contents on entry do not matter.  Calls
+ *              that share a workspace must be ordered on one stream.
+ * Shapes: n_in, n_out and every rank a positive multiple of 32; ldx >= n_in,
+ *   ldy >= n_out, both multiples of 8.  tokens >= 0; tokens == 0 is a no-op
+ *   (nothing launched, pointers unchecked).
+ * Alignment: x, y, u_bits, vt_bits, h, g, l and workspace 16-byte aligned.
+ * Numerics: 1..32 tokens run the decode kernels, which take x as fp16 on the
+ *   tensor cores: |x| must stay below 65504 (else LB_ERR_RANGE is raised on
+ *   the device status word and y is undefined).  Larger batches run the
+ *   prefill kernels, which read x as bf16 directly.
+ * Errors: LB_ERR_INVALID_ARGUMENT (null pointers, negative sizes),
+ *   LB_ERR_UNSUPPORTED_SHAPE, LB_ERR_MISALIGNED, LB_ERR_WORKSPACE_TOO_SMALL,
+ *   LB_ERR_NOT_SUPPORTED_DEVICE, LB_ERR_CUDA (launch failure).  Conditions
+ *   found while the kernels run are reported by lb_device_status. */
+LB_API lb_status lb_linear_forward(const uint16_t *x, int64_t tokens, int64_t n_in, int64_t n_out,
+                            int64_t ldx, const lb_path *main, const lb_path *residual,
+                            uint16_t *y, int64_t ldy, void *workspace, size_t workspace_bytes,
+                            void *stream);
+
+/* Synchronise `stream`, then read and clear the current device's status word,
+ * which kernels set when a device-side condition stops them (a bounded wait
+ * that gave up, an fp16 overflow).  *out receives LB_OK or the first such
+ * condition.  Returns LB_ERR_CUDA if the synchronisation itself fails. */
+LB_API lb_status lb_device_status(void *stream, lb_status *out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LB_H */

@@ -1,0 +1,145 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+function include/lb.h declares, answers the host-only queries, and rejects bad
+arguments before it touches CUDA.  No call here reaches a kernel."""
+import ctypes
+import re
+
+import pytest
+
+import binarized_rank_linear_b200 as lb
+import oracle
+from binarized_rank_linear_b200 import build as lb_build
+from binarized_rank_linear_b200 import synth
+
+
+@pytest.fixture(scope="module")
+def L():
+    lb_build.build()
+    return lb.lib()
+
+
+def declared_functions():
+    text = open(lb.HEADER_PATH).read()
+    return sorted(set(re.findall(r"LB_API\s+[\w\s\*]+?\b(lb_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("lb_pack_signs", "lb_linear_forward", "lb_rank_for_budget", "lb_packed_ld_words",
+                     "lb_packed_bytes", "lb_forward_workspace_bytes", "lb_device_status",
+                     "lb_status_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), f"{name} missing from {lb.LIB_PATH}"
+
+
+def test_status_strings(L):
+    for code in range(0, 9):
+        s = lb.status_string(code)
+        assert s.startswith("LB_") and "UNKNOWN" not in s
+    assert lb.status_string(99) == "LB_ERR_UNKNOWN"
+
+
+def test_packed_ld_and_bytes_match_the_oracle_packer(L):
+    for cols in (1, 31, 32, 33, 288, 800, 1024, 4096, 11008, 28672):
+        assert lb.packed_ld_words(cols) == -(-cols // 32)
+    assert lb.packed_ld_words(0) == -1
+    assert lb.packed_bytes(lb.LB_FACTOR_U, 28672, 288) == 28672 * 9 * 4
+    assert lb.packed_bytes(lb.LB_FACTOR_V, 8192, 288) == 288 * 256 * 4
+    assert lb.packed_bytes(lb.LB_FACTOR_U, 0, 32) == 0
+
+
+@pytest.mark.parametrize("name", sorted(synth.CONFIGS))
+def test_rank_rule_matches_oracle_and_table(L, name):
+    c = synth.CONFIGS[name]
+    r = lb.rank_for_budget(c.n_in, c.n_out, c.eff_num, c.eff_den, c.paths, 32)
+    assert r == c.rank == oracle.rank_for_budget(c.n_in, c.n_out, c.eff_num, c.eff_den, c.paths, 32)
+
+
+def test_rank_rule_random_against_oracle(L):
+    import random
+    rnd = random.Random(3)
+    for _ in range(500):
+        n_in, n_out = rnd.randint(1, 1 << 18), rnd.randint(1, 1 << 18)
+        num, den = rnd.randint(1, 200), rnd.randint(1, 200)
+        paths, align = rnd.choice([1, 2]), rnd.choice([1, 8, 32, 64])
+        expect = oracle.rank_for_budget(n_in, n_out, num, den, paths, align)
+        r = ctypes.c_int64(-1)
+        st = L.lb_rank_for_budget(n_in, n_out, num, den, paths, align, ctypes.byref(r))
+        assert r.value == expect
+        assert st == (lb.LB_OK if expect > 0 else lb.LB_ERR_UNSUPPORTED_SHAPE)
+
+
+def test_rank_rule_rejects_bad_arguments(L):
+    r = ctypes.c_int64(5)
+    assert L.lb_rank_for_budget(0, 10, 1, 1, 1, 1, ctypes.byref(r)) == lb.LB_ERR_INVALID_ARGUMENT
+    assert L.lb_rank_for_budget(10, 10, 1, 1, 3, 1, ctypes.byref(r)) == lb.LB_ERR_INVALID_ARGUMENT
+    assert L.lb_rank_for_budget(10, 10, 1, 0, 1, 1, ctypes.byref(r)) == lb.LB_ERR_INVALID_ARGUMENT
+    assert L.lb_rank_for_budget(10, 10, 1, 1, 1, 1, None) == lb.LB_ERR_INVALID_ARGUMENT
+    # no int64 overflow for huge (valid) inputs
+    big = 1 << 40
+    assert L.lb_rank_for_budget(big, big, 1, 1, 1, 1, ctypes.byref(r)) == lb.LB_OK
+    assert r.value == big // 2
+
+
+def test_workspace_query(L):
+    for name in ("tiny", "llama2_7b_q", "llama2_70b_gate"):
+        c = synth.CONFIGS[name]
+        for m in (1, 8, 32):
+            assert lb.forward_workspace_bytes(m, c.n_in, c.n_out, c.rank,
+                                              c.rank if c.paths == 2 else 0) > 0
+    assert lb.forward_workspace_bytes(0, 256, 256, 32, 0) == 0
+    assert lb.forward_workspace_bytes(1, 256, 256, 0, 0) == 0
+
+
+FAKE = 0x10000          # 16-byte aligned, never dereferenced: every call below fails its checks first
+
+
+def fake_path(rank=32, **over):
+    d = dict(u_bits=FAKE, vt_bits=FAKE, h=FAKE, g=FAKE, l=FAKE, rank=rank, u_ld=0, vt_ld=0)
+    d.update(over)
+    return lb.LbPath(**d)
+
+
+def forward(L, x=FAKE, tokens=1, n_in=256, n_out=256, ldx=256, main=None, residual=None, y=FAKE,
+            ldy=256, ws=FAKE, ws_bytes=1 << 20):
+    main = fake_path() if main is None else main
+    return L.lb_linear_forward(x, tokens, n_in, n_out, ldx, ctypes.byref(main),
+                               ctypes.byref(residual) if residual is not None else None, y, ldy, ws,
+                               ws_bytes, None)
+
+
+def test_forward_rejects_bad_arguments_before_any_cuda_call(L):
+    assert forward(L, tokens=-1) == lb.LB_ERR_INVALID_ARGUMENT
+    assert forward(L, tokens=0, x=0, y=0) == lb.LB_OK                 # no-op
+    assert forward(L, x=0) == lb.LB_ERR_INVALID_ARGUMENT
+    assert forward(L, y=0) == lb.LB_ERR_INVALID_ARGUMENT
+    assert forward(L, n_in=250, ldx=256) == lb.LB_ERR_UNSUPPORTED_SHAPE
+    assert forward(L, n_out=100, ldy=256) == lb.LB_ERR_UNSUPPORTED_SHAPE
+    assert forward(L, ldx=128) == lb.LB_ERR_INVALID_ARGUMENT
+    assert forward(L, ldx=260) == lb.LB_ERR_MISALIGNED
+    assert forward(L, x=FAKE + 2) == lb.LB_ERR_MISALIGNED
+    assert forward(L, main=fake_path(rank=48)) == lb.LB_ERR_UNSUPPORTED_SHAPE
+    assert forward(L, main=fake_path(rank=0)) == lb.LB_ERR_INVALID_ARGUMENT
+    assert forward(L, main=fake_path(u_bits=0)) == lb.LB_ERR_INVALID_ARGUMENT
+    assert forward(L, main=fake_path(g=FAKE + 4)) == lb.LB_ERR_MISALIGNED
+    assert forward(L, main=fake_path(vt_ld=7)) == lb.LB_ERR_INVALID_ARGUMENT   # < ceil(256/32)
+    assert forward(L, residual=fake_path(l=0)) == lb.LB_ERR_INVALID_ARGUMENT
+    assert forward(L, ws_bytes=16) == lb.LB_ERR_WORKSPACE_TOO_SMALL
+    assert forward(L, ws=0) == lb.LB_ERR_INVALID_ARGUMENT
+    assert forward(L, ws=FAKE + 8) == lb.LB_ERR_MISALIGNED
+
+
+def test_pack_rejects_bad_arguments_before_any_cuda_call(L):
+    P = L.lb_pack_signs
+    assert P(0, lb.LB_I8, lb.LB_FACTOR_U, 4, 32, 32, FAKE, 1, None) == lb.LB_ERR_INVALID_ARGUMENT
+    assert P(FAKE, 9, lb.LB_FACTOR_U, 4, 32, 32, FAKE, 1, None) == lb.LB_ERR_INVALID_ARGUMENT
+    assert P(FAKE, lb.LB_I8, 5, 4, 32, 32, FAKE, 1, None) == lb.LB_ERR_INVALID_ARGUMENT
+    assert P(FAKE, lb.LB_I8, lb.LB_FACTOR_U, 4, 32, 16, FAKE, 1, None) == lb.LB_ERR_INVALID_ARGUMENT
+    assert P(FAKE, lb.LB_I8, lb.LB_FACTOR_U, 4, 64, 64, FAKE, 1, None) == lb.LB_ERR_INVALID_ARGUMENT
+    assert P(FAKE, lb.LB_I8, lb.LB_FACTOR_V, 64, 32, 32, FAKE, 1, None) == lb.LB_ERR_INVALID_ARGUMENT
+    assert P(FAKE + 1, lb.LB_F32, lb.LB_FACTOR_U, 4, 32, 32, FAKE, 1, None) == lb.LB_ERR_MISALIGNED
+    assert P(FAKE, lb.LB_F32, lb.LB_FACTOR_U, 4, 32, 32, FAKE + 2, 1, None) == lb.LB_ERR_MISALIGNED

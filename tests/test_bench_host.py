@@ -1,0 +1,73 @@
+"""Host-side logic of bench.py: the algorithmic byte and FLOP counts of the
+workload table, and the replica aggregation (max over ranks) on two gloo
+processes."""
+import os
+
+import pytest
+
+import bench
+from binarized_rank_linear_b200 import synth
+
+# per-call algorithmic bytes / flops of the workload table (packed sign bits +
+# fp16 scales + bf16 x and y; flops of the two contractions)
+EXPECTED = {
+    ("tiny", 1): (4160, 32768),
+    ("llama2_7b_q", 1): (2150400, 33554432),
+    ("llama2_7b_q", 8): (2265088, 268435456),
+    ("llama2_7b_gate", 1): (3114624, 48332800),
+    ("llama2_7b_gate", 32): (4051072, 48332800 * 32),
+    ("llama2_70b_gate", 1): (2876544, 42467328),
+    ("qwen3_14b_gate", 8192): (375320832, 803158884352),
+}
+
+
+@pytest.mark.parametrize("key", sorted(EXPECTED))
+def test_algorithmic_counts(key):
+    name, m = key
+    c = synth.CONFIGS[name]
+    ranks = [c.rank] * c.paths
+    nb, nf = EXPECTED[key]
+    assert bench.algorithmic_bytes(c.n_in, c.n_out, ranks, m) == nb
+    assert bench.algorithmic_flops(c.n_in, c.n_out, ranks, m) == nf
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ms = [12.5, 30.0][rank]
+        mx = bench.max_over_ranks(ms, world)
+        bench.barrier(world)
+        q.put((rank, mx, bench.aggregate(100.0, mx / 1e3, world)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_replicas_take_the_slowest_rank():
+    import socket
+
+    import torch.multiprocessing as mp
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for rank, mx, value in res:
+        assert mx == 30.0                       # max over ranks
+        assert value == pytest.approx(2 * 100.0 / 0.030)   # both ranks' units / slowest time
+
+
+def test_reference_arm_non_zero_ranks_exit(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    bench.main(["--impl", "reference", "--steps", "3", "--warmup", "3"])
+    assert capsys.readouterr().out == ""

@@ -1,0 +1,198 @@
+"""lb_linear_forward on the GPU against the fp64 oracle.
+
+Every workload of the synthetic table runs at each of its token counts; the
+prefill workloads (8192 tokens) are checked on a sample of token rows that
+the oracle computes one by one.  Edge cases: the token sweep around the
+decode/prefill boundary, ragged shapes with r1 != r2, an integer-exact case
+that must match bit for bit, sign-flip invariance (bitwise), determinism,
+workspace contents, strided outputs and canaries, and the status word.
+"""
+import numpy as np
+import pytest
+
+import binarized_rank_linear_b200 as lb
+import oracle
+from binarized_rank_linear_b200 import synth
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+def torch():
+    import torch as t
+    return t
+
+
+DECODE_CASES = [(name, m) for name, c in sorted(synth.CONFIGS.items()) if c.tokens[0] <= 32
+                for m in c.tokens]
+
+
+@pytest.mark.parametrize("name,tokens", DECODE_CASES)
+def test_decode_configs(name, tokens):
+    layer = synth.make_config(name, tokens)
+    y = gu.bf16_to_f64(gu.run_gpu(layer))
+    gu.assert_close(y, gu.oracle_y(layer), f"{name} M={tokens}")
+
+
+PREFILL = [name for name, c in sorted(synth.CONFIGS.items()) if c.tokens[0] > 32]
+
+
+@pytest.mark.parametrize("name", PREFILL)
+def test_prefill_configs_sampled(name):
+    layer = synth.make_config(name)
+    M = layer["x"].shape[0]
+    y = gu.bf16_to_f64(gu.run_gpu(layer))
+    rng = np.random.default_rng(1)
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, M - 1], rng.choice(M, 27, replace=False)]))
+    gu.assert_close(y[rows], gu.oracle_y(layer, rows), f"{name} sampled rows")
+    assert np.all(np.isfinite(y))
+
+
+@pytest.mark.parametrize("tokens", [1, 2, 7, 8, 9, 16, 17, 31, 32, 33, 64, 255, 256, 257])
+def test_token_sweep_ragged_shape(tokens):
+    layer = synth.make_layer(384, 160, [64, 96], tokens, config_id=500)
+    y = gu.bf16_to_f64(gu.run_gpu(layer))
+    gu.assert_close(y, gu.oracle_y(layer), f"M={tokens}")
+
+
+@pytest.mark.parametrize("n_in,n_out,ranks", [(32, 32, [32]), (96, 64, [32]), (64, 800, [32, 64]),
+                                              (1056, 224, [160, 32]), (4096, 96, [288])])
+def test_small_and_asymmetric_shapes(n_in, n_out, ranks):
+    for tokens in (1, 5, 40):
+        layer = synth.make_layer(n_in, n_out, ranks, tokens, config_id=600 + n_in + n_out)
+        y = gu.bf16_to_f64(gu.run_gpu(layer))
+        gu.assert_close(y, gu.oracle_y(layer), f"{n_in}x{n_out} r={ranks} M={tokens}")
+
+
+def integer_layer(n_in, n_out, ranks, tokens, seed):
+    rng = np.random.default_rng(seed)
+    paths = []
+    for r in ranks:
+        paths.append(dict(sv=(1 - 2 * rng.integers(0, 2, (n_in, r))).astype(np.int8),
+                          su=(1 - 2 * rng.integers(0, 2, (n_out, r))).astype(np.int8),
+                          h=np.ones(n_out, np.float16), g=np.ones(n_in, np.float16),
+                          l=np.ones(r, np.float16)))
+    xf = rng.integers(-1, 2, (tokens, n_in)).astype(np.float32)
+    xf[rng.random((tokens, n_in)) < 0.9] = 0.0       # keep |y| small
+    x = (xf.view(np.uint32) >> 16).astype(np.uint16)
+    return dict(x=x, paths=paths, n_in=n_in, n_out=n_out)
+
+
+def bf16_rne(v: np.ndarray) -> np.ndarray:
+    return synth.f32_to_bf16_bits(v.astype(np.float32))
+
+
+@pytest.mark.parametrize("tokens", [1, 3, 8, 32, 40])
+def test_integer_exact_is_bitwise(tokens):
+    """Unit scales and x in {-1, 0, 1}: every intermediate is a small integer,
+    exact in fp16, bf16 and fp32, so the GPU must equal the oracle (rounded
+    to bf16) bit for bit.  Pins sign orientation, pack layout and transposes."""
+    layer = integer_layer(512, 224, [64, 32], tokens, tokens)
+    ref = gu.oracle_y(layer)
+    assert np.abs(ref).max() <= 256 and np.array_equal(ref, np.rint(ref))
+    got = gu.bf16_bits(gu.run_gpu(layer))
+    assert np.array_equal(got, bf16_rne(ref))
+
+
+@pytest.mark.parametrize("tokens", [1, 8, 300])
+def test_sign_flip_invariance_is_bitwise(tokens):
+    layer = synth.make_layer(1024, 512, [96, 64], tokens, config_id=700)
+    y0 = gu.bf16_bits(gu.run_gpu(layer))
+    rng = np.random.default_rng(2)
+    for p in layer["paths"]:
+        cols = rng.random(p["su"].shape[1]) < 0.5
+        p["su"] = np.where(cols[None, :], -p["su"], p["su"]).astype(np.int8)
+        p["sv"] = np.where(cols[None, :], -p["sv"], p["sv"]).astype(np.int8)
+    y1 = gu.bf16_bits(gu.run_gpu(layer))
+    assert np.array_equal(y0, y1)
+
+
+def test_deterministic_and_workspace_independent():
+    t = torch()
+    layer = synth.make_config("llama2_7b_gate", 16)
+    paths = gu.device_paths(layer)
+    x = gu.bf16_tensor(layer["x"])
+    c = synth.CONFIGS["llama2_7b_gate"]
+    need = lb.forward_workspace_bytes(16, c.n_in, c.n_out, c.rank, c.rank)
+    outs = []
+    for fill in (0, 0xFF, 0x7C):
+        ws = t.full((need,), fill, dtype=t.uint8, device="cuda")
+        outs.append(gu.bf16_bits(lb.linear_forward(x, paths[0], paths[1], workspace=ws)))
+    assert all(np.array_equal(outs[0], o) for o in outs[1:])
+
+
+def test_strided_io_and_canaries():
+    t = torch()
+    layer = synth.make_layer(256, 128, [32, 64], 5, config_id=800)
+    paths = gu.device_paths(layer)
+    xb = t.zeros((5, 264), dtype=t.bfloat16, device="cuda")
+    xb[:, :256] = gu.bf16_tensor(layer["x"])
+    ybig = t.full((7, 136), 12345.0, dtype=t.bfloat16, device="cuda")
+    y = ybig[:5, :128]
+    lb.linear_forward(xb[:, :256], paths[0], paths[1], y=y)
+    t.cuda.synchronize()
+    gu.assert_close(gu.bf16_to_f64(y.contiguous()), gu.oracle_y(layer), "strided")
+    assert bool((ybig[:, 128:] == 12345.0).all()) and bool((ybig[5:] == 12345.0).all())
+
+
+def test_bad_arguments_write_nothing():
+    t = torch()
+    layer = synth.make_layer(256, 128, [32], 3, config_id=801)
+    paths = gu.device_paths(layer)
+    x = gu.bf16_tensor(layer["x"])
+    y = t.full((3, 128), 7.0, dtype=t.bfloat16, device="cuda")
+    ws = t.empty(1 << 20, dtype=t.uint8, device="cuda")
+    c = paths[0].as_c()
+    L = lb.lib()
+    import ctypes
+    for args in [(x.data_ptr(), 3, 250, 128, 256), (x.data_ptr() + 2, 3, 256, 128, 256),
+                 (x.data_ptr(), 3, 256, 128, 100)]:
+        st = L.lb_linear_forward(*args, ctypes.byref(c), None, y.data_ptr(), 128, ws.data_ptr(),
+                                 ws.numel(), None)
+        assert st != lb.LB_OK
+    st = L.lb_linear_forward(x.data_ptr(), 3, 256, 128, 256, ctypes.byref(c), None, y.data_ptr(), 128,
+                             ws.data_ptr(), 16, None)
+    assert st == lb.LB_ERR_WORKSPACE_TOO_SMALL
+    t.cuda.synchronize()
+    assert bool((y == 7.0).all())
+    assert lb.device_status() == lb.LB_OK
+
+
+def test_zero_tokens_is_a_noop():
+    t = torch()
+    layer = synth.make_layer(256, 128, [32], 1, config_id=802)
+    paths = gu.device_paths(layer)
+    x = t.empty((0, 256), dtype=t.bfloat16, device="cuda")
+    y = lb.linear_forward(x, paths[0])
+    assert y.shape == (0, 128)
+
+
+def test_range_overflow_sets_status_not_fault():
+    """|x| beyond the fp16 range on the decode path raises LB_ERR_RANGE on the
+    status word (the kernels keep running; nothing faults)."""
+    layer = synth.make_layer(256, 128, [32], 2, config_id=803)
+    big = np.full((2, 256), 1e6, dtype=np.float32)
+    layer["x"] = synth.f32_to_bf16_bits(big)
+    assert lb.device_status() == lb.LB_OK
+    gu.run_gpu(layer)
+    assert lb.device_status() == lb.LB_ERR_RANGE
+    assert lb.device_status() == lb.LB_OK          # read clears it
+
+
+def test_non_default_stream():
+    t = torch()
+    layer = synth.make_config("llama2_7b_q", 8)
+    paths = gu.device_paths(layer)
+    x = gu.bf16_tensor(layer["x"])
+    s = t.cuda.Stream()
+    with t.cuda.stream(s):
+        y = lb.linear_forward(x, paths[0], paths[1], stream=s)
+    s.synchronize()
+    gu.assert_close(gu.bf16_to_f64(y), gu.oracle_y(layer), "side stream")
+
+
+def test_layer_object():
+    layer = synth.make_config("tiny")
+    mod = lb.LittleBitLinear.from_factors(layer["paths"])
+    y = mod(gu.bf16_tensor(layer["x"]))
+    gu.assert_close(gu.bf16_to_f64(y), gu.oracle_y(layer), "module")
