@@ -181,10 +181,8 @@ def dense_weight(paths: list[dict]) -> np.ndarray:
 # --------------------------------------------------------------------------
 
 def packed_ld_words(cols: int) -> int:
-    """Words per packed row: ceil(cols / 32) rounded up to a multiple of 4
-    (16-byte rows)."""
-    w = -(-int(cols) // 32)
-    return -(-w // 4) * 4
+    """Smallest packed row stride: ceil(cols / 32) words (rows are dense)."""
+    return -(-int(cols) // 32)
 
 
 def _negative_mask(src: np.ndarray, dtype: str) -> np.ndarray:
