@@ -41,6 +41,9 @@ __device__ __forceinline__ void cp_async4(void *dst, const void *src, uint32_t s
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+// Wait until at most N of this thread's committed groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;\n" :: "n"(N) : "memory"); }
 
 // ---------------------------------------------------------------- PDL
 // Wait until the grids this one depends on (programmatic stream
@@ -97,6 +100,13 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32
 
 // ---------------------------------------------------------------- numerics
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b16) { return __uint_as_float(b16 << 16); }
+
+__device__ __forceinline__ float f16_bits_to_float(uint16_t b)
+{
+    float f;
+    asm("cvt.f32.f16 %0, %1;\n" : "=f"(f) : "h"(b));
+    return f;
+}
 
 // Two floats -> packed fp16x2 (round to nearest even); lo in bits 0..15.
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi)

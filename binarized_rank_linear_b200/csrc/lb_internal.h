@@ -46,6 +46,12 @@ struct ForwardArgs {
 };
 
 // Decode path (1..32 tokens per launch pair; larger batches are sliced).
+// Up to kSmallMaxTokens tokens run on CUDA cores (nibble tables, lb_gemv.cu),
+// more on the register tensor cores (lb_decode.cu).
+constexpr int kSmallMaxTokens = 4;
+size_t small_workspace_bytes(int M, const int *ranks, int npaths);
+cudaError_t small_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M);
+cudaError_t small_prepare_device(const DeviceInfo &dev);
 constexpr int kDecodeMaxTokens = 32;
 size_t decode_workspace_bytes(int tokens, int n_in, int n_out, const int *ranks, int npaths);
 cudaError_t decode_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream);

@@ -162,10 +162,11 @@ LB_API size_t lb_forward_workspace_bytes(int64_t tokens, int64_t n_in, int64_t n
  *   ldy >= n_out, both multiples of 8.  tokens >= 0; tokens == 0 is a no-op
  *   (nothing launched, pointers unchecked).
  * Alignment: x, y, u_bits, vt_bits, h, g, l and workspace 16-byte aligned.
- * Numerics: 1..32 tokens run the decode kernels, which take x as fp16 on the
- *   tensor cores: |x| must stay below 65504 (else LB_ERR_RANGE is raised on
- *   the device status word and y is undefined).  Larger batches run the
- *   prefill kernels, which read x as bf16 directly.
+ * Numerics: all sums accumulate in fp32 and y is rounded to bf16 once.
+ *   1..4 tokens run on CUDA cores in fp32 throughout.  5..32 tokens feed the
+ *   tensor cores fp16 operands: g (.) x and the latent z must stay below
+ *   65504 in magnitude (else LB_ERR_RANGE is raised on the device status word
+ *   and y is undefined).  Larger batches run the prefill kernels.
  * Errors: LB_ERR_INVALID_ARGUMENT (null pointers, negative sizes),
  *   LB_ERR_UNSUPPORTED_SHAPE, LB_ERR_MISALIGNED, LB_ERR_WORKSPACE_TOO_SMALL,
  *   LB_ERR_NOT_SUPPORTED_DEVICE, LB_ERR_CUDA (launch failure).  Conditions

@@ -168,15 +168,27 @@ def test_zero_tokens_is_a_noop():
 
 
 def test_range_overflow_sets_status_not_fault():
-    """|x| beyond the fp16 range on the decode path raises LB_ERR_RANGE on the
-    status word (the kernels keep running; nothing faults)."""
-    layer = synth.make_layer(256, 128, [32], 2, config_id=803)
-    big = np.full((2, 256), 1e6, dtype=np.float32)
+    """g (.) x beyond the fp16 range on the tensor-core decode path (5..32
+    tokens) raises LB_ERR_RANGE on the status word (the kernels keep running;
+    nothing faults)."""
+    layer = synth.make_layer(256, 128, [32], 8, config_id=803)
+    big = np.full((8, 256), 1e8, dtype=np.float32)
     layer["x"] = synth.f32_to_bf16_bits(big)
     assert lb.device_status() == lb.LB_OK
     gu.run_gpu(layer)
     assert lb.device_status() == lb.LB_ERR_RANGE
     assert lb.device_status() == lb.LB_OK          # read clears it
+
+
+def test_small_batch_path_is_fp32_throughout():
+    """1..4 tokens run in fp32 up to the bf16 output: inputs far beyond the
+    fp16 range are fine there."""
+    layer = synth.make_layer(256, 128, [32, 64], 3, config_id=804)
+    xf = oracle.bf16_bits_to_f64(layer["x"]) * 2.0 ** 40
+    layer["x"] = synth.f32_to_bf16_bits(xf.astype(np.float32))
+    y = gu.bf16_to_f64(gu.run_gpu(layer))
+    gu.assert_close(y, gu.oracle_y(layer), "x * 2^40")
+    assert lb.device_status() == lb.LB_OK
 
 
 def test_non_default_stream():
