@@ -35,6 +35,10 @@ constexpr int kT = 512;           // threads per CTA
 constexpr int kNW = kT / 32;      // warps per CTA
 constexpr int kMaxChunkWords = 64;
 constexpr size_t kMaxPartialBytes = 96 * 1024;
+// A nibble table is 16 floats, stored 20 floats (80 bytes) apart: the 16-byte
+// stores of consecutive threads building consecutive tables then start in 8
+// different bank groups, and a lookup still reads one 64-byte table.
+constexpr int kTab = 20;
 
 __host__ __device__ __forceinline__ int quads_of_words(int w) { return (w + 3) / 4; }
 // Row stride in words for bit rows that 16-byte copies fill: a multiple of 4
@@ -102,8 +106,8 @@ __global__ void __launch_bounds__(kT) small_latent_kernel(const SmallLatentParam
     uint16_t *lraw = reinterpret_cast<uint16_t *>(sbits + 32 * p.rg * p.S);  // [32 rg]
     uint16_t *graw = lraw + 32 * p.rg;                                       // [2][ccols]
     uint16_t *xraw = graw + 2 * ccols;                                       // [2][M][ccols]
-    float4 *tab = reinterpret_cast<float4 *>(xraw + 2 * ccols * M);          // [M][cw][8][4]
-    float *red = reinterpret_cast<float *>(tab + 32 * cw * M);               // [kNW][32][MT]
+    float4 *tab = reinterpret_cast<float4 *>(xraw + 2 * ccols * M);          // [M][cw][8][kTab / 4]
+    float *red = reinterpret_cast<float *>(tab + 8 * cw * M * (kTab / 4));   // [kNW][32][MT]
 
     // (1) weights, all asynchronous: sign bits, l slice, g of the first chunk
     if ((ld & 3) == 0) {
@@ -168,7 +172,7 @@ __global__ void __launch_bounds__(kT) small_latent_kernel(const SmallLatentParam
             const float v1 = f16_bits_to_float(gq.x >> 16) * bf16_bits_to_float(xq.x >> 16);
             const float v2 = f16_bits_to_float(gq.y & 0xffff) * bf16_bits_to_float(xq.y & 0xffff);
             const float v3 = f16_bits_to_float(gq.y >> 16) * bf16_bits_to_float(xq.y >> 16);
-            nibble_table(v0, v1, v2, v3, tab + 4 * (m * 8 * cw + wi));
+            nibble_table(v0, v1, v2, v3, tab + (kTab / 4) * (m * 8 * cw + wi));
         }
         __syncthreads();
         // (4) one lookup per 4 sign bits of the row
@@ -182,7 +186,7 @@ __global__ void __launch_bounds__(kT) small_latent_kernel(const SmallLatentParam
                     const int nib = (bits >> (4 * i)) & 15;
 #pragma unroll
                     for (int m = 0; m < MT; ++m) {
-                        const float v = tb[((m * cw + wl) * 8 + i) * 16 + nib];
+                        const float v = tb[((m * cw + wl) * 8 + i) * kTab + nib];
                         if (i & 1) acc2[m] += v;
                         else acc[m] += v;
                     }
@@ -243,8 +247,8 @@ __global__ void __launch_bounds__(kT) small_expand_kernel(const SmallExpandParam
     uint16_t *const sh1 = sh0 + 32 * p.rg;
     uint16_t *const sl = sh1 + (two ? 32 * p.rg : 0);                        // [R] (zmode 1)
     float *const zr = reinterpret_cast<float *>(sl + (p.zmode ? R : 0));     // [cs or 1][R][M]
-    float4 *const tab = reinterpret_cast<float4 *>(zr + (p.zmode ? p.cs : 1) * R * M);  // [M][WT][8][4]
-    float *const red = reinterpret_cast<float *>(tab + 32 * WT * M);        // [kNW][32][MT]
+    float4 *const tab = reinterpret_cast<float4 *>(zr + (p.zmode ? p.cs : 1) * R * M);  // [M][WT][8][kTab / 4]
+    float *const red = reinterpret_cast<float *>(tab + 8 * WT * M * (kTab / 4));        // [kNW][32][MT]
 
     // (1) weights: this CTA's rows of U, h and (zmode 1) l, asynchronously
     for (int pp = 0; pp < p.npaths; ++pp) {
@@ -294,7 +298,7 @@ __global__ void __launch_bounds__(kT) small_expand_kernel(const SmallExpandParam
             }
             v[j] = s;
         }
-        nibble_table(v[0], v[1], v[2], v[3], tab + 4 * (m * 8 * WT + wi));
+        nibble_table(v[0], v[1], v[2], v[3], tab + (kTab / 4) * (m * 8 * WT + wi));
     }
     __syncthreads();
 
@@ -319,7 +323,7 @@ __global__ void __launch_bounds__(kT) small_expand_kernel(const SmallExpandParam
             for (int i = 0; i < 8; ++i) {
                 const int nib = (bits >> (4 * i)) & 15;
 #pragma unroll
-                for (int m = 0; m < MT; ++m) s[m] += tb[((m * WT + w) * 8 + i) * 16 + nib];
+                for (int m = 0; m < MT; ++m) s[m] += tb[((m * WT + w) * 8 + i) * kTab + nib];
             }
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
@@ -360,7 +364,7 @@ size_t small_latent_smem(int rg, int S, int cw, int M)
 {
     const int MT = M <= 1 ? 1 : (M <= 2 ? 2 : 4);
     return (size_t)32 * rg * S * 4 + (size_t)64 * rg + (size_t)128 * cw + (size_t)128 * cw * M +
-           (size_t)512 * cw * M + (size_t)kNW * 32 * MT * 4;
+           (size_t)32 * kTab * cw * M + (size_t)kNW * 32 * MT * 4;
 }
 
 SmallLatentPlan make_small_latent_plan(int rg, int cs, int M, int n_in, const int *ranks, int npaths,
@@ -426,7 +430,7 @@ size_t small_expand_smem(int rg, const int *S, int npaths, int M, int zmode, int
     for (int pp = 0; pp < npaths; ++pp) b += (size_t)32 * rg * S[pp] * 4 + 16 + (size_t)64 * rg;
     if (zmode) b += (size_t)2 * R;
     b += (size_t)(zmode ? cs : 1) * R * M * 4;
-    b += (size_t)(R / 32) * 8 * 64 * M;
+    b += (size_t)(R / 32) * 8 * 4 * kTab * M;
     b += (size_t)kNW * 32 * MT * 4;
     return b;
 }
