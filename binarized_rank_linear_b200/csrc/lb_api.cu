@@ -61,7 +61,7 @@ lb_status device_info(lb::DeviceInfo *out)
         cudaGetLastError();
         return LB_ERR_CUDA;
     }
-    if (lb::decode_prepare_device(info) != cudaSuccess) {
+    if (lb::decode_prepare_device(info) != cudaSuccess || lb::prefill_prepare_device(info) != cudaSuccess) {
         cudaGetLastError();
         return LB_ERR_CUDA;
     }
@@ -97,6 +97,7 @@ lb_status check_path(const lb_path *p, int64_t n_in, int64_t n_out, lb::PathDesc
 
 size_t workspace_for(int64_t tokens, int64_t n_in, int64_t n_out, const int *ranks, int npaths)
 {
+    if (tokens > lb::kDecodeMaxTokens) return lb::prefill_workspace_bytes((int)tokens, ranks, npaths);
     return lb::decode_workspace_bytes((int)tokens, (int)n_in, (int)n_out, ranks, npaths);
 }
 
@@ -228,7 +229,9 @@ lb_status lb_linear_forward(const uint16_t *x, int64_t tokens, int64_t n_in, int
     lb::DeviceInfo dev;
     st = device_info(&dev);
     if (st != LB_OK) return st;
-    const cudaError_t e = lb::decode_forward(a, dev, static_cast<cudaStream_t>(stream));
+    const cudaError_t e = a.tokens > lb::kDecodeMaxTokens
+                              ? lb::prefill_forward(a, dev, static_cast<cudaStream_t>(stream))
+                              : lb::decode_forward(a, dev, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
         cudaGetLastError();
         return LB_ERR_CUDA;

@@ -57,4 +57,10 @@ size_t decode_workspace_bytes(int tokens, int n_in, int n_out, const int *ranks,
 cudaError_t decode_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 cudaError_t decode_prepare_device(const DeviceInfo &dev);
 
+// Prefill path (more than kDecodeMaxTokens tokens): two tcgen05 GEMMs with the
+// binary operand expanded in shared memory (lb_prefill.cu).
+size_t prefill_workspace_bytes(int tokens, const int *ranks, int npaths);
+cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream);
+cudaError_t prefill_prepare_device(const DeviceInfo &dev);
+
 }  // namespace lb
