@@ -38,11 +38,15 @@ namespace lb {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int kThreads = 192;
+constexpr int kProducerWarps = 8;
+constexpr int kThreads = 64 + 32 * kProducerWarps;
+constexpr int kPrefetch = 2;  // K-blocks of sign bits (and g) staged ahead of the one being expanded
 constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KB
 constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
 constexpr uint32_t TMEM_COLS = 256;
-constexpr size_t kSmem = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + 256;
+constexpr uint32_t BITS_BYTES = BN * 8;  // a K-block of sign bits: 64 bits per B row
+constexpr uint32_t G_BYTES = 2 * BK * 2;  // a K-block of g for both paths
+constexpr size_t kSmem = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES + BITS_BYTES + G_BYTES) + 256;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // give up on a wait after 2 s
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -150,6 +154,19 @@ __device__ __forceinline__ uint32_t sw128_offset(int row, int chunk)
     return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+// Barrier over the producer warps (named barrier 1) returning the AND of `ok`.
+__device__ __forceinline__ bool producers_all(bool ok)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, 1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)ok), "n"(32 * kProducerWarps)
+        : "memory");
+    return r != 0;
+}
+
 // Two packed 16-bit scales with the sign bits (bit 0 -> low half, bit 1 ->
 // high half) of a 2-bit group applied.
 __device__ __forceinline__ uint32_t signed_scales(uint32_t scale2, uint32_t bits2)
@@ -179,7 +196,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;  // SW128 tiles need 1024-byte alignment
     const uint32_t sA = base, sB = base + STAGES * A_BYTES;
-    const uint32_t bars = sB + STAGES * B_BYTES;  // full[4], empty[4], accum, then the tmem address
+    const uint32_t sBits = sB + STAGES * B_BYTES;      // ring of packed sign bits, [stage][row][8 bytes]
+    const uint32_t sG = sBits + STAGES * BITS_BYTES;   // ring of g (mode 1), [stage][path][64]
+    const uint32_t bars = sG + STAGES * G_BYTES;       // full[4], empty[4], accum, then the tmem address
     const uint32_t full0 = bars, empty0 = bars + 8 * STAGES, accum = bars + 16 * STAGES;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + (bars + 16 * STAGES + 8 - raw));
     __shared__ int abort_shared;
@@ -191,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             for (int s = 0; s < STAGES; ++s) {
-                mbar_init(full0 + 8 * s, 1 + 4);  // TMA arrive.expect_tx + 4 producer warps
+                mbar_init(full0 + 8 * s, 1 + kProducerWarps);  // TMA arrive.expect_tx + producer warps
                 mbar_init(empty0 + 8 * s, 1);     // one tcgen05.commit
             }
             mbar_init(accum, 1);
@@ -248,106 +267,122 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(accum);
         }
     } else {
-        // ---------------- B producers: 128 threads, 4 rows x 8 chunks per warp step
+        // ---------------- B producers: 8 warps, 4 rows x 8 chunks per warp step
+        const int pt = tid - 64;    // producer thread 0 .. 255; also the B row it stages bits for
         const int wb = warp - 2;
-        const int jc = lane & 7;    // 16-byte chunk (8 columns) of the row
+        const int jc = lane & 7;     // 16-byte chunk (8 columns) of the row
         const int rsub = lane >> 3;  // row within a group of 4
-        // per thread: 16 rows n = 16 * g... (g = wb + 4 t) * 4 + rsub, fixed across K-blocks
-        int rowN[16];
-        int rowp[16];  // path-local row (mode 1) / global output row (mode 2); -1 = outside
-        uint32_t hs[16][2];
+        constexpr int RPT = BN / (4 * kProducerWarps);  // rows per thread per K-block
+        uint32_t hs0[RPT], hs1[RPT];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const int n = 4 * (wb + 4 * t) + rsub;
-            const int nn = n0 + n;
-            rowN[t] = n;
-            if (nn >= p.N) {
-                rowp[t] = -1;
-                hs[t][0] = hs[t][1] = 0u;
-            } else if (MODE == 1) {
-                rowp[t] = nn;
-                hs[t][0] = hs[t][1] = 0u;
-            } else {
-                rowp[t] = nn;
+        for (int t = 0; t < RPT; ++t) {
+            const int nn = n0 + 4 * (wb + kProducerWarps * t) + rsub;
+            hs0[t] = hs1[t] = 0u;
+            if (MODE == 2 && nn < p.N) {
                 const uint32_t h0 = p.s0[nn], h1 = p.s1 ? p.s1[nn] : 0u;
-                hs[t][0] = h0 | (h0 << 16);
-                hs[t][1] = h1 | (h1 << 16);
+                hs0[t] = h0 | (h0 << 16);
+                hs1[t] = h1 | (h1 << 16);
             }
+        }
+        // Stage the sign bits (and g) of K-block kb into ring slot kb % STAGES:
+        // producer thread pt copies the two words of B row pt; 16 threads copy g.
+        auto stage_bits = [&](int kb) {
+            const int slot = kb % STAGES;
+            const int nn = n0 + pt;
+            uint32_t *dst = reinterpret_cast<uint32_t *>(smem_raw + (sBits + slot * BITS_BYTES + pt * 8 - raw));
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+                const int kc = kb * BK + 32 * w;  // first column of this word
+                const uint32_t *src = p.bits0;
+                bool real = nn < p.N && kc < p.K;
+                if (real) {
+                    if (MODE == 1) {
+                        const bool sec = nn >= p.r0;
+                        src = (sec ? p.bits1 : p.bits0) + (int64_t)(sec ? nn - p.r0 : nn) * (sec ? p.bld1 : p.bld0) +
+                              (kc >> 5);
+                    } else {
+                        const bool sec = kc >= p.r0;
+                        src = (sec ? p.bits1 : p.bits0) + (int64_t)nn * (sec ? p.bld1 : p.bld0) +
+                              ((sec ? kc - p.r0 : kc) >> 5);
+                    }
+                }
+                cp_async4(dst + w, src, real ? 4u : 0u);
+            }
+            if (MODE == 1 && pt < 16) {
+                const int pp = pt >> 3, c = pt & 7;
+                const int k0 = kb * BK + 8 * c;
+                const uint16_t *gs = pp ? p.s1 : p.s0;
+                const bool real = gs != nullptr && k0 < p.K;
+                cp_async16(smem_raw + (sG + slot * G_BYTES + pp * (BK * 2) + c * 16 - raw), real ? gs + k0 : p.s0,
+                           real ? 16u : 0u);
+            }
+        };
+        // exactly kPrefetch groups ahead of the loop (empty when there are fewer
+        // K-blocks), so wait_group<kPrefetch> below always covers block kb
+        for (int kb = 0; kb < kPrefetch; ++kb) {
+            if (kb < nk) stage_bits(kb);
+            cp_async_commit();
         }
         for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-            if (!mbar_wait(empty0 + 8 * s, ph ^ 1u) || abort_flag) {
+            if (kb + kPrefetch < nk) stage_bits(kb + kPrefetch);
+            cp_async_commit();  // one group per K-block on every thread (possibly empty)
+            cp_async_wait_group<kPrefetch>();
+            // wait for the MMA to release stage s, then one barrier over the
+            // producer threads that both publishes every thread's staged bits
+            // and makes the give-up decision the same for all of them (a
+            // plain bar.sync would wait forever for a thread that left)
+            bool ok = mbar_wait(empty0 + 8 * s, ph ^ 1u) && !abort_flag;
+            ok = producers_all(ok);
+            if (!ok) {
                 abort_flag = 1;
                 break;
             }
-            const int k0 = kb * BK + 8 * jc;  // first column of this thread's chunk
+            const uint8_t *bits = smem_raw + (sBits + s * BITS_BYTES - raw);
+            const int k0 = kb * BK + 8 * jc;
             const bool kin = k0 < p.K;
             const uint32_t tile = sB + s * B_BYTES;
+            uint32_t g0[4] = {0u, 0u, 0u, 0u}, g1[4] = {0u, 0u, 0u, 0u};
             if (MODE == 1) {
-                // scale by column: g_p[k0 .. k0+7] rounded to bf16 (both paths)
-                uint32_t g2[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
-                if (kin) {
+                // g of this chunk, both paths, rounded to bf16 pairs
+                const uint4 q0 = *reinterpret_cast<const uint4 *>(smem_raw + (sG + s * G_BYTES + jc * 16 - raw));
+                const uint4 q1 = *reinterpret_cast<const uint4 *>(smem_raw + (sG + s * G_BYTES + BK * 2 + jc * 16 - raw));
+                const uint32_t w0[4] = {q0.x, q0.y, q0.z, q0.w}, w1[4] = {q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
-                    for (int pp = 0; pp < 2; ++pp) {
-                        const uint16_t *gs = pp ? p.s1 : p.s0;
-                        if (gs) {
-                            const uint4 q = __ldg(reinterpret_cast<const uint4 *>(gs + k0));
-                            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const float lo = f16_bits_to_float((uint16_t)(w[i] & 0xffffu));
-                                const float hi = f16_bits_to_float((uint16_t)(w[i] >> 16));
-                                g2[pp][i] = (uint32_t)float_to_bf16_bits(lo) | ((uint32_t)float_to_bf16_bits(hi) << 16);
-                            }
-                        }
-                    }
+                for (int i = 0; i < 4; ++i) {
+                    g0[i] = (uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w0[i] & 0xffffu))) |
+                            ((uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w0[i] >> 16))) << 16);
+                    g1[i] = (uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w1[i] & 0xffffu))) |
+                            ((uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w1[i] >> 16))) << 16);
                 }
+            }
+            const bool sec2 = MODE == 2 && k0 >= p.r0;  // mode 2: path of this chunk's columns
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    const int nn = rowp[t];
-                    if (nn >= 0 && kin) {
-                        const bool sec = nn >= p.r0;
-                        const int row = sec ? nn - p.r0 : nn;
-                        const uint32_t *b = (sec ? p.bits1 : p.bits0) + (int64_t)row * (sec ? p.bld1 : p.bld0);
-                        const uint32_t byte = (__ldg(b + (k0 >> 5)) >> (k0 & 31)) & 0xffu;
-                        v = make_uint4(signed_scales(sec ? g2[1][0] : g2[0][0], byte),
-                                       signed_scales(sec ? g2[1][1] : g2[0][1], byte >> 2),
-                                       signed_scales(sec ? g2[1][2] : g2[0][2], byte >> 4),
-                                       signed_scales(sec ? g2[1][3] : g2[0][3], byte >> 6));
-                    }
-                    const uint32_t dst = tile + sw128_offset(rowN[t], jc);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
-                                 "r"(v.w)
-                                 : "memory");
+            for (int t = 0; t < RPT; ++t) {
+                const int n = 4 * (wb + kProducerWarps * t) + rsub;
+                const uint32_t byte = bits[n * 8 + jc];  // zero for rows/columns outside the matrix
+                uint4 v;
+                if (MODE == 1) {
+                    const bool sec = n0 + n >= p.r0;
+                    v = make_uint4(signed_scales(sec ? g1[0] : g0[0], byte), signed_scales(sec ? g1[1] : g0[1], byte >> 2),
+                                   signed_scales(sec ? g1[2] : g0[2], byte >> 4),
+                                   signed_scales(sec ? g1[3] : g0[3], byte >> 6));
+                } else {
+                    const uint32_t h = (n0 + n < p.N && kin) ? (sec2 ? hs1[t] : hs0[t]) : 0u;
+                    v = make_uint4(signed_scales(h, byte), signed_scales(h, byte >> 2), signed_scales(h, byte >> 4),
+                                   signed_scales(h, byte >> 6));
                 }
-            } else {
-                // scale by row (h of the chunk's path); bits from the path's U row
-                const bool sec = k0 >= p.r0;
-                const int kk = sec ? k0 - p.r0 : k0;
-                const uint32_t *bits = sec ? p.bits1 : p.bits0;
-                const int64_t bld = sec ? p.bld1 : p.bld0;
-#pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    const int nn = rowp[t];
-                    if (nn >= 0 && kin) {
-                        const uint32_t byte = (__ldg(bits + (int64_t)nn * bld + (kk >> 5)) >> (kk & 31)) & 0xffu;
-                        const uint32_t h = sec ? hs[t][1] : hs[t][0];
-                        v = make_uint4(signed_scales(h, byte), signed_scales(h, byte >> 2), signed_scales(h, byte >> 4),
-                                       signed_scales(h, byte >> 6));
-                    }
-                    const uint32_t dst = tile + sw128_offset(rowN[t], jc);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
-                                 "r"(v.w)
-                                 : "memory");
-                }
+                const uint32_t dst = tile + sw128_offset(n, jc);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
+                             "r"(v.w)
+                             : "memory");
             }
             fence_async_shared();
             __syncwarp();
             if (lane == 0) mbar_arrive(full0 + 8 * s);
         }
+        cp_async_wait_all();
 
         // ---------------- epilogue: tensor memory -> registers -> global
         bool ok = !abort_flag;
@@ -357,8 +392,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int quad = warp & 3;  // warp w reads tensor-memory lanes 32 (w % 4) ..
         const int m = m0 + 32 * quad + lane;
+        const int cbeg = ((warp - 2) / 4) * (BN / 2);  // two warps per lane quadrant: column halves
         bool overflow = false;
-        for (int c0 = 0; c0 < BN; c0 += 16) {
+        for (int c0 = cbeg; c0 < cbeg + BN / 2; c0 += 16) {
             uint32_t v[16];
             if (ok) tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)c0, v);
             const int nn = n0 + c0;
