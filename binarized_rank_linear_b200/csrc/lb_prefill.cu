@@ -19,7 +19,7 @@
 //               swizzle, no multicast)
 //   warp 1      one thread issues tcgen05.mma (M = 128, N = 256, K = 16) and
 //               commits each stage back to its producers
-//   warps 2..5  expand the packed sign bits of the stage's B tile into
+//   warps 2..9  one B row per thread: expand the row's packed sign bits into
 //               +-scale values in the same swizzled layout, then read the
 //               accumulator out of tensor memory and store the tile
 // Stages are handed over with mbarriers (4-deep ring).  Every wait is bounded
@@ -40,13 +40,13 @@ namespace {
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int kProducerWarps = 8;
 constexpr int kThreads = 64 + 32 * kProducerWarps;
-constexpr int kPrefetch = 2;  // K-blocks of sign bits (and g) staged ahead of the one being expanded
+constexpr int kPrefetch = 3;  // K-blocks of sign bits (and g) staged ahead of the one being expanded
 constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KB
 constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t BITS_BYTES = BN * 8;  // a K-block of sign bits: 64 bits per B row
 constexpr uint32_t G_BYTES = 2 * BK * 2;  // a K-block of g for both paths
-constexpr size_t kSmem = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES + BITS_BYTES + G_BYTES) + 256;
+constexpr size_t kSmem = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES + BITS_BYTES + 2 * G_BYTES) + 256;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // give up on a wait after 2 s
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -146,13 +146,9 @@ __device__ __forceinline__ uint32_t instr_desc(uint32_t fmt)
     return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
-// Byte offset of element (row, k) of a 128-byte-swizzled K-major tile whose
-// rows are 64 two-byte elements: 16-byte chunk k/8 of row `row` is stored at
-// chunk position (k/8) ^ (row % 8).
-__device__ __forceinline__ uint32_t sw128_offset(int row, int chunk)
-{
-    return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
-}
+// Tiles are K-major with 128-byte swizzle: row `row` holds 64 two-byte
+// elements in 128 bytes, and its 16-byte chunk j (elements 8j .. 8j + 7) is
+// stored at chunk position j ^ (row % 8).
 
 // Barrier over the producer warps (named barrier 1) returning the AND of `ok`.
 __device__ __forceinline__ bool producers_all(bool ok)
@@ -165,13 +161,6 @@ __device__ __forceinline__ bool producers_all(bool ok)
         : "r"((uint32_t)ok), "n"(32 * kProducerWarps)
         : "memory");
     return r != 0;
-}
-
-// Two packed 16-bit scales with the sign bits (bit 0 -> low half, bit 1 ->
-// high half) of a 2-bit group applied.
-__device__ __forceinline__ uint32_t signed_scales(uint32_t scale2, uint32_t bits2)
-{
-    return scale2 ^ (((bits2 & 3u) * 0x40008000u) & 0x80008000u);
 }
 
 // ---------------------------------------------------------------- kernel
@@ -197,8 +186,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;  // SW128 tiles need 1024-byte alignment
     const uint32_t sA = base, sB = base + STAGES * A_BYTES;
     const uint32_t sBits = sB + STAGES * B_BYTES;      // ring of packed sign bits, [stage][row][8 bytes]
-    const uint32_t sG = sBits + STAGES * BITS_BYTES;   // ring of g (mode 1), [stage][path][64]
-    const uint32_t bars = sG + STAGES * G_BYTES;       // full[4], empty[4], accum, then the tmem address
+    const uint32_t sG16 = sBits + STAGES * BITS_BYTES;  // ring of g as given (mode 1), [stage][path][64]
+    const uint32_t sGbf = sG16 + STAGES * G_BYTES;      // the same rounded to bf16
+    const uint32_t bars = sGbf + STAGES * G_BYTES;      // full[4], empty[4], accum, then the tmem address
     const uint32_t full0 = bars, empty0 = bars + 8 * STAGES, accum = bars + 16 * STAGES;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + (bars + 16 * STAGES + 8 - raw));
     __shared__ int abort_shared;
@@ -267,115 +257,127 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(accum);
         }
     } else {
-        // ---------------- B producers: 8 warps, 4 rows x 8 chunks per warp step
-        const int pt = tid - 64;    // producer thread 0 .. 255; also the B row it stages bits for
-        const int wb = warp - 2;
-        const int jc = lane & 7;     // 16-byte chunk (8 columns) of the row
-        const int rsub = lane >> 3;  // row within a group of 4
-        constexpr int RPT = BN / (4 * kProducerWarps);  // rows per thread per K-block
-        uint32_t hs0[RPT], hs1[RPT];
-#pragma unroll
-        for (int t = 0; t < RPT; ++t) {
-            const int nn = n0 + 4 * (wb + kProducerWarps * t) + rsub;
-            hs0[t] = hs1[t] = 0u;
-            if (MODE == 2 && nn < p.N) {
-                const uint32_t h0 = p.s0[nn], h1 = p.s1 ? p.s1[nn] : 0u;
-                hs0[t] = h0 | (h0 << 16);
-                hs1[t] = h1 | (h1 << 16);
+        // ---------------- B producers: 8 warps, producer thread pt owns B row pt
+        // of the tile.  Each K-block it copies the row's 64 sign bits into a
+        // ring slot with its own asynchronous copies, so it needs no barrier to
+        // read them back; the scales are shared, so those go through a barrier.
+        const int pt = tid - 64;
+        const int nn = n0 + pt;  // row of B (mode 1: latent index; mode 2: output row)
+        const uint32_t x7 = (uint32_t)(pt & 7);  // the row's 128-byte swizzle: logical chunk j sits at chunk j ^ x7
+        const bool row_in = nn < p.N;
+        const bool sec_row = MODE == 1 && nn >= p.r0;  // mode 1: the row's path
+        uint32_t hs0 = 0u, hs1 = 0u;                   // mode 2: h of the row, both halves
+        if (MODE == 2 && row_in) {
+            const uint32_t h0 = p.s0[nn], h1 = p.s1 ? p.s1[nn] : 0u;
+            hs0 = h0 | (h0 << 16);
+            hs1 = h1 | (h1 << 16);
+        }
+        const uint32_t *row_bits0 = nullptr;  // mode 1: the row's packed words; mode 2: path 0 row
+        const uint32_t *row_bits1 = nullptr;  // mode 2: path 1 row
+        if (row_in) {
+            if (MODE == 1)
+                row_bits0 = sec_row ? p.bits1 + (int64_t)(nn - p.r0) * p.bld1 : p.bits0 + (int64_t)nn * p.bld0;
+            else {
+                row_bits0 = p.bits0 + (int64_t)nn * p.bld0;
+                if (p.bits1) row_bits1 = p.bits1 + (int64_t)nn * p.bld1;
             }
         }
-        // Stage the sign bits (and g) of K-block kb into ring slot kb % STAGES:
-        // producer thread pt copies the two words of B row pt; 16 threads copy g.
-        auto stage_bits = [&](int kb) {
+        const int kwords = p.K >> 5, r0w = p.r0 >> 5;
+        // Stage K-block kb: the row's two packed words, and (mode 1) one 16-byte
+        // piece of g per thread 0..15 (path pt / 8, chunk pt % 8) in fp16.
+        auto stage = [&](int kb) {
             const int slot = kb % STAGES;
-            const int nn = n0 + pt;
-            uint32_t *dst = reinterpret_cast<uint32_t *>(smem_raw + (sBits + slot * BITS_BYTES + pt * 8 - raw));
+            uint8_t *dst = smem_raw + (sBits + slot * BITS_BYTES + pt * 8 - raw);
 #pragma unroll
             for (int w = 0; w < 2; ++w) {
-                const int kc = kb * BK + 32 * w;  // first column of this word
+                const int wd = 2 * kb + w;  // word of the concatenated row
                 const uint32_t *src = p.bits0;
-                bool real = nn < p.N && kc < p.K;
+                bool real = row_in && wd < kwords;
                 if (real) {
-                    if (MODE == 1) {
-                        const bool sec = nn >= p.r0;
-                        src = (sec ? p.bits1 : p.bits0) + (int64_t)(sec ? nn - p.r0 : nn) * (sec ? p.bld1 : p.bld0) +
-                              (kc >> 5);
-                    } else {
-                        const bool sec = kc >= p.r0;
-                        src = (sec ? p.bits1 : p.bits0) + (int64_t)nn * (sec ? p.bld1 : p.bld0) +
-                              ((sec ? kc - p.r0 : kc) >> 5);
-                    }
+                    if (MODE == 1) src = row_bits0 + wd;
+                    else src = wd < r0w ? row_bits0 + wd : row_bits1 + (wd - r0w);
                 }
-                cp_async4(dst + w, src, real ? 4u : 0u);
+                cp_async4(dst + 4 * w, src, real ? 4u : 0u);
             }
             if (MODE == 1 && pt < 16) {
                 const int pp = pt >> 3, c = pt & 7;
                 const int k0 = kb * BK + 8 * c;
                 const uint16_t *gs = pp ? p.s1 : p.s0;
                 const bool real = gs != nullptr && k0 < p.K;
-                cp_async16(smem_raw + (sG + slot * G_BYTES + pp * (BK * 2) + c * 16 - raw), real ? gs + k0 : p.s0,
-                           real ? 16u : 0u);
+                cp_async16(smem_raw + (sG16 + slot * G_BYTES + pt * 16 - raw), real ? gs + k0 : p.s0, real ? 16u : 0u);
             }
         };
-        // exactly kPrefetch groups ahead of the loop (empty when there are fewer
-        // K-blocks), so wait_group<kPrefetch> below always covers block kb
+        // Mode 1: thread pt < 16 rounds its own fp16 piece of K-block kb to bf16
+        // and publishes it (the next producer barrier makes it visible).
+        auto convert_g = [&](int kb) {
+            if (MODE == 1 && pt < 16) {
+                const int slot = kb % STAGES;
+                const uint4 q = *reinterpret_cast<const uint4 *>(smem_raw + (sG16 + slot * G_BYTES + pt * 16 - raw));
+                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+                uint32_t o[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    o[i] = (uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[i] & 0xffffu))) |
+                           ((uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[i] >> 16))) << 16);
+                *reinterpret_cast<uint4 *>(smem_raw + (sGbf + slot * G_BYTES + pt * 16 - raw)) =
+                    make_uint4(o[0], o[1], o[2], o[3]);
+            }
+        };
+        // kPrefetch groups ahead (empty ones past the end), so that in
+        // iteration kb wait_group<kPrefetch - 1> leaves blocks <= kb + 1 landed
         for (int kb = 0; kb < kPrefetch; ++kb) {
-            if (kb < nk) stage_bits(kb);
+            if (kb < nk) stage(kb);
             cp_async_commit();
         }
+        cp_async_wait_group<kPrefetch - 1>();
+        convert_g(0);
         for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-            if (kb + kPrefetch < nk) stage_bits(kb + kPrefetch);
+            if (kb + kPrefetch < nk) stage(kb + kPrefetch);
             cp_async_commit();  // one group per K-block on every thread (possibly empty)
-            cp_async_wait_group<kPrefetch>();
+            cp_async_wait_group<kPrefetch - 1>();
             // wait for the MMA to release stage s, then one barrier over the
-            // producer threads that both publishes every thread's staged bits
-            // and makes the give-up decision the same for all of them (a
-            // plain bar.sync would wait forever for a thread that left)
+            // producer threads that both publishes the bf16 g of this block and
+            // makes the give-up decision the same for all of them (a plain
+            // bar.sync would wait forever for a thread that left)
             bool ok = mbar_wait(empty0 + 8 * s, ph ^ 1u) && !abort_flag;
             ok = producers_all(ok);
             if (!ok) {
                 abort_flag = 1;
                 break;
             }
-            const uint8_t *bits = smem_raw + (sBits + s * BITS_BYTES - raw);
-            const int k0 = kb * BK + 8 * jc;
-            const bool kin = k0 < p.K;
-            const uint32_t tile = sB + s * B_BYTES;
-            uint32_t g0[4] = {0u, 0u, 0u, 0u}, g1[4] = {0u, 0u, 0u, 0u};
+            if (kb + 1 < nk) convert_g(kb + 1);  // its slot was last read three blocks ago
+            // the row's 64 sign bits: byte j holds columns 8j .. 8j + 7
+            const uint2 wb2 = *reinterpret_cast<const uint2 *>(smem_raw + (sBits + s * BITS_BYTES + pt * 8 - raw));
+            uint4 sc[8];  // per chunk: the four packed scale words
             if (MODE == 1) {
-                // g of this chunk, both paths, rounded to bf16 pairs
-                const uint4 q0 = *reinterpret_cast<const uint4 *>(smem_raw + (sG + s * G_BYTES + jc * 16 - raw));
-                const uint4 q1 = *reinterpret_cast<const uint4 *>(smem_raw + (sG + s * G_BYTES + BK * 2 + jc * 16 - raw));
-                const uint32_t w0[4] = {q0.x, q0.y, q0.z, q0.w}, w1[4] = {q1.x, q1.y, q1.z, q1.w};
+                const uint8_t *gb = smem_raw + (sGbf + s * G_BYTES + (sec_row ? BK * 2 : 0) - raw);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    g0[i] = (uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w0[i] & 0xffffu))) |
-                            ((uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w0[i] >> 16))) << 16);
-                    g1[i] = (uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w1[i] & 0xffffu))) |
-                            ((uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w1[i] >> 16))) << 16);
+                for (int q = 0; q < 8; ++q) sc[q] = *reinterpret_cast<const uint4 *>(gb + 16 * q);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int k0 = kb * BK + 8 * q;  // first column of the chunk
+                    const uint32_t h = k0 < p.K ? (k0 >= p.r0 ? hs1 : hs0) : 0u;
+                    sc[q] = make_uint4(h, h, h, h);
                 }
             }
-            const bool sec2 = MODE == 2 && k0 >= p.r0;  // mode 2: path of this chunk's columns
+            // chunk q of the row goes to chunk position q ^ x7 (the tile is
+            // 1024-byte aligned, so the XOR acts on address bits 4..6 alone);
+            // the 8 rows of a store phase then cover all 32 banks
+            const uint32_t rowx = (sB + s * B_BYTES + pt * 128) | (x7 << 4);
 #pragma unroll
-            for (int t = 0; t < RPT; ++t) {
-                const int n = 4 * (wb + kProducerWarps * t) + rsub;
-                const uint32_t byte = bits[n * 8 + jc];  // zero for rows/columns outside the matrix
-                uint4 v;
-                if (MODE == 1) {
-                    const bool sec = n0 + n >= p.r0;
-                    v = make_uint4(signed_scales(sec ? g1[0] : g0[0], byte), signed_scales(sec ? g1[1] : g0[1], byte >> 2),
-                                   signed_scales(sec ? g1[2] : g0[2], byte >> 4),
-                                   signed_scales(sec ? g1[3] : g0[3], byte >> 6));
-                } else {
-                    const uint32_t h = (n0 + n < p.N && kin) ? (sec2 ? hs1[t] : hs0[t]) : 0u;
-                    v = make_uint4(signed_scales(h, byte), signed_scales(h, byte >> 2), signed_scales(h, byte >> 4),
-                                   signed_scales(h, byte >> 6));
-                }
-                const uint32_t dst = tile + sw128_offset(n, jc);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
-                             "r"(v.w)
+            for (int q = 0; q < 8; ++q) {
+                const uint32_t b = __byte_perm(q < 4 ? wb2.x : wb2.y, 0u, 0x4440u | (uint32_t)(q & 3));
+                // (b * K_i) puts sign bit 2i at bit 15 and bit 2i + 1 at bit 31
+                // (the two shifted copies of the byte do not overlap: no carries)
+                const uint32_t v0 = ((b * 0x40008000u) & 0x80008000u) ^ sc[q].x;
+                const uint32_t v1 = ((b * 0x10002000u) & 0x80008000u) ^ sc[q].y;
+                const uint32_t v2 = ((b * 0x04000800u) & 0x80008000u) ^ sc[q].z;
+                const uint32_t v3 = ((b * 0x01000200u) & 0x80008000u) ^ sc[q].w;
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowx ^ (16u * q)), "r"(v0), "r"(v1),
+                             "r"(v2), "r"(v3)
                              : "memory");
             }
             fence_async_shared();
