@@ -33,6 +33,12 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t 
                  :: "r"(smem_u32(dst)), "l"(src), "r"(src_bytes) : "memory");
 }
 
+__device__ __forceinline__ void cp_async8(void *dst, const void *src, uint32_t src_bytes = 8)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n"
+                 :: "r"(smem_u32(dst)), "l"(src), "r"(src_bytes) : "memory");
+}
+
 __device__ __forceinline__ void cp_async4(void *dst, const void *src, uint32_t src_bytes = 4)
 {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n"

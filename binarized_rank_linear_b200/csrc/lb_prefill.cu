@@ -46,7 +46,10 @@ constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t BITS_BYTES = BN * 8;  // a K-block of sign bits: 64 bits per B row
 constexpr uint32_t G_BYTES = 2 * BK * 2;  // a K-block of g for both paths
-constexpr size_t kSmem = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES + BITS_BYTES + 2 * G_BYTES) + 256;
+// per stage: A tile, B tile, sign bits; per producer warp: its own g ring as
+// given (STAGES deep) and rounded to bf16 (2 deep)
+constexpr size_t kSmem =
+    1024 + (size_t)STAGES * (A_BYTES + B_BYTES + BITS_BYTES) + (size_t)kProducerWarps * (STAGES + 2) * G_BYTES + 256;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // give up on a wait after 2 s
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -150,23 +153,11 @@ __device__ __forceinline__ uint32_t instr_desc(uint32_t fmt)
 // elements in 128 bytes, and its 16-byte chunk j (elements 8j .. 8j + 7) is
 // stored at chunk position j ^ (row % 8).
 
-// Barrier over the producer warps (named barrier 1) returning the AND of `ok`.
-__device__ __forceinline__ bool producers_all(bool ok)
-{
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.and.pred p, 1, %2, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)ok), "n"(32 * kProducerWarps)
-        : "memory");
-    return r != 0;
-}
-
 // ---------------------------------------------------------------- kernel
 struct SignGemmParams {
     int M, N, K;
     int r0;  // mode 1: B rows [0, r0) are path 0; mode 2: K columns [0, r0) are path 0
+    int bits8;  // every K-block's two words of a row can be fetched as one aligned 8-byte copy
     const uint32_t *bits0, *bits1;
     int64_t bld0, bld1;          // words per packed row
     const uint16_t *s0, *s1;     // mode 1: g (fp16, length K); mode 2: h (fp16, length N)
@@ -186,9 +177,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;  // SW128 tiles need 1024-byte alignment
     const uint32_t sA = base, sB = base + STAGES * A_BYTES;
     const uint32_t sBits = sB + STAGES * B_BYTES;      // ring of packed sign bits, [stage][row][8 bytes]
-    const uint32_t sG16 = sBits + STAGES * BITS_BYTES;  // ring of g as given (mode 1), [stage][path][64]
-    const uint32_t sGbf = sG16 + STAGES * G_BYTES;      // the same rounded to bf16
-    const uint32_t bars = sGbf + STAGES * G_BYTES;      // full[4], empty[4], accum, then the tmem address
+    const uint32_t sG16 = sBits + STAGES * BITS_BYTES;  // mode 1, per producer warp: g as given, [warp][stage][path][64]
+    const uint32_t sGbf = sG16 + kProducerWarps * STAGES * G_BYTES;  // the same rounded to bf16, [warp][2][path][64]
+    const uint32_t bars = sGbf + kProducerWarps * 2 * G_BYTES;       // full[4], empty[4], accum, then the tmem address
     const uint32_t full0 = bars, empty0 = bars + 8 * STAGES, accum = bars + 16 * STAGES;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + (bars + 16 * STAGES + 8 - raw));
     __shared__ int abort_shared;
@@ -259,9 +250,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ---------------- B producers: 8 warps, producer thread pt owns B row pt
         // of the tile.  Each K-block it copies the row's 64 sign bits into a
-        // ring slot with its own asynchronous copies, so it needs no barrier to
-        // read them back; the scales are shared, so those go through a barrier.
+        // ring slot with its own asynchronous copies, and each warp keeps its
+        // own copy of g, so the producer warps never wait for one another:
+        // they only meet at the stage barriers the MMA thread waits on.
         const int pt = tid - 64;
+        const int wb = warp - 2;
         const int nn = n0 + pt;  // row of B (mode 1: latent index; mode 2: output row)
         const uint32_t x7 = (uint32_t)(pt & 7);  // the row's 128-byte swizzle: logical chunk j sits at chunk j ^ x7
         const bool row_in = nn < p.N;
@@ -283,43 +276,52 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         const int kwords = p.K >> 5, r0w = p.r0 >> 5;
-        // Stage K-block kb: the row's two packed words, and (mode 1) one 16-byte
-        // piece of g per thread 0..15 (path pt / 8, chunk pt % 8) in fp16.
+        const uint32_t g16w = sG16 + (uint32_t)wb * STAGES * G_BYTES, gbfw = sGbf + (uint32_t)wb * 2 * G_BYTES;
+        // Stage K-block kb: the row's two packed words (one 8-byte copy when
+        // both sit 8-byte aligned in one path), and (mode 1) lanes 0..15 copy
+        // one 16-byte piece of g each (path lane / 8, chunk lane % 8).
         auto stage = [&](int kb) {
             const int slot = kb % STAGES;
             uint8_t *dst = smem_raw + (sBits + slot * BITS_BYTES + pt * 8 - raw);
-#pragma unroll
-            for (int w = 0; w < 2; ++w) {
-                const int wd = 2 * kb + w;  // word of the concatenated row
+            const int wd = 2 * kb;  // first word of the block in the concatenated row
+            if (p.bits8) {
                 const uint32_t *src = p.bits0;
-                bool real = row_in && wd < kwords;
-                if (real) {
-                    if (MODE == 1) src = row_bits0 + wd;
-                    else src = wd < r0w ? row_bits0 + wd : row_bits1 + (wd - r0w);
+                uint32_t bytes = 0u;
+                if (row_in && wd < kwords) {
+                    src = (MODE == 1 || wd < r0w) ? row_bits0 + wd : row_bits1 + (wd - r0w);
+                    bytes = wd + 1 < kwords ? 8u : 4u;
                 }
-                cp_async4(dst + 4 * w, src, real ? 4u : 0u);
+                cp_async8(dst, src, bytes);
+            } else {
+#pragma unroll
+                for (int w = 0; w < 2; ++w) {
+                    const uint32_t *src = p.bits0;
+                    const bool real = row_in && wd + w < kwords;
+                    if (real) src = (MODE == 1 || wd + w < r0w) ? row_bits0 + wd + w : row_bits1 + (wd + w - r0w);
+                    cp_async4(dst + 4 * w, src, real ? 4u : 0u);
+                }
             }
-            if (MODE == 1 && pt < 16) {
-                const int pp = pt >> 3, c = pt & 7;
+            if (MODE == 1 && lane < 16) {
+                const int pp = lane >> 3, c = lane & 7;
                 const int k0 = kb * BK + 8 * c;
                 const uint16_t *gs = pp ? p.s1 : p.s0;
                 const bool real = gs != nullptr && k0 < p.K;
-                cp_async16(smem_raw + (sG16 + slot * G_BYTES + pt * 16 - raw), real ? gs + k0 : p.s0, real ? 16u : 0u);
+                cp_async16(smem_raw + (g16w + slot * G_BYTES + lane * 16 - raw), real ? gs + k0 : p.s0,
+                           real ? 16u : 0u);
             }
         };
-        // Mode 1: thread pt < 16 rounds its own fp16 piece of K-block kb to bf16
-        // and publishes it (the next producer barrier makes it visible).
+        // Mode 1: lanes 0..15 round their own fp16 piece of K-block kb to bf16
+        // into the warp's slot kb % 2 (the warp reads it after a __syncwarp).
         auto convert_g = [&](int kb) {
-            if (MODE == 1 && pt < 16) {
-                const int slot = kb % STAGES;
-                const uint4 q = *reinterpret_cast<const uint4 *>(smem_raw + (sG16 + slot * G_BYTES + pt * 16 - raw));
+            if (MODE == 1 && lane < 16) {
+                const uint4 q = *reinterpret_cast<const uint4 *>(smem_raw + (g16w + (kb % STAGES) * G_BYTES + lane * 16 - raw));
                 const uint32_t w[4] = {q.x, q.y, q.z, q.w};
                 uint32_t o[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     o[i] = (uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[i] & 0xffffu))) |
                            ((uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[i] >> 16))) << 16);
-                *reinterpret_cast<uint4 *>(smem_raw + (sGbf + slot * G_BYTES + pt * 16 - raw)) =
+                *reinterpret_cast<uint4 *>(smem_raw + (gbfw + (kb & 1) * G_BYTES + lane * 16 - raw)) =
                     make_uint4(o[0], o[1], o[2], o[3]);
             }
         };
@@ -331,28 +333,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         cp_async_wait_group<kPrefetch - 1>();
         convert_g(0);
+        __syncwarp();
         for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
             if (kb + kPrefetch < nk) stage(kb + kPrefetch);
             cp_async_commit();  // one group per K-block on every thread (possibly empty)
             cp_async_wait_group<kPrefetch - 1>();
-            // wait for the MMA to release stage s, then one barrier over the
-            // producer threads that both publishes the bf16 g of this block and
-            // makes the give-up decision the same for all of them (a plain
-            // bar.sync would wait forever for a thread that left)
+            // wait for the MMA to release stage s; the give-up decision is
+            // made per warp (the arrive below is per warp)
             bool ok = mbar_wait(empty0 + 8 * s, ph ^ 1u) && !abort_flag;
-            ok = producers_all(ok);
+            ok = __all_sync(0xffffffffu, ok);
             if (!ok) {
                 abort_flag = 1;
                 break;
             }
-            if (kb + 1 < nk) convert_g(kb + 1);  // its slot was last read three blocks ago
+            // slot (kb + 1) % 2 was last read in the previous iteration, before its __syncwarp
+            if (kb + 1 < nk) convert_g(kb + 1);
             // the row's 64 sign bits: byte j holds columns 8j .. 8j + 7
             const uint2 wb2 = *reinterpret_cast<const uint2 *>(smem_raw + (sBits + s * BITS_BYTES + pt * 8 - raw));
             uint4 sc[8];  // per chunk: the four packed scale words
             if (MODE == 1) {
-                const uint8_t *gb = smem_raw + (sGbf + s * G_BYTES + (sec_row ? BK * 2 : 0) - raw);
+                const uint8_t *gb = smem_raw + (gbfw + (kb & 1) * G_BYTES + (sec_row ? BK * 2 : 0) - raw);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) sc[q] = *reinterpret_cast<const uint4 *>(gb + 16 * q);
             } else {
@@ -468,6 +470,9 @@ cudaError_t encode_a(CUtensorMap *tm, const void *ptr, int rows, int cols, int64
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// True when every row of a packed matrix starts 8-byte aligned.
+bool even8(const uint32_t *bits, int64_t ld) { return (reinterpret_cast<uintptr_t>(bits) & 7u) == 0 && ld % 2 == 0; }
+
 }  // namespace
 
 cudaError_t prefill_prepare_device(const DeviceInfo &dev)
@@ -504,6 +509,7 @@ cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStr
     p1.N = R;
     p1.K = a.n_in;
     p1.r0 = r0;
+    p1.bits8 = even8(a.path[0].vt_bits, a.path[0].vt_ld) && (a.npaths < 2 || even8(a.path[1].vt_bits, a.path[1].vt_ld));
     p1.bits0 = a.path[0].vt_bits;
     p1.bld0 = a.path[0].vt_ld;
     p1.s0 = a.path[0].g;
@@ -531,6 +537,7 @@ cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStr
     p2.N = a.n_out;
     p2.K = R;
     p2.r0 = r0;
+    p2.bits8 = even8(a.path[0].u_bits, a.path[0].u_ld) && (a.npaths < 2 || (r0 % 64 == 0 && even8(a.path[1].u_bits, a.path[1].u_ld)));
     p2.bits0 = a.path[0].u_bits;
     p2.bld0 = a.path[0].u_ld;
     p2.s0 = a.path[0].h;
