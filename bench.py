@@ -44,7 +44,7 @@ from binarized_rank_linear_b200 import synth  # noqa: E402
 METRIC = "LittleBitLinear µs/call & HBM GB/s (batch 1); prefill TFLOP/s; % of roofline"
 DECODE_MAX_TOKENS = 32
 L2_BYTES = 126 * 1024 * 1024
-KERNEL_SOURCES = ["lb_common.cuh", "lb_decode.cu", "lb_internal.h", "lb_api.cu"]
+CSRC = os.path.join(ROOT, "binarized_rank_linear_b200", "csrc")
 
 
 # ---------------------------------------------------------------- workload arithmetic
@@ -67,10 +67,12 @@ def workload_name(c, tokens):
 
 
 def source_hash():
+    """Hash of every kernel source: a traffic figure taken on other sources is stale."""
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "binarized_rank_linear_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    for f in sorted(os.listdir(CSRC)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(CSRC, f), "rb") as fh:
+                h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -415,14 +417,17 @@ def run_lb(args, world, rank, local):
         achieved = nbytes / per_call_s / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm"], "traffic": load_traffic(args.config, tokens),
-                "kernel": "lb_linear_forward call (latent_kernel + expand_kernel, PDL-chained)",
+                "kernel": ("lb_linear_forward call: small_latent_kernel + small_expand_kernel (CUDA cores, PDL-chained)"
+                           if tokens <= 4 else
+                           "lb_linear_forward call: latent_kernel + expand_kernel (mma.sync, PDL-chained)"),
                 "peak_source": peaks["source"]}
     else:
         achieved = nflops / per_call_s / 1e12
         pk = peaks["bf16_sustained"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
                 "frac": achieved / pk, "traffic": load_traffic(args.config, tokens),
-                "kernel": "lb_linear_forward call", "peak_source": peaks["source"] + " (sustained)"}
+                "kernel": "lb_linear_forward call: sign_gemm_kernel<1> + sign_gemm_kernel<2> (tcgen05)",
+                "peak_source": peaks["source"] + " (sustained)"}
     cpu = None
     if world == 1 and not args.no_cpu:
         import oracle
@@ -444,7 +449,7 @@ def run_lb(args, world, rank, local):
            "e2e": {"value": e2e_value, "unit": "GB/s" if decode else "TFLOP/s",
                    "h2d_bytes_per_step": 2 * tokens * c.n_in, "d2h_bytes_per_step": 2 * tokens * c.n_out,
                    "steps": e2e_steps},
-           "gpu_launches": 2 * args.steps * -(-tokens // DECODE_MAX_TOKENS) if decode else None,
+           "gpu_launches": 2 * args.steps,  # contraction 1 + contraction 2 per call, decode and prefill
            "impl": "lb"}
     print(json.dumps(out), flush=True)
 
