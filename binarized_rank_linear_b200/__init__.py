@@ -87,6 +87,9 @@ def lib() -> ctypes.CDLL:
             L.lb_linear_forward.restype = i32
             L.lb_linear_forward.argtypes = [vp, i64, i64, i64, i64, ctypes.POINTER(LbPath),
                                             ctypes.POINTER(LbPath), vp, i64, vp, sz, vp]
+            L.lb_linear_forward_fixed_scratch.restype = i32
+            L.lb_linear_forward_fixed_scratch.argtypes = [vp, i64, i64, i64, i64, ctypes.POINTER(LbPath),
+                                                          ctypes.POINTER(LbPath), vp, i64, vp]
             L.lb_device_status.restype = i32
             L.lb_device_status.argtypes = [vp, ctypes.POINTER(i32)]
             _lib = L
@@ -211,6 +214,26 @@ def linear_forward(x, main: PackedPath, residual: PackedPath | None = None, y=No
         ctypes.byref(cr) if cr is not None else None, y.data_ptr(), y.stride(0),
         workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream)),
         "lb_linear_forward")
+    return y
+
+
+def linear_forward_fixed_scratch(x, main: PackedPath, residual: PackedPath | None = None, y=None,
+                                 stream=None):
+    """``lb_linear_forward_fixed_scratch``: as :func:`linear_forward` for
+    1..32 tokens, with the library's fixed device scratch instead of a
+    workspace.  Allocates y with torch when not given (the C call itself
+    allocates nothing)."""
+    torch = _torch()
+    tokens, n_in = x.shape
+    n_out = main.h.shape[0]
+    if y is None:
+        y = torch.empty((tokens, n_out), dtype=torch.bfloat16, device=x.device)
+    cm = main.as_c()
+    cr = residual.as_c() if residual is not None else None
+    _check(lib().lb_linear_forward_fixed_scratch(
+        x.data_ptr(), tokens, n_in, n_out, x.stride(0), ctypes.byref(cm),
+        ctypes.byref(cr) if cr is not None else None, y.data_ptr(), y.stride(0), _stream_handle(stream)),
+        "lb_linear_forward_fixed_scratch")
     return y
 
 

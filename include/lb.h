@@ -176,6 +176,40 @@ LB_API lb_status lb_linear_forward(const uint16_t *x, int64_t tokens, int64_t n_
                             uint16_t *y, int64_t ldy, void *workspace, size_t workspace_bytes,
                             void *stream);
 
+/* ---------------------------------------------------------- fixed scratch
+ * lb_linear_forward_fixed_scratch: lb_linear_forward for 1..32 tokens with
+ * no workspace argument.  The pages have no counterpart; this is a service of
+ * this library.
+ *
+ * It is meant for callers that cannot give the library device memory at call
+ * time: a plain C host program with no device allocator of its own, a
+ * runtime that reserves all of its device memory once under a fixed budget,
+ * or a latency-critical loop in which allocating (and the device-wide
+ * synchronisation that cudaMalloc and cudaFree imply) is not allowed.  The
+ * call allocates nothing.  The scratch it uses is a fixed array of
+ * LB_FIXED_SCRATCH_BYTES that is part of the library's device code, one per
+ * device.
+ *
+ * Arguments, results, numerics and errors are those of lb_linear_forward
+ * without `workspace` / `workspace_bytes`, with these differences:
+ *   - tokens must be 0..32 (the decode path); more -> LB_ERR_UNSUPPORTED_SHAPE;
+ *   - a shape whose lb_forward_workspace_bytes exceeds LB_FIXED_SCRATCH_BYTES
+ *     -> LB_ERR_WORKSPACE_TOO_SMALL (nothing is launched);
+ *   - the first call on each device looks up the array's device address
+ *     (once; later calls reuse it).  Make that first call, with the device
+ *     current, before any stream capture.  If the lookup fails the call
+ *     returns LB_ERR_CUDA.
+ * Nothing in the array has to start at zero: each call writes every byte it
+ * later reads.  All calls on one device share the one array, so two calls
+ * that could run at the same time (different streams, or different host
+ * threads without ordering between them) race and give undefined results;
+ * order them, e.g. on one stream. */
+#define LB_FIXED_SCRATCH_BYTES (1u << 20)
+LB_API lb_status lb_linear_forward_fixed_scratch(const uint16_t *x, int64_t tokens, int64_t n_in,
+                                          int64_t n_out, int64_t ldx, const lb_path *main,
+                                          const lb_path *residual, uint16_t *y, int64_t ldy,
+                                          void *stream);
+
 /* Synchronise `stream`, then read and clear the current device's status word,
  * which kernels set when a device-side condition stops them (a bounded wait
  * that gave up, an fp16 overflow).  *out receives LB_OK or the first such

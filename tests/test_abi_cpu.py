@@ -143,3 +143,29 @@ def test_pack_rejects_bad_arguments_before_any_cuda_call(L):
     assert P(FAKE, lb.LB_I8, lb.LB_FACTOR_V, 64, 32, 32, FAKE, 1, None) == lb.LB_ERR_INVALID_ARGUMENT
     assert P(FAKE + 1, lb.LB_F32, lb.LB_FACTOR_U, 4, 32, 32, FAKE, 1, None) == lb.LB_ERR_MISALIGNED
     assert P(FAKE, lb.LB_F32, lb.LB_FACTOR_U, 4, 32, 32, FAKE + 2, 1, None) == lb.LB_ERR_MISALIGNED
+
+
+def forward_fixed(L, x=FAKE, tokens=1, n_in=256, n_out=256, ldx=256, main=None, residual=None, y=FAKE,
+                  ldy=256):
+    main = fake_path() if main is None else main
+    return L.lb_linear_forward_fixed_scratch(x, tokens, n_in, n_out, ldx, ctypes.byref(main),
+                                             ctypes.byref(residual) if residual is not None else None,
+                                             y, ldy, None)
+
+
+def test_fixed_scratch_rejects_before_any_cuda_call(L):
+    """The fixed-scratch entry serves 1..32 tokens and shapes whose scratch
+    fits LB_FIXED_SCRATCH_BYTES (1 MiB); everything else is refused on the
+    host, before the device is touched."""
+    assert forward_fixed(L, tokens=0) == lb.LB_OK
+    assert forward_fixed(L, tokens=-1) == lb.LB_ERR_INVALID_ARGUMENT
+    assert forward_fixed(L, tokens=33) == lb.LB_ERR_UNSUPPORTED_SHAPE
+    assert forward_fixed(L, x=0) == lb.LB_ERR_INVALID_ARGUMENT
+    assert forward_fixed(L, y=0) == lb.LB_ERR_INVALID_ARGUMENT
+    assert L.lb_linear_forward_fixed_scratch(FAKE, 1, 256, 256, 256, None, None, FAKE, 256,
+                                             None) == lb.LB_ERR_INVALID_ARGUMENT
+    # two rank-32768 paths at 32 tokens need 4 MiB of latent scratch
+    big = fake_path(rank=32768)
+    assert L.lb_forward_workspace_bytes(32, 4096, 4096, 32768, 32768) > (1 << 20)
+    assert forward_fixed(L, tokens=32, n_in=4096, n_out=4096, ldx=4096, ldy=4096, main=big,
+                         residual=big) == lb.LB_ERR_WORKSPACE_TOO_SMALL
