@@ -78,12 +78,24 @@ __device__ __forceinline__ void cluster_sync()
     asm volatile("barrier.cluster.arrive.release.aligned;\n"
                  "barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
 }
+// Split cluster barrier: arrive early, wait later (no memory ordering; used
+// to know that every CTA of the cluster has started before touching its
+// shared memory).
+__device__ __forceinline__ void cluster_arrive_relaxed()
+{
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;\n" ::: "memory"); }
 // Address of `p` (a shared-memory variable of this CTA) in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t map_shared_rank(const void *p, uint32_t rank)
 {
     uint32_t out;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
     return out;
+}
+__device__ __forceinline__ void st_shared_cluster_f32(uint32_t addr, float v)
+{
+    asm volatile("st.shared::cluster.f32 [%0], %1;\n" ::"r"(addr), "f"(v) : "memory");
 }
 __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr)
 {

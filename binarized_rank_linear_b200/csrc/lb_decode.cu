@@ -806,7 +806,9 @@ cudaError_t decode_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStre
     for (int m0 = 0; m0 < a.tokens; m0 += kDecodeMaxTokens) {
         const int M = std::min(kDecodeMaxTokens, a.tokens - m0);
         cudaError_t e;
-        if (M <= kSmallMaxTokens) e = small_forward(a, dev, stream, m0, M);
+        const int ranks[2] = {a.path[0].rank, a.npaths > 1 ? a.path[1].rank : 0};
+        if (M <= kSmallMaxTokens && small_fits(M, a.n_in, a.n_out, ranks, a.npaths, dev))
+            e = small_forward(a, dev, stream, m0, M);
         else if (M <= 8) e = launch_decode<1>(a, dev, stream, m0, M);
         else if (M <= 16) e = launch_decode<2>(a, dev, stream, m0, M);
         else e = launch_decode<4>(a, dev, stream, m0, M);

@@ -51,6 +51,9 @@ struct ForwardArgs {
 constexpr int kSmallMaxTokens = 4;
 size_t small_workspace_bytes(int M, const int *ranks, int npaths);
 cudaError_t small_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M);
+// False when the shapes do not fit the small path (its latent tables must fit
+// shared memory); the tensor-core decode path takes those.
+bool small_fits(int M, int n_in, int n_out, const int *ranks, int npaths, const DeviceInfo &dev);
 cudaError_t small_prepare_device(const DeviceInfo &dev);
 constexpr int kDecodeMaxTokens = 32;
 size_t decode_workspace_bytes(int tokens, int n_in, int n_out, const int *ranks, int npaths);
