@@ -65,12 +65,6 @@ __device__ __forceinline__ uint4 ldg_early_v4(const void *p)
     asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
 }
-__device__ __forceinline__ uint2 ldg_early_v2(const void *p)
-{
-    uint2 v;
-    asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-    return v;
-}
 __device__ __forceinline__ uint32_t ldg_early_u32(const void *p)
 {
     uint32_t v;
@@ -135,9 +129,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const Small1Para
 
     if (p.cs > 1) cluster_arrive_relaxed();  // waited for before the partials go to the first CTA
 
-    // (1) weights, all before the dependency wait: this lane's sign words
-    // (row row0 + lane, words wa ..), the g of this thread's first tables and
-    // l of the CTA's rows, into registers
+    // (1) this lane's sign words (row row0 + lane, words wa ..) into
+    // registers, before the dependency wait.  (Fetching g and l this early as
+    // well measured slower at the Llama-2-7B q_proj shape, so they come later.)
     uint32_t bw[kWW];
     {
         const int64_t ld = second ? p.vt_ld1 : p.vt_ld0;
@@ -145,15 +139,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const Small1Para
     }
     const uint16_t *g = (second ? p.g1 : p.g0) + 32 * c0;
     const int ntab = 8 * (c1 - c0);
-    constexpr int kPre = 2;  // tables per thread whose g is fetched early
-    uint2 gq[kPre];
-#pragma unroll
-    for (int k = 0; k < kPre; ++k) {
-        const int t = tid + k * nthr;
-        gq[k] = t < ntab ? ldg_early_v2(g + 4 * t) : make_uint2(0u, 0u);
-    }
     const uint16_t *l = second ? p.l1 : p.l0;
-    const uint16_t lr = tid < 32 ? ldg_early_u16(l + row0 + tid) : (uint16_t)0;
     if (p.early) pdl_launch_dependents();
 
     // (2) x comes from the previous kernel: tables of v = g (.) x for the
@@ -162,11 +148,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const Small1Para
     float4 *tab = reinterpret_cast<float4 *>(smem);  // [M][cww * 8][kTab / 4]
     float *red = reinterpret_cast<float *>(smem) + (size_t)M * cww * 8 * kTab;  // [warps][32][MT]
     float *part = red + nwarps * 32 * MT;                                       // [cs][32][MT] (first CTA)
-    float *ls = part + kMaxCluster * 32 * MT;                                   // [32]
-    for (int t = tid, k = 0; t < ntab; t += nthr, ++k) {
-        uint2 gw;
-        if (k < kPre) gw = k == 0 ? gq[0] : gq[1];
-        else gw = __ldg(reinterpret_cast<const uint2 *>(g + 4 * t));
+    for (int t = tid; t < ntab; t += nthr) {
+        const uint2 gw = __ldg(reinterpret_cast<const uint2 *>(g + 4 * t));
         for (int m = 0; m < M; ++m) {
             const uint2 xq = __ldg(reinterpret_cast<const uint2 *>(p.x + (int64_t)m * p.ldx + 32 * c0 + 4 * t));
             const float v0 = f16_bits_to_float(gw.x & 0xffff) * bf16_bits_to_float(xq.x & 0xffff);
@@ -176,7 +159,6 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const Small1Para
             nibble_table(v0, v1, v2, v3, tab + (kTab / 4) * (m * cww * 8 + t));
         }
     }
-    if (tid < 32) ls[tid] = f16_bits_to_float(lr);
     __syncthreads();
 
     // (3) one lookup per 4 sign bits; two chains per token
@@ -214,7 +196,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const Small1Para
         const int r = e / M, m = e - r * M;
         float s = 0.f;
         for (int w = 0; w < nwarps; ++w) s += red[(w * 32 + r) * MT + m];
-        if (p.cs == 1) p.z[(int64_t)(kg0 + r) * M + m] = s * ls[r];
+        if (p.cs == 1) p.z[(int64_t)(kg0 + r) * M + m] = s * f16_bits_to_float(l[row0 + r]);
         else st_shared_cluster_f32(map_shared_rank(part + (split * 32 + r) * MT + m, 0), s);
     }
     if (p.cs > 1) {
@@ -224,7 +206,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const Small1Para
                 const int r = e / M, m = e - r * M;
                 float s = 0.f;
                 for (int c = 0; c < p.cs; ++c) s += part[(c * 32 + r) * MT + m];
-                p.z[(int64_t)(kg0 + r) * M + m] = s * ls[r];
+                p.z[(int64_t)(kg0 + r) * M + m] = s * f16_bits_to_float(l[row0 + r]);
             }
         }
     }
@@ -366,7 +348,7 @@ struct Small2Plan {
 
 size_t small1_smem(int warps, int ww, int M, int MT)
 {
-    return (size_t)M * warps * ww * 8 * kTab * 4 + (size_t)(warps + kMaxCluster) * 32 * MT * 4 + 32 * 4;
+    return (size_t)M * warps * ww * 8 * kTab * 4 + (size_t)(warps + kMaxCluster) * 32 * MT * 4;
 }
 size_t small2_smem(int warps, int WT, int M, int MT)
 {
