@@ -51,6 +51,35 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 template <int N>
 __device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;\n" :: "n"(N) : "memory"); }
 
+// Loads issued where they stand in the program: weights fetched ahead of use
+// (at kernel entry, or K-blocks ahead) so that their latency overlaps other
+// work.  The compiler does not move a volatile asm past another one (such as
+// a dependency wait or a barrier), nor sink it to the first use of its result.
+__device__ __forceinline__ uint4 ldg_early_v4(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint2 ldg_early_v2(const void *p)
+{
+    uint2 v;
+    asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint32_t ldg_early_u32(const void *p)
+{
+    uint32_t v;
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint16_t ldg_early_u16(const void *p)
+{
+    uint16_t v;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
 // ---------------------------------------------------------------- PDL
 // Wait until the grids this one depends on (programmatic stream
 // serialisation) have completed and their writes are visible.  A no-op when

@@ -56,28 +56,6 @@ __device__ __forceinline__ void nibble_table(float v0, float v1, float v2, float
     dst[3] = make_float4(a - c, -b - c, b - c, -a - c);
 }
 
-// Loads issued where they stand in the program: the weights are fetched at
-// kernel entry so that their DRAM latency overlaps the dependency wait, and a
-// volatile asm is not moved past the (volatile) wait by the compiler.
-__device__ __forceinline__ uint4 ldg_early_v4(const void *p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-    return v;
-}
-__device__ __forceinline__ uint32_t ldg_early_u32(const void *p)
-{
-    uint32_t v;
-    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
-    return v;
-}
-__device__ __forceinline__ uint16_t ldg_early_u16(const void *p)
-{
-    uint16_t v;
-    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
-    return v;
-}
-
 // Words [0, n) of a packed row into registers (n <= kWW); the rest are zero.
 __device__ __forceinline__ void load_words(uint32_t (&w)[kWW], const uint32_t *src, int n)
 {

@@ -38,18 +38,15 @@ namespace lb {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int kProducerWarps = 8;
+constexpr int kGroupWarps = 8;                   // producer warps per K-block: one B row per thread
+constexpr int kProducerWarps = 2 * kGroupWarps;  // two groups take alternate K-blocks
 constexpr int kThreads = 64 + 32 * kProducerWarps;
-constexpr int kPrefetch = 3;  // K-blocks of sign bits (and g) staged ahead of the one being expanded
 constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KB
 constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
 constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t BITS_BYTES = BN * 8;  // a K-block of sign bits: 64 bits per B row
 constexpr uint32_t G_BYTES = 2 * BK * 2;  // a K-block of g for both paths
-// per stage: A tile, B tile, sign bits; per producer warp: its own g ring as
-// given (STAGES deep) and rounded to bf16 (2 deep)
-constexpr size_t kSmem =
-    1024 + (size_t)STAGES * (A_BYTES + B_BYTES + BITS_BYTES) + (size_t)kProducerWarps * (STAGES + 2) * G_BYTES + 256;
+// per stage: A tile, B tile; per producer warp: two slots of g rounded to bf16
+constexpr size_t kSmem = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + (size_t)kProducerWarps * 2 * G_BYTES + 256;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // give up on a wait after 2 s
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -176,9 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;  // SW128 tiles need 1024-byte alignment
     const uint32_t sA = base, sB = base + STAGES * A_BYTES;
-    const uint32_t sBits = sB + STAGES * B_BYTES;      // ring of packed sign bits, [stage][row][8 bytes]
-    const uint32_t sG16 = sBits + STAGES * BITS_BYTES;  // mode 1, per producer warp: g as given, [warp][stage][path][64]
-    const uint32_t sGbf = sG16 + kProducerWarps * STAGES * G_BYTES;  // the same rounded to bf16, [warp][2][path][64]
+    const uint32_t sGbf = sB + STAGES * B_BYTES;  // mode 1, per producer warp: g in bf16, [warp][2][path][64]
     const uint32_t bars = sGbf + kProducerWarps * 2 * G_BYTES;       // full[4], empty[4], accum, then the tmem address
     const uint32_t full0 = bars, empty0 = bars + 8 * STAGES, accum = bars + 16 * STAGES;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + (bars + 16 * STAGES + 8 - raw));
@@ -191,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             for (int s = 0; s < STAGES; ++s) {
-                mbar_init(full0 + 8 * s, 1 + kProducerWarps);  // TMA arrive.expect_tx + producer warps
+                mbar_init(full0 + 8 * s, 1 + kGroupWarps);  // TMA arrive.expect_tx + one group's warps
                 mbar_init(empty0 + 8 * s, 1);     // one tcgen05.commit
             }
             mbar_init(accum, 1);
@@ -248,15 +243,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(accum);
         }
     } else {
-        // ---------------- B producers: 8 warps, producer thread pt owns B row pt
-        // of the tile.  Each K-block it copies the row's 64 sign bits into a
-        // ring slot with its own asynchronous copies, and each warp keeps its
-        // own copy of g, so the producer warps never wait for one another:
-        // they only meet at the stage barriers the MMA thread waits on.
+        // ---------------- B producers: 16 warps in two groups.  Group q expands
+        // the K-blocks kb = q, q + 2, ..., one B row per thread, so every warp
+        // has two MMA periods for each of its blocks and its latency (barrier
+        // wait, expansion, arrive) hides behind the other group's block.  The
+        // row's sign words (and, in mode 1, a piece of g) are loaded into
+        // registers four K-blocks ahead of use.
         const int pt = tid - 64;
-        const int wb = warp - 2;
-        const int nn = n0 + pt;  // row of B (mode 1: latent index; mode 2: output row)
-        const uint32_t x7 = (uint32_t)(pt & 7);  // the row's 128-byte swizzle: logical chunk j sits at chunk j ^ x7
+        const int grp = pt >> 8;        // 0 or 1
+        const int row = pt & (BN - 1);  // B row within the tile
+        const int wl = warp - 2;        // producer warp 0 .. 15
+        const int nn = n0 + row;        // row of B (mode 1: latent index; mode 2: output row)
+        const uint32_t x7 = (uint32_t)(row & 7);  // the row's 128-byte swizzle: logical chunk j sits at chunk j ^ x7
         const bool row_in = nn < p.N;
         const bool sec_row = MODE == 1 && nn >= p.r0;  // mode 1: the row's path
         uint32_t hs0 = 0u, hs1 = 0u;                   // mode 2: h of the row, both halves
@@ -276,85 +274,70 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         const int kwords = p.K >> 5, r0w = p.r0 >> 5;
-        const uint32_t g16w = sG16 + (uint32_t)wb * STAGES * G_BYTES, gbfw = sGbf + (uint32_t)wb * 2 * G_BYTES;
-        // Stage K-block kb: the row's two packed words (one 8-byte copy when
-        // both sit 8-byte aligned in one path), and (mode 1) lanes 0..15 copy
-        // one 16-byte piece of g each (path lane / 8, chunk lane % 8).
-        auto stage = [&](int kb) {
-            const int slot = kb % STAGES;
-            uint8_t *dst = smem_raw + (sBits + slot * BITS_BYTES + pt * 8 - raw);
-            const int wd = 2 * kb;  // first word of the block in the concatenated row
-            if (p.bits8) {
-                const uint32_t *src = p.bits0;
-                uint32_t bytes = 0u;
-                if (row_in && wd < kwords) {
-                    src = (MODE == 1 || wd < r0w) ? row_bits0 + wd : row_bits1 + (wd - r0w);
-                    bytes = wd + 1 < kwords ? 8u : 4u;
-                }
-                cp_async8(dst, src, bytes);
-            } else {
-#pragma unroll
-                for (int w = 0; w < 2; ++w) {
-                    const uint32_t *src = p.bits0;
-                    const bool real = row_in && wd + w < kwords;
-                    if (real) src = (MODE == 1 || wd + w < r0w) ? row_bits0 + wd + w : row_bits1 + (wd + w - r0w);
-                    cp_async4(dst + 4 * w, src, real ? 4u : 0u);
+        const uint32_t gbfw = sGbf + (uint32_t)wl * 2 * G_BYTES;  // this warp's two bf16 g slots
+        auto word_ptr = [&](int w) { return (MODE == 1 || w < r0w) ? row_bits0 + w : row_bits1 + (w - r0w); };
+        // The row's two words of K-block kb (zero past the end of the row).
+        auto load_bits = [&](int kb) {
+            uint2 v = make_uint2(0u, 0u);
+            const int wd = 2 * kb;
+            if (row_in && wd < kwords) {
+                if (p.bits8 && wd + 1 < kwords) {
+                    v = ldg_early_v2(word_ptr(wd));
+                } else {
+                    v.x = ldg_early_u32(word_ptr(wd));
+                    if (wd + 1 < kwords) v.y = ldg_early_u32(word_ptr(wd + 1));
                 }
             }
+            return v;
+        };
+        // Mode 1: lanes 0..15 fetch one 16-byte piece of g of K-block kb (path
+        // lane / 8, columns 8 (lane % 8) ..), as given (fp16).
+        auto load_g = [&](int kb) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
             if (MODE == 1 && lane < 16) {
-                const int pp = lane >> 3, c = lane & 7;
-                const int k0 = kb * BK + 8 * c;
+                const int pp = lane >> 3, k0 = kb * BK + 8 * (lane & 7);
                 const uint16_t *gs = pp ? p.s1 : p.s0;
-                const bool real = gs != nullptr && k0 < p.K;
-                cp_async16(smem_raw + (g16w + slot * G_BYTES + lane * 16 - raw), real ? gs + k0 : p.s0,
-                           real ? 16u : 0u);
+                if (gs != nullptr && k0 < p.K) v = ldg_early_v4(gs + k0);
             }
+            return v;
         };
-        // Mode 1: lanes 0..15 round their own fp16 piece of K-block kb to bf16
-        // into the warp's slot kb % 2 (the warp reads it after a __syncwarp).
-        auto convert_g = [&](int kb) {
-            if (MODE == 1 && lane < 16) {
-                const uint4 q = *reinterpret_cast<const uint4 *>(smem_raw + (g16w + (kb % STAGES) * G_BYTES + lane * 16 - raw));
-                const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-                uint32_t o[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    o[i] = (uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[i] & 0xffffu))) |
-                           ((uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[i] >> 16))) << 16);
-                *reinterpret_cast<uint4 *>(smem_raw + (gbfw + (kb & 1) * G_BYTES + lane * 16 - raw)) =
-                    make_uint4(o[0], o[1], o[2], o[3]);
+        uint2 nb0 = load_bits(grp), nb1 = load_bits(grp + 2);
+        uint4 ng0 = load_g(grp), ng1 = load_g(grp + 2);
+        for (int kb = grp, j = 0; kb < nk; kb += 2, ++j) {
+            const uint2 wb2 = nb0;
+            const uint4 gcur = ng0;
+            nb0 = nb1;
+            ng0 = ng1;
+            if (kb + 4 < nk) {
+                nb1 = load_bits(kb + 4);
+                ng1 = load_g(kb + 4);
             }
-        };
-        // kPrefetch groups ahead (empty ones past the end), so that in
-        // iteration kb wait_group<kPrefetch - 1> leaves blocks <= kb + 1 landed
-        for (int kb = 0; kb < kPrefetch; ++kb) {
-            if (kb < nk) stage(kb);
-            cp_async_commit();
-        }
-        cp_async_wait_group<kPrefetch - 1>();
-        convert_g(0);
-        __syncwarp();
-        for (int kb = 0; kb < nk; ++kb) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-            if (kb + kPrefetch < nk) stage(kb + kPrefetch);
-            cp_async_commit();  // one group per K-block on every thread (possibly empty)
-            cp_async_wait_group<kPrefetch - 1>();
-            // wait for the MMA to release stage s; the give-up decision is
-            // made per warp (the arrive below is per warp)
+            // wait for the MMA to release stage s (it last held block kb - 4,
+            // this group's previous use of it); the decision is per warp
             bool ok = mbar_wait(empty0 + 8 * s, ph ^ 1u) && !abort_flag;
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) {
                 abort_flag = 1;
                 break;
             }
-            // slot (kb + 1) % 2 was last read in the previous iteration, before its __syncwarp
-            if (kb + 1 < nk) convert_g(kb + 1);
-            // the row's 64 sign bits: byte j holds columns 8j .. 8j + 7
-            const uint2 wb2 = *reinterpret_cast<const uint2 *>(smem_raw + (sBits + s * BITS_BYTES + pt * 8 - raw));
             uint4 sc[8];  // per chunk: the four packed scale words
             if (MODE == 1) {
-                const uint8_t *gb = smem_raw + (gbfw + (kb & 1) * G_BYTES + (sec_row ? BK * 2 : 0) - raw);
+                // lanes 0..15 round this block's g to bf16 into the warp's slot
+                // j % 2 (last read two iterations ago, before a __syncwarp)
+                if (lane < 16) {
+                    const uint32_t w[4] = {gcur.x, gcur.y, gcur.z, gcur.w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        o[i] = (uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[i] & 0xffffu))) |
+                               ((uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[i] >> 16))) << 16);
+                    *reinterpret_cast<uint4 *>(smem_raw + (gbfw + (j & 1) * G_BYTES + lane * 16 - raw)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                __syncwarp();
+                const uint8_t *gb = smem_raw + (gbfw + (j & 1) * G_BYTES + (sec_row ? BK * 2 : 0) - raw);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) sc[q] = *reinterpret_cast<const uint4 *>(gb + 16 * q);
             } else {
@@ -368,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // chunk q of the row goes to chunk position q ^ x7 (the tile is
             // 1024-byte aligned, so the XOR acts on address bits 4..6 alone);
             // the 8 rows of a store phase then cover all 32 banks
-            const uint32_t rowx = (sB + s * B_BYTES + pt * 128) | (x7 << 4);
+            const uint32_t rowx = (sB + s * B_BYTES + row * 128) | (x7 << 4);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const uint32_t b = __byte_perm(q < 4 ? wb2.x : wb2.y, 0u, 0x4440u | (uint32_t)(q & 3));
@@ -386,7 +369,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(full0 + 8 * s);
         }
-        cp_async_wait_all();
 
         // ---------------- epilogue: tensor memory -> registers -> global
         bool ok = !abort_flag;
@@ -396,9 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int quad = warp & 3;  // warp w reads tensor-memory lanes 32 (w % 4) ..
         const int m = m0 + 32 * quad + lane;
-        const int cbeg = ((warp - 2) / 4) * (BN / 2);  // two warps per lane quadrant: column halves
+        const int cbeg = ((warp - 2) / 4) * (BN / 4);  // four warps per lane quadrant: column quarters
         bool overflow = false;
-        for (int c0 = cbeg; c0 < cbeg + BN / 2; c0 += 16) {
+        for (int c0 = cbeg; c0 < cbeg + BN / 4; c0 += 16) {
             uint32_t v[16];
             if (ok) tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)c0, v);
             const int nn = n0 + c0;
