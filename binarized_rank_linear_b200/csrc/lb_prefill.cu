@@ -14,18 +14,21 @@
 // to bf16); contraction 2 runs fp16 x fp16 (z rounded to fp16; h exact).
 // Accumulation is fp32 in tensor memory.
 //
-// One CTA computes a 128 x 256 tile of C = A . B^T:
-//   warp 0      allocates tensor memory and streams A tiles with TMA (128-byte
-//               swizzle, no multicast)
-//   warp 1      one thread issues tcgen05.mma (M = 128, N = 256, K = 16) and
-//               commits each stage back to its producers
-//   warps 2..9  one B row per thread: expand the row's packed sign bits into
-//               +-scale values in the same swizzled layout, then read the
-//               accumulator out of tensor memory and store the tile
+// A persistent grid (one CTA per SM) walks the 128 x 256 tiles of C = A . B^T.
+// In each CTA:
+//   warp 0       allocates tensor memory (two 256-column accumulators) and
+//                streams A tiles with TMA (128-byte swizzle, no multicast)
+//   warp 1       one thread issues tcgen05.mma (M = 128, N = 256, K = 16)
+//   warps 2..17  two groups of 8 taking alternate K-blocks, one B row per
+//                thread: expand the row's packed sign bits into +-scale
+//                values in the same swizzled layout
+//   warps 18..21 read a finished accumulator out of tensor memory and store
+//                the tile, while the MMA fills the other accumulator
 // Stages are handed over with mbarriers (4-deep ring).  Every wait is bounded
 // in time: a wait that gives up sets LB_ERR_DEVICE_TIMEOUT on the status word
 // and the CTA winds down (drains its copies, frees tensor memory) instead of
 // hanging.
+#include <algorithm>
 #include <cstdint>
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -40,10 +43,11 @@ namespace {
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int kGroupWarps = 8;                   // producer warps per K-block: one B row per thread
 constexpr int kProducerWarps = 2 * kGroupWarps;  // two groups take alternate K-blocks
-constexpr int kThreads = 64 + 32 * kProducerWarps;
+constexpr int kEpiWarps = 4;                     // one per tensor-memory lane quadrant
+constexpr int kThreads = 32 * (2 + kProducerWarps + kEpiWarps);
 constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KB
 constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
-constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
 constexpr uint32_t G_BYTES = 2 * BK * 2;  // a K-block of g for both paths
 // per stage: A tile, B tile; per producer warp: two slots of g rounded to bf16
 constexpr size_t kSmem = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + (size_t)kProducerWarps * 2 * G_BYTES + 256;
@@ -164,6 +168,12 @@ struct SignGemmParams {
     int *status;
 };
 
+// Persistent: CTA c computes the 128 x 256 tiles t = c, c + gridDim.x, ...
+// (tile t is rows (t % tiles_m) * 128 and columns (t / tiles_m) * 256, so the
+// CTAs running at once share the same few columns of B).  Its K-blocks form
+// one sequence over all its tiles, so stages, phases and the producer groups'
+// alternation run on across tile boundaries.  Two accumulators in tensor
+// memory let the epilogue warps drain tile i while the MMA runs tile i + 1.
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     sign_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const SignGemmParams p)
@@ -174,22 +184,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;  // SW128 tiles need 1024-byte alignment
     const uint32_t sA = base, sB = base + STAGES * A_BYTES;
     const uint32_t sGbf = sB + STAGES * B_BYTES;  // mode 1, per producer warp: g in bf16, [warp][2][path][64]
-    const uint32_t bars = sGbf + kProducerWarps * 2 * G_BYTES;       // full[4], empty[4], accum, then the tmem address
-    const uint32_t full0 = bars, empty0 = bars + 8 * STAGES, accum = bars + 16 * STAGES;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + (bars + 16 * STAGES + 8 - raw));
+    const uint32_t bars = sGbf + kProducerWarps * 2 * G_BYTES;
+    // full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain, then the tmem address
+    const uint32_t full0 = bars, empty0 = bars + 8 * STAGES, accf0 = bars + 16 * STAGES;
+    const uint32_t acce0 = accf0 + 16, drain = acce0 + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + (drain + 8 - raw));
     __shared__ int abort_shared;
     volatile int &abort_flag = abort_shared;  // set by whichever role gives up; read by all
 
-    const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
+    const int tiles_m = (p.M + BM - 1) / BM;
+    const int ntiles = tiles_m * ((p.N + BN - 1) / BN);
+    const int G = gridDim.x, c = blockIdx.x;
+    const int my_tiles = c < ntiles ? (ntiles - c + G - 1) / G : 0;
     const int nk = (p.K + BK - 1) / BK;
+    const int nblocks = my_tiles * nk;  // this CTA's K-blocks, all tiles
 
     if (warp == 0) {
         if (lane == 0) {
             for (int s = 0; s < STAGES; ++s) {
                 mbar_init(full0 + 8 * s, 1 + kGroupWarps);  // TMA arrive.expect_tx + one group's warps
-                mbar_init(empty0 + 8 * s, 1);     // one tcgen05.commit
+                mbar_init(empty0 + 8 * s, 1);               // one tcgen05.commit
             }
-            mbar_init(accum, 1);
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(accf0 + 8 * b, 1);          // one tcgen05.commit
+                mbar_init(acce0 + 8 * b, kEpiWarps);  // every epilogue warp
+            }
+            mbar_init(drain, 1);
             abort_flag = 0;
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         }
@@ -205,116 +225,151 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- A producer (TMA)
         if (lane == 0) {
             int issued = 0;
-            for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % STAGES;
-                const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+            for (int gb = 0; gb < nblocks; ++gb) {
+                const int i = gb / nk, kb = gb - i * nk;
+                const int t = c + i * G;
+                const int s = gb % STAGES;
+                const uint32_t ph = (uint32_t)(gb / STAGES) & 1u;
                 if (!mbar_wait(empty0 + 8 * s, ph ^ 1u) || abort_flag) {
                     abort_flag = 1;
                     break;
                 }
                 mbar_arrive_expect_tx(full0 + 8 * s, A_BYTES);
-                tma_load_2d(sA + s * A_BYTES, &tmA, kb * BK, m0, full0 + 8 * s);
+                tma_load_2d(sA + s * A_BYTES, &tmA, kb * BK, (t % tiles_m) * BM, full0 + 8 * s);
                 ++issued;
             }
             if (abort_flag) {
                 // let copies already in flight land before the CTA goes away
-                for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
-                    mbar_wait(full0 + 8 * (kb % STAGES), (uint32_t)(kb / STAGES) & 1u);
+                for (int gb = (issued > STAGES ? issued - STAGES : 0); gb < issued; ++gb)
+                    mbar_wait(full0 + 8 * (gb % STAGES), (uint32_t)(gb / STAGES) & 1u);
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer
+        // ---------------- MMA issuer: tile i accumulates in columns 256 (i % 2) ..
         if (lane == 0) {
             const uint32_t idesc = instr_desc(MODE == 1 ? 1u : 0u);
-            for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % STAGES;
-                const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-                if (!mbar_wait(full0 + 8 * s, ph) || abort_flag) {
+            int gb = 0;
+            for (int i = 0; i < my_tiles && !abort_flag; ++i) {
+                const int b = i & 1;
+                // the epilogue has drained this accumulator (tile i - 2)
+                if (!mbar_wait(acce0 + 8 * b, (uint32_t)((i >> 1) & 1) ^ 1u)) {
                     abort_flag = 1;
                     break;
                 }
                 tc_fence_after();
-                const uint64_t ad = smem_desc(sA + s * A_BYTES), bd = smem_desc(sB + s * B_BYTES);
+                const uint32_t acc = tmem + (uint32_t)(b * BN);
+                for (int kb = 0; kb < nk; ++kb, ++gb) {
+                    const int s = gb % STAGES;
+                    const uint32_t ph = (uint32_t)(gb / STAGES) & 1u;
+                    if (!mbar_wait(full0 + 8 * s, ph) || abort_flag) {
+                        abort_flag = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = smem_desc(sA + s * A_BYTES), bd = smem_desc(sB + s * B_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk)  // +32 bytes along K per step of 16
-                    umma(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
-                umma_commit(empty0 + 8 * s);
+                    for (int kk = 0; kk < BK / 16; ++kk)  // +32 bytes along K per step of 16
+                        umma(acc, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                    umma_commit(empty0 + 8 * s);
+                }
+                if (abort_flag) break;
+                umma_commit(accf0 + 8 * b);
             }
-            umma_commit(accum);
+            // every MMA issued has finished before the CTA frees tensor memory
+            umma_commit(drain);
+            if (!mbar_wait(drain, 0)) abort_flag = 1;
         }
-    } else {
+    } else if (warp < 2 + kProducerWarps) {
         // ---------------- B producers: 16 warps in two groups.  Group q expands
-        // the K-blocks kb = q, q + 2, ..., one B row per thread, so every warp
-        // has two MMA periods for each of its blocks and its latency (barrier
-        // wait, expansion, arrive) hides behind the other group's block.  The
-        // row's sign words (and, in mode 1, a piece of g) are loaded into
-        // registers four K-blocks ahead of use.
+        // the blocks gb = q, q + 2, ... of the CTA's K-block sequence, one B
+        // row per thread, so every warp has two MMA periods for each of its
+        // blocks and its latency (barrier wait, expansion, arrive) hides
+        // behind the other group's block.  What a block needs from memory
+        // (the row's sign words; g in mode 1, h in mode 2) is loaded into
+        // registers four blocks ahead of use.
         const int pt = tid - 64;
         const int grp = pt >> 8;        // 0 or 1
         const int row = pt & (BN - 1);  // B row within the tile
         const int wl = warp - 2;        // producer warp 0 .. 15
-        const int nn = n0 + row;        // row of B (mode 1: latent index; mode 2: output row)
         const uint32_t x7 = (uint32_t)(row & 7);  // the row's 128-byte swizzle: logical chunk j sits at chunk j ^ x7
-        const bool row_in = nn < p.N;
-        const bool sec_row = MODE == 1 && nn >= p.r0;  // mode 1: the row's path
-        uint32_t hs0 = 0u, hs1 = 0u;                   // mode 2: h of the row, both halves
-        if (MODE == 2 && row_in) {
-            const uint32_t h0 = p.s0[nn], h1 = p.s1 ? p.s1[nn] : 0u;
-            hs0 = h0 | (h0 << 16);
-            hs1 = h1 | (h1 << 16);
-        }
-        const uint32_t *row_bits0 = nullptr;  // mode 1: the row's packed words; mode 2: path 0 row
-        const uint32_t *row_bits1 = nullptr;  // mode 2: path 1 row
-        if (row_in) {
-            if (MODE == 1)
-                row_bits0 = sec_row ? p.bits1 + (int64_t)(nn - p.r0) * p.bld1 : p.bits0 + (int64_t)nn * p.bld0;
-            else {
-                row_bits0 = p.bits0 + (int64_t)nn * p.bld0;
-                if (p.bits1) row_bits1 = p.bits1 + (int64_t)nn * p.bld1;
-            }
-        }
         const int kwords = p.K >> 5, r0w = p.r0 >> 5;
         const uint32_t gbfw = sGbf + (uint32_t)wl * 2 * G_BYTES;  // this warp's two bf16 g slots
-        auto word_ptr = [&](int w) { return (MODE == 1 || w < r0w) ? row_bits0 + w : row_bits1 + (w - r0w); };
-        // The row's two words of K-block kb (zero past the end of the row).
-        auto load_bits = [&](int kb) {
-            uint2 v = make_uint2(0u, 0u);
-            const int wd = 2 * kb;
+        struct Pref {
+            uint2 bits;      // the row's two sign words of the block (zero outside the matrix)
+            uint4 g;         // mode 1, lanes 0..15: g of path lane / 8, columns 8 (lane % 8) .. (fp16)
+            uint32_t h0, h1; // mode 2: h of the row, both paths (fp16)
+        };
+        // Position of a block in the sequence, advanced without divisions:
+        // tile iteration, K-block, and this thread's B row in that tile.
+        struct Cursor {
+            int gb, i, kb, nn;
+        };
+        auto cursor_at = [&](int gb) {
+            Cursor u;
+            u.gb = gb;
+            u.i = gb / nk;
+            u.kb = gb - u.i * nk;
+            u.nn = ((c + u.i * G) / tiles_m) * BN + row;
+            return u;
+        };
+        auto advance2 = [&](Cursor &u) {
+            u.gb += 2;
+            u.kb += 2;
+            if (u.kb >= nk) {
+                while (u.kb >= nk) {
+                    u.kb -= nk;
+                    ++u.i;
+                }
+                u.nn = ((c + u.i * G) / tiles_m) * BN + row;
+            }
+        };
+        auto fetch = [&](const Cursor &u) {
+            Pref f;
+            f.bits = make_uint2(0u, 0u);
+            f.g = make_uint4(0u, 0u, 0u, 0u);
+            f.h0 = f.h1 = 0u;
+            if (u.gb >= nblocks) return f;
+            const int kb = u.kb, nn = u.nn;
+            const bool row_in = nn < p.N;
+            const int wd = 2 * kb;  // first word of the block in the (concatenated) row
             if (row_in && wd < kwords) {
-                if (p.bits8 && wd + 1 < kwords) {
-                    v = ldg_early_v2(word_ptr(wd));
+                const uint32_t *rb0, *rb1 = nullptr;
+                if (MODE == 1) {
+                    const bool sec = nn >= p.r0;
+                    rb0 = sec ? p.bits1 + (int64_t)(nn - p.r0) * p.bld1 : p.bits0 + (int64_t)nn * p.bld0;
                 } else {
-                    v.x = ldg_early_u32(word_ptr(wd));
-                    if (wd + 1 < kwords) v.y = ldg_early_u32(word_ptr(wd + 1));
+                    rb0 = p.bits0 + (int64_t)nn * p.bld0;
+                    if (p.bits1) rb1 = p.bits1 + (int64_t)nn * p.bld1;
+                }
+                auto wp = [&](int w) { return (MODE == 1 || w < r0w) ? rb0 + w : rb1 + (w - r0w); };
+                if (p.bits8 && wd + 1 < kwords) {
+                    f.bits = ldg_early_v2(wp(wd));
+                } else {
+                    f.bits.x = ldg_early_u32(wp(wd));
+                    if (wd + 1 < kwords) f.bits.y = ldg_early_u32(wp(wd + 1));
                 }
             }
-            return v;
-        };
-        // Mode 1: lanes 0..15 fetch one 16-byte piece of g of K-block kb (path
-        // lane / 8, columns 8 (lane % 8) ..), as given (fp16).
-        auto load_g = [&](int kb) {
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
             if (MODE == 1 && lane < 16) {
                 const int pp = lane >> 3, k0 = kb * BK + 8 * (lane & 7);
                 const uint16_t *gs = pp ? p.s1 : p.s0;
-                if (gs != nullptr && k0 < p.K) v = ldg_early_v4(gs + k0);
+                if (gs != nullptr && k0 < p.K) f.g = ldg_early_v4(gs + k0);
             }
-            return v;
+            if (MODE == 2 && row_in) {
+                f.h0 = ldg_early_u16(p.s0 + nn);
+                if (p.s1) f.h1 = ldg_early_u16(p.s1 + nn);
+            }
+            return f;
         };
-        uint2 nb0 = load_bits(grp), nb1 = load_bits(grp + 2);
-        uint4 ng0 = load_g(grp), ng1 = load_g(grp + 2);
-        for (int kb = grp, j = 0; kb < nk; kb += 2, ++j) {
-            const uint2 wb2 = nb0;
-            const uint4 gcur = ng0;
-            nb0 = nb1;
-            ng0 = ng1;
-            if (kb + 4 < nk) {
-                nb1 = load_bits(kb + 4);
-                ng1 = load_g(kb + 4);
-            }
-            const int s = kb % STAGES;
-            const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-            // wait for the MMA to release stage s (it last held block kb - 4,
+        Cursor u = cursor_at(grp), ua = cursor_at(grp + 4);  // this block, and the one four ahead
+        Pref f0 = fetch(u), f1 = fetch(cursor_at(grp + 2));
+        for (int j = 0; u.gb < nblocks; ++j, advance2(u), advance2(ua)) {
+            const Pref cur = f0;
+            f0 = f1;
+            f1 = fetch(ua);
+            const int gb = u.gb, kb = u.kb, nn = u.nn;
+            const int s = gb % STAGES;
+            const uint32_t ph = (uint32_t)(gb / STAGES) & 1u;
+            // wait for the MMA to release stage s (it last held block gb - 4,
             // this group's previous use of it); the decision is per warp
             bool ok = mbar_wait(empty0 + 8 * s, ph ^ 1u) && !abort_flag;
             ok = __all_sync(0xffffffffu, ok);
@@ -327,20 +382,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // lanes 0..15 round this block's g to bf16 into the warp's slot
                 // j % 2 (last read two iterations ago, before a __syncwarp)
                 if (lane < 16) {
-                    const uint32_t w[4] = {gcur.x, gcur.y, gcur.z, gcur.w};
+                    const uint32_t w[4] = {cur.g.x, cur.g.y, cur.g.z, cur.g.w};
                     uint32_t o[4];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        o[i] = (uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[i] & 0xffffu))) |
-                               ((uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[i] >> 16))) << 16);
+                    for (int q = 0; q < 4; ++q)
+                        o[q] = (uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[q] & 0xffffu))) |
+                               ((uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[q] >> 16))) << 16);
                     *reinterpret_cast<uint4 *>(smem_raw + (gbfw + (j & 1) * G_BYTES + lane * 16 - raw)) =
                         make_uint4(o[0], o[1], o[2], o[3]);
                 }
                 __syncwarp();
-                const uint8_t *gb = smem_raw + (gbfw + (j & 1) * G_BYTES + (sec_row ? BK * 2 : 0) - raw);
+                const bool sec_row = nn >= p.r0;  // the row's path
+                const uint8_t *gb_ = smem_raw + (gbfw + (j & 1) * G_BYTES + (sec_row ? BK * 2 : 0) - raw);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) sc[q] = *reinterpret_cast<const uint4 *>(gb + 16 * q);
+                for (int q = 0; q < 8; ++q) sc[q] = *reinterpret_cast<const uint4 *>(gb_ + 16 * q);
             } else {
+                const uint32_t hs0 = cur.h0 | (cur.h0 << 16), hs1 = cur.h1 | (cur.h1 << 16);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const int k0 = kb * BK + 8 * q;  // first column of the chunk
@@ -354,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t rowx = (sB + s * B_BYTES + row * 128) | (x7 << 4);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                const uint32_t b = __byte_perm(q < 4 ? wb2.x : wb2.y, 0u, 0x4440u | (uint32_t)(q & 3));
+                const uint32_t b = __byte_perm(q < 4 ? cur.bits.x : cur.bits.y, 0u, 0x4440u | (uint32_t)(q & 3));
                 // (b * K_i) puts sign bit 2i at bit 15 and bit 2i + 1 at bit 31
                 // (the two shifted copies of the byte do not overlap: no carries)
                 const uint32_t v0 = ((b * 0x40008000u) & 0x80008000u) ^ sc[q].x;
@@ -369,46 +426,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(full0 + 8 * s);
         }
-
-        // ---------------- epilogue: tensor memory -> registers -> global
-        bool ok = !abort_flag;
-        if (ok) ok = mbar_wait(accum, 0);
-        ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
-        if (!ok) abort_flag = 1;
-        tc_fence_after();
-        const int quad = warp & 3;  // warp w reads tensor-memory lanes 32 (w % 4) ..
-        const int m = m0 + 32 * quad + lane;
-        const int cbeg = ((warp - 2) / 4) * (BN / 4);  // four warps per lane quadrant: column quarters
+    } else {
+        // ---------------- epilogue: warp w drains tensor-memory lanes 32 (w % 4)
+        // .. of each tile's accumulator, then hands the accumulator back
+        const int quad = warp & 3;
         bool overflow = false;
-        for (int c0 = cbeg; c0 < cbeg + BN / 4; c0 += 16) {
-            uint32_t v[16];
-            if (ok) tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)c0, v);
-            const int nn = n0 + c0;
-            if (!ok || m >= p.M || nn >= p.N) continue;
-            uint32_t o[8];
-            if (MODE == 1) {
-                // z = l (.) c, rounded to fp16 (the operand of contraction 2)
-                const bool sec = nn >= p.r0;
-                const uint16_t *lp = sec ? p.l1 + (nn - p.r0) : p.l0 + nn;
-                const uint4 la = __ldg(reinterpret_cast<const uint4 *>(lp));
-                const uint4 lb = __ldg(reinterpret_cast<const uint4 *>(lp + 8));
-                const uint32_t lw[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float z0 = __uint_as_float(v[2 * i]) * f16_bits_to_float((uint16_t)(lw[i] & 0xffffu));
-                    const float z1 = __uint_as_float(v[2 * i + 1]) * f16_bits_to_float((uint16_t)(lw[i] >> 16));
-                    overflow |= beyond_f16(z0) | beyond_f16(z1);
-                    o[i] = pack_half2(z0, z1);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    o[i] = (uint32_t)float_to_bf16_bits(__uint_as_float(v[2 * i])) |
-                           ((uint32_t)float_to_bf16_bits(__uint_as_float(v[2 * i + 1])) << 16);
+        for (int i = 0; i < my_tiles; ++i) {
+            const int b = i & 1;
+            const int t = c + i * G;
+            const int m = (t % tiles_m) * BM + 32 * quad + lane;
+            const int n0 = (t / tiles_m) * BN;
+            bool ok = !abort_flag && mbar_wait(accf0 + 8 * b, (uint32_t)((i >> 1) & 1));
+            ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+            if (!ok) {
+                abort_flag = 1;
+                break;
             }
-            uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + (int64_t)m * p.ldo + nn);
-            dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-            dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+            tc_fence_after();
+            for (int c0 = 0; c0 < BN; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * BN + c0), v);
+                const int nn = n0 + c0;
+                if (m >= p.M || nn >= p.N) continue;
+                uint32_t o[8];
+                if (MODE == 1) {
+                    // z = l (.) c, rounded to fp16 (the operand of contraction 2)
+                    const bool sec = nn >= p.r0;
+                    const uint16_t *lp = sec ? p.l1 + (nn - p.r0) : p.l0 + nn;
+                    const uint4 la = __ldg(reinterpret_cast<const uint4 *>(lp));
+                    const uint4 lb = __ldg(reinterpret_cast<const uint4 *>(lp + 8));
+                    const uint32_t lw[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const float z0 = __uint_as_float(v[2 * q]) * f16_bits_to_float((uint16_t)(lw[q] & 0xffffu));
+                        const float z1 = __uint_as_float(v[2 * q + 1]) * f16_bits_to_float((uint16_t)(lw[q] >> 16));
+                        overflow |= beyond_f16(z0) | beyond_f16(z1);
+                        o[q] = pack_half2(z0, z1);
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        o[q] = (uint32_t)float_to_bf16_bits(__uint_as_float(v[2 * q])) |
+                               ((uint32_t)float_to_bf16_bits(__uint_as_float(v[2 * q + 1])) << 16);
+                }
+                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + (int64_t)m * p.ldo + nn);
+                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce0 + 8 * b);
         }
         if (overflow) set_status(p.status, LB_ERR_RANGE);
     }
@@ -505,8 +572,8 @@ cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStr
     p1.out = z;
     p1.ldo = R;
     p1.status = dev.status;
-    dim3 grid1((unsigned)((M + BM - 1) / BM), (unsigned)((R + BN - 1) / BN));
-    sign_gemm_kernel<1><<<grid1, kThreads, kSmem, stream>>>(tx, p1);
+    const int tiles1 = ((M + BM - 1) / BM) * ((R + BN - 1) / BN);
+    sign_gemm_kernel<1><<<std::min(tiles1, dev.sm_count), kThreads, kSmem, stream>>>(tx, p1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
@@ -531,8 +598,8 @@ cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStr
     p2.out = a.y;
     p2.ldo = a.ldy;
     p2.status = dev.status;
-    dim3 grid2((unsigned)((M + BM - 1) / BM), (unsigned)((a.n_out + BN - 1) / BN));
-    sign_gemm_kernel<2><<<grid2, kThreads, kSmem, stream>>>(tz, p2);
+    const int tiles2 = ((M + BM - 1) / BM) * ((a.n_out + BN - 1) / BN);
+    sign_gemm_kernel<2><<<std::min(tiles2, dev.sm_count), kThreads, kSmem, stream>>>(tz, p2);
     return cudaGetLastError();
 }
 
