@@ -40,17 +40,31 @@
 namespace lb {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int kGroupWarps = 8;                   // producer warps per K-block: one B row per thread
-constexpr int kProducerWarps = 2 * kGroupWarps;  // two groups take alternate K-blocks
-constexpr int kEpiWarps = 4;                     // one per tensor-memory lane quadrant
-constexpr int kThreads = 32 * (2 + kProducerWarps + kEpiWarps);
-constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KB
-constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
-constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
-constexpr uint32_t G_BYTES = 2 * BK * 2;  // a K-block of g for both paths
-// per stage: A tile, B tile; per producer warp: two slots of g rounded to bf16
-constexpr size_t kSmem = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + (size_t)kProducerWarps * 2 * G_BYTES + 256;
+constexpr int BM = 128, BN = 256, BK = 64;  // one MMA: M = 128, N = 256; K-blocks of 64
+constexpr int kGroupWarps = 8;                // producer warps per K-block: one B row per thread
+constexpr uint32_t B_BYTES = BN * BK * 2;     // 32 KB
+constexpr uint32_t TMEM_COLS = 2 * BN;        // two 256-column accumulators
+constexpr uint32_t G_BYTES = 2 * BK * 2;      // a K-block of g for both paths
+
+// Two tile shapes.  H = 1: a CTA tile is 128 x 256; the two accumulators
+// double-buffer consecutive tiles, and two producer groups take alternate
+// K-blocks.  H = 2: a CTA tile is 256 x 256, two M = 128 halves that share
+// each expanded B tile (half the sign expansion per flop); the two
+// accumulators hold the halves of one tile, and one producer group has twice
+// as long per K-block.
+template <int H>
+struct Shape {
+    static constexpr int kStages = H == 1 ? 4 : 3;
+    static constexpr int kGroups = H == 1 ? 2 : 1;
+    static constexpr int kProducerWarps = kGroupWarps * kGroups;
+    static constexpr int kEpiWarps = 4 * H;  // per accumulator in use, one per tensor-memory lane quadrant
+    static constexpr int kThreads = 32 * (2 + kProducerWarps + kEpiWarps);
+    static constexpr int kTileM = BM * H;
+    static constexpr uint32_t kABytes = (uint32_t)kTileM * BK * 2;  // 16 or 32 KB
+    // per stage: A tile, B tile; per producer warp: two slots of g rounded to bf16
+    static constexpr size_t kSmem =
+        1024 + (size_t)kStages * (kABytes + B_BYTES) + (size_t)kProducerWarps * 2 * G_BYTES + 256;
+};
 constexpr unsigned long long kWaitNs = 2000000000ull;  // give up on a wait after 2 s
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -127,12 +141,17 @@ __device__ __forceinline__ void umma_commit(uint32_t bar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16])
+// 32 consecutive fp32 columns of this warp's 32 lanes, one register each,
+// then wait for them (one wait per 32 columns).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
 {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
         : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -174,10 +193,14 @@ struct SignGemmParams {
 // one sequence over all its tiles, so stages, phases and the producer groups'
 // alternation run on across tile boundaries.  Two accumulators in tensor
 // memory let the epilogue warps drain tile i while the MMA runs tile i + 1.
-template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int MODE, int H>
+__global__ void __launch_bounds__(Shape<H>::kThreads, 1)
     sign_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const SignGemmParams p)
 {
+    using S = Shape<H>;
+    constexpr int STAGES = S::kStages;
+    constexpr uint32_t A_BYTES = S::kABytes;
+    constexpr int kProducerWarps = S::kProducerWarps;
     extern __shared__ uint8_t smem_raw[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t raw = smem_u32(smem_raw);
@@ -192,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ int abort_shared;
     volatile int &abort_flag = abort_shared;  // set by whichever role gives up; read by all
 
-    const int tiles_m = (p.M + BM - 1) / BM;
+    const int tiles_m = (p.M + S::kTileM - 1) / S::kTileM;
     const int ntiles = tiles_m * ((p.N + BN - 1) / BN);
     const int G = gridDim.x, c = blockIdx.x;
     const int my_tiles = c < ntiles ? (ntiles - c + G - 1) / G : 0;
@@ -207,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int b = 0; b < 2; ++b) {
                 mbar_init(accf0 + 8 * b, 1);          // one tcgen05.commit
-                mbar_init(acce0 + 8 * b, kEpiWarps);  // every epilogue warp
+                mbar_init(acce0 + 8 * b, S::kEpiWarps);  // every epilogue warp
             }
             mbar_init(drain, 1);
             abort_flag = 0;
@@ -235,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 mbar_arrive_expect_tx(full0 + 8 * s, A_BYTES);
-                tma_load_2d(sA + s * A_BYTES, &tmA, kb * BK, (t % tiles_m) * BM, full0 + 8 * s);
+                tma_load_2d(sA + s * A_BYTES, &tmA, kb * BK, (t % tiles_m) * S::kTileM, full0 + 8 * s);
                 ++issued;
             }
             if (abort_flag) {
@@ -245,14 +268,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer: tile i accumulates in columns 256 (i % 2) ..
+        // ---------------- MMA issuer.  H = 1: tile i accumulates in columns
+        // 256 (i % 2) ..; H = 2: half h of every tile accumulates in columns 256 h ..
         if (lane == 0) {
             const uint32_t idesc = instr_desc(MODE == 1 ? 1u : 0u);
             int gb = 0;
             for (int i = 0; i < my_tiles && !abort_flag; ++i) {
-                const int b = i & 1;
-                // the epilogue has drained this accumulator (tile i - 2)
-                if (!mbar_wait(acce0 + 8 * b, (uint32_t)((i >> 1) & 1) ^ 1u)) {
+                const int b = H == 1 ? (i & 1) : 0;  // hand-over barriers of the accumulator(s)
+                const int use = H == 1 ? (i >> 1) : i;
+                // the epilogue has drained the accumulator(s) (tile i - 2, or i - 1)
+                if (!mbar_wait(acce0 + 8 * b, (uint32_t)(use & 1) ^ 1u)) {
                     abort_flag = 1;
                     break;
                 }
@@ -266,10 +291,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t ad = smem_desc(sA + s * A_BYTES), bd = smem_desc(sB + s * B_BYTES);
+                    const uint64_t bd = smem_desc(sB + s * B_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)  // +32 bytes along K per step of 16
-                        umma(acc, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                    for (int h = 0; h < H; ++h) {
+                        // half h: A rows 128 h .. (16 KB further on, a whole number of 8-row atoms)
+                        const uint64_t ad = smem_desc(sA + s * A_BYTES + (uint32_t)h * (BM * BK * 2));
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)  // +32 bytes along K per step of 16
+                            umma(acc + (uint32_t)(h * BN), ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                    }
                     umma_commit(empty0 + 8 * s);
                 }
                 if (abort_flag) break;
@@ -280,15 +310,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(drain, 0)) abort_flag = 1;
         }
     } else if (warp < 2 + kProducerWarps) {
-        // ---------------- B producers: 16 warps in two groups.  Group q expands
-        // the blocks gb = q, q + 2, ... of the CTA's K-block sequence, one B
-        // row per thread, so every warp has two MMA periods for each of its
-        // blocks and its latency (barrier wait, expansion, arrive) hides
-        // behind the other group's block.  What a block needs from memory
-        // (the row's sign words; g in mode 1, h in mode 2) is loaded into
-        // registers four blocks ahead of use.
+        // ---------------- B producers: groups of 8 warps, one B row per thread.
+        // H = 1: two groups; group q expands the blocks gb = q, q + 2, ... of
+        // the CTA's K-block sequence, so every warp has two MMA periods for
+        // each of its blocks and its latency (barrier wait, expansion, arrive)
+        // hides behind the other group's block.  H = 2: one group; a block
+        // feeds two MMA halves, so it has two MMA periods as well.  What a
+        // block needs from memory (the row's sign words; g in mode 1, h in
+        // mode 2) is loaded into registers two of the group's blocks ahead.
         const int pt = tid - 64;
-        const int grp = pt >> 8;        // 0 or 1
+        constexpr int NG = S::kGroups;  // block stride of a group
+        const int grp = pt >> 8;        // 0 .. NG - 1
         const int row = pt & (BN - 1);  // B row within the tile
         const int wl = warp - 2;        // producer warp 0 .. 15
         const uint32_t x7 = (uint32_t)(row & 7);  // the row's 128-byte swizzle: logical chunk j sits at chunk j ^ x7
@@ -312,9 +344,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             u.nn = ((c + u.i * G) / tiles_m) * BN + row;
             return u;
         };
-        auto advance2 = [&](Cursor &u) {
-            u.gb += 2;
-            u.kb += 2;
+        auto advance = [&](Cursor &u) {
+            u.gb += NG;
+            u.kb += NG;
             if (u.kb >= nk) {
                 while (u.kb >= nk) {
                     u.kb -= nk;
@@ -360,9 +392,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             return f;
         };
-        Cursor u = cursor_at(grp), ua = cursor_at(grp + 4);  // this block, and the one four ahead
-        Pref f0 = fetch(u), f1 = fetch(cursor_at(grp + 2));
-        for (int j = 0; u.gb < nblocks; ++j, advance2(u), advance2(ua)) {
+        Cursor u = cursor_at(grp), ua = cursor_at(grp + 2 * NG);  // this block, and the group's block two ahead
+        Pref f0 = fetch(u), f1 = fetch(cursor_at(grp + NG));
+        for (int j = 0; u.gb < nblocks; ++j, advance(u), advance(ua)) {
             const Pref cur = f0;
             f0 = f1;
             f1 = fetch(ua);
@@ -428,24 +460,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------- epilogue: warp w drains tensor-memory lanes 32 (w % 4)
-        // .. of each tile's accumulator, then hands the accumulator back
+        // .. of a finished accumulator (H = 2: warps 4 e .. 4 e + 3 of the
+        // epilogue drain half e), then hands the accumulator back
         const int quad = warp & 3;
+        const int eh = H == 1 ? 0 : (warp - 2 - kProducerWarps) >> 2;
         bool overflow = false;
         for (int i = 0; i < my_tiles; ++i) {
-            const int b = i & 1;
+            const int b = H == 1 ? (i & 1) : 0;
+            const int use = H == 1 ? (i >> 1) : i;
             const int t = c + i * G;
-            const int m = (t % tiles_m) * BM + 32 * quad + lane;
+            const int m = (t % tiles_m) * S::kTileM + eh * BM + 32 * quad + lane;
             const int n0 = (t / tiles_m) * BN;
-            bool ok = !abort_flag && mbar_wait(accf0 + 8 * b, (uint32_t)((i >> 1) & 1));
+            bool ok = !abort_flag && mbar_wait(accf0 + 8 * b, (uint32_t)(use & 1));
             ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
             if (!ok) {
                 abort_flag = 1;
                 break;
             }
             tc_fence_after();
-            for (int c0 = 0; c0 < BN; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * BN + c0), v);
+            for (int c32 = 0; c32 < BN; c32 += 32) {
+                uint32_t vv[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)((b + eh) * BN + c32), vv);
+#pragma unroll
+              for (int half = 0; half < 2; ++half) {
+                const int c0 = c32 + 16 * half;
+                const uint32_t *v = vv + 16 * half;
                 const int nn = n0 + c0;
                 if (m >= p.M || nn >= p.N) continue;
                 uint32_t o[8];
@@ -472,6 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + (int64_t)m * p.ldo + nn);
                 dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
                 dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+              }
             }
             tc_fence_before();
             __syncwarp();
@@ -505,12 +545,12 @@ cudaError_t get_encoder()
 }
 
 // 2-D map over a row-major [rows x cols] matrix of 2-byte elements with row
-// stride `ld` elements; boxes of 64 columns x 128 rows, 128-byte swizzle.
-cudaError_t encode_a(CUtensorMap *tm, const void *ptr, int rows, int cols, int64_t ld, bool bf16)
+// stride `ld` elements; boxes of 64 columns x box_rows rows, 128-byte swizzle.
+cudaError_t encode_a(CUtensorMap *tm, const void *ptr, int rows, int cols, int64_t ld, bool bf16, int box_rows)
 {
     const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
-    const cuuint32_t box[2] = {BK, BM};
+    const cuuint32_t box[2] = {BK, (cuuint32_t)box_rows};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = g_encode(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
                                 const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -522,16 +562,44 @@ cudaError_t encode_a(CUtensorMap *tm, const void *ptr, int rows, int cols, int64
 // True when every row of a packed matrix starts 8-byte aligned.
 bool even8(const uint32_t *bits, int64_t ld) { return (reinterpret_cast<uintptr_t>(bits) & 7u) == 0 && ld % 2 == 0; }
 
+// One contraction on a persistent grid.  The tile shape follows a makespan
+// model: H = 2 expands half the sign bits per flop, which measured about 1.6x
+// the H = 1 throughput while the expansion bounds the kernel, but it has half
+// as many tiles; take it when ceil(tiles_2 / SMs) * 2 / 1.6 <= ceil(tiles_1 / SMs).
+// A is x (mode 1, bf16) or z (mode 2, fp16), row-major with stride lda.
+template <int MODE>
+cudaError_t launch_sign_gemm(const SignGemmParams &p, const void *a, int64_t lda, const DeviceInfo &dev,
+                             cudaStream_t stream)
+{
+    const int tn = (p.N + BN - 1) / BN;
+    const int t1 = ((p.M + BM - 1) / BM) * tn, t2 = ((p.M + 2 * BM - 1) / (2 * BM)) * tn;
+    const int w1 = (t1 + dev.sm_count - 1) / dev.sm_count, w2 = (t2 + dev.sm_count - 1) / dev.sm_count;
+    const int H = 5 * w2 <= 4 * w1 ? 2 : 1;
+    CUtensorMap tm;
+    cudaError_t e = encode_a(&tm, a, p.M, p.K, lda, MODE == 1, BM * H);
+    if (e != cudaSuccess) return e;
+    if (H == 2)
+        sign_gemm_kernel<MODE, 2><<<std::min(t2, dev.sm_count), Shape<2>::kThreads, Shape<2>::kSmem, stream>>>(tm, p);
+    else
+        sign_gemm_kernel<MODE, 1><<<std::min(t1, dev.sm_count), Shape<1>::kThreads, Shape<1>::kSmem, stream>>>(tm, p);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t prefill_prepare_device(const DeviceInfo &dev)
 {
     (void)dev;
     cudaError_t e = get_encoder();
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(sign_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(sign_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sign_gemm_kernel<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Shape<1>::kSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sign_gemm_kernel<2, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Shape<1>::kSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sign_gemm_kernel<1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Shape<2>::kSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sign_gemm_kernel<2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Shape<2>::kSmem);
+    return e;
 }
 
 size_t prefill_workspace_bytes(int tokens, const int *ranks, int npaths)
@@ -550,9 +618,6 @@ cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStr
     if (e != cudaSuccess) return e;
 
     // contraction 1: Z = (X . B1^T) (.) l
-    CUtensorMap tx;
-    e = encode_a(&tx, a.x, M, a.n_in, a.ldx, true);
-    if (e != cudaSuccess) return e;
     SignGemmParams p1{};
     p1.M = M;
     p1.N = R;
@@ -572,15 +637,10 @@ cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStr
     p1.out = z;
     p1.ldo = R;
     p1.status = dev.status;
-    const int tiles1 = ((M + BM - 1) / BM) * ((R + BN - 1) / BN);
-    sign_gemm_kernel<1><<<std::min(tiles1, dev.sm_count), kThreads, kSmem, stream>>>(tx, p1);
-    e = cudaGetLastError();
+    e = launch_sign_gemm<1>(p1, a.x, a.ldx, dev, stream);
     if (e != cudaSuccess) return e;
 
     // contraction 2: Y = Z . B2^T
-    CUtensorMap tz;
-    e = encode_a(&tz, z, M, R, R, false);
-    if (e != cudaSuccess) return e;
     SignGemmParams p2{};
     p2.M = M;
     p2.N = a.n_out;
@@ -598,9 +658,7 @@ cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStr
     p2.out = a.y;
     p2.ldo = a.ldy;
     p2.status = dev.status;
-    const int tiles2 = ((M + BM - 1) / BM) * ((a.n_out + BN - 1) / BN);
-    sign_gemm_kernel<2><<<std::min(tiles2, dev.sm_count), kThreads, kSmem, stream>>>(tz, p2);
-    return cudaGetLastError();
+    return launch_sign_gemm<2>(p2, z, R, dev, stream);
 }
 
 }  // namespace lb
