@@ -55,6 +55,18 @@ def test_token_sweep_ragged_shape(tokens):
     gu.assert_close(y, gu.oracle_y(layer), f"M={tokens}")
 
 
+@pytest.mark.parametrize("n_in,n_out,ranks", [(256, 5120, [64, 32]), (64, 32, [2432, 2432])])
+def test_prefill_tile_shapes_ragged(n_in, n_out, ranks):
+    """1000 tokens over many output tiles: on a 148-SM part the wide
+    contraction runs 256-row CTA tiles (two 128-row halves sharing each
+    expanded sign tile), the narrow one 128-row tiles.  1000 = 3 x 256 + 232
+    leaves the last tile's second half partly outside the batch, and a latent
+    of 96 (first case) is one and a half K-blocks."""
+    layer = synth.make_layer(n_in, n_out, ranks, 1000, config_id=700 + n_out)
+    y = gu.bf16_to_f64(gu.run_gpu(layer))
+    gu.assert_close(y, gu.oracle_y(layer), f"{n_in}x{n_out} r={ranks} M=1000")
+
+
 @pytest.mark.parametrize("n_in,n_out,ranks", [(32, 32, [32]), (96, 64, [32]), (64, 800, [32, 64]),
                                               (1056, 224, [160, 32]), (4096, 96, [288])])
 def test_small_and_asymmetric_shapes(n_in, n_out, ranks):
