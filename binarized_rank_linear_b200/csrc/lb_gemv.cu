@@ -107,27 +107,35 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const Small1Para
 
     if (p.cs > 1) cluster_arrive_relaxed();  // waited for before the partials go to the first CTA
 
-    // (1) this lane's sign words (row row0 + lane, words wa ..) into
-    // registers, before the dependency wait.  (Fetching g and l this early as
-    // well measured slower at the Llama-2-7B q_proj shape, so they come later.)
+    // (1) weights, before the dependency wait: this lane's sign words (row
+    // row0 + lane, words wa ..) into registers; the CTA's slice of g and l of
+    // its rows into shared memory with asynchronous copies
     uint32_t bw[kWW];
     {
         const int64_t ld = second ? p.vt_ld1 : p.vt_ld0;
         load_words(bw, (second ? p.vt1 : p.vt0) + (int64_t)(row0 + lane) * ld + wa, nwd);
     }
-    const uint16_t *g = (second ? p.g1 : p.g0) + 32 * c0;
     const int ntab = 8 * (c1 - c0);
-    const uint16_t *l = second ? p.l1 : p.l0;
+    float4 *tab = reinterpret_cast<float4 *>(smem);  // [M][cww * 8][kTab / 4]
+    float *red = reinterpret_cast<float *>(smem) + (size_t)M * cww * 8 * kTab;  // [warps][32][MT]
+    float *part = red + nwarps * 32 * MT;                                       // [cs][32][MT] (first CTA)
+    uint16_t *gsm = reinterpret_cast<uint16_t *>(part + kMaxCluster * 32 * MT);  // [cww * 32]
+    uint16_t *lsm = gsm + cww * 32;                                              // [32]
+    {
+        const uint16_t *g = (second ? p.g1 : p.g0) + 32 * c0;
+        for (int e = tid; e < 4 * (c1 - c0); e += nthr) cp_async16(gsm + 8 * e, g + 8 * e);
+        if (tid < 4) cp_async16(lsm + 8 * tid, (second ? p.l1 : p.l0) + row0 + 8 * tid);
+        cp_async_commit();
+    }
     if (p.early) pdl_launch_dependents();
 
     // (2) x comes from the previous kernel: tables of v = g (.) x for the
     // CTA's columns, token-major
     pdl_wait();
-    float4 *tab = reinterpret_cast<float4 *>(smem);  // [M][cww * 8][kTab / 4]
-    float *red = reinterpret_cast<float *>(smem) + (size_t)M * cww * 8 * kTab;  // [warps][32][MT]
-    float *part = red + nwarps * 32 * MT;                                       // [cs][32][MT] (first CTA)
+    cp_async_wait_all();
+    __syncthreads();
     for (int t = tid; t < ntab; t += nthr) {
-        const uint2 gw = __ldg(reinterpret_cast<const uint2 *>(g + 4 * t));
+        const uint2 gw = *reinterpret_cast<const uint2 *>(gsm + 4 * t);
         for (int m = 0; m < M; ++m) {
             const uint2 xq = __ldg(reinterpret_cast<const uint2 *>(p.x + (int64_t)m * p.ldx + 32 * c0 + 4 * t));
             const float v0 = f16_bits_to_float(gw.x & 0xffff) * bf16_bits_to_float(xq.x & 0xffff);
@@ -174,7 +182,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const Small1Para
         const int r = e / M, m = e - r * M;
         float s = 0.f;
         for (int w = 0; w < nwarps; ++w) s += red[(w * 32 + r) * MT + m];
-        if (p.cs == 1) p.z[(int64_t)(kg0 + r) * M + m] = s * f16_bits_to_float(l[row0 + r]);
+        if (p.cs == 1) p.z[(int64_t)(kg0 + r) * M + m] = s * f16_bits_to_float(lsm[r]);
         else st_shared_cluster_f32(map_shared_rank(part + (split * 32 + r) * MT + m, 0), s);
     }
     if (p.cs > 1) {
@@ -184,7 +192,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const Small1Para
                 const int r = e / M, m = e - r * M;
                 float s = 0.f;
                 for (int c = 0; c < p.cs; ++c) s += part[(c * 32 + r) * MT + m];
-                p.z[(int64_t)(kg0 + r) * M + m] = s * f16_bits_to_float(l[row0 + r]);
+                p.z[(int64_t)(kg0 + r) * M + m] = s * f16_bits_to_float(lsm[r]);
             }
         }
     }
@@ -326,7 +334,8 @@ struct Small2Plan {
 
 size_t small1_smem(int warps, int ww, int M, int MT)
 {
-    return (size_t)M * warps * ww * 8 * kTab * 4 + (size_t)(warps + kMaxCluster) * 32 * MT * 4;
+    return (size_t)M * warps * ww * 8 * kTab * 4 + (size_t)(warps + kMaxCluster) * 32 * MT * 4 +
+           (size_t)warps * ww * 32 * 2 + 64;
 }
 size_t small2_smem(int warps, int WT, int M, int MT)
 {
@@ -431,7 +440,11 @@ cudaError_t launch_small(const ForwardArgs &a, const DeviceInfo &dev, cudaStream
     }
     E.ks = p2.ks;
     E.ww = p2.ww;
-    E.early = 0;
+    // Releasing the next kernel on the stream (the next layer's contraction
+    // 1) at entry overlaps its weight loads with this kernel, but its CTAs
+    // then compete for SMs: measured faster when this grid is light (at most
+    // 8 warps per SM), slower when it is not.
+    E.early = (int64_t)p2.ctas * p2.warps <= 8 * (int64_t)dev.sm_count ? 1 : 0;
     E.y = a.y + (int64_t)m0 * a.ldy;
     E.ldy = a.ldy;
 
