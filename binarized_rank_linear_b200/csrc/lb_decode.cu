@@ -786,6 +786,7 @@ cudaError_t prepare_nt(const DeviceInfo &dev)
 cudaError_t decode_prepare_device(const DeviceInfo &dev)
 {
     cudaError_t e = small_prepare_device(dev);
+    if (e == cudaSuccess) e = mid_prepare_device(dev);
     if (e == cudaSuccess) e = prepare_nt<1>(dev);
     if (e == cudaSuccess) e = prepare_nt<2>(dev);
     if (e == cudaSuccess) e = prepare_nt<4>(dev);
@@ -798,7 +799,8 @@ size_t decode_workspace_bytes(int tokens, int n_in, int n_out, const int *ranks,
     (void)n_out;
     const int M = std::min(tokens, kDecodeMaxTokens);
     const size_t mma = std::max(latent_frag_bytes(M, ranks, npaths, nullptr), kMaxPartialBytes);
-    return std::max(mma, small_workspace_bytes(std::min(M, kSmallMaxTokens), ranks, npaths));
+    return std::max(std::max(mma, mid_workspace_bytes(M, ranks, npaths)),
+                    small_workspace_bytes(std::min(M, kSmallMaxTokens), ranks, npaths));
 }
 
 cudaError_t decode_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream)
@@ -809,6 +811,7 @@ cudaError_t decode_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStre
         const int ranks[2] = {a.path[0].rank, a.npaths > 1 ? a.path[1].rank : 0};
         if (M <= kSmallMaxTokens && small_fits(M, a.n_in, a.n_out, ranks, a.npaths, dev))
             e = small_forward(a, dev, stream, m0, M);
+        else if (M <= kMidMaxTokens) e = mid_forward(a, dev, stream, m0, M);
         else if (M <= 8) e = launch_decode<1>(a, dev, stream, m0, M);
         else if (M <= 16) e = launch_decode<2>(a, dev, stream, m0, M);
         else e = launch_decode<4>(a, dev, stream, m0, M);

@@ -60,6 +60,13 @@ size_t decode_workspace_bytes(int tokens, int n_in, int n_out, const int *ranks,
 cudaError_t decode_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 cudaError_t decode_prepare_device(const DeviceInfo &dev);
 
+// 5..32 tokens per launch pair on tcgen05 with the sign matrix as the
+// 128-row MMA operand (lb_mid.cu); x is sliced in batches of at most 32.
+constexpr int kMidMaxTokens = 32;
+size_t mid_workspace_bytes(int tokens, const int *ranks, int npaths);
+cudaError_t mid_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M);
+cudaError_t mid_prepare_device(const DeviceInfo &dev);
+
 // Prefill path (more than kDecodeMaxTokens tokens): two tcgen05 GEMMs with the
 // binary operand expanded in shared memory (lb_prefill.cu).
 size_t prefill_workspace_bytes(int tokens, const int *ranks, int npaths);

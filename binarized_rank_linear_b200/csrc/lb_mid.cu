@@ -1,0 +1,482 @@
+// lb_mid.cu - the forward pass for 5..32 tokens, on tcgen05 tensor cores.
+//
+// The layer (sesamedisk.com, "Samsung LittleBit 13B Model", section "What the
+// method actually computes", Proposition 1) as two skinny products in which
+// the sign matrix is the 128-row MMA operand and the few tokens are the N
+// dimension (16 or 32):
+//
+//   contraction 1:  C1[k, m] = sum_i W1[k, i] x[m, i],  W1[k, i] = sign(V_p[i, k]) g_p[i]   (bf16)
+//                   z[m, k]  = l_k C1[k, m], rounded to fp16 (the operand of contraction 2)
+//   contraction 2:  C2[o, m] = sum_k W2[o, k] z[m, k],  W2[o, k] = sign(U_p[o, k]) h_p[o]   (fp16)
+//                   y[m, o]  = C2[o, m], rounded to bf16
+//
+// with both paths of residual compensation concatenated (rows of W1, columns
+// of W2).  Every sign bit is expanded into shared memory exactly once per
+// call, whatever the number of tokens.
+//
+// A CTA takes one 128-row tile of W and a range of its K-blocks.  The `cs`
+// CTAs that split the K-blocks of a tile form a thread-block cluster: each
+// sends the rows of its partial accumulator that CTA r finalises to CTA r
+// (distributed shared memory), and every CTA adds what it received in
+// cluster-rank order, so results do not depend on timing.
+//   warp 0      allocates tensor memory, waits for the previous kernel, then
+//               streams the token tiles (x or z) with TMA (no multicast)
+//   warp 1      one thread issues tcgen05.mma (M = 128, N = 16 or 32, K = 16)
+//   warps 2..9  two groups of 4 taking alternate K-blocks, one W row per
+//               thread: expand the row's packed signs into +-scale values in
+//               128-byte-swizzled shared memory; warps 2..5 then read the
+//               accumulator and finish the tile
+// Every wait on an mbarrier is bounded in time; a wait that gives up sets
+// LB_ERR_DEVICE_TIMEOUT and the CTA winds down.
+#include <algorithm>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "lb_common.cuh"
+#include "lb_internal.h"
+#include "lb_tc.cuh"
+
+namespace lb {
+namespace {
+
+using namespace tc;
+
+constexpr int TM = 128, BK = 64, STAGES = 4;
+constexpr int kGroupWarps = 4;                  // one W row per thread: 128 rows
+constexpr int kProducerWarps = 2 * kGroupWarps;  // two groups take alternate K-blocks
+constexpr int kThreads = 32 * (2 + kProducerWarps);
+constexpr int kMaxCluster = 8;
+constexpr uint32_t A_BYTES = TM * BK * 2;  // expanded W tile, 16 KB
+constexpr uint32_t G_BYTES = 2 * BK * 2;   // a K-block of g for both paths
+constexpr uint32_t TMEM_COLS = 32;
+
+template <int NT>
+struct MidShape {
+    static constexpr uint32_t kBBytes = (uint32_t)NT * BK * 2;  // token tile
+    static constexpr uint32_t kRedBytes = (uint32_t)TM * NT * 4;  // partials received, [cs][128 / cs][NT]
+    static constexpr size_t kSmem =
+        1024 + (size_t)STAGES * (A_BYTES + kBBytes) + kRedBytes + (size_t)kProducerWarps * 2 * G_BYTES + 256;
+};
+
+struct MidParams {
+    int M;       // tokens (at most NT)
+    int rows;    // rows of W: mode 1 R (both paths), mode 2 n_out
+    int K;       // mode 1 n_in, mode 2 R
+    int r0;      // mode 1: rows [0, r0) are path 0; mode 2: K columns [0, r0) are path 0
+    int bits8;   // every K-block's two words of a row can be fetched as one aligned 8-byte load
+    const uint32_t *bits0, *bits1;
+    int64_t bld0, bld1;       // words per packed row
+    const uint16_t *s0, *s1;  // mode 1: g (length K); mode 2: h (length rows)
+    const uint16_t *l0, *l1;  // mode 1: latent scale
+    int cs;                   // CTAs per tile (cluster size), splitting the K-blocks
+    int kpc;                  // K-blocks per CTA
+    void *out;                // mode 1: z fp16 [M][ldo]; mode 2: y bf16 [M][ldo]
+    int64_t ldo;
+    int *status;
+};
+
+// One finished value: mode 1 z[m][nn] = l_nn c (fp16; true if it does not
+// fit), mode 2 y[m][nn] (bf16).
+template <int MODE>
+__device__ __forceinline__ bool put_value(const MidParams &p, int m, int nn, float s)
+{
+    uint16_t *out = static_cast<uint16_t *>(p.out) + (int64_t)m * p.ldo + nn;
+    if (MODE == 1) {
+        const uint16_t lv = nn < p.r0 ? p.l0[nn] : p.l1[nn - p.r0];
+        const float z = s * f16_bits_to_float(lv);
+        *out = (uint16_t)(pack_half2(z, 0.f) & 0xffffu);
+        return beyond_f16(z);
+    }
+    *out = float_to_bf16_bits(s);
+    return false;
+}
+
+template <int MODE, int NT>
+__global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const MidParams p)
+{
+    using S = MidShape<NT>;
+    constexpr uint32_t B_BYTES = S::kBBytes;
+    extern __shared__ uint8_t smem_raw[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;  // SW128 tiles need 1024-byte alignment
+    const uint32_t sA = base, sB = base + STAGES * A_BYTES;
+    const uint32_t sRed = sB + STAGES * B_BYTES;  // partials received from the cluster, [cs][rpr][NT] fp32
+    const uint32_t sGbf = sRed + S::kRedBytes;    // mode 1, per producer warp: g in bf16, [warp][2][path][64]
+    const uint32_t bars = sGbf + kProducerWarps * 2 * G_BYTES;
+    // full[STAGES], empty[STAGES], acc_full, drain, then the tmem address
+    const uint32_t full0 = bars, empty0 = bars + 8 * STAGES, accf = bars + 16 * STAGES, drain = accf + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + (drain + 8 - raw));
+    __shared__ int abort_shared;
+    volatile int &abort_flag = abort_shared;
+
+    const int cs = p.cs;
+    const int tile = blockIdx.x / cs, split = blockIdx.x - tile * cs;  // split = rank in the cluster
+    const int nk = (p.K + BK - 1) / BK;
+    const int kb0 = split * p.kpc, nkb = max(0, min(nk, kb0 + p.kpc) - kb0);
+    if (cs > 1) cluster_arrive_relaxed();  // waited for before partials go to other CTAs
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int s = 0; s < STAGES; ++s) {
+                mbar_init(full0 + 8 * s, 1 + kGroupWarps);  // TMA arrive.expect_tx + one group's warps
+                mbar_init(empty0 + 8 * s, 1);               // one tcgen05.commit
+            }
+            mbar_init(accf, 1);
+            mbar_init(drain, 1);
+            abort_flag = 0;
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+        __syncwarp();
+        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    uint32_t acc_row[NT];  // warps 2..5: this thread's row of the accumulator
+#pragma unroll
+    for (int m = 0; m < NT; ++m) acc_row[m] = 0u;
+
+    if (warp == 0) {
+        // ---------------- token tiles (TMA); the tokens come from the previous kernel
+        if (lane == 0) {
+            pdl_wait();
+            int issued = 0;
+            for (int j = 0; j < nkb; ++j) {
+                const int s = j % STAGES;
+                const uint32_t ph = (uint32_t)(j / STAGES) & 1u;
+                if (!mbar_wait(empty0 + 8 * s, ph ^ 1u) || abort_flag) {
+                    abort_flag = 1;
+                    break;
+                }
+                mbar_arrive_expect_tx(full0 + 8 * s, B_BYTES);
+                tma_load_2d(sB + s * B_BYTES, &tmB, (kb0 + j) * BK, 0, full0 + 8 * s);
+                ++issued;
+            }
+            if (abort_flag) {
+                for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+                    mbar_wait(full0 + 8 * (j % STAGES), (uint32_t)(j / STAGES) & 1u);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = instr_desc(MODE == 1 ? 1u : 0u, TM, NT);
+            for (int j = 0; j < nkb; ++j) {
+                const int s = j % STAGES;
+                const uint32_t ph = (uint32_t)(j / STAGES) & 1u;
+                if (!mbar_wait(full0 + 8 * s, ph) || abort_flag) {
+                    abort_flag = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t ad = smem_desc(sA + s * A_BYTES), bd = smem_desc(sB + s * B_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk)  // +32 bytes along K per step of 16
+                    umma(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (j | kk) != 0);
+                umma_commit(empty0 + 8 * s);
+            }
+            umma_commit(accf);
+            // every MMA issued has finished before the CTA frees tensor memory
+            umma_commit(drain);
+            if (!mbar_wait(drain, 0)) abort_flag = 1;
+        }
+    } else {
+        // ---------------- producers: group grp expands blocks j = grp, grp + 2, ...
+        // of this CTA's K range, one W row per thread; what a block needs from
+        // memory (the row's sign words; g in mode 1) is loaded into registers
+        // two of the group's blocks ahead
+        const int pw = warp - 2;  // producer warp 0 .. 7
+        const int grp = pw >> 2;
+        const int row = ((pw & 3) << 5) | lane;  // W row within the tile
+        const int nn = tile * TM + row;
+        const uint32_t x7 = (uint32_t)(row & 7);  // the row's 128-byte swizzle
+        const bool row_in = nn < p.rows;
+        const bool sec_row = MODE == 1 && nn >= p.r0;  // mode 1: the row's path
+        const int kwords = p.K >> 5, r0w = p.r0 >> 5;
+        const uint32_t gbfw = sGbf + (uint32_t)pw * 2 * G_BYTES;  // this warp's two bf16 g slots
+        const uint32_t *rb0 = nullptr, *rb1 = nullptr;
+        uint32_t hs0 = 0u, hs1 = 0u;  // mode 2: h of the row, both paths, both halves
+        if (row_in) {
+            if (MODE == 1) {
+                rb0 = sec_row ? p.bits1 + (int64_t)(nn - p.r0) * p.bld1 : p.bits0 + (int64_t)nn * p.bld0;
+            } else {
+                rb0 = p.bits0 + (int64_t)nn * p.bld0;
+                if (p.bits1) rb1 = p.bits1 + (int64_t)nn * p.bld1;
+                const uint32_t h0 = ldg_early_u16(p.s0 + nn), h1 = p.s1 ? ldg_early_u16(p.s1 + nn) : 0u;
+                hs0 = h0 | (h0 << 16);
+                hs1 = h1 | (h1 << 16);
+            }
+        }
+        auto wp = [&](int w) { return (MODE == 1 || w < r0w) ? rb0 + w : rb1 + (w - r0w); };
+        struct Pref {
+            uint2 bits;  // the row's two sign words of the block (zero outside the matrix)
+            uint4 g;     // mode 1, lanes 0..15: g of path lane / 8, columns 8 (lane % 8) .. (fp16)
+        };
+        auto fetch = [&](int j) {
+            Pref f;
+            f.bits = make_uint2(0u, 0u);
+            f.g = make_uint4(0u, 0u, 0u, 0u);
+            if (j >= nkb) return f;
+            const int kb = kb0 + j, wd = 2 * kb;
+            if (row_in && wd < kwords) {
+                if (p.bits8 && wd + 1 < kwords) {
+                    f.bits = ldg_early_v2(wp(wd));
+                } else {
+                    f.bits.x = ldg_early_u32(wp(wd));
+                    if (wd + 1 < kwords) f.bits.y = ldg_early_u32(wp(wd + 1));
+                }
+            }
+            if (MODE == 1 && lane < 16) {
+                const int pp = lane >> 3, k0 = kb * BK + 8 * (lane & 7);
+                const uint16_t *gs = pp ? p.s1 : p.s0;
+                if (gs != nullptr && k0 < p.K) f.g = ldg_early_v4(gs + k0);
+            }
+            return f;
+        };
+        Pref f0 = fetch(grp), f1 = fetch(grp + 2);
+        for (int j = grp, it = 0; j < nkb; j += 2, ++it) {
+            const Pref cur = f0;
+            f0 = f1;
+            f1 = fetch(j + 4);
+            const int kb = kb0 + j;
+            const int s = j % STAGES;
+            const uint32_t ph = (uint32_t)(j / STAGES) & 1u;
+            bool ok = mbar_wait(empty0 + 8 * s, ph ^ 1u) && !abort_flag;
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) {
+                abort_flag = 1;
+                break;
+            }
+            uint4 sc[8];  // per chunk: the four packed scale words
+            if (MODE == 1) {
+                // lanes 0..15 round this block's g to bf16 into the warp's slot
+                // it % 2 (last read two iterations ago, before a __syncwarp)
+                if (lane < 16) {
+                    const uint32_t w[4] = {cur.g.x, cur.g.y, cur.g.z, cur.g.w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        o[q] = (uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[q] & 0xffffu))) |
+                               ((uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[q] >> 16))) << 16);
+                    *reinterpret_cast<uint4 *>(smem_raw + (gbfw + (it & 1) * G_BYTES + lane * 16 - raw)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                __syncwarp();
+                const uint8_t *gb = smem_raw + (gbfw + (it & 1) * G_BYTES + (sec_row ? BK * 2 : 0) - raw);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) sc[q] = *reinterpret_cast<const uint4 *>(gb + 16 * q);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int k0 = kb * BK + 8 * q;  // first column of the chunk
+                    const uint32_t h = k0 < p.K ? (k0 >= p.r0 ? hs1 : hs0) : 0u;
+                    sc[q] = make_uint4(h, h, h, h);
+                }
+            }
+            const uint32_t rowx = (sA + s * A_BYTES + row * 128) | (x7 << 4);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                store_sign_chunk(rowx ^ (16u * q), __byte_perm(q < 4 ? cur.bits.x : cur.bits.y, 0u, 0x4440u | (uint32_t)(q & 3)),
+                                 sc[q]);
+            fence_async_shared();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full0 + 8 * s);
+        }
+        // warps 2..5: this thread's row 32 (warp % 4) + lane of the accumulator
+        if (pw < 4) {
+            bool ok = !abort_flag && mbar_wait(accf, 0);
+            ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+            if (!ok) abort_flag = 1;
+            tc_fence_after();
+            if (ok && nkb > 0) {
+                const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+                if (NT == 16) {
+                    uint32_t v[16];
+                    tmem_ld16(ta, v);
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) acc_row[m] = v[m];
+                } else {
+                    uint32_t v[32];
+                    tmem_ld32(ta, v);
+#pragma unroll
+                    for (int m = 0; m < NT; ++m) acc_row[m] = v[m & 31];
+                }
+            }
+        }
+    }
+
+    // ---------------- finish: every partial of the tile added in rank order
+    pdl_launch_dependents();
+    __syncwarp();
+    const bool holder = warp >= 2 && warp < 6;  // these threads hold an accumulator row
+    bool overflow = false;
+    if (cs == 1) {
+        if (holder) {
+            pdl_wait();  // y / z may still be in use by the previous kernel
+            const int nn = tile * TM + 32 * (warp & 3) + lane;
+            if (nn < p.rows) {
+#pragma unroll
+                for (int m = 0; m < NT; ++m)
+                    if (m < p.M) overflow |= put_value<MODE>(p, m, nn, __uint_as_float(acc_row[m]));
+            }
+        }
+    } else {
+        // CTA r finalises rows r * rpr .. of the tile: every CTA sends it its
+        // partials of those rows, then adds what it received
+        const int rpr = TM / cs;
+        cluster_wait();  // every CTA of the cluster is running
+        if (holder) {
+            const int rho = 32 * (warp & 3) + lane;
+            const int dst = rho / rpr, q = rho - dst * rpr;
+            const uint32_t ra = map_shared_addr(sRed + (uint32_t)((split * rpr + q) * NT) * 4u, (uint32_t)dst);
+#pragma unroll
+            for (int m4 = 0; m4 < NT; m4 += 4)
+                st_shared_cluster_v4(ra + 4u * m4, acc_row[m4], acc_row[m4 + 1], acc_row[m4 + 2], acc_row[m4 + 3]);
+        }
+        cluster_sync();  // every partial has arrived
+        pdl_wait();
+        const float *red = reinterpret_cast<const float *>(smem_raw + (sRed - raw));
+        for (int e = tid; e < rpr * p.M; e += kThreads) {
+            const int m = e / rpr, q = e - m * rpr;
+            float s = 0.f;
+            for (int c = 0; c < cs; ++c) s += red[(c * rpr + q) * NT + m];
+            const int nn = tile * TM + split * rpr + q;
+            if (nn < p.rows) overflow |= put_value<MODE>(p, m, nn, s);
+        }
+    }
+    if (overflow) set_status(p.status, LB_ERR_RANGE);
+
+    tc_fence_before();
+    __syncthreads();
+    if (abort_flag && tid == 0) set_status(p.status, LB_ERR_DEVICE_TIMEOUT);
+    if (warp == 0) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+// CTAs per tile: a power of two (each finalises 128 / cs rows of the tile),
+// at most a portable cluster, enough to give about two CTAs per SM (each uses
+// about 100 KB of shared memory), and never a CTA without a K-block.
+int pick_split(int tiles, int nk, int sm_count)
+{
+    const int want = std::max(1, std::min(kMaxCluster, (2 * sm_count) / std::max(1, tiles)));
+    int cs = 1;
+    while (2 * cs <= want && 2 * cs <= nk) cs *= 2;
+    while (cs > 1 && (cs - 1) * ((nk + cs - 1) / cs) >= nk) cs /= 2;
+    return cs;
+}
+
+template <int MODE, int NT>
+cudaError_t launch_mid(MidParams p, const void *b, int64_t ldb, const DeviceInfo &dev, cudaStream_t stream)
+{
+    const int tiles = (p.rows + TM - 1) / TM, nk = (p.K + BK - 1) / BK;
+    p.cs = pick_split(tiles, nk, dev.sm_count);
+    p.kpc = (nk + p.cs - 1) / p.cs;
+    CUtensorMap tm;
+    cudaError_t e = encode_2d(&tm, b, p.M, p.K, ldb, MODE == 1, NT);
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)p.cs;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(tiles * p.cs));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = MidShape<NT>::kSmem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.cs > 1 ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, mid_gemm_kernel<MODE, NT>, tm, p);
+}
+
+template <int NT>
+cudaError_t mid_forward_nt(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M)
+{
+    const int r0 = a.path[0].rank, r1 = a.npaths > 1 ? a.path[1].rank : 0;
+    const int R = r0 + r1;
+    uint16_t *z = static_cast<uint16_t *>(a.workspace);  // [M][R] fp16
+    const uint16_t *x = a.x + (int64_t)m0 * a.ldx;
+
+    // contraction 1: z = l (.) (W1 x^T), rows = latent indices of both paths
+    MidParams p1{};
+    p1.M = M;
+    p1.rows = R;
+    p1.K = a.n_in;
+    p1.r0 = r0;
+    p1.bits8 = even8(a.path[0].vt_bits, a.path[0].vt_ld) && (a.npaths < 2 || even8(a.path[1].vt_bits, a.path[1].vt_ld));
+    p1.bits0 = a.path[0].vt_bits;
+    p1.bld0 = a.path[0].vt_ld;
+    p1.s0 = a.path[0].g;
+    p1.l0 = a.path[0].l;
+    if (a.npaths > 1) {
+        p1.bits1 = a.path[1].vt_bits;
+        p1.bld1 = a.path[1].vt_ld;
+        p1.s1 = a.path[1].g;
+        p1.l1 = a.path[1].l;
+    }
+    p1.out = z;
+    p1.ldo = R;
+    p1.status = dev.status;
+    cudaError_t e = launch_mid<1, NT>(p1, x, a.ldx, dev, stream);
+    if (e != cudaSuccess) return e;
+
+    // contraction 2: y = W2 z^T, rows = outputs
+    MidParams p2{};
+    p2.M = M;
+    p2.rows = a.n_out;
+    p2.K = R;
+    p2.r0 = r0;
+    p2.bits8 = even8(a.path[0].u_bits, a.path[0].u_ld) && (a.npaths < 2 || (r0 % 64 == 0 && even8(a.path[1].u_bits, a.path[1].u_ld)));
+    p2.bits0 = a.path[0].u_bits;
+    p2.bld0 = a.path[0].u_ld;
+    p2.s0 = a.path[0].h;
+    if (a.npaths > 1) {
+        p2.bits1 = a.path[1].u_bits;
+        p2.bld1 = a.path[1].u_ld;
+        p2.s1 = a.path[1].h;
+    }
+    p2.out = a.y + (int64_t)m0 * a.ldy;
+    p2.ldo = a.ldy;
+    p2.status = dev.status;
+    return launch_mid<2, NT>(p2, z, R, dev, stream);
+}
+
+}  // namespace
+
+cudaError_t mid_prepare_device(const DeviceInfo &dev)
+{
+    (void)dev;
+    cudaError_t e = get_encoder();
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(mid_gemm_kernel<1, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MidShape<16>::kSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(mid_gemm_kernel<2, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MidShape<16>::kSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(mid_gemm_kernel<1, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MidShape<32>::kSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(mid_gemm_kernel<2, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MidShape<32>::kSmem);
+    return e;
+}
+
+size_t mid_workspace_bytes(int tokens, const int *ranks, int npaths)
+{
+    const size_t R = (size_t)ranks[0] + (npaths > 1 ? ranks[1] : 0);
+    return (size_t)std::min(tokens, kMidMaxTokens) * R * 2;
+}
+
+cudaError_t mid_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M)
+{
+    if (M <= 16) return mid_forward_nt<16>(a, dev, stream, m0, M);
+    return mid_forward_nt<32>(a, dev, stream, m0, M);
+}
+
+}  // namespace lb

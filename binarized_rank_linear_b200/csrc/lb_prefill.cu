@@ -30,15 +30,16 @@
 // hanging.
 #include <algorithm>
 #include <cstdint>
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "lb_common.cuh"
 #include "lb_internal.h"
+#include "lb_tc.cuh"
 
 namespace lb {
 namespace {
+
+using namespace tc;
 
 constexpr int BM = 128, BN = 256, BK = 64;  // one MMA: M = 128, N = 256; K-blocks of 64
 constexpr int kGroupWarps = 8;                // producer warps per K-block: one B row per thread
@@ -65,110 +66,6 @@ struct Shape {
     static constexpr size_t kSmem =
         1024 + (size_t)kStages * (kABytes + B_BYTES) + (size_t)kProducerWarps * 2 * G_BYTES + 256;
 };
-constexpr unsigned long long kWaitNs = 2000000000ull;  // give up on a wait after 2 s
-
-// ---------------------------------------------------------------- PTX wrappers
-__device__ __forceinline__ unsigned long long globaltimer()
-{
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar)
-{
-    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
-{
-    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
-                 "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
-{
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return done != 0;
-}
-// Wait for the phase with the given parity to complete, for at most kWaitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
-{
-    if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = globaltimer();
-    for (;;) {
-        for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer() - t0 > kWaitNs) return false;
-    }
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *tm, int x, int y, uint32_t bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(dst), "l"(tm), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-__device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t cols)
-{
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(cols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols)
-{
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
-}
-__device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
-        : "memory");
-}
-__device__ __forceinline__ void umma_commit(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-// 32 consecutive fp32 columns of this warp's 32 lanes, one register each,
-// then wait for them (one wait per 32 columns).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
-          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
-// 128 bytes, 8-row atoms 1024 bytes apart.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr)
-{
-    return (uint64_t)((addr >> 4) & 0x3FFF) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
-}
-// Instruction descriptor for kind::f16: fp32 accumulate, K-major A and B,
-// M = 128, N = 256; `fmt` 0 = fp16 operands, 1 = bf16 operands.
-__device__ __forceinline__ uint32_t instr_desc(uint32_t fmt)
-{
-    return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-}
-
 // Tiles are K-major with 128-byte swizzle: row `row` holds 64 two-byte
 // elements in 128 bytes, and its 16-byte chunk j (elements 8j .. 8j + 7) is
 // stored at chunk position j ^ (row % 8).
@@ -271,7 +168,7 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
         // ---------------- MMA issuer.  H = 1: tile i accumulates in columns
         // 256 (i % 2) ..; H = 2: half h of every tile accumulates in columns 256 h ..
         if (lane == 0) {
-            const uint32_t idesc = instr_desc(MODE == 1 ? 1u : 0u);
+            const uint32_t idesc = instr_desc(MODE == 1 ? 1u : 0u, BM, BN);
             int gb = 0;
             for (int i = 0; i < my_tiles && !abort_flag; ++i) {
                 const int b = H == 1 ? (i & 1) : 0;  // hand-over barriers of the accumulator(s)
@@ -443,16 +340,8 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
             const uint32_t rowx = (sB + s * B_BYTES + row * 128) | (x7 << 4);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                const uint32_t b = __byte_perm(q < 4 ? cur.bits.x : cur.bits.y, 0u, 0x4440u | (uint32_t)(q & 3));
-                // (b * K_i) puts sign bit 2i at bit 15 and bit 2i + 1 at bit 31
-                // (the two shifted copies of the byte do not overlap: no carries)
-                const uint32_t v0 = ((b * 0x40008000u) & 0x80008000u) ^ sc[q].x;
-                const uint32_t v1 = ((b * 0x10002000u) & 0x80008000u) ^ sc[q].y;
-                const uint32_t v2 = ((b * 0x04000800u) & 0x80008000u) ^ sc[q].z;
-                const uint32_t v3 = ((b * 0x01000200u) & 0x80008000u) ^ sc[q].w;
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowx ^ (16u * q)), "r"(v0), "r"(v1),
-                             "r"(v2), "r"(v3)
-                             : "memory");
+                store_sign_chunk(rowx ^ (16u * q), __byte_perm(q < 4 ? cur.bits.x : cur.bits.y, 0u, 0x4440u | (uint32_t)(q & 3)),
+                                 sc[q]);
             }
             fence_async_shared();
             __syncwarp();
@@ -531,37 +420,6 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-
-cudaError_t get_encoder()
-{
-    if (g_encode) return cudaSuccess;
-    cudaDriverEntryPointQueryResult q;
-    void *fn = nullptr;
-    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
-    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    return cudaSuccess;
-}
-
-// 2-D map over a row-major [rows x cols] matrix of 2-byte elements with row
-// stride `ld` elements; boxes of 64 columns x box_rows rows, 128-byte swizzle.
-cudaError_t encode_a(CUtensorMap *tm, const void *ptr, int rows, int cols, int64_t ld, bool bf16, int box_rows)
-{
-    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
-    const cuuint32_t box[2] = {BK, (cuuint32_t)box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = g_encode(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                                const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
-// True when every row of a packed matrix starts 8-byte aligned.
-bool even8(const uint32_t *bits, int64_t ld) { return (reinterpret_cast<uintptr_t>(bits) & 7u) == 0 && ld % 2 == 0; }
-
 // One contraction on a persistent grid.  The tile shape follows a makespan
 // model: H = 2 expands half the sign bits per flop, which measured about 1.6x
 // the H = 1 throughput while the expansion bounds the kernel, but it has half
@@ -576,7 +434,7 @@ cudaError_t launch_sign_gemm(const SignGemmParams &p, const void *a, int64_t lda
     const int w1 = (t1 + dev.sm_count - 1) / dev.sm_count, w2 = (t2 + dev.sm_count - 1) / dev.sm_count;
     const int H = 5 * w2 <= 4 * w1 ? 2 : 1;
     CUtensorMap tm;
-    cudaError_t e = encode_a(&tm, a, p.M, p.K, lda, MODE == 1, BM * H);
+    cudaError_t e = encode_2d(&tm, a, p.M, p.K, lda, MODE == 1, BM * H);
     if (e != cudaSuccess) return e;
     if (H == 2)
         sign_gemm_kernel<MODE, 2><<<std::min(t2, dev.sm_count), Shape<2>::kThreads, Shape<2>::kSmem, stream>>>(tm, p);
