@@ -53,7 +53,10 @@ constexpr uint32_t TMEM_COLS = 32;
 template <int NT>
 struct MidShape {
     static constexpr uint32_t kBBytes = (uint32_t)NT * BK * 2;  // token tile
-    static constexpr uint32_t kRedBytes = (uint32_t)TM * NT * 4;  // partials received, [cs][128 / cs][NT]
+    // partials received, [cs][128 / cs][kRedStride] fp32: rows padded by 4
+    // floats so that 16-byte accesses of consecutive rows cover every bank
+    static constexpr int kRedStride = NT + 4;
+    static constexpr uint32_t kRedBytes = (uint32_t)TM * kRedStride * 4;
     static constexpr size_t kSmem =
         1024 + (size_t)STAGES * (A_BYTES + kBBytes) + kRedBytes + (size_t)kProducerWarps * 2 * G_BYTES + 256;
 };
@@ -75,20 +78,31 @@ struct MidParams {
     int *status;
 };
 
-// One finished value: mode 1 z[m][nn] = l_nn c (fp16; true if it does not
-// fit), mode 2 y[m][nn] (bf16).
-template <int MODE>
-__device__ __forceinline__ bool put_value(const MidParams &p, int m, int nn, float s)
+// One finished row nn of the tile for every token: mode 1 z[m][nn] =
+// l_nn c[m] (fp16; returns true if a value does not fit), mode 2 y[m][nn]
+// (bf16).  A warp's lanes take consecutive rows, so each token's stores are
+// contiguous.
+template <int MODE, int NT>
+__device__ __forceinline__ bool finish_row(const MidParams &p, int nn, const float (&c)[NT])
 {
-    uint16_t *out = static_cast<uint16_t *>(p.out) + (int64_t)m * p.ldo + nn;
+    uint16_t *out = static_cast<uint16_t *>(p.out) + nn;
+    bool overflow = false;
     if (MODE == 1) {
-        const uint16_t lv = nn < p.r0 ? p.l0[nn] : p.l1[nn - p.r0];
-        const float z = s * f16_bits_to_float(lv);
-        *out = (uint16_t)(pack_half2(z, 0.f) & 0xffffu);
-        return beyond_f16(z);
+        const float lv = f16_bits_to_float(nn < p.r0 ? p.l0[nn] : p.l1[nn - p.r0]);
+#pragma unroll
+        for (int m = 0; m < NT; ++m) {
+            if (m < p.M) {
+                const float z = c[m] * lv;
+                out[(int64_t)m * p.ldo] = (uint16_t)(pack_half2(z, 0.f) & 0xffffu);
+                overflow |= beyond_f16(z);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int m = 0; m < NT; ++m)
+            if (m < p.M) out[(int64_t)m * p.ldo] = float_to_bf16_bits(c[m]);
     }
-    *out = float_to_bf16_bits(s);
-    return false;
+    return overflow;
 }
 
 template <int MODE, int NT>
@@ -142,6 +156,7 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
     if (warp == 0) {
         // ---------------- token tiles (TMA); the tokens come from the previous kernel
         if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(&tmB) : "memory");
             pdl_wait();
             int issued = 0;
             for (int j = 0; j < nkb; ++j) {
@@ -317,11 +332,10 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
         if (holder) {
             pdl_wait();  // y / z may still be in use by the previous kernel
             const int nn = tile * TM + 32 * (warp & 3) + lane;
-            if (nn < p.rows) {
+            float c[NT];
 #pragma unroll
-                for (int m = 0; m < NT; ++m)
-                    if (m < p.M) overflow |= put_value<MODE>(p, m, nn, __uint_as_float(acc_row[m]));
-            }
+            for (int m = 0; m < NT; ++m) c[m] = __uint_as_float(acc_row[m]);
+            if (nn < p.rows) overflow = finish_row<MODE, NT>(p, nn, c);
         }
     } else {
         // CTA r finalises rows r * rpr .. of the tile: every CTA sends it its
@@ -331,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
         if (holder) {
             const int rho = 32 * (warp & 3) + lane;
             const int dst = rho / rpr, q = rho - dst * rpr;
-            const uint32_t ra = map_shared_addr(sRed + (uint32_t)((split * rpr + q) * NT) * 4u, (uint32_t)dst);
+            const uint32_t ra = map_shared_addr(sRed + (uint32_t)((split * rpr + q) * S::kRedStride) * 4u, (uint32_t)dst);
 #pragma unroll
             for (int m4 = 0; m4 < NT; m4 += 4)
                 st_shared_cluster_v4(ra + 4u * m4, acc_row[m4], acc_row[m4 + 1], acc_row[m4 + 2], acc_row[m4 + 3]);
@@ -339,12 +353,23 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
         cluster_sync();  // every partial has arrived
         pdl_wait();
         const float *red = reinterpret_cast<const float *>(smem_raw + (sRed - raw));
-        for (int e = tid; e < rpr * p.M; e += kThreads) {
-            const int m = e / rpr, q = e - m * rpr;
-            float s = 0.f;
-            for (int c = 0; c < cs; ++c) s += red[(c * rpr + q) * NT + m];
+        for (int q = tid; q < rpr; q += kThreads) {  // one row per thread, every token
+            float c[NT];
+#pragma unroll
+            for (int m = 0; m < NT; ++m) c[m] = 0.f;
+            for (int r = 0; r < cs; ++r) {
+                const float4 *src = reinterpret_cast<const float4 *>(red + (r * rpr + q) * S::kRedStride);
+#pragma unroll
+                for (int m4 = 0; m4 < NT / 4; ++m4) {
+                    const float4 v = src[m4];
+                    c[4 * m4] += v.x;
+                    c[4 * m4 + 1] += v.y;
+                    c[4 * m4 + 2] += v.z;
+                    c[4 * m4 + 3] += v.w;
+                }
+            }
             const int nn = tile * TM + split * rpr + q;
-            if (nn < p.rows) overflow |= put_value<MODE>(p, m, nn, s);
+            if (nn < p.rows) overflow |= finish_row<MODE, NT>(p, nn, c);
         }
     }
     if (overflow) set_status(p.status, LB_ERR_RANGE);
