@@ -33,23 +33,10 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t 
                  :: "r"(smem_u32(dst)), "l"(src), "r"(src_bytes) : "memory");
 }
 
-__device__ __forceinline__ void cp_async8(void *dst, const void *src, uint32_t src_bytes = 8)
-{
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;\n"
-                 :: "r"(smem_u32(dst)), "l"(src), "r"(src_bytes) : "memory");
-}
 
-__device__ __forceinline__ void cp_async4(void *dst, const void *src, uint32_t src_bytes = 4)
-{
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n"
-                 :: "r"(smem_u32(dst)), "l"(src), "r"(src_bytes) : "memory");
-}
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
-// Wait until at most N of this thread's committed groups are still in flight.
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;\n" :: "n"(N) : "memory"); }
 
 // Loads issued where they stand in the program: weights fetched ahead of use
 // (at kernel entry, or K-blocks ahead) so that their latency overlaps other
@@ -88,19 +75,6 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\
 // Let the next grid on the stream start its prologue early.
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
-// ---------------------------------------------------------------- clusters
-__device__ __forceinline__ uint32_t cluster_ctarank()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ uint32_t cluster_nctarank()
-{
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_nctarank;\n" : "=r"(r));
-    return r;
-}
 // Full cluster barrier with release/acquire semantics for shared::cluster memory.
 __device__ __forceinline__ void cluster_sync()
 {
@@ -138,24 +112,7 @@ __device__ __forceinline__ void st_shared_cluster_v4(uint32_t addr, uint32_t a, 
     asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");
 }
-__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr)
-{
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
 
-// ---------------------------------------------------------------- tensor cores
-// D = A * B + D, m16n8k16, A/B fp16, accumulate fp32 (register operands).
-__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                              uint32_t a3, uint32_t b0, uint32_t b1)
-{
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
 
 // ---------------------------------------------------------------- numerics
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b16) { return __uint_as_float(b16 << 16); }

@@ -45,9 +45,9 @@ struct ForwardArgs {
     size_t workspace_bytes;
 };
 
-// Decode path (1..32 tokens per launch pair; larger batches are sliced).
-// Up to kSmallMaxTokens tokens run on CUDA cores (nibble tables, lb_gemv.cu),
-// more on the register tensor cores (lb_decode.cu).
+// Decode path (1..32 tokens per launch pair; larger batches are sliced,
+// lb_decode.cu).  Up to kSmallMaxTokens tokens run on CUDA cores (nibble
+// tables, lb_gemv.cu) when the shapes fit it, the rest on tcgen05 (lb_mid.cu).
 constexpr int kSmallMaxTokens = 4;
 size_t small_workspace_bytes(int M, const int *ranks, int npaths);
 cudaError_t small_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M);

@@ -163,10 +163,11 @@ LB_API size_t lb_forward_workspace_bytes(int64_t tokens, int64_t n_in, int64_t n
  *   (nothing launched, pointers unchecked).
  * Alignment: x, y, u_bits, vt_bits, h, g, l and workspace 16-byte aligned.
  * Numerics: all sums accumulate in fp32 and y is rounded to bf16 once.
- *   1..4 tokens run on CUDA cores in fp32 throughout.  5..32 tokens feed the
- *   tensor cores fp16 operands: g (.) x and the latent z must stay below
- *   65504 in magnitude (else LB_ERR_RANGE is raised on the device status word
- *   and y is undefined).  Larger batches run the prefill kernels.
+ *   1..4 tokens run on CUDA cores in fp32 throughout.  More tokens run on
+ *   the tensor cores: contraction 1 with bf16 operands (x as given, g
+ *   rounded to bf16), contraction 2 with fp16 operands (the latent z rounded
+ *   to fp16, h exact); z must stay below 65504 in magnitude (else
+ *   LB_ERR_RANGE is raised on the device status word and y is undefined).
  * Errors: LB_ERR_INVALID_ARGUMENT (null pointers, negative sizes),
  *   LB_ERR_UNSUPPORTED_SHAPE, LB_ERR_MISALIGNED, LB_ERR_WORKSPACE_TOO_SMALL,
  *   LB_ERR_NOT_SUPPORTED_DEVICE, LB_ERR_CUDA (launch failure).  Conditions
