@@ -85,6 +85,14 @@ def _load():
             lib.oracle_forward.argtypes = [
                 ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                 ctypes.POINTER(_Path), ctypes.c_int, ctypes.c_void_p]
+            lib.oracle_latent.restype = ctypes.c_int
+            lib.oracle_latent.argtypes = [
+                ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                ctypes.POINTER(_Path), ctypes.c_int, ctypes.c_void_p]
+            lib.oracle_expand.restype = ctypes.c_int
+            lib.oracle_expand.argtypes = [
+                ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                ctypes.POINTER(_Path), ctypes.c_int, ctypes.c_void_p]
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_num_threads.argtypes = []
             _lib = lib
@@ -159,6 +167,50 @@ def forward(x: np.ndarray, paths: list[dict]) -> np.ndarray:
                                 len(P), y.ctypes.data)
     if rc != 0:
         raise RuntimeError(f"oracle_forward failed ({rc})")
+    return y
+
+
+def _c_paths(P):
+    arr = (_Path * len(P))()
+    for j, p in enumerate(P):
+        arr[j] = _Path(p["rank"], p["su"].ctypes.data, p["sv"].ctypes.data,
+                       p["h"].ctypes.data, p["g"].ctypes.data, p["l"].ctypes.data)
+    return arr
+
+
+def latent(x: np.ndarray, paths: list[dict]) -> np.ndarray:
+    """fp64 first half of the forward pass (input scale, contraction 1,
+    latent scale): ``z[m, off_p + k] = l_k sum_i sv[i, k] g_i x[m, i]``, the
+    paths side by side (path 0 first).  Returns float64 ``[tokens, sum r_p]``.
+    Same arguments as :func:`forward`."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    if x.ndim != 2:
+        raise ValueError("x must be [tokens, n_in]")
+    P = [_as_path_arrays(p) for p in paths]
+    for p in P:
+        if p["sv"].shape[0] != x.shape[1]:
+            raise ValueError("V_sign does not match x")
+    z = np.empty((x.shape[0], sum(p["rank"] for p in P)), dtype=np.float64)
+    rc = _load().oracle_latent(x.ctypes.data, x.shape[0], x.shape[1], _c_paths(P), len(P), z.ctypes.data)
+    if rc != 0:
+        raise RuntimeError(f"oracle_latent failed ({rc})")
+    return z
+
+
+def expand(z: np.ndarray, paths: list[dict]) -> np.ndarray:
+    """fp64 second half of the forward pass (contraction 2, row scale, sum of
+    the paths) from a latent laid out as :func:`latent` returns it.
+    ``expand(latent(x, P), P)`` equals ``forward(x, P)`` exactly.  Returns
+    float64 ``[tokens, n_out]``."""
+    z = np.ascontiguousarray(z, dtype=np.float64)
+    P = [_as_path_arrays(p) for p in paths]
+    if z.ndim != 2 or z.shape[1] != sum(p["rank"] for p in P):
+        raise ValueError("z must be [tokens, sum of the ranks]")
+    n_out = P[0]["su"].shape[0]
+    y = np.empty((z.shape[0], n_out), dtype=np.float64)
+    rc = _load().oracle_expand(z.ctypes.data, z.shape[0], n_out, _c_paths(P), len(P), y.ctypes.data)
+    if rc != 0:
+        raise RuntimeError(f"oracle_expand failed ({rc})")
     return y
 
 

@@ -139,3 +139,105 @@ int oracle_forward(const double *x, int64_t tokens, int64_t n_in, int64_t n_out,
     free(t); free(c); free(z);
     return 0;
 }
+
+/* The first half of the forward pass alone (steps 1 to 3): the latent
+ *   z[m][off_p + k] = l_k * sum_i sv[i][k] * g_i * x[m][i]
+ * for every path p, paths side by side (off_p = sum of the ranks before p),
+ * z [tokens x sum_p rank_p].  Same steps and order as oracle_forward.
+ * Returns 0 on success, -1 on a bad argument, -2 when out of memory. */
+int oracle_latent(const double *x, int64_t tokens, int64_t n_in, const oracle_path *paths, int npaths,
+                  double *z)
+{
+    if (tokens < 0 || n_in <= 0 || npaths < 1 || !paths)
+        return -1;
+    if (tokens == 0)
+        return 0;
+    if (!x || !z)
+        return -1;
+    int64_t R = 0;
+    for (int p = 0; p < npaths; ++p) {
+        if (paths[p].rank <= 0 || !paths[p].sv || !paths[p].g || !paths[p].l)
+            return -1;
+        R += paths[p].rank;
+    }
+    double *t = (double *)malloc(sizeof(double) * (size_t)n_in);
+    if (!t)
+        return -2;
+    for (int64_t m = 0; m < tokens; ++m) {
+        const double *xm = x + m * n_in;
+        int64_t off = 0;
+        for (int p = 0; p < npaths; ++p) {
+            const oracle_path *P = &paths[p];
+            const int64_t r = P->rank;
+            double *zm = z + m * R + off;
+            for (int64_t i = 0; i < n_in; ++i)      /* step 1 */
+                t[i] = P->g[i] * xm[i];
+#pragma omp parallel
+            {
+                int nth = 1, tid = 0;
+#ifdef _OPENMP
+                nth = omp_get_num_threads();
+                tid = omp_get_thread_num();
+#endif
+                int64_t k0 = r * tid / nth, k1 = r * (tid + 1) / nth;
+                for (int64_t k = k0; k < k1; ++k)
+                    zm[k] = 0.0;
+                for (int64_t i = 0; i < n_in; ++i) { /* step 2, i ascending */
+                    const int8_t *row = P->sv + i * r;
+                    const double ti = t[i];
+                    for (int64_t k = k0; k < k1; ++k)
+                        zm[k] += (double)row[k] * ti;
+                }
+            }
+            for (int64_t k = 0; k < r; ++k)         /* step 3 */
+                zm[k] = P->l[k] * zm[k];
+            off += r;
+        }
+    }
+    free(t);
+    return 0;
+}
+
+/* The second half alone (steps 4 and 5): from a latent z laid out as
+ * oracle_latent writes it,
+ *   y[m][o] = sum_p h_{p,o} * sum_k su[o][k] * z[m][off_p + k]
+ * (k ascending, paths in order; y [tokens x n_out]).  Same steps and order
+ * as oracle_forward, so oracle_expand(oracle_latent(x)) equals
+ * oracle_forward(x) exactly. */
+int oracle_expand(const double *z, int64_t tokens, int64_t n_out, const oracle_path *paths, int npaths,
+                  double *y)
+{
+    if (tokens < 0 || n_out <= 0 || npaths < 1 || !paths)
+        return -1;
+    if (tokens == 0)
+        return 0;
+    if (!z || !y)
+        return -1;
+    int64_t R = 0;
+    for (int p = 0; p < npaths; ++p) {
+        if (paths[p].rank <= 0 || !paths[p].su || !paths[p].h)
+            return -1;
+        R += paths[p].rank;
+    }
+    for (int64_t m = 0; m < tokens; ++m) {
+        double *ym = y + m * n_out;
+        for (int64_t o = 0; o < n_out; ++o)
+            ym[o] = 0.0;
+        int64_t off = 0;
+        for (int p = 0; p < npaths; ++p) {
+            const oracle_path *P = &paths[p];
+            const int64_t r = P->rank;
+            const double *zm = z + m * R + off;
+#pragma omp parallel for schedule(static)
+            for (int64_t o = 0; o < n_out; ++o) {
+                const int8_t *row = P->su + o * r;
+                double e = 0.0;
+                for (int64_t k = 0; k < r; ++k)
+                    e += (double)row[k] * zm[k];
+                ym[o] += P->h[o] * e;
+            }
+            off += r;
+        }
+    }
+    return 0;
+}

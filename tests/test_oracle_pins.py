@@ -269,3 +269,54 @@ def test_unmutated_oracle_passes_pins():
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_pins_catch_planted_mistakes(name):
     assert not _pins_pass(MUTANTS[name]), f"mutant {name} slipped through the pins"
+
+
+# ---------------------------------------------------------------- the two halves
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_latent_then_expand_is_forward_bitwise(seed):
+    """expand(latent(x)) takes exactly the forward pass's steps in the same
+    order, so it equals forward(x) bit for bit (the forward pass is pinned
+    above)."""
+    x, paths = random_layer(np.random.default_rng(40 + seed), 48, 40, [7, 12], 3)
+    z = oracle.latent(x, paths)
+    assert z.shape == (3, 19)
+    assert np.array_equal(oracle.expand(z, paths), oracle.forward(x, paths))
+
+
+def _exact_scales(rng, n):
+    """Scales whose products are exact in fp64 (small binary fractions)."""
+    return rng.choice([-2.0, -0.75, -0.5, 0.25, 0.5, 1.0, 1.5, 3.0], n)
+
+
+def test_latent_closed_form_on_hadamard_columns():
+    """V_sign = Sylvester H (rows i, columns k) and x = 2.5 e_j: the latent is
+    z_k = l_k g_j 2.5 H[j, k], exactly; the second path (columns of H in
+    reverse order) follows in the same row, after the first path's."""
+    n = 32
+    H = sylvester(n)
+    rng = np.random.default_rng(7)
+    p1 = dict(su=H, sv=H, h=_exact_scales(rng, n), g=_exact_scales(rng, n), l=_exact_scales(rng, n))
+    p2 = dict(su=H[:, ::-1], sv=H[:, ::-1], h=_exact_scales(rng, n), g=_exact_scales(rng, n),
+              l=_exact_scales(rng, n))
+    for j in (0, 5, 31):
+        x = np.zeros((1, n))
+        x[0, j] = 2.5
+        z = oracle.latent(x, [p1, p2])[0]
+        assert np.array_equal(z[:n], p1["l"] * p1["g"][j] * 2.5 * H[j, :])
+        assert np.array_equal(z[n:], p2["l"] * p2["g"][j] * 2.5 * H[j, ::-1])
+
+
+def test_expand_closed_form_on_hadamard_rows():
+    """U_sign = Sylvester H (rows o, columns k) and a latent 1.5 e_k in path 1
+    and -0.5 e_k' in path 2: y_o = 1.5 h1_o H[o, k] - 0.5 h2_o H[o, k'], exactly."""
+    n = 32
+    H = sylvester(n)
+    rng = np.random.default_rng(8)
+    p1 = dict(su=H, sv=H, h=_exact_scales(rng, n), g=_exact_scales(rng, n), l=_exact_scales(rng, n))
+    p2 = dict(su=H[::-1], sv=H, h=_exact_scales(rng, n), g=_exact_scales(rng, n), l=_exact_scales(rng, n))
+    for k, k2 in ((0, 3), (17, 31)):
+        z = np.zeros((1, 2 * n))
+        z[0, k] = 1.5
+        z[0, n + k2] = -0.5
+        y = oracle.expand(z, [p1, p2])[0]
+        assert np.array_equal(y, 1.5 * p1["h"] * H[:, k] + (-0.5) * p2["h"] * H[::-1][:, k2])
