@@ -87,6 +87,12 @@ def lib() -> ctypes.CDLL:
             L.lb_linear_forward.restype = i32
             L.lb_linear_forward.argtypes = [vp, i64, i64, i64, i64, ctypes.POINTER(LbPath),
                                             ctypes.POINTER(LbPath), vp, i64, vp, sz, vp]
+            L.lb_latent_forward.restype = i32
+            L.lb_latent_forward.argtypes = [vp, i64, i64, i64, ctypes.POINTER(LbPath), ctypes.POINTER(LbPath),
+                                            vp, i64, vp]
+            L.lb_expand_forward.restype = i32
+            L.lb_expand_forward.argtypes = [vp, i64, i64, i64, ctypes.POINTER(LbPath), ctypes.POINTER(LbPath),
+                                            vp, i64, vp]
             L.lb_linear_forward_fixed_scratch.restype = i32
             L.lb_linear_forward_fixed_scratch.argtypes = [vp, i64, i64, i64, i64, ctypes.POINTER(LbPath),
                                                           ctypes.POINTER(LbPath), vp, i64, vp]
@@ -214,6 +220,39 @@ def linear_forward(x, main: PackedPath, residual: PackedPath | None = None, y=No
         ctypes.byref(cr) if cr is not None else None, y.data_ptr(), y.stride(0),
         workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream)),
         "lb_linear_forward")
+    return y
+
+
+def latent_forward(x, main: PackedPath, residual: PackedPath | None = None, z=None, stream=None):
+    """``lb_latent_forward``: x bf16 [tokens, n_in] -> z fp16 [tokens, r_main
+    + r_residual] (the latent of both paths, main first).  Allocates z with
+    torch when not given (the C call allocates nothing)."""
+    torch = _torch()
+    tokens, n_in = x.shape
+    R = main.rank + (residual.rank if residual is not None else 0)
+    if z is None:
+        z = torch.empty((tokens, R), dtype=torch.float16, device=x.device)
+    cm = main.as_c()
+    cr = residual.as_c() if residual is not None else None
+    _check(lib().lb_latent_forward(
+        x.data_ptr(), tokens, n_in, x.stride(0), ctypes.byref(cm), ctypes.byref(cr) if cr is not None else None,
+        z.data_ptr(), z.stride(0), _stream_handle(stream)), "lb_latent_forward")
+    return z
+
+
+def expand_forward(z, main: PackedPath, residual: PackedPath | None = None, y=None, stream=None):
+    """``lb_expand_forward``: z fp16 [tokens, r_main + r_residual] -> y bf16
+    [tokens, n_out].  Allocates y with torch when not given."""
+    torch = _torch()
+    tokens = z.shape[0]
+    n_out = main.h.shape[0]
+    if y is None:
+        y = torch.empty((tokens, n_out), dtype=torch.bfloat16, device=z.device)
+    cm = main.as_c()
+    cr = residual.as_c() if residual is not None else None
+    _check(lib().lb_expand_forward(
+        z.data_ptr(), tokens, n_out, z.stride(0), ctypes.byref(cm), ctypes.byref(cr) if cr is not None else None,
+        y.data_ptr(), y.stride(0), _stream_handle(stream)), "lb_expand_forward")
     return y
 
 

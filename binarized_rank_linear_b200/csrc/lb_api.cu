@@ -95,6 +95,37 @@ lb_status check_path(const lb_path *p, int64_t n_in, int64_t n_out, lb::PathDesc
     return LB_OK;
 }
 
+// Checks the half of a path that one contraction alone uses: the V side
+// (vt_bits, g, l against n_in) for the latent, the U side (u_bits, h) for the
+// expansion; the other half is not read and may be null.
+lb_status check_half(const lb_path *p, bool v_side, int64_t n_in, lb::PathDesc *d)
+{
+    if (!p) return LB_ERR_INVALID_ARGUMENT;
+    if (p->rank <= 0 || p->u_ld < 0 || p->vt_ld < 0) return LB_ERR_INVALID_ARGUMENT;
+    if (p->rank % 32 != 0 || p->rank > kMaxRank) return LB_ERR_UNSUPPORTED_SHAPE;
+    *d = lb::PathDesc{};
+    d->rank = (int)p->rank;
+    if (v_side) {
+        if (!p->vt_bits || !p->g || !p->l) return LB_ERR_INVALID_ARGUMENT;
+        const int64_t vt_ld = p->vt_ld ? p->vt_ld : ceil_words(n_in);
+        if (vt_ld < ceil_words(n_in)) return LB_ERR_INVALID_ARGUMENT;
+        if (!aligned16(p->vt_bits) || !aligned16(p->g) || !aligned16(p->l)) return LB_ERR_MISALIGNED;
+        d->vt_bits = p->vt_bits;
+        d->g = p->g;
+        d->l = p->l;
+        d->vt_ld = vt_ld;
+    } else {
+        if (!p->u_bits || !p->h) return LB_ERR_INVALID_ARGUMENT;
+        const int64_t u_ld = p->u_ld ? p->u_ld : ceil_words(p->rank);
+        if (u_ld < ceil_words(p->rank)) return LB_ERR_INVALID_ARGUMENT;
+        if (!aligned16(p->u_bits) || !aligned16(p->h)) return LB_ERR_MISALIGNED;
+        d->u_bits = p->u_bits;
+        d->h = p->h;
+        d->u_ld = u_ld;
+    }
+    return LB_OK;
+}
+
 size_t workspace_for(int64_t tokens, int64_t n_in, int64_t n_out, const int *ranks, int npaths)
 {
     if (tokens > lb::kDecodeMaxTokens) return lb::prefill_workspace_bytes((int)tokens, ranks, npaths);
@@ -233,6 +264,66 @@ lb_status lb_linear_forward(const uint16_t *x, int64_t tokens, int64_t n_in, int
                               ? lb::prefill_forward(a, dev, static_cast<cudaStream_t>(stream))
                               : lb::decode_forward(a, dev, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    return LB_OK;
+}
+
+lb_status lb_latent_forward(const uint16_t *x, int64_t tokens, int64_t n_in, int64_t ldx, const lb_path *main,
+                            const lb_path *residual, uint16_t *z, int64_t ldz, void *stream)
+{
+    if (tokens < 0 || n_in <= 0) return LB_ERR_INVALID_ARGUMENT;
+    if (tokens == 0) return LB_OK;
+    if (!x || !z || !main) return LB_ERR_INVALID_ARGUMENT;
+    if (ldx < n_in) return LB_ERR_INVALID_ARGUMENT;
+    if (n_in % 32 != 0 || n_in > kMaxDim || tokens > kMaxTokens) return LB_ERR_UNSUPPORTED_SHAPE;
+    lb::ForwardArgs a{};
+    a.npaths = residual ? 2 : 1;
+    lb_status st = check_half(main, true, n_in, &a.path[0]);
+    if (st == LB_OK && residual) st = check_half(residual, true, n_in, &a.path[1]);
+    if (st != LB_OK) return st;
+    const int64_t R = a.path[0].rank + (a.npaths > 1 ? a.path[1].rank : 0);
+    if (ldz < R) return LB_ERR_INVALID_ARGUMENT;
+    if (ldx % 8 != 0 || ldz % 8 != 0 || !aligned16(x) || !aligned16(z)) return LB_ERR_MISALIGNED;
+    a.x = x;
+    a.ldx = ldx;
+    a.tokens = (int)tokens;
+    a.n_in = (int)n_in;
+    lb::DeviceInfo dev;
+    st = device_info(&dev);
+    if (st != LB_OK) return st;
+    if (lb::latent_launch(a, dev, static_cast<cudaStream_t>(stream), z, ldz) != cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    return LB_OK;
+}
+
+lb_status lb_expand_forward(const uint16_t *z, int64_t tokens, int64_t n_out, int64_t ldz, const lb_path *main,
+                            const lb_path *residual, uint16_t *y, int64_t ldy, void *stream)
+{
+    if (tokens < 0 || n_out <= 0) return LB_ERR_INVALID_ARGUMENT;
+    if (tokens == 0) return LB_OK;
+    if (!z || !y || !main) return LB_ERR_INVALID_ARGUMENT;
+    if (ldy < n_out) return LB_ERR_INVALID_ARGUMENT;
+    if (n_out % 32 != 0 || n_out > kMaxDim || tokens > kMaxTokens) return LB_ERR_UNSUPPORTED_SHAPE;
+    lb::ForwardArgs a{};
+    a.npaths = residual ? 2 : 1;
+    lb_status st = check_half(main, false, 0, &a.path[0]);
+    if (st == LB_OK && residual) st = check_half(residual, false, 0, &a.path[1]);
+    if (st != LB_OK) return st;
+    const int64_t R = a.path[0].rank + (a.npaths > 1 ? a.path[1].rank : 0);
+    if (ldz < R) return LB_ERR_INVALID_ARGUMENT;
+    if (ldz % 8 != 0 || ldy % 8 != 0 || !aligned16(z) || !aligned16(y)) return LB_ERR_MISALIGNED;
+    a.tokens = (int)tokens;
+    a.n_out = (int)n_out;
+    a.y = y;
+    a.ldy = ldy;
+    lb::DeviceInfo dev;
+    st = device_info(&dev);
+    if (st != LB_OK) return st;
+    if (lb::expand_launch(a, dev, static_cast<cudaStream_t>(stream), z, ldz) != cudaSuccess) {
         cudaGetLastError();
         return LB_ERR_CUDA;
     }

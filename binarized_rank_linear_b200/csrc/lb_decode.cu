@@ -1,7 +1,8 @@
 // lb_decode.cu - the forward pass for 1..32 tokens: dispatch between the
 // CUDA-core path (1..4 tokens, lb_gemv.cu) and the tcgen05 path (5..32
 // tokens, lb_mid.cu).  Larger batches handed to this file are sliced into
-// pieces of at most 32 tokens.
+// pieces of at most 32 tokens.  Also the dispatch of either contraction on
+// its own (the split latent entry points).
 //
 // The layer (sesamedisk.com, "Samsung LittleBit 13B Model", section "What the
 // method actually computes", Proposition 1) is computed by a pair of
@@ -43,6 +44,19 @@ cudaError_t decode_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStre
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
+}
+
+cudaError_t latent_launch(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, uint16_t *z, int64_t ldz)
+{
+    return a.tokens > kDecodeMaxTokens ? prefill_latent(a, dev, stream, z, ldz)
+                                       : mid_latent(a, dev, stream, 0, a.tokens, z, ldz);
+}
+
+cudaError_t expand_launch(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, const uint16_t *z,
+                          int64_t ldz)
+{
+    return a.tokens > kDecodeMaxTokens ? prefill_expand(a, dev, stream, z, ldz)
+                                       : mid_expand(a, dev, stream, 0, a.tokens, z, ldz);
 }
 
 }  // namespace lb

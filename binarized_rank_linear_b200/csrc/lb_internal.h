@@ -66,11 +66,25 @@ constexpr int kMidMaxTokens = 32;
 size_t mid_workspace_bytes(int tokens, const int *ranks, int npaths);
 cudaError_t mid_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M);
 cudaError_t mid_prepare_device(const DeviceInfo &dev);
+cudaError_t mid_latent(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M, uint16_t *z,
+                       int64_t ldz);
+cudaError_t mid_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M,
+                       const uint16_t *z, int64_t ldz);
 
 // Prefill path (more than kDecodeMaxTokens tokens): two tcgen05 GEMMs with the
 // binary operand expanded in shared memory (lb_prefill.cu).
 size_t prefill_workspace_bytes(int tokens, const int *ranks, int npaths);
 cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 cudaError_t prefill_prepare_device(const DeviceInfo &dev);
+cudaError_t prefill_latent(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, uint16_t *z, int64_t ldz);
+cudaError_t prefill_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, const uint16_t *z,
+                           int64_t ldz);
+
+// Either contraction alone, the latent in caller memory: z fp16 [tokens][ldz]
+// (token-major, the paths side by side, path 0 first); any number of tokens
+// (up to 32 on the lb_mid.cu kernels, more on the prefill kernels).
+cudaError_t latent_launch(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, uint16_t *z, int64_t ldz);
+cudaError_t expand_launch(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, const uint16_t *z,
+                          int64_t ldz);
 
 }  // namespace lb

@@ -423,15 +423,15 @@ cudaError_t launch_mid(MidParams p, const void *b, int64_t ldb, const DeviceInfo
     return cudaLaunchKernelEx(&cfg, mid_gemm_kernel<MODE, NT>, tm, p);
 }
 
+// Contraction 1 of tokens m0 .. m0 + M: z = l (.) (W1 x^T), rows = latent
+// indices of both paths, into z fp16 [M][ldz] (token-major).
 template <int NT>
-cudaError_t mid_forward_nt(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M)
+cudaError_t mid_latent_nt(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M, uint16_t *z,
+                          int64_t ldz)
 {
     const int r0 = a.path[0].rank, r1 = a.npaths > 1 ? a.path[1].rank : 0;
     const int R = r0 + r1;
-    uint16_t *z = static_cast<uint16_t *>(a.workspace);  // [M][R] fp16
     const uint16_t *x = a.x + (int64_t)m0 * a.ldx;
-
-    // contraction 1: z = l (.) (W1 x^T), rows = latent indices of both paths
     MidParams p1{};
     p1.M = M;
     p1.rows = R;
@@ -449,12 +449,19 @@ cudaError_t mid_forward_nt(const ForwardArgs &a, const DeviceInfo &dev, cudaStre
         p1.l1 = a.path[1].l;
     }
     p1.out = z;
-    p1.ldo = R;
+    p1.ldo = ldz;
     p1.status = dev.status;
-    cudaError_t e = launch_mid<1, NT>(p1, x, a.ldx, dev, stream);
-    if (e != cudaSuccess) return e;
+    return launch_mid<1, NT>(p1, x, a.ldx, dev, stream);
+}
 
-    // contraction 2: y = W2 z^T, rows = outputs
+// Contraction 2 of tokens m0 .. m0 + M from z fp16 [M][ldz]: y = W2 z^T,
+// rows = outputs.
+template <int NT>
+cudaError_t mid_expand_nt(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M,
+                          const uint16_t *z, int64_t ldz)
+{
+    const int r0 = a.path[0].rank, r1 = a.npaths > 1 ? a.path[1].rank : 0;
+    const int R = r0 + r1;
     MidParams p2{};
     p2.M = M;
     p2.rows = a.n_out;
@@ -472,7 +479,7 @@ cudaError_t mid_forward_nt(const ForwardArgs &a, const DeviceInfo &dev, cudaStre
     p2.out = a.y + (int64_t)m0 * a.ldy;
     p2.ldo = a.ldy;
     p2.status = dev.status;
-    return launch_mid<2, NT>(p2, z, R, dev, stream);
+    return launch_mid<2, NT>(p2, z, ldz, dev, stream);
 }
 
 }  // namespace
@@ -498,10 +505,26 @@ size_t mid_workspace_bytes(int tokens, const int *ranks, int npaths)
     return (size_t)std::min(tokens, kMidMaxTokens) * R * 2;
 }
 
+cudaError_t mid_latent(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M, uint16_t *z,
+                       int64_t ldz)
+{
+    if (M <= 16) return mid_latent_nt<16>(a, dev, stream, m0, M, z, ldz);
+    return mid_latent_nt<32>(a, dev, stream, m0, M, z, ldz);
+}
+
+cudaError_t mid_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M,
+                       const uint16_t *z, int64_t ldz)
+{
+    if (M <= 16) return mid_expand_nt<16>(a, dev, stream, m0, M, z, ldz);
+    return mid_expand_nt<32>(a, dev, stream, m0, M, z, ldz);
+}
+
 cudaError_t mid_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M)
 {
-    if (M <= 16) return mid_forward_nt<16>(a, dev, stream, m0, M);
-    return mid_forward_nt<32>(a, dev, stream, m0, M);
+    const int R = a.path[0].rank + (a.npaths > 1 ? a.path[1].rank : 0);
+    uint16_t *z = static_cast<uint16_t *>(a.workspace);  // [M][R] fp16
+    const cudaError_t e = mid_latent(a, dev, stream, m0, M, z, R);
+    return e != cudaSuccess ? e : mid_expand(a, dev, stream, m0, M, z, R);
 }
 
 }  // namespace lb

@@ -466,12 +466,11 @@ size_t prefill_workspace_bytes(int tokens, const int *ranks, int npaths)
     return (size_t)tokens * R * 2 + 256;
 }
 
-cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream)
+cudaError_t prefill_latent(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, uint16_t *z, int64_t ldz)
 {
     const int M = a.tokens;
     const int r0 = a.path[0].rank, r1 = a.npaths > 1 ? a.path[1].rank : 0;
     const int R = r0 + r1;
-    uint16_t *z = static_cast<uint16_t *>(a.workspace);  // [M x R] fp16
     cudaError_t e = get_encoder();
     if (e != cudaSuccess) return e;
 
@@ -493,9 +492,18 @@ cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStr
         p1.l1 = a.path[1].l;
     }
     p1.out = z;
-    p1.ldo = R;
+    p1.ldo = ldz;
     p1.status = dev.status;
-    e = launch_sign_gemm<1>(p1, a.x, a.ldx, dev, stream);
+    return launch_sign_gemm<1>(p1, a.x, a.ldx, dev, stream);
+}
+
+cudaError_t prefill_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, const uint16_t *z,
+                           int64_t ldz)
+{
+    const int M = a.tokens;
+    const int r0 = a.path[0].rank, r1 = a.npaths > 1 ? a.path[1].rank : 0;
+    const int R = r0 + r1;
+    cudaError_t e = get_encoder();
     if (e != cudaSuccess) return e;
 
     // contraction 2: Y = Z . B2^T
@@ -516,7 +524,15 @@ cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStr
     p2.out = a.y;
     p2.ldo = a.ldy;
     p2.status = dev.status;
-    return launch_sign_gemm<2>(p2, z, R, dev, stream);
+    return launch_sign_gemm<2>(p2, z, ldz, dev, stream);
+}
+
+cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream)
+{
+    const int R = a.path[0].rank + (a.npaths > 1 ? a.path[1].rank : 0);
+    uint16_t *z = static_cast<uint16_t *>(a.workspace);  // [M x R] fp16
+    const cudaError_t e = prefill_latent(a, dev, stream, z, R);
+    return e != cudaSuccess ? e : prefill_expand(a, dev, stream, z, R);
 }
 
 }  // namespace lb

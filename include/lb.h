@@ -177,6 +177,40 @@ LB_API lb_status lb_linear_forward(const uint16_t *x, int64_t tokens, int64_t n_
                             uint16_t *y, int64_t ldy, void *workspace, size_t workspace_bytes,
                             void *stream);
 
+/* ---------------------------------------------------------- split halves
+ * The two halves of lb_linear_forward on their own, with the r-wide latent
+ * in caller memory.  For factorised key and value projections a model can
+ * cache this latent instead of the full-width keys and values (sesamedisk.com,
+ * "Samsung LittleBit 13B Model", section "The real result": the KV cache
+ * shrinks because the smaller latent state is cached).
+ *
+ * Latent layout: z fp16 [tokens x ldz], row-major (token-major), row stride
+ * ldz elements >= r_main + r_residual and a multiple of 8; row m holds the
+ * main path's r_main latents, then the residual path's.  16-byte aligned.
+ *
+ * lb_latent_forward (steps 1-3 of Proposition 1):
+ *     z[m][off_p + k] = l_p[k] * sum_i sign(V_p[i][k]) * g_p[i] * x[m][i]
+ *   Uses vt_bits, vt_ld, g, l and rank of each path (u_bits and h are not
+ *   read and may be NULL).  x as in lb_linear_forward.
+ * lb_expand_forward (steps 4-5):
+ *     y[m][o] = sum_p h_p[o] * sum_k sign(U_p[o][k]) * z[m][off_p + k]
+ *   Uses u_bits, u_ld, h and rank (vt_bits, g and l are not read and may be
+ *   NULL).  y as in lb_linear_forward.
+ * Numerics (any number of tokens, all on the tensor cores): contraction 1 in
+ *   bf16 x bf16 (g rounded to bf16), contraction 2 in fp16 x fp16 (h
+ *   exact), fp32 accumulation; z is rounded to fp16 (nearest even) and must
+ *   stay below 65504 in magnitude (else LB_ERR_RANGE on the device status
+ *   word and z is undefined); y is rounded to bf16 once.
+ * No workspace; nothing is allocated.  Errors as lb_linear_forward; tokens
+ *   == 0 is a no-op.  A z written by lb_latent_forward and read by
+ *   lb_expand_forward on the same stream needs no other synchronisation. */
+LB_API lb_status lb_latent_forward(const uint16_t *x, int64_t tokens, int64_t n_in, int64_t ldx,
+                            const lb_path *main, const lb_path *residual, uint16_t *z, int64_t ldz,
+                            void *stream);
+LB_API lb_status lb_expand_forward(const uint16_t *z, int64_t tokens, int64_t n_out, int64_t ldz,
+                            const lb_path *main, const lb_path *residual, uint16_t *y, int64_t ldy,
+                            void *stream);
+
 /* ---------------------------------------------------------- fixed scratch
  * lb_linear_forward_fixed_scratch: lb_linear_forward for 1..32 tokens with
  * no workspace argument.  The pages have no counterpart; this is a service of

@@ -169,3 +169,32 @@ def test_fixed_scratch_rejects_before_any_cuda_call(L):
     assert L.lb_forward_workspace_bytes(32, 4096, 4096, 32768, 32768) > (1 << 20)
     assert forward_fixed(L, tokens=32, n_in=4096, n_out=4096, ldx=4096, ldy=4096, main=big,
                          residual=big) == lb.LB_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_split_halves_reject_bad_arguments_before_any_cuda_call(L):
+    """lb_latent_forward checks the V half of each path and lb_expand_forward
+    the U half; the other half may be null.  Everything is refused on the
+    host before the device is touched."""
+    lat = lambda **kw: L.lb_latent_forward(
+        kw.get("x", FAKE), kw.get("tokens", 1), kw.get("n_in", 256), kw.get("ldx", 256),
+        ctypes.byref(kw.get("main", fake_path(u_bits=0, h=0))), None, kw.get("z", FAKE), kw.get("ldz", 32), None)
+    exp = lambda **kw: L.lb_expand_forward(
+        kw.get("z", FAKE), kw.get("tokens", 1), kw.get("n_out", 256), kw.get("ldz", 32),
+        ctypes.byref(kw.get("main", fake_path(vt_bits=0, g=0, l=0))), None, kw.get("y", FAKE), kw.get("ldy", 256),
+        None)
+    for f in (lat, exp):
+        assert f(tokens=0) == lb.LB_OK
+        assert f(tokens=-1) == lb.LB_ERR_INVALID_ARGUMENT
+        assert f(z=0) == lb.LB_ERR_INVALID_ARGUMENT
+        assert f(ldz=16) == lb.LB_ERR_INVALID_ARGUMENT          # below the rank
+        assert f(ldz=36) == lb.LB_ERR_MISALIGNED                 # not a multiple of 8
+        assert f(z=FAKE + 2) == lb.LB_ERR_MISALIGNED
+        assert f(main=fake_path(rank=48)) == lb.LB_ERR_UNSUPPORTED_SHAPE
+    assert lat(x=0) == lb.LB_ERR_INVALID_ARGUMENT
+    assert lat(n_in=48, ldx=48) == lb.LB_ERR_UNSUPPORTED_SHAPE
+    assert lat(main=fake_path(g=0)) == lb.LB_ERR_INVALID_ARGUMENT  # the V half is required
+    assert lat(main=fake_path(vt_bits=FAKE + 4)) == lb.LB_ERR_MISALIGNED
+    assert exp(y=0) == lb.LB_ERR_INVALID_ARGUMENT
+    assert exp(n_out=48, ldy=48) == lb.LB_ERR_UNSUPPORTED_SHAPE
+    assert exp(main=fake_path(h=0)) == lb.LB_ERR_INVALID_ARGUMENT  # the U half is required
+    assert exp(main=fake_path(u_bits=FAKE + 4)) == lb.LB_ERR_MISALIGNED
