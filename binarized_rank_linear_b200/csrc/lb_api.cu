@@ -128,7 +128,7 @@ lb_status check_half(const lb_path *p, bool v_side, int64_t n_in, lb::PathDesc *
 
 size_t workspace_for(int64_t tokens, int64_t n_in, int64_t n_out, const int *ranks, int npaths)
 {
-    if (tokens > lb::kDecodeMaxTokens) return lb::prefill_workspace_bytes((int)tokens, ranks, npaths);
+    if (tokens > lb::kMidMaxTokens) return lb::prefill_workspace_bytes((int)tokens, ranks, npaths);
     return lb::decode_workspace_bytes((int)tokens, (int)n_in, (int)n_out, ranks, npaths);
 }
 
@@ -260,7 +260,7 @@ lb_status lb_linear_forward(const uint16_t *x, int64_t tokens, int64_t n_in, int
     lb::DeviceInfo dev;
     st = device_info(&dev);
     if (st != LB_OK) return st;
-    const cudaError_t e = a.tokens > lb::kDecodeMaxTokens
+    const cudaError_t e = a.tokens > lb::kMidMaxTokens
                               ? lb::prefill_forward(a, dev, static_cast<cudaStream_t>(stream))
                               : lb::decode_forward(a, dev, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {

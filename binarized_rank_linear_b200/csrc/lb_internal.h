@@ -45,9 +45,10 @@ struct ForwardArgs {
     size_t workspace_bytes;
 };
 
-// Decode path (1..32 tokens per launch pair; larger batches are sliced,
-// lb_decode.cu).  Up to kSmallMaxTokens tokens run on CUDA cores (nibble
-// tables, lb_gemv.cu) when the shapes fit it, the rest on tcgen05 (lb_mid.cu).
+// Decode path (up to kMidMaxTokens tokens per launch pair; lb_decode.cu).
+// Up to kSmallMaxTokens tokens run on CUDA cores (nibble tables, lb_gemv.cu)
+// when the shapes fit it, the rest on tcgen05 (lb_mid.cu).  kDecodeMaxTokens
+// bounds the fixed-scratch entry point.
 constexpr int kSmallMaxTokens = 4;
 size_t small_workspace_bytes(int M, const int *ranks, int npaths);
 cudaError_t small_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M);
@@ -60,9 +61,9 @@ size_t decode_workspace_bytes(int tokens, int n_in, int n_out, const int *ranks,
 cudaError_t decode_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 cudaError_t decode_prepare_device(const DeviceInfo &dev);
 
-// 5..32 tokens per launch pair on tcgen05 with the sign matrix as the
-// 128-row MMA operand (lb_mid.cu); x is sliced in batches of at most 32.
-constexpr int kMidMaxTokens = 32;
+// Up to kMidMaxTokens tokens per launch pair on tcgen05 with the sign matrix
+// as the 128-row MMA operand and the tokens as N (lb_mid.cu).
+constexpr int kMidMaxTokens = 128;
 size_t mid_workspace_bytes(int tokens, const int *ranks, int npaths);
 cudaError_t mid_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M);
 cudaError_t mid_prepare_device(const DeviceInfo &dev);
@@ -71,7 +72,7 @@ cudaError_t mid_latent(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t
 cudaError_t mid_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M,
                        const uint16_t *z, int64_t ldz);
 
-// Prefill path (more than kDecodeMaxTokens tokens): two tcgen05 GEMMs with the
+// Prefill path (more than kMidMaxTokens tokens): two tcgen05 GEMMs with the
 // binary operand expanded in shared memory (lb_prefill.cu).
 size_t prefill_workspace_bytes(int tokens, const int *ranks, int npaths);
 cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream);

@@ -1,9 +1,9 @@
-// lb_mid.cu - the forward pass for 5..32 tokens, on tcgen05 tensor cores.
+// lb_mid.cu - the forward pass for 5..128 tokens, on tcgen05 tensor cores.
 //
 // The layer (sesamedisk.com, "Samsung LittleBit 13B Model", section "What the
 // method actually computes", Proposition 1) as two skinny products in which
-// the sign matrix is the 128-row MMA operand and the few tokens are the N
-// dimension (16 or 32):
+// the sign matrix is the 128-row MMA operand and the tokens are the N
+// dimension (16, 32, 64 or 128):
 //
 //   contraction 1:  C1[k, m] = sum_i W1[k, i] x[m, i],  W1[k, i] = sign(V_p[i, k]) g_p[i]   (bf16)
 //                   z[m, k]  = l_k C1[k, m], rounded to fp16 (the operand of contraction 2)
@@ -21,7 +21,7 @@
 // cluster-rank order, so results do not depend on timing.
 //   warp 0      allocates tensor memory, waits for the previous kernel, then
 //               streams the token tiles (x or z) with TMA (no multicast)
-//   warp 1      one thread issues tcgen05.mma (M = 128, N = 16 or 32, K = 16)
+//   warp 1      one thread issues tcgen05.mma (M = 128, N = 16 .. 128, K = 16)
 //   warps 2..9  two groups of 4 taking alternate K-blocks, one W row per
 //               thread: expand the row's packed signs into +-scale values in
 //               128-byte-swizzled shared memory; warps 2..5 then read the
@@ -48,10 +48,13 @@ constexpr int kThreads = 32 * (2 + kProducerWarps);
 constexpr int kMaxCluster = 8;
 constexpr uint32_t A_BYTES = TM * BK * 2;  // expanded W tile, 16 KB
 constexpr uint32_t G_BYTES = 2 * BK * 2;   // a K-block of g for both paths
-constexpr uint32_t TMEM_COLS = 32;
 
+// NT = token columns of the MMA (16, 32, 64 or 128); the accumulator is read
+// out in chunks of CH columns.
 template <int NT>
 struct MidShape {
+    static constexpr int CH = NT < 32 ? NT : 32;
+    static constexpr uint32_t kTmemCols = NT < 32 ? 32 : NT;
     static constexpr uint32_t kBBytes = (uint32_t)NT * BK * 2;  // token tile
     // partials received, [cs][128 / cs][kRedStride] fp32: rows padded by 4
     // floats so that 16-byte accesses of consecutive rows cover every bank
@@ -59,6 +62,7 @@ struct MidShape {
     static constexpr uint32_t kRedBytes = (uint32_t)TM * kRedStride * 4;
     static constexpr size_t kSmem =
         1024 + (size_t)STAGES * (A_BYTES + kBBytes) + kRedBytes + (size_t)kProducerWarps * 2 * G_BYTES + 256;
+    static constexpr int kCtasPerSm = 2 * kSmem <= 227 * 1024 ? 2 : 1;
 };
 
 struct MidParams {
@@ -78,31 +82,48 @@ struct MidParams {
     int *status;
 };
 
-// One finished row nn of the tile for every token: mode 1 z[m][nn] =
-// l_nn c[m] (fp16; returns true if a value does not fit), mode 2 y[m][nn]
-// (bf16).  A warp's lanes take consecutive rows, so each token's stores are
-// contiguous.
-template <int MODE, int NT>
-__device__ __forceinline__ bool finish_row(const MidParams &p, int nn, const float (&c)[NT])
+// Finished values of row nn of the tile for the tokens c0 .. c0 + CH - 1:
+// mode 1 z[m][nn] = l_nn c (fp16; returns true if a value does not fit),
+// mode 2 y[m][nn] (bf16).  A warp's lanes take consecutive rows, so each
+// token's stores are contiguous.
+template <int MODE, int CH>
+__device__ __forceinline__ bool finish_chunk(const MidParams &p, int nn, int c0, const float (&c)[CH])
 {
     uint16_t *out = static_cast<uint16_t *>(p.out) + nn;
     bool overflow = false;
     if (MODE == 1) {
         const float lv = f16_bits_to_float(nn < p.r0 ? p.l0[nn] : p.l1[nn - p.r0]);
 #pragma unroll
-        for (int m = 0; m < NT; ++m) {
-            if (m < p.M) {
-                const float z = c[m] * lv;
-                out[(int64_t)m * p.ldo] = (uint16_t)(pack_half2(z, 0.f) & 0xffffu);
+        for (int j = 0; j < CH; ++j) {
+            if (c0 + j < p.M) {
+                const float z = c[j] * lv;
+                out[(int64_t)(c0 + j) * p.ldo] = (uint16_t)(pack_half2(z, 0.f) & 0xffffu);
                 overflow |= beyond_f16(z);
             }
         }
     } else {
 #pragma unroll
-        for (int m = 0; m < NT; ++m)
-            if (m < p.M) out[(int64_t)m * p.ldo] = float_to_bf16_bits(c[m]);
+        for (int j = 0; j < CH; ++j)
+            if (c0 + j < p.M) out[(int64_t)(c0 + j) * p.ldo] = float_to_bf16_bits(c[j]);
     }
     return overflow;
+}
+
+// CH accumulator columns c0 .. of this warp's 32 lanes (zero when the
+// accumulator was never written); warp-collective.
+template <int CH>
+__device__ __forceinline__ void acc_chunk(uint32_t taddr, bool valid, float (&c)[CH])
+{
+    if (valid) {
+        uint32_t v[CH];
+        if constexpr (CH == 16) tmem_ld16(taddr, v);
+        else tmem_ld32(taddr, v);
+#pragma unroll
+        for (int j = 0; j < CH; ++j) c[j] = __uint_as_float(v[j]);
+    } else {
+#pragma unroll
+        for (int j = 0; j < CH; ++j) c[j] = 0.f;
+    }
 }
 
 template <int MODE, int NT>
@@ -142,16 +163,14 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         }
         __syncwarp();
-        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+        tmem_alloc(smem_u32(tmem_slot), S::kTmemCols);
         tc_fence_before();
     }
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    uint32_t acc_row[NT];  // warps 2..5: this thread's row of the accumulator
-#pragma unroll
-    for (int m = 0; m < NT; ++m) acc_row[m] = 0u;
+    bool acc_ok = false;  // warps 2..5: the accumulator is complete and holds this CTA's K-blocks
 
     if (warp == 0) {
         // ---------------- token tiles (TMA); the tokens come from the previous kernel
@@ -306,36 +325,26 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
             ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
             if (!ok) abort_flag = 1;
             tc_fence_after();
-            if (ok && nkb > 0) {
-                const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-                if (NT == 16) {
-                    uint32_t v[16];
-                    tmem_ld16(ta, v);
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) acc_row[m] = v[m];
-                } else {
-                    uint32_t v[32];
-                    tmem_ld32(ta, v);
-#pragma unroll
-                    for (int m = 0; m < NT; ++m) acc_row[m] = v[m & 31];
-                }
-            }
+            acc_ok = ok && nkb > 0;
         }
     }
 
     // ---------------- finish: every partial of the tile added in rank order
     pdl_launch_dependents();
     __syncwarp();
-    const bool holder = warp >= 2 && warp < 6;  // these threads hold an accumulator row
+    constexpr int CH = S::CH;
+    const bool holder = warp >= 2 && warp < 6;  // these warps read accumulator rows 32 (warp % 4) ..
+    const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     bool overflow = false;
     if (cs == 1) {
         if (holder) {
             pdl_wait();  // y / z may still be in use by the previous kernel
             const int nn = tile * TM + 32 * (warp & 3) + lane;
-            float c[NT];
-#pragma unroll
-            for (int m = 0; m < NT; ++m) c[m] = __uint_as_float(acc_row[m]);
-            if (nn < p.rows) overflow = finish_row<MODE, NT>(p, nn, c);
+            for (int c0 = 0; c0 < NT; c0 += CH) {
+                float c[CH];
+                acc_chunk<CH>(ta + (uint32_t)c0, acc_ok, c);
+                if (nn < p.rows) overflow |= finish_chunk<MODE, CH>(p, nn, c0, c);
+            }
         }
     } else {
         // CTA r finalises rows r * rpr .. of the tile: every CTA sends it its
@@ -346,30 +355,37 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
             const int rho = 32 * (warp & 3) + lane;
             const int dst = rho / rpr, q = rho - dst * rpr;
             const uint32_t ra = map_shared_addr(sRed + (uint32_t)((split * rpr + q) * S::kRedStride) * 4u, (uint32_t)dst);
+            for (int c0 = 0; c0 < NT; c0 += CH) {
+                float c[CH];
+                acc_chunk<CH>(ta + (uint32_t)c0, acc_ok, c);
 #pragma unroll
-            for (int m4 = 0; m4 < NT; m4 += 4)
-                st_shared_cluster_v4(ra + 4u * m4, acc_row[m4], acc_row[m4 + 1], acc_row[m4 + 2], acc_row[m4 + 3]);
+                for (int j = 0; j < CH; j += 4)
+                    st_shared_cluster_v4(ra + 4u * (c0 + j), __float_as_uint(c[j]), __float_as_uint(c[j + 1]),
+                                         __float_as_uint(c[j + 2]), __float_as_uint(c[j + 3]));
+            }
         }
         cluster_sync();  // every partial has arrived
         pdl_wait();
         const float *red = reinterpret_cast<const float *>(smem_raw + (sRed - raw));
         for (int q = tid; q < rpr; q += kThreads) {  // one row per thread, every token
-            float c[NT];
-#pragma unroll
-            for (int m = 0; m < NT; ++m) c[m] = 0.f;
-            for (int r = 0; r < cs; ++r) {
-                const float4 *src = reinterpret_cast<const float4 *>(red + (r * rpr + q) * S::kRedStride);
-#pragma unroll
-                for (int m4 = 0; m4 < NT / 4; ++m4) {
-                    const float4 v = src[m4];
-                    c[4 * m4] += v.x;
-                    c[4 * m4 + 1] += v.y;
-                    c[4 * m4 + 2] += v.z;
-                    c[4 * m4 + 3] += v.w;
-                }
-            }
             const int nn = tile * TM + split * rpr + q;
-            if (nn < p.rows) overflow |= finish_row<MODE, NT>(p, nn, c);
+            for (int c0 = 0; c0 < NT; c0 += CH) {
+                float c[CH];
+#pragma unroll
+                for (int j = 0; j < CH; ++j) c[j] = 0.f;
+                for (int r = 0; r < cs; ++r) {
+                    const float4 *src = reinterpret_cast<const float4 *>(red + (r * rpr + q) * S::kRedStride + c0);
+#pragma unroll
+                    for (int j4 = 0; j4 < CH / 4; ++j4) {
+                        const float4 v = src[j4];
+                        c[4 * j4] += v.x;
+                        c[4 * j4 + 1] += v.y;
+                        c[4 * j4 + 2] += v.z;
+                        c[4 * j4 + 3] += v.w;
+                    }
+                }
+                if (nn < p.rows) overflow |= finish_chunk<MODE, CH>(p, nn, c0, c);
+            }
         }
     }
     if (overflow) set_status(p.status, LB_ERR_RANGE);
@@ -380,17 +396,17 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
     if (warp == 0) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        tmem_dealloc(tmem, S::kTmemCols);
     }
 }
 
 // ---------------------------------------------------------------- host side
 // CTAs per tile: a power of two (each finalises 128 / cs rows of the tile),
-// at most a portable cluster, enough to give about two CTAs per SM (each uses
-// about 100 KB of shared memory), and never a CTA without a K-block.
-int pick_split(int tiles, int nk, int sm_count)
+// at most a portable cluster, enough to fill the CTA slots (one or two per
+// SM, as shared memory allows), and never a CTA without a K-block.
+int pick_split(int tiles, int nk, int slots)
 {
-    const int want = std::max(1, std::min(kMaxCluster, (2 * sm_count) / std::max(1, tiles)));
+    const int want = std::max(1, std::min(kMaxCluster, slots / std::max(1, tiles)));
     int cs = 1;
     while (2 * cs <= want && 2 * cs <= nk) cs *= 2;
     while (cs > 1 && (cs - 1) * ((nk + cs - 1) / cs) >= nk) cs /= 2;
@@ -401,7 +417,7 @@ template <int MODE, int NT>
 cudaError_t launch_mid(MidParams p, const void *b, int64_t ldb, const DeviceInfo &dev, cudaStream_t stream)
 {
     const int tiles = (p.rows + TM - 1) / TM, nk = (p.K + BK - 1) / BK;
-    p.cs = pick_split(tiles, nk, dev.sm_count);
+    p.cs = pick_split(tiles, nk, MidShape<NT>::kCtasPerSm * dev.sm_count);
     p.kpc = (nk + p.cs - 1) / p.cs;
     CUtensorMap tm;
     cudaError_t e = encode_2d(&tm, b, p.M, p.K, ldb, MODE == 1, NT);
@@ -482,21 +498,27 @@ cudaError_t mid_expand_nt(const ForwardArgs &a, const DeviceInfo &dev, cudaStrea
     return launch_mid<2, NT>(p2, z, ldz, dev, stream);
 }
 
+
+template <int NT>
+cudaError_t prepare_nt(cudaError_t e)
+{
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(mid_gemm_kernel<1, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MidShape<NT>::kSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(mid_gemm_kernel<2, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MidShape<NT>::kSmem);
+    return e;
+}
+
 }  // namespace
 
 cudaError_t mid_prepare_device(const DeviceInfo &dev)
 {
     (void)dev;
     cudaError_t e = get_encoder();
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(mid_gemm_kernel<1, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MidShape<16>::kSmem);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(mid_gemm_kernel<2, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MidShape<16>::kSmem);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(mid_gemm_kernel<1, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MidShape<32>::kSmem);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(mid_gemm_kernel<2, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MidShape<32>::kSmem);
-    return e;
+    e = prepare_nt<16>(e);
+    e = prepare_nt<32>(e);
+    e = prepare_nt<64>(e);
+    return prepare_nt<128>(e);
 }
 
 size_t mid_workspace_bytes(int tokens, const int *ranks, int npaths)
@@ -509,14 +531,18 @@ cudaError_t mid_latent(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t
                        int64_t ldz)
 {
     if (M <= 16) return mid_latent_nt<16>(a, dev, stream, m0, M, z, ldz);
-    return mid_latent_nt<32>(a, dev, stream, m0, M, z, ldz);
+    if (M <= 32) return mid_latent_nt<32>(a, dev, stream, m0, M, z, ldz);
+    if (M <= 64) return mid_latent_nt<64>(a, dev, stream, m0, M, z, ldz);
+    return mid_latent_nt<128>(a, dev, stream, m0, M, z, ldz);
 }
 
 cudaError_t mid_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M,
                        const uint16_t *z, int64_t ldz)
 {
     if (M <= 16) return mid_expand_nt<16>(a, dev, stream, m0, M, z, ldz);
-    return mid_expand_nt<32>(a, dev, stream, m0, M, z, ldz);
+    if (M <= 32) return mid_expand_nt<32>(a, dev, stream, m0, M, z, ldz);
+    if (M <= 64) return mid_expand_nt<64>(a, dev, stream, m0, M, z, ldz);
+    return mid_expand_nt<128>(a, dev, stream, m0, M, z, ldz);
 }
 
 cudaError_t mid_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M)
