@@ -132,6 +132,14 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
     return r;
 }
 
+// Two floats -> packed bf16x2 (round to nearest even); lo in bits 0..15.
+__device__ __forceinline__ uint32_t pack_bf162(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 // float -> bf16 bits, round to nearest even.
 __device__ __forceinline__ uint16_t float_to_bf16_bits(float v)
 {

@@ -1,4 +1,4 @@
-// lb_prefill.cu - the forward pass for more than 32 tokens, on tcgen05 tensor cores.
+// lb_prefill.cu - the forward pass for more than 128 tokens, on tcgen05 tensor cores.
 //
 // The layer (sesamedisk.com, "Samsung LittleBit 13B Model", section "What the
 // method actually computes", Proposition 1) is two dense contractions once
@@ -14,14 +14,15 @@
 // to bf16); contraction 2 runs fp16 x fp16 (z rounded to fp16; h exact).
 // Accumulation is fp32 in tensor memory.
 //
-// A persistent grid (one CTA per SM) walks the 128 x 256 tiles of C = A . B^T.
+// A persistent grid (one CTA per SM) walks the 128 x bn tiles of C = A . B^T,
+// bn a multiple of 32 up to 256 chosen per call (see launch_sign_gemm).
 // In each CTA:
 //   warp 0       allocates tensor memory (two 256-column accumulators) and
 //                streams A tiles with TMA (128-byte swizzle, no multicast)
-//   warp 1       one thread issues tcgen05.mma (M = 128, N = 256, K = 16)
+//   warp 1       one thread issues tcgen05.mma (M = 128, N = bn, K = 16)
 //   warps 2..17  two groups of 8 taking alternate K-blocks, one B row per
-//                thread: expand the row's packed sign bits into +-scale
-//                values in the same swizzled layout
+//                thread (rows past bn idle): expand the row's packed sign
+//                bits into +-scale values in the same swizzled layout
 //   warps 18..21 read a finished accumulator out of tensor memory and store
 //                the tile, while the MMA fills the other accumulator
 // Stages are handed over with mbarriers (4-deep ring).  Every wait is bounded
@@ -41,11 +42,12 @@ namespace {
 
 using namespace tc;
 
-constexpr int BM = 128, BN = 256, BK = 64;  // one MMA: M = 128, N = 256; K-blocks of 64
+constexpr int BM = 128, BN = 256, BK = 64;  // one MMA: M = 128, N = bn <= 256; K-blocks of 64
 constexpr int kGroupWarps = 8;                // producer warps per K-block: one B row per thread
 constexpr uint32_t B_BYTES = BN * BK * 2;     // 32 KB
 constexpr uint32_t TMEM_COLS = 2 * BN;        // two 256-column accumulators
 constexpr uint32_t G_BYTES = 2 * BK * 2;      // a K-block of g for both paths
+constexpr uint32_t OUT_BYTES = 32 * 64;       // an output box: 32 rows x 32 two-byte columns
 
 // Two tile shapes.  H = 1: a CTA tile is 128 x 256; the two accumulators
 // double-buffer consecutive tiles, and two producer groups take alternate
@@ -62,9 +64,13 @@ struct Shape {
     static constexpr int kThreads = 32 * (2 + kProducerWarps + kEpiWarps);
     static constexpr int kTileM = BM * H;
     static constexpr uint32_t kABytes = (uint32_t)kTileM * BK * 2;  // 16 or 32 KB
-    // per stage: A tile, B tile; per producer warp: two slots of g rounded to bf16
-    static constexpr size_t kSmem =
-        1024 + (size_t)kStages * (kABytes + B_BYTES) + (size_t)kProducerWarps * 2 * G_BYTES + 256;
+    static constexpr int kOutBufs = H == 1 ? 2 : 1;  // output boxes per epilogue warp
+    // per stage: A tile, B tile; per epilogue warp: its output boxes and the
+    // tile's latent scale in fp32 (mode 1); per producer warp: two slots of g
+    // rounded to bf16
+    static constexpr size_t kSmem = 1024 + (size_t)kStages * (kABytes + B_BYTES) +
+                                    (size_t)kEpiWarps * (kOutBufs * OUT_BYTES + BN * 4) +
+                                    (size_t)kProducerWarps * 2 * G_BYTES + 256;
 };
 // Tiles are K-major with 128-byte swizzle: row `row` holds 64 two-byte
 // elements in 128 bytes, and its 16-byte chunk j (elements 8j .. 8j + 7) is
@@ -73,6 +79,7 @@ struct Shape {
 // ---------------------------------------------------------------- kernel
 struct SignGemmParams {
     int M, N, K;
+    int bn;  // tile width along N: a multiple of 32, at most BN
     int r0;  // mode 1: B rows [0, r0) are path 0; mode 2: K columns [0, r0) are path 0
     int bits8;  // every K-block's two words of a row can be fetched as one aligned 8-byte copy
     const uint32_t *bits0, *bits1;
@@ -84,15 +91,16 @@ struct SignGemmParams {
     int *status;
 };
 
-// Persistent: CTA c computes the 128 x 256 tiles t = c, c + gridDim.x, ...
-// (tile t is rows (t % tiles_m) * 128 and columns (t / tiles_m) * 256, so the
+// Persistent: CTA c computes the tiles t = c, c + gridDim.x, ...
+// (tile t is rows (t % tiles_m) * 128 H and columns (t / tiles_m) * bn, so the
 // CTAs running at once share the same few columns of B).  Its K-blocks form
 // one sequence over all its tiles, so stages, phases and the producer groups'
 // alternation run on across tile boundaries.  Two accumulators in tensor
 // memory let the epilogue warps drain tile i while the MMA runs tile i + 1.
 template <int MODE, int H>
 __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
-    sign_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const SignGemmParams p)
+    sign_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmOut,
+                     const SignGemmParams p)
 {
     using S = Shape<H>;
     constexpr int STAGES = S::kStages;
@@ -103,8 +111,10 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;  // SW128 tiles need 1024-byte alignment
     const uint32_t sA = base, sB = base + STAGES * A_BYTES;
-    const uint32_t sGbf = sB + STAGES * B_BYTES;  // mode 1, per producer warp: g in bf16, [warp][2][path][64]
-    const uint32_t bars = sGbf + kProducerWarps * 2 * G_BYTES;
+    const uint32_t sOut = sB + STAGES * B_BYTES;  // per epilogue warp: kOutBufs output boxes
+    const uint32_t sGbf = sOut + S::kEpiWarps * S::kOutBufs * OUT_BYTES;  // mode 1, per producer warp: g in bf16, [warp][2][path][64]
+    const uint32_t sLf = sGbf + kProducerWarps * 2 * G_BYTES;  // mode 1, per epilogue warp: l of the tile in fp32
+    const uint32_t bars = sLf + S::kEpiWarps * BN * 4;
     // full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain, then the tmem address
     const uint32_t full0 = bars, empty0 = bars + 8 * STAGES, accf0 = bars + 16 * STAGES;
     const uint32_t acce0 = accf0 + 16, drain = acce0 + 16;
@@ -113,7 +123,8 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
     volatile int &abort_flag = abort_shared;  // set by whichever role gives up; read by all
 
     const int tiles_m = (p.M + S::kTileM - 1) / S::kTileM;
-    const int ntiles = tiles_m * ((p.N + BN - 1) / BN);
+    const int ntiles = tiles_m * ((p.N + p.bn - 1) / p.bn);
+    const int busy_warps = (p.bn + 31) >> 5;  // producer warps per group with rows in the tile
     const int G = gridDim.x, c = blockIdx.x;
     const int my_tiles = c < ntiles ? (ntiles - c + G - 1) / G : 0;
     const int nk = (p.K + BK - 1) / BK;
@@ -122,7 +133,7 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             for (int s = 0; s < STAGES; ++s) {
-                mbar_init(full0 + 8 * s, 1 + kGroupWarps);  // TMA arrive.expect_tx + one group's warps
+                mbar_init(full0 + 8 * s, 1 + busy_warps);  // TMA arrive.expect_tx + one group's busy warps
                 mbar_init(empty0 + 8 * s, 1);               // one tcgen05.commit
             }
             for (int b = 0; b < 2; ++b) {
@@ -168,7 +179,7 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
         // ---------------- MMA issuer.  H = 1: tile i accumulates in columns
         // 256 (i % 2) ..; H = 2: half h of every tile accumulates in columns 256 h ..
         if (lane == 0) {
-            const uint32_t idesc = instr_desc(MODE == 1 ? 1u : 0u, BM, BN);
+            const uint32_t idesc = instr_desc(MODE == 1 ? 1u : 0u, BM, p.bn);
             int gb = 0;
             for (int i = 0; i < my_tiles && !abort_flag; ++i) {
                 const int b = H == 1 ? (i & 1) : 0;  // hand-over barriers of the accumulator(s)
@@ -223,6 +234,9 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
         const uint32_t x7 = (uint32_t)(row & 7);  // the row's 128-byte swizzle: logical chunk j sits at chunk j ^ x7
         const int kwords = p.K >> 5, r0w = p.r0 >> 5;
         const uint32_t gbfw = sGbf + (uint32_t)wl * 2 * G_BYTES;  // this warp's two bf16 g slots
+        // a warp whose rows all lie past bn takes no part (the stage barriers
+        // count only the busy warps)
+        const int my_blocks = (wl & (kGroupWarps - 1)) < busy_warps ? nblocks : 0;
         struct Pref {
             uint2 bits;      // the row's two sign words of the block (zero outside the matrix)
             uint4 g;         // mode 1, lanes 0..15: g of path lane / 8, columns 8 (lane % 8) .. (fp16)
@@ -238,7 +252,7 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
             u.gb = gb;
             u.i = gb / nk;
             u.kb = gb - u.i * nk;
-            u.nn = ((c + u.i * G) / tiles_m) * BN + row;
+            u.nn = ((c + u.i * G) / tiles_m) * p.bn + row;
             return u;
         };
         auto advance = [&](Cursor &u) {
@@ -249,7 +263,7 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
                     u.kb -= nk;
                     ++u.i;
                 }
-                u.nn = ((c + u.i * G) / tiles_m) * BN + row;
+                u.nn = ((c + u.i * G) / tiles_m) * p.bn + row;
             }
         };
         auto fetch = [&](const Cursor &u) {
@@ -257,9 +271,9 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
             f.bits = make_uint2(0u, 0u);
             f.g = make_uint4(0u, 0u, 0u, 0u);
             f.h0 = f.h1 = 0u;
-            if (u.gb >= nblocks) return f;
+            if (u.gb >= my_blocks) return f;
             const int kb = u.kb, nn = u.nn;
-            const bool row_in = nn < p.N;
+            const bool row_in = row < p.bn && nn < p.N;
             const int wd = 2 * kb;  // first word of the block in the (concatenated) row
             if (row_in && wd < kwords) {
                 const uint32_t *rb0, *rb1 = nullptr;
@@ -291,7 +305,7 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
         };
         Cursor u = cursor_at(grp), ua = cursor_at(grp + 2 * NG);  // this block, and the group's block two ahead
         Pref f0 = fetch(u), f1 = fetch(cursor_at(grp + NG));
-        for (int j = 0; u.gb < nblocks; ++j, advance(u), advance(ua)) {
+        for (int j = 0; u.gb < my_blocks; ++j, advance(u), advance(ua)) {
             const Pref cur = f0;
             f0 = f1;
             f1 = fetch(ua);
@@ -338,10 +352,12 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
             // 1024-byte aligned, so the XOR acts on address bits 4..6 alone);
             // the 8 rows of a store phase then cover all 32 banks
             const uint32_t rowx = (sB + s * B_BYTES + row * 128) | (x7 << 4);
+            if (row < p.bn) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                store_sign_chunk(rowx ^ (16u * q), __byte_perm(q < 4 ? cur.bits.x : cur.bits.y, 0u, 0x4440u | (uint32_t)(q & 3)),
-                                 sc[q]);
+                for (int q = 0; q < 8; ++q) {
+                    store_sign_chunk(rowx ^ (16u * q),
+                                     __byte_perm(q < 4 ? cur.bits.x : cur.bits.y, 0u, 0x4440u | (uint32_t)(q & 3)), sc[q]);
+                }
             }
             fence_async_shared();
             __syncwarp();
@@ -350,16 +366,36 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
     } else {
         // ---------------- epilogue: warp w drains tensor-memory lanes 32 (w % 4)
         // .. of a finished accumulator (H = 2: warps 4 e .. 4 e + 3 of the
-        // epilogue drain half e), then hands the accumulator back
+        // epilogue drain half e), then hands the accumulator back.  Each
+        // 32-column chunk of the warp's 32 rows goes out as one bulk tensor
+        // store: the lanes (one row each) write the converted chunk into a
+        // swizzled box in shared memory, and lane 0 issues the store.  Rows or
+        // columns past the matrix are clipped by the store itself.
         const int quad = warp & 3;
-        const int eh = H == 1 ? 0 : (warp - 2 - kProducerWarps) >> 2;
+        const int ew = warp - 2 - kProducerWarps;  // epilogue warp 0 .. kEpiWarps - 1
+        const int eh = H == 1 ? 0 : ew >> 2;
+        const uint32_t obox = sOut + (uint32_t)ew * S::kOutBufs * OUT_BYTES;  // the warp's boxes
+        const uint32_t lsm = sLf + (uint32_t)ew * BN * 4;                        // the warp's fp32 l
+        const uint32_t rsw = (uint32_t)((lane >> 1) & 3);  // the row's 64-byte swizzle
+        int nst = 0;  // boxes this warp has stored
         bool overflow = false;
         for (int i = 0; i < my_tiles; ++i) {
             const int b = H == 1 ? (i & 1) : 0;
             const int use = H == 1 ? (i >> 1) : i;
             const int t = c + i * G;
-            const int m = (t % tiles_m) * S::kTileM + eh * BM + 32 * quad + lane;
-            const int n0 = (t / tiles_m) * BN;
+            const int m0 = (t % tiles_m) * S::kTileM + eh * BM + 32 * quad;  // the warp's first row
+            const bool row_in = m0 + lane < p.M;
+            const int n0 = (t / tiles_m) * p.bn;
+            if (MODE == 1) {
+                // the tile's latent scale, widened to fp32 once (lane j takes
+                // columns j, j + 32, ...) while the accumulator fills
+                for (int cc = lane; cc < p.bn && n0 + cc < p.N; cc += 32) {
+                    const int nn = n0 + cc;
+                    const float lv = f16_bits_to_float(nn >= p.r0 ? p.l1[nn - p.r0] : p.l0[nn]);
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(lsm + 4u * (uint32_t)cc), "f"(lv) : "memory");
+                }
+                __syncwarp();
+            }
             bool ok = !abort_flag && mbar_wait(accf0 + 8 * b, (uint32_t)(use & 1));
             ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
             if (!ok) {
@@ -367,45 +403,54 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
                 break;
             }
             tc_fence_after();
-            for (int c32 = 0; c32 < BN; c32 += 32) {
-                uint32_t vv[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)((b + eh) * BN + c32), vv);
-#pragma unroll
-              for (int half = 0; half < 2; ++half) {
-                const int c0 = c32 + 16 * half;
-                const uint32_t *v = vv + 16 * half;
-                const int nn = n0 + c0;
-                if (m >= p.M || nn >= p.N) continue;
-                uint32_t o[8];
+            for (int c32 = 0; c32 < p.bn && n0 + c32 < p.N; c32 += 32) {
+                const int nn = n0 + c32;
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)((b + eh) * BN + c32), v);
+                uint32_t o[16];
                 if (MODE == 1) {
-                    // z = l (.) c, rounded to fp16 (the operand of contraction 2)
-                    const bool sec = nn >= p.r0;
-                    const uint16_t *lp = sec ? p.l1 + (nn - p.r0) : p.l0 + nn;
-                    const uint4 la = __ldg(reinterpret_cast<const uint4 *>(lp));
-                    const uint4 lb = __ldg(reinterpret_cast<const uint4 *>(lp + 8));
-                    const uint32_t lw[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
+                    // z = l (.) c, rounded to fp16 (the operand of contraction 2);
+                    // every lane reads the same l (a shared-memory broadcast)
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float z0 = __uint_as_float(v[2 * q]) * f16_bits_to_float((uint16_t)(lw[q] & 0xffffu));
-                        const float z1 = __uint_as_float(v[2 * q + 1]) * f16_bits_to_float((uint16_t)(lw[q] >> 16));
-                        overflow |= beyond_f16(z0) | beyond_f16(z1);
-                        o[q] = pack_half2(z0, z1);
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        float4 lq;
+                        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                     : "=f"(lq.x), "=f"(lq.y), "=f"(lq.z), "=f"(lq.w)
+                                     : "r"(lsm + 4u * (uint32_t)(c32 + 4 * q4)));
+                        const float z0 = __uint_as_float(v[4 * q4]) * lq.x, z1 = __uint_as_float(v[4 * q4 + 1]) * lq.y;
+                        const float z2 = __uint_as_float(v[4 * q4 + 2]) * lq.z, z3 = __uint_as_float(v[4 * q4 + 3]) * lq.w;
+                        overflow |= row_in && (beyond_f16(z0) | beyond_f16(z1) | beyond_f16(z2) | beyond_f16(z3));
+                        o[2 * q4] = pack_half2(z0, z1);
+                        o[2 * q4 + 1] = pack_half2(z2, z3);
                     }
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        o[q] = (uint32_t)float_to_bf16_bits(__uint_as_float(v[2 * q])) |
-                               ((uint32_t)float_to_bf16_bits(__uint_as_float(v[2 * q + 1])) << 16);
+                    for (int q = 0; q < 16; ++q) o[q] = pack_bf162(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1]));
                 }
-                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + (int64_t)m * p.ldo + nn);
-                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-              }
+                if (m0 >= p.M) continue;  // the warp's rows all lie past the matrix
+                const uint32_t box = obox + (uint32_t)(nst % S::kOutBufs) * OUT_BYTES;
+                const uint32_t rowa = box + (uint32_t)lane * 64;  // this lane's row of the box
+                // the store that last used this box has finished reading it
+                if (lane == 0) bulk_wait_read<S::kOutBufs - 1>();
+                __syncwarp();
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowa + (((uint32_t)q ^ rsw) << 4)),
+                                 "r"(o[4 * q]), "r"(o[4 * q + 1]), "r"(o[4 * q + 2]), "r"(o[4 * q + 3])
+                                 : "memory");
+                fence_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmOut, nn, m0, box);
+                    bulk_commit();
+                }
+                ++nst;
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(acce0 + 8 * b);
         }
+        if (lane == 0) bulk_wait_all();
         if (overflow) set_status(p.status, LB_ERR_RANGE);
     }
 
@@ -420,26 +465,64 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-// One contraction on a persistent grid.  The tile shape follows a makespan
-// model: H = 2 expands half the sign bits per flop, which measured about 1.6x
-// the H = 1 throughput while the expansion bounds the kernel, but it has half
-// as many tiles; take it when ceil(tiles_2 / SMs) * 2 / 1.6 <= ceil(tiles_1 / SMs).
+// The tile shape of one contraction, from a makespan model fitted to timings
+// of this kernel on B200 (Qwen3-14B and Llama-2-7B shapes, 256 to 8192
+// tokens).  A CTA spends per K-block of a tile, in tenths of a nanosecond,
+//   H = 1:  max(4800, 2000 + 20 bn)    (two producer groups alternate)
+//   H = 2:  max(8000, 5500 + 18 bn)    (one group feeds both halves)
+// where the constant floors are the producers' latency per block and the
+// slopes the sign expansion and MMA, plus per tile 500 ns (H = 1: its
+// epilogue overlaps the next tile) or 3000 ns (H = 2: both accumulators hold
+// the one tile, so the MMA waits for its epilogue).  The makespan is
+// ceil(tiles / SMs) tiles.  Of the widths giving each column-tile count only
+// the narrowest (rounded up to 32, the output box width) is worth trying;
+// ties (widths whose blocks all sit at the floor) go to more tiles, i.e. less
+// work per CTA.
+struct TilePlan {
+    int H, bn, tiles;
+};
+
+TilePlan plan_tiles(int M, int N, int K, int sms)
+{
+    const long nk = (K + BK - 1) / BK;
+    TilePlan best{1, BN, 0};
+    long best_cost = -1;
+    for (int H = 1; H <= 2; ++H) {
+        const int tm = (M + BM * H - 1) / (BM * H);
+        for (int tn = (N + BN - 1) / BN; tn <= (N + 31) / 32; ++tn) {
+            const int bn = ((N + tn - 1) / tn + 31) & ~31;
+            if ((N + bn - 1) / bn != tn) continue;
+            const int tiles = tm * tn, waves = (tiles + sms - 1) / sms;
+            const long per_block = H == 1 ? std::max(4800, 2000 + 20 * bn) : std::max(8000, 5500 + 18 * bn);
+            const long cost = (long)waves * (nk * per_block + (H == 1 ? 5000 : 30000));
+            if (best_cost < 0 || cost < best_cost || (cost == best_cost && tiles > best.tiles)) {
+                best_cost = cost;
+                best = TilePlan{H, bn, tiles};
+            }
+        }
+    }
+    return best;
+}
+
+// One contraction on a persistent grid of min(tiles, SMs) CTAs.
 // A is x (mode 1, bf16) or z (mode 2, fp16), row-major with stride lda.
 template <int MODE>
-cudaError_t launch_sign_gemm(const SignGemmParams &p, const void *a, int64_t lda, const DeviceInfo &dev,
+cudaError_t launch_sign_gemm(SignGemmParams p, const void *a, int64_t lda, const DeviceInfo &dev,
                              cudaStream_t stream)
 {
-    const int tn = (p.N + BN - 1) / BN;
-    const int t1 = ((p.M + BM - 1) / BM) * tn, t2 = ((p.M + 2 * BM - 1) / (2 * BM)) * tn;
-    const int w1 = (t1 + dev.sm_count - 1) / dev.sm_count, w2 = (t2 + dev.sm_count - 1) / dev.sm_count;
-    const int H = 5 * w2 <= 4 * w1 ? 2 : 1;
-    CUtensorMap tm;
+    const TilePlan tp = plan_tiles(p.M, p.N, p.K, dev.sm_count);
+    const int H = tp.H;
+    p.bn = tp.bn;
+    CUtensorMap tm, tmo;
     cudaError_t e = encode_2d(&tm, a, p.M, p.K, lda, MODE == 1, BM * H);
+    // the output: z fp16 (mode 1) or y bf16 (mode 2), [M x N] with stride ldo
+    if (e == cudaSuccess) e = encode_store_2d(&tmo, p.out, p.M, p.N, p.ldo, MODE == 2);
     if (e != cudaSuccess) return e;
+    const int grid = std::min(tp.tiles, dev.sm_count);
     if (H == 2)
-        sign_gemm_kernel<MODE, 2><<<std::min(t2, dev.sm_count), Shape<2>::kThreads, Shape<2>::kSmem, stream>>>(tm, p);
+        sign_gemm_kernel<MODE, 2><<<grid, Shape<2>::kThreads, Shape<2>::kSmem, stream>>>(tm, tmo, p);
     else
-        sign_gemm_kernel<MODE, 1><<<std::min(t1, dev.sm_count), Shape<1>::kThreads, Shape<1>::kSmem, stream>>>(tm, p);
+        sign_gemm_kernel<MODE, 1><<<grid, Shape<1>::kThreads, Shape<1>::kSmem, stream>>>(tm, tmo, p);
     return cudaGetLastError();
 }
 

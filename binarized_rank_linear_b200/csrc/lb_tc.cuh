@@ -61,6 +61,24 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
         if (globaltimer() - t0 > kWaitNs) return false;
     }
 }
+// Bulk tensor store of one box from shared memory; completion is tracked by
+// the issuing thread's bulk async-groups.  Rows or columns of the box outside
+// the tensor are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *tm, int x, int y, uint32_t src)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(tm), "r"(x), "r"(y),
+                 "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until at most N of this thread's bulk groups still read shared memory
+template <int N>
+__device__ __forceinline__ void bulk_wait_read()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// wait until all of this thread's bulk groups have completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *tm, int x, int y, uint32_t bar)
 {
     asm volatile(
@@ -166,6 +184,25 @@ inline cudaError_t get_encoder()
     if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     return cudaSuccess;
+}
+
+// 2-D map over a row-major [rows x cols] matrix of 2-byte elements with row
+// stride `ld` elements; boxes of 32 columns x 32 rows, 64-byte swizzle: the
+// shared-memory box is 32 rows of 64 bytes, and 16-byte chunk q of row r sits
+// at chunk position q ^ ((r >> 1) & 3) (address bits 4..5 XOR bits 7..8).
+// For bulk stores of a tile's output.
+inline cudaError_t encode_store_2d(CUtensorMap *tm, void *ptr, int rows, int cols, int64_t ld, bool bf16)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 g_encode = encoder_slot();
+    if (!g_encode) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    const cuuint32_t box[2] = {32, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ptr,
+                                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 // 2-D map over a row-major [rows x cols] matrix of 2-byte elements with row

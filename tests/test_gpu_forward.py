@@ -57,14 +57,36 @@ def test_token_sweep_ragged_shape(tokens):
 
 @pytest.mark.parametrize("n_in,n_out,ranks", [(256, 5120, [64, 32]), (64, 32, [2432, 2432])])
 def test_prefill_tile_shapes_ragged(n_in, n_out, ranks):
-    """1000 tokens over many output tiles: on a 148-SM part the wide
-    contraction runs 256-row CTA tiles (two 128-row halves sharing each
-    expanded sign tile), the narrow one 128-row tiles.  1000 = 3 x 256 + 232
-    leaves the last tile's second half partly outside the batch, and a latent
-    of 96 (first case) is one and a half K-blocks."""
+    """1000 tokens over many output tiles: 1000 = 7 x 128 + 104 leaves the
+    last row tile partly outside the batch, and a latent of 96 (first case)
+    is one and a half K-blocks; the second case has a 4864-wide latent, so
+    contraction 1 runs more tiles than there are SMs."""
     layer = synth.make_layer(n_in, n_out, ranks, 1000, config_id=700 + n_out)
     y = gu.bf16_to_f64(gu.run_gpu(layer))
     gu.assert_close(y, gu.oracle_y(layer), f"{n_in}x{n_out} r={ranks} M=1000")
+
+
+# Shapes whose contractions take each family of the prefill kernel's tile
+# plans on a 148-SM B200 (128-row tiles of width 32 .. 256, one or two waves;
+# 256-row tiles at 2100 tokens), each checked whole against the oracle.  The
+# plan is the library's choice; the ids record which one each shape took when
+# the cases were picked.
+TILE_PLAN_CASES = [
+    pytest.param(129, 256, 256, [32, 32], id="m129-c1-w32"),
+    pytest.param(129, 256, 4096, [32, 32], id="m129-c2-w64"),
+    pytest.param(520, 256, 2048, [32, 32], id="m520-c2-w96"),
+    pytest.param(1000, 256, 2048, [32, 32], id="m1000-c2-w128"),
+    pytest.param(700, 256, 4096, [32, 32], id="m700-c2-w192"),
+    pytest.param(2600, 256, 2048, [32, 32], id="m2600-c2-w160-2waves"),
+    pytest.param(2100, 256, 4096, [160, 160], id="m2100-c2-h2-w256"),
+]
+
+
+@pytest.mark.parametrize("tokens,n_in,n_out,ranks", TILE_PLAN_CASES)
+def test_prefill_tile_plans(tokens, n_in, n_out, ranks):
+    layer = synth.make_layer(n_in, n_out, ranks, tokens, config_id=900 + n_out + sum(ranks))
+    y = gu.bf16_to_f64(gu.run_gpu(layer))
+    gu.assert_close(y, gu.oracle_y(layer), f"{n_in}x{n_out} r={ranks} M={tokens}")
 
 
 @pytest.mark.parametrize("n_in,n_out,ranks", [(32, 32, [32]), (96, 64, [32]), (64, 800, [32, 64]),
@@ -94,7 +116,7 @@ def bf16_rne(v: np.ndarray) -> np.ndarray:
     return synth.f32_to_bf16_bits(v.astype(np.float32))
 
 
-@pytest.mark.parametrize("tokens", [1, 3, 8, 32, 40])
+@pytest.mark.parametrize("tokens", [1, 3, 8, 32, 40, 129, 300, 1000])
 def test_integer_exact_is_bitwise(tokens):
     """Unit scales and x in {-1, 0, 1}: every intermediate is a small integer,
     exact in fp16, bf16 and fp32, so the GPU must equal the oracle (rounded
