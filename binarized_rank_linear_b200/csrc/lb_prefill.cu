@@ -64,13 +64,15 @@ struct Shape {
     static constexpr int kThreads = 32 * (2 + kProducerWarps + kEpiWarps);
     static constexpr int kTileM = BM * H;
     static constexpr uint32_t kABytes = (uint32_t)kTileM * BK * 2;  // 16 or 32 KB
-    static constexpr int kOutBufs = H == 1 ? 2 : 1;  // output boxes per epilogue warp
+    static constexpr int kOutBufs = 1;  // output boxes per epilogue warp
+    static constexpr int kRing = 2;     // sign-word slots per producer thread
     // per stage: A tile, B tile; per epilogue warp: its output boxes and the
     // tile's latent scale in fp32 (mode 1); per producer warp: two slots of g
-    // rounded to bf16
+    // rounded to bf16; per producer thread: kRing slots of sign words
     static constexpr size_t kSmem = 1024 + (size_t)kStages * (kABytes + B_BYTES) +
                                     (size_t)kEpiWarps * (kOutBufs * OUT_BYTES + BN * 4) +
-                                    (size_t)kProducerWarps * 2 * G_BYTES + 256;
+                                    (size_t)kProducerWarps * (2 * G_BYTES + 32 * 8 * kRing) + 256;
+    static_assert(kSmem <= 232448, "shared memory per CTA");
 };
 // Tiles are K-major with 128-byte swizzle: row `row` holds 64 two-byte
 // elements in 128 bytes, and its 16-byte chunk j (elements 8j .. 8j + 7) is
@@ -114,7 +116,8 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
     const uint32_t sOut = sB + STAGES * B_BYTES;  // per epilogue warp: kOutBufs output boxes
     const uint32_t sGbf = sOut + S::kEpiWarps * S::kOutBufs * OUT_BYTES;  // mode 1, per producer warp: g in bf16, [warp][2][path][64]
     const uint32_t sLf = sGbf + kProducerWarps * 2 * G_BYTES;  // mode 1, per epilogue warp: l of the tile in fp32
-    const uint32_t bars = sLf + S::kEpiWarps * BN * 4;
+    const uint32_t sRing = sLf + S::kEpiWarps * BN * 4;  // per producer thread: kRing 8-byte sign-word slots
+    const uint32_t bars = sRing + kProducerWarps * 32 * 8 * S::kRing;
     // full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain, then the tmem address
     const uint32_t full0 = bars, empty0 = bars + 8 * STAGES, accf0 = bars + 16 * STAGES;
     const uint32_t acce0 = accf0 + 16, drain = acce0 + 16;
@@ -223,25 +226,33 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
         // the CTA's K-block sequence, so every warp has two MMA periods for
         // each of its blocks and its latency (barrier wait, expansion, arrive)
         // hides behind the other group's block.  H = 2: one group; a block
-        // feeds two MMA halves, so it has two MMA periods as well.  What a
-        // block needs from memory (the row's sign words; g in mode 1, h in
-        // mode 2) is loaded into registers two of the group's blocks ahead.
+        // feeds two MMA halves, so it has two MMA periods as well.
+        // What a block needs from memory arrives without a register holding a
+        // load in flight across blocks (copying such a register would wait
+        // for the load):
+        //   sign words  copied asynchronously (cp.async) into the thread's
+        //               slot of a ring in shared memory, kRing of the group's
+        //               blocks ahead, and waited for just before use;
+        //   g (mode 1)  lanes 0..15 copy a block's 64 values of each path
+        //               (fp16) into the warp's g slot the same way, and round
+        //               them to bf16 in place just before use;
+        //   h (mode 2)  depends on the row only, so it is loaded once per
+        //               tile, a tile ahead.
         const int pt = tid - 64;
         constexpr int NG = S::kGroups;  // block stride of a group
+        constexpr int RING = S::kRing;
+        static_assert(RING == 2, "the warp's two g slots double as the g ring");
+        constexpr uint32_t RING_STRIDE = (uint32_t)kProducerWarps * 32 * 8;  // bytes between ring slots
         const int grp = pt >> 8;        // 0 .. NG - 1
         const int row = pt & (BN - 1);  // B row within the tile
         const int wl = warp - 2;        // producer warp 0 .. 15
         const uint32_t x7 = (uint32_t)(row & 7);  // the row's 128-byte swizzle: logical chunk j sits at chunk j ^ x7
         const int kwords = p.K >> 5, r0w = p.r0 >> 5;
         const uint32_t gbfw = sGbf + (uint32_t)wl * 2 * G_BYTES;  // this warp's two bf16 g slots
+        const uint32_t ring = sRing + (uint32_t)pt * 8;           // this thread's slot 0 (8 bytes)
         // a warp whose rows all lie past bn takes no part (the stage barriers
         // count only the busy warps)
         const int my_blocks = (wl & (kGroupWarps - 1)) < busy_warps ? nblocks : 0;
-        struct Pref {
-            uint2 bits;      // the row's two sign words of the block (zero outside the matrix)
-            uint4 g;         // mode 1, lanes 0..15: g of path lane / 8, columns 8 (lane % 8) .. (fp16)
-            uint32_t h0, h1; // mode 2: h of the row, both paths (fp16)
-        };
         // Position of a block in the sequence, advanced without divisions:
         // tile iteration, K-block, and this thread's B row in that tile.
         struct Cursor {
@@ -266,16 +277,24 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
                 u.nn = ((c + u.i * G) / tiles_m) * p.bn + row;
             }
         };
-        auto fetch = [&](const Cursor &u) {
-            Pref f;
-            f.bits = make_uint2(0u, 0u);
-            f.g = make_uint4(0u, 0u, 0u, 0u);
-            f.h0 = f.h1 = 0u;
-            if (u.gb >= my_blocks) return f;
-            const int kb = u.kb, nn = u.nn;
-            const bool row_in = row < p.bn && nn < p.N;
-            const int wd = 2 * kb;  // first word of the block in the (concatenated) row
-            if (row_in && wd < kwords) {
+        // Start the copies of block u's two sign words into ring slot `slot`
+        // (zeros outside the matrix) and, mode 1, lanes 0..15, of its g into
+        // the warp's g slot `slot`: one cp.async group.
+        auto copy_block = [&](const Cursor &u, int slot) {
+            if (MODE == 1 && u.gb < my_blocks && lane < 16) {
+                // lane: path lane / 8, columns 8 (lane % 8) .. 8 (lane % 8) + 7 of the block
+                const int pp = lane >> 3, k0 = u.kb * BK + 8 * (lane & 7);
+                const uint16_t *gs = pp ? p.s1 : p.s0;
+                const uint32_t gdst = gbfw + (uint32_t)slot * G_BYTES + (uint32_t)lane * 16;
+                if (gs != nullptr && k0 < p.K)
+                    cp_async16s(gdst, gs + k0);
+                else
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(gdst), "r"(0u) : "memory");
+            }
+            const uint32_t dst = ring + (uint32_t)slot * RING_STRIDE;
+            const int wd = 2 * u.kb;  // first word of the block in the (concatenated) row
+            if (u.gb < my_blocks && row < p.bn && u.nn < p.N && wd < kwords) {
+                const int nn = u.nn;
                 const uint32_t *rb0, *rb1 = nullptr;
                 if (MODE == 1) {
                     const bool sec = nn >= p.r0;
@@ -286,61 +305,81 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
                 }
                 auto wp = [&](int w) { return (MODE == 1 || w < r0w) ? rb0 + w : rb1 + (w - r0w); };
                 if (p.bits8 && wd + 1 < kwords) {
-                    f.bits = ldg_early_v2(wp(wd));
+                    cp_async8(dst, wp(wd));
                 } else {
-                    f.bits.x = ldg_early_u32(wp(wd));
-                    if (wd + 1 < kwords) f.bits.y = ldg_early_u32(wp(wd + 1));
+                    cp_async4(dst, wp(wd));
+                    if (wd + 1 < kwords)
+                        cp_async4(dst + 4, wp(wd + 1));
+                    else
+                        asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst + 4), "r"(0u) : "memory");
                 }
+            } else if (u.gb < my_blocks) {
+                asm volatile("st.shared.v2.u32 [%0], {%1, %1};" ::"r"(dst), "r"(0u) : "memory");
             }
-            if (MODE == 1 && lane < 16) {
-                const int pp = lane >> 3, k0 = kb * BK + 8 * (lane & 7);
-                const uint16_t *gs = pp ? p.s1 : p.s0;
-                if (gs != nullptr && k0 < p.K) f.g = ldg_early_v4(gs + k0);
-            }
-            if (MODE == 2 && row_in) {
-                f.h0 = ldg_early_u16(p.s0 + nn);
-                if (p.s1) f.h1 = ldg_early_u16(p.s1 + nn);
-            }
-            return f;
+            cp_async_commit();  // one group per block (empty past the end), so the waits count blocks
         };
-        Cursor u = cursor_at(grp), ua = cursor_at(grp + 2 * NG);  // this block, and the group's block two ahead
-        Pref f0 = fetch(u), f1 = fetch(cursor_at(grp + NG));
+        // mode 2: h of this thread's row in tile iteration i, both paths (fp16 pair)
+        auto fetch_h = [&](int i) {
+            uint32_t hv = 0u;
+            const int nn = ((c + i * G) / tiles_m) * p.bn + row;
+            if (MODE == 2 && i < my_tiles && row < p.bn && nn < p.N) {
+                hv = ldg_early_u16(p.s0 + nn);
+                if (p.s1) hv |= (uint32_t)ldg_early_u16(p.s1 + nn) << 16;
+            }
+            return hv;
+        };
+        Cursor u = cursor_at(grp), ua = cursor_at(grp + RING * NG);  // this block, and the group's block RING ahead
+        {
+            Cursor w = u;
+            for (int d = 0; d < RING; ++d, advance(w)) copy_block(w, d);
+        }
+        int hi = -2;                  // tile iteration whose h is in hcur (none yet; hnext is for hi + 1)
+        uint32_t hcur = 0u, hnext = 0u;
         for (int j = 0; u.gb < my_blocks; ++j, advance(u), advance(ua)) {
-            const Pref cur = f0;
-            f0 = f1;
-            f1 = fetch(ua);
             const int gb = u.gb, kb = u.kb, nn = u.nn;
+            if (MODE == 2 && u.i != hi) {  // first block of a tile for this group
+                hcur = u.i == hi + 1 ? hnext : fetch_h(u.i);
+                hnext = fetch_h(u.i + 1);
+                hi = u.i;
+            }
             const int s = gb % STAGES;
             const uint32_t ph = (uint32_t)(gb / STAGES) & 1u;
-            // wait for the MMA to release stage s (it last held block gb - 4,
-            // this group's previous use of it); the decision is per warp
+            // wait for the MMA to release stage s (it last held block
+            // gb - STAGES); the decision is per warp
             bool ok = mbar_wait(empty0 + 8 * s, ph ^ 1u) && !abort_flag;
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) {
                 abort_flag = 1;
                 break;
             }
+            // this block's copies have landed (at most RING - 1 younger
+            // groups still pending)
+            cp_async_wait_group<RING - 1>();
+            const int slot = j % RING;
             uint4 sc[8];  // per chunk: the four packed scale words
             if (MODE == 1) {
-                // lanes 0..15 round this block's g to bf16 into the warp's slot
-                // j % 2 (last read two iterations ago, before a __syncwarp)
+                // lanes 0..15 round their 8 values of g to bf16 in place
+                const uint32_t gsl = gbfw + (uint32_t)slot * G_BYTES;
                 if (lane < 16) {
-                    const uint32_t w[4] = {cur.g.x, cur.g.y, cur.g.z, cur.g.w};
-                    uint32_t o[4];
+                    uint32_t w[4];
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                                 : "r"(gsl + (uint32_t)lane * 16)
+                                 : "memory");
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        o[q] = (uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[q] & 0xffffu))) |
-                               ((uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[q] >> 16))) << 16);
-                    *reinterpret_cast<uint4 *>(smem_raw + (gbfw + (j & 1) * G_BYTES + lane * 16 - raw)) =
-                        make_uint4(o[0], o[1], o[2], o[3]);
+                        w[q] = pack_bf162(f16_bits_to_float((uint16_t)(w[q] & 0xffffu)), f16_bits_to_float((uint16_t)(w[q] >> 16)));
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(gsl + (uint32_t)lane * 16), "r"(w[0]),
+                                 "r"(w[1]), "r"(w[2]), "r"(w[3])
+                                 : "memory");
                 }
                 __syncwarp();
                 const bool sec_row = nn >= p.r0;  // the row's path
-                const uint8_t *gb_ = smem_raw + (gbfw + (j & 1) * G_BYTES + (sec_row ? BK * 2 : 0) - raw);
+                const uint8_t *gb_ = smem_raw + (gsl + (sec_row ? BK * 2 : 0) - raw);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) sc[q] = *reinterpret_cast<const uint4 *>(gb_ + 16 * q);
             } else {
-                const uint32_t hs0 = cur.h0 | (cur.h0 << 16), hs1 = cur.h1 | (cur.h1 << 16);
+                const uint32_t hs0 = (hcur & 0xffffu) * 0x10001u, hs1 = (hcur >> 16) * 0x10001u;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const int k0 = kb * BK + 8 * q;  // first column of the chunk
@@ -348,6 +387,11 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
                     sc[q] = make_uint4(h, h, h, h);
                 }
             }
+            uint2 bits;
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                         : "=r"(bits.x), "=r"(bits.y)
+                         : "r"(ring + (uint32_t)slot * RING_STRIDE)
+                         : "memory");
             // chunk q of the row goes to chunk position q ^ x7 (the tile is
             // 1024-byte aligned, so the XOR acts on address bits 4..6 alone);
             // the 8 rows of a store phase then cover all 32 banks
@@ -355,14 +399,19 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
             if (row < p.bn) {
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    store_sign_chunk(rowx ^ (16u * q),
-                                     __byte_perm(q < 4 ? cur.bits.x : cur.bits.y, 0u, 0x4440u | (uint32_t)(q & 3)), sc[q]);
+                    store_sign_chunk(rowx ^ (16u * q), __byte_perm(q < 4 ? bits.x : bits.y, 0u, 0x4440u | (uint32_t)(q & 3)),
+                                     sc[q]);
                 }
             }
             fence_async_shared();
             __syncwarp();
             if (lane == 0) mbar_arrive(full0 + 8 * s);
+            // refill the slots (their contents are used above, and every lane
+            // is past its reads after the __syncwarp) with the group's block
+            // RING ahead
+            copy_block(ua, slot);
         }
+        cp_async_wait_all();  // no copy may land after the CTA is gone
     } else {
         // ---------------- epilogue: warp w drains tensor-memory lanes 32 (w % 4)
         // .. of a finished accumulator (H = 2: warps 4 e .. 4 e + 3 of the

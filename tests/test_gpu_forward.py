@@ -98,7 +98,7 @@ def test_small_and_asymmetric_shapes(n_in, n_out, ranks):
         gu.assert_close(y, gu.oracle_y(layer), f"{n_in}x{n_out} r={ranks} M={tokens}")
 
 
-def integer_layer(n_in, n_out, ranks, tokens, seed):
+def integer_layer(n_in, n_out, ranks, tokens, seed, zero_frac=0.9):
     rng = np.random.default_rng(seed)
     paths = []
     for r in ranks:
@@ -107,7 +107,7 @@ def integer_layer(n_in, n_out, ranks, tokens, seed):
                           h=np.ones(n_out, np.float16), g=np.ones(n_in, np.float16),
                           l=np.ones(r, np.float16)))
     xf = rng.integers(-1, 2, (tokens, n_in)).astype(np.float32)
-    xf[rng.random((tokens, n_in)) < 0.9] = 0.0       # keep |y| small
+    xf[rng.random((tokens, n_in)) < zero_frac] = 0.0  # keep |y| small
     x = (xf.view(np.uint32) >> 16).astype(np.uint16)
     return dict(x=x, paths=paths, n_in=n_in, n_out=n_out)
 
@@ -121,7 +121,8 @@ def test_integer_exact_is_bitwise(tokens):
     """Unit scales and x in {-1, 0, 1}: every intermediate is a small integer,
     exact in fp16, bf16 and fp32, so the GPU must equal the oracle (rounded
     to bf16) bit for bit.  Pins sign orientation, pack layout and transposes."""
-    layer = integer_layer(512, 224, [64, 32], tokens, tokens)
+    # sparser x for the larger batches keeps every |y| within 256
+    layer = integer_layer(512, 224, [64, 32], tokens, tokens, 0.9 if tokens < 100 else 0.97)
     ref = gu.oracle_y(layer)
     assert np.abs(ref).max() <= 256 and np.array_equal(ref, np.rint(ref))
     got = gu.bf16_bits(gu.run_gpu(layer))
