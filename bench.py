@@ -270,6 +270,158 @@ def run_reference(args, world, rank):
 
 # ---------------------------------------------------------------- the GPU arm
 
+def kernel_label(tokens):
+    if tokens <= 4:
+        return "lb_linear_forward call: small1_kernel + small2_kernel (CUDA cores, PDL-chained)"
+    if tokens <= 128:
+        return ("lb_linear_forward call: mid_gemm_kernel<1> + mid_gemm_kernel<2> "
+                "(tcgen05, sign matrix as the 128-row operand, PDL-chained)")
+    return "lb_linear_forward call: sign_gemm_kernel<1> + sign_gemm_kernel<2> (tcgen05, persistent)"
+
+
+def dense_baseline(layer, x, steps, stream, device):
+    """The layer as the dense bf16 matrix W = sum_p diag(h_p) S_U diag(l_p)
+    S_V^T diag(g_p), applied with one cuBLAS GEMM per call (torch.matmul): the comparison the pages' kernel speedup
+    figure makes (littlebitllm.com, "How small"; the single-kernel speedup
+    quoted for a Llama2-70B layer).  W is built with plain PyTorch ops on the
+    GPU; copies rotate past twice the L2 cache, as the packed weights do."""
+    import torch
+    W = None
+    for p in layer["paths"]:
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        su, sv = t(p["su"]).float(), t(p["sv"]).float()
+        h, g, l = (t(p[k].view(np.int16)).view(torch.float16).float() for k in ("h", "g", "l"))
+        term = (h[:, None] * su * l[None, :]) @ (sv * g[:, None]).t()
+        W = term if W is None else W + term
+    W = W.to(torch.bfloat16)
+    w_bytes = W.numel() * 2
+    nsets = max(1, min(64, -(-2 * L2_BYTES // w_bytes) + 1))
+    Ws = [W] + [W.clone() for _ in range(nsets - 1)]
+    y = torch.empty((x.shape[0], W.shape[0]), dtype=torch.bfloat16, device=device)
+    per_graph = max(nsets, 32)
+    cap = torch.cuda.Stream(device)
+    torch.matmul(x, Ws[0].t(), out=y)  # warm the cuBLAS handle before capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        for i in range(per_graph):
+            torch.matmul(x, Ws[i % nsets].t(), out=y)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    reps = max(1, min(200, steps // per_graph))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * per_graph)
+    return {"us_per_call": us, "kind": "cuBLAS bf16 GEMM (torch.matmul) on the dense weight, CUDA graphs",
+            "dense_weight_bytes": w_bytes, "weight_sets": nsets}
+
+
+# A decoder block's linears in the order a forward pass runs them, as
+# (workload, count) from the table in binarized_rank_linear_b200/synth.py.
+BLOCKS = {
+    "llama2_7b": [("llama2_7b_q", 4), ("llama2_7b_gate", 2), ("llama2_7b_down", 1)],  # q k v o, gate up, down
+    "qwen3_14b": [("qwen3_14b_qo", 1), ("qwen3_14b_kv", 2), ("qwen3_14b_qo", 1),       # q, k v, o
+                  ("qwen3_14b_gate", 2), ("qwen3_14b_down", 1)],                      # gate up, down
+}
+
+
+def run_block(args, world, rank, local):
+    """One step is a whole decoder block's linears at `tokens` tokens, called
+    back to back on one stream (each call's launches PDL-chained to the
+    previous one) from CUDA graphs; weights rotate past twice the L2 cache."""
+    import torch
+    import binarized_rank_linear_b200 as lb
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    tokens = args.tokens or 1
+    seq = [name for name, n in BLOCKS[args.block] for _ in range(n)]
+    layers, nbytes, nflops = [], 0, 0
+    for j, name in enumerate(seq):
+        c = synth.CONFIGS[name]
+        ranks = [c.rank] * c.paths
+        nbytes += algorithmic_bytes(c.n_in, c.n_out, ranks, tokens)
+        nflops += algorithmic_flops(c.n_in, c.n_out, ranks, tokens)
+        lay = synth.make_config(name, tokens, seed=j)
+        paths = []
+        for p in lay["paths"]:
+            dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+            paths.append(lb.PackedPath.from_factors(dev(p["su"]), dev(p["sv"]), dev(p["h"]), dev(p["g"]), dev(p["l"])))
+        x = torch.from_numpy(lay["x"].view(np.int16)).to(device).view(torch.bfloat16)
+        y = torch.empty((tokens, c.n_out), dtype=torch.bfloat16, device=device)
+        ws = torch.empty(max(16, lb.forward_workspace_bytes(tokens, c.n_in, c.n_out, c.rank,
+                                                            c.rank if c.paths > 1 else 0)),
+                         dtype=torch.uint8, device=device)
+        layers.append((paths, x, y, ws))
+    set_bytes = sum(p.u_bits.numel() * 4 + p.vt_bits.numel() * 4 for lay in layers for p in lay[0])
+    nsets = max(1, min(64, -(-2 * L2_BYTES // set_bytes) + 1))
+
+    def clone(p):
+        return lb.PackedPath(p.u_bits.clone(), p.vt_bits.clone(), p.h.clone(), p.g.clone(), p.l.clone(), p.rank)
+
+    sets = [[lay[0] for lay in layers]] + [[[clone(p) for p in lay[0]] for lay in layers] for _ in range(nsets - 1)]
+
+    def block(i):
+        for (paths0, x, y, ws), paths in zip(layers, sets[i % nsets]):
+            lb.linear_forward(x, paths[0], paths[1] if len(paths) > 1 else None, y=y, workspace=ws)
+
+    block(0)
+    torch.cuda.synchronize()
+    assert lb.device_status() == lb.LB_OK
+    per_graph = max(1, min(2 * nsets, 64))
+    cap = torch.cuda.Stream(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        for i in range(per_graph):
+            block(i)
+    for _ in range(max(1, args.warmup // per_graph)):
+        g.replay()
+    torch.cuda.synchronize()
+    reps = max(1, args.steps // per_graph)
+    stream = torch.cuda.current_stream(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    with clk:
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    steps = reps * per_graph
+    per_block_s = ms / 1e3 / steps
+    assert lb.device_status() == lb.LB_OK
+    if rank != 0:
+        return
+    decode = tokens <= DECODE_MAX_TOKENS
+    peaks = load_peaks()
+    achieved = (nbytes / per_block_s / 1e9) if decode else (nflops / per_block_s / 1e12)
+    pk = peaks["hbm"] if decode else peaks["bf16_sustained"]
+    out = {"metric": "decoder block of LittleBit linears: us/block, " + ("HBM GB/s" if decode else "TFLOP/s"),
+           "value": aggregate(((nbytes / 1e9) if decode else (nflops / 1e12)) * steps, ms / 1e3, world),
+           "unit": "GB/s" if decode else "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
+           "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f16", "data": "synthetic",
+           "config": {"workload": "%s block (%s) at %d tokens" % (args.block, ", ".join(seq), tokens),
+                      "tokens": tokens, "linears": len(seq), "weight_sets": nsets,
+                      "launch": "CUDA graphs of %d blocks" % per_graph},
+           "us_per_block": per_block_s * 1e6, "algorithmic_bytes_per_block": nbytes,
+           "algorithmic_flops_per_block": nflops,
+           "roofline": {"bound": "hbm" if decode else "tensor", "achieved": achieved, "peak": pk,
+                        "unit": "GB/s" if decode else "TFLOP/s", "frac": achieved / pk, "traffic": None,
+                        "peak_source": peaks["source"]},
+           "clocks": clk.summary(), "gpu_launches": 2 * len(seq) * steps, "impl": "lb"}
+    print(json.dumps(out), flush=True)
+
+
 def run_lb(args, world, rank, local):
     import torch
     import binarized_rank_linear_b200 as lb
@@ -410,6 +562,8 @@ def run_lb(args, world, rank, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
     e2e_value = aggregate(units * e2e_steps, e2e_ms / 1e3, world)
 
+    dense = dense_baseline(layer, x, args.steps, stream, device) if args.dense_baseline else None
+
     if rank != 0:
         return
     peaks = load_peaks()
@@ -417,16 +571,14 @@ def run_lb(args, world, rank, local):
         achieved = nbytes / per_call_s / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm"], "traffic": load_traffic(args.config, tokens),
-                "kernel": ("lb_linear_forward call: small_latent_kernel + small_expand_kernel (CUDA cores, PDL-chained)"
-                           if tokens <= 4 else
-                           "lb_linear_forward call: latent_kernel + expand_kernel (mma.sync, PDL-chained)"),
+                "kernel": kernel_label(tokens),
                 "peak_source": peaks["source"]}
     else:
         achieved = nflops / per_call_s / 1e12
         pk = peaks["bf16_sustained"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
                 "frac": achieved / pk, "traffic": load_traffic(args.config, tokens),
-                "kernel": "lb_linear_forward call: sign_gemm_kernel<1> + sign_gemm_kernel<2> (tcgen05)",
+                "kernel": kernel_label(tokens),
                 "peak_source": peaks["source"] + " (sustained)"}
     cpu = None
     if world == 1 and not args.no_cpu:
@@ -451,6 +603,9 @@ def run_lb(args, world, rank, local):
                    "steps": e2e_steps},
            "gpu_launches": 2 * args.steps,  # contraction 1 + contraction 2 per call, decode and prefill
            "impl": "lb"}
+    if dense is not None:
+        dense["speedup"] = dense["us_per_call"] / (per_call_s * 1e6)
+        out["dense_baseline"] = dense
     print(json.dumps(out), flush=True)
 
 
@@ -466,6 +621,10 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=5000)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-parity", action="store_true")
+    ap.add_argument("--block", choices=sorted(BLOCKS), default=None,
+                    help="time a whole decoder block's linears chained (tokens default 1)")
+    ap.add_argument("--dense-baseline", action="store_true",
+                    help="also time a cuBLAS bf16 GEMM on the reconstructed dense weight (same tokens)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -475,7 +634,7 @@ def main(argv=None):
         return
     world, rank, local = dist_setup(args.gpus)
     try:
-        run_lb(args, world, rank, local)
+        (run_block if args.block else run_lb)(args, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -71,3 +71,24 @@ def test_reference_arm_non_zero_ranks_exit(monkeypatch, capsys):
     monkeypatch.setenv("WORLD_SIZE", "2")
     bench.main(["--impl", "reference", "--steps", "3", "--warmup", "3"])
     assert capsys.readouterr().out == ""
+
+
+def test_blocks_are_the_models_linears():
+    """--block: every entry names a workload of the table, and the linears'
+    shapes chain as a decoder block does (attention in -> model width, MLP
+    up -> intermediate width, down -> model width)."""
+    for name, seq in bench.BLOCKS.items():
+        linears = [synth.CONFIGS[w] for w, n in seq for _ in range(n)]
+        assert len(linears) == 7
+        width = linears[0].n_in
+        assert all(c.n_in == width for c in linears[:3])           # q, k, v read the block input
+        assert linears[3].n_out == width                          # o writes the model width
+        gate, up, down = linears[4:]
+        assert gate.n_in == up.n_in == width and gate.n_out == up.n_out == down.n_in
+        assert down.n_out == width
+
+
+def test_kernel_labels_follow_the_dispatch():
+    assert "small1_kernel" in bench.kernel_label(1) and "small1_kernel" in bench.kernel_label(4)
+    assert "mid_gemm_kernel" in bench.kernel_label(5) and "mid_gemm_kernel" in bench.kernel_label(128)
+    assert "sign_gemm_kernel" in bench.kernel_label(129)
