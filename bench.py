@@ -321,26 +321,30 @@ def dense_baseline(layer, x, steps, stream, device):
             "dense_weight_bytes": w_bytes, "weight_sets": nsets}
 
 
-# A decoder block's linears in the order a forward pass runs them, as
-# (workload, count) from the table in binarized_rank_linear_b200/synth.py.
+# A decoder block's linears in the order a forward pass runs them, grouped by
+# the input they read (workload names from binarized_rank_linear_b200/synth.py):
+# q k v, o, gate up, down.
 BLOCKS = {
-    "llama2_7b": [("llama2_7b_q", 4), ("llama2_7b_gate", 2), ("llama2_7b_down", 1)],  # q k v o, gate up, down
-    "qwen3_14b": [("qwen3_14b_qo", 1), ("qwen3_14b_kv", 2), ("qwen3_14b_qo", 1),       # q, k v, o
-                  ("qwen3_14b_gate", 2), ("qwen3_14b_down", 1)],                      # gate up, down
+    "llama2_7b": [["llama2_7b_q"] * 3, ["llama2_7b_q"], ["llama2_7b_gate"] * 2, ["llama2_7b_down"]],
+    "qwen3_14b": [["qwen3_14b_qo", "qwen3_14b_kv", "qwen3_14b_kv"], ["qwen3_14b_qo"], ["qwen3_14b_gate"] * 2,
+                  ["qwen3_14b_down"]],
 }
 
 
 def run_block(args, world, rank, local):
     """One step is a whole decoder block's linears at `tokens` tokens, called
     back to back on one stream (each call's launches PDL-chained to the
-    previous one) from CUDA graphs; weights rotate past twice the L2 cache."""
+    previous one) from CUDA graphs; weights rotate past twice the L2 cache.
+    With --fused the linears that read the same input (q k v; gate up) run
+    as one lb_linear_forward_siblings call."""
     import torch
     import binarized_rank_linear_b200 as lb
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     tokens = args.tokens or 1
-    seq = [name for name, n in BLOCKS[args.block] for _ in range(n)]
+    groups = BLOCKS[args.block]
+    seq = [name for grp in groups for name in grp]
     layers, nbytes, nflops = [], 0, 0
     for j, name in enumerate(seq):
         c = synth.CONFIGS[name]
@@ -366,9 +370,24 @@ def run_block(args, world, rank, local):
 
     sets = [[lay[0] for lay in layers]] + [[[clone(p) for p in lay[0]] for lay in layers] for _ in range(nsets - 1)]
 
+    # fused: one shared x and workspace per group
+    gstart = np.cumsum([0] + [len(grp) for grp in groups])
+    gx, gws = [], []
+    for a, b in zip(gstart[:-1], gstart[1:]):
+        gx.append(layers[a][1])
+        spec = [(layers[k][0][0], layers[k][0][1] if len(layers[k][0]) > 1 else None) for k in range(a, b)]
+        gws.append(torch.empty(max(16, lb.siblings_workspace_bytes(tokens, gx[-1].shape[1], spec)),
+                               dtype=torch.uint8, device=device))
+
     def block(i):
-        for (paths0, x, y, ws), paths in zip(layers, sets[i % nsets]):
-            lb.linear_forward(x, paths[0], paths[1] if len(paths) > 1 else None, y=y, workspace=ws)
+        s = sets[i % nsets]
+        if not args.fused:
+            for (paths0, x, y, ws), paths in zip(layers, s):
+                lb.linear_forward(x, paths[0], paths[1] if len(paths) > 1 else None, y=y, workspace=ws)
+            return
+        for gi, (a, b) in enumerate(zip(gstart[:-1], gstart[1:])):
+            lb.linear_forward_siblings(gx[gi], [(s[k][0], s[k][1] if len(s[k]) > 1 else None) for k in range(a, b)],
+                                       ys=[layers[k][2] for k in range(a, b)], workspace=gws[gi])
 
     block(0)
     torch.cuda.synchronize()
@@ -412,13 +431,16 @@ def run_block(args, world, rank, local):
            "dtype": "f16", "data": "synthetic",
            "config": {"workload": "%s block (%s) at %d tokens" % (args.block, ", ".join(seq), tokens),
                       "tokens": tokens, "linears": len(seq), "weight_sets": nsets,
+                      "calls": ("one lb_linear_forward_siblings call per input group (%d)" % len(groups))
+                      if args.fused else "one lb_linear_forward call per linear",
                       "launch": "CUDA graphs of %d blocks" % per_graph},
            "us_per_block": per_block_s * 1e6, "algorithmic_bytes_per_block": nbytes,
            "algorithmic_flops_per_block": nflops,
            "roofline": {"bound": "hbm" if decode else "tensor", "achieved": achieved, "peak": pk,
                         "unit": "GB/s" if decode else "TFLOP/s", "frac": achieved / pk, "traffic": None,
                         "peak_source": peaks["source"]},
-           "clocks": clk.summary(), "gpu_launches": 2 * len(seq) * steps, "impl": "lb"}
+           "clocks": clk.summary(),
+           "gpu_launches": 2 * (len(groups) if args.fused and tokens <= 4 else len(seq)) * steps, "impl": "lb"}
     print(json.dumps(out), flush=True)
 
 
@@ -623,6 +645,8 @@ def main(argv=None):
     ap.add_argument("--no-parity", action="store_true")
     ap.add_argument("--block", choices=sorted(BLOCKS), default=None,
                     help="time a whole decoder block's linears chained (tokens default 1)")
+    ap.add_argument("--fused", action="store_true",
+                    help="with --block: linears that share their input run as one siblings call")
     ap.add_argument("--dense-baseline", action="store_true",
                     help="also time a cuBLAS bf16 GEMM on the reconstructed dense weight (same tokens)")
     args = ap.parse_args(argv)

@@ -62,6 +62,15 @@ _lock = threading.Lock()
 _lib = None
 
 
+class LbProjection(ctypes.Structure):
+    """``lb_projection`` (include/lb.h): one layer of a group that shares x."""
+    _fields_ = [("n_out", ctypes.c_int64), ("main", ctypes.POINTER(LbPath)), ("residual", ctypes.POINTER(LbPath)),
+                ("y", ctypes.c_void_p), ("ldy", ctypes.c_int64)]
+
+
+MAX_SIBLINGS = 4
+
+
 def lib() -> ctypes.CDLL:
     """Load ``liblb.so`` (once).  Raises if it has not been built."""
     global _lib
@@ -96,6 +105,10 @@ def lib() -> ctypes.CDLL:
             L.lb_linear_forward_fixed_scratch.restype = i32
             L.lb_linear_forward_fixed_scratch.argtypes = [vp, i64, i64, i64, i64, ctypes.POINTER(LbPath),
                                                           ctypes.POINTER(LbPath), vp, i64, vp]
+            L.lb_siblings_workspace_bytes.restype = sz
+            L.lb_siblings_workspace_bytes.argtypes = [i64, i64, i32, ctypes.POINTER(LbProjection)]
+            L.lb_linear_forward_siblings.restype = i32
+            L.lb_linear_forward_siblings.argtypes = [vp, i64, i64, i64, i32, ctypes.POINTER(LbProjection), vp, sz, vp]
             L.lb_device_status.restype = i32
             L.lb_device_status.argtypes = [vp, ctypes.POINTER(i32)]
             _lib = L
@@ -221,6 +234,46 @@ def linear_forward(x, main: PackedPath, residual: PackedPath | None = None, y=No
         workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream)),
         "lb_linear_forward")
     return y
+
+
+def _projections(layers, ys):
+    """ctypes array of lb_projection for [(main, residual or None), ...] and
+    their outputs; the LbPath structs are returned too, to keep them alive."""
+    keep = []
+    arr = (LbProjection * len(layers))()
+    for j, ((main, residual), y) in enumerate(zip(layers, ys)):
+        cm = main.as_c()
+        cr = residual.as_c() if residual is not None else None
+        keep += [cm, cr]
+        arr[j].n_out = main.h.shape[0]
+        arr[j].main = ctypes.pointer(cm)
+        arr[j].residual = ctypes.pointer(cr) if cr is not None else None
+        arr[j].y = y.data_ptr() if y is not None else None
+        arr[j].ldy = y.stride(0) if y is not None else main.h.shape[0]
+    return arr, keep
+
+
+def siblings_workspace_bytes(tokens: int, n_in: int, layers) -> int:
+    arr, _keep = _projections(layers, [None] * len(layers))
+    return int(lib().lb_siblings_workspace_bytes(tokens, n_in, len(layers), arr))
+
+
+def linear_forward_siblings(x, layers, ys=None, workspace=None, stream=None):
+    """``lb_linear_forward_siblings``: several layers that read the same x,
+    given as [(main, residual or None), ...]; returns their outputs (bf16
+    [tokens, n_out_j]), allocated with torch when not given."""
+    torch = _torch()
+    tokens, n_in = x.shape
+    if ys is None:
+        ys = [torch.empty((tokens, main.h.shape[0]), dtype=torch.bfloat16, device=x.device) for main, _ in layers]
+    arr, _keep = _projections(layers, ys)
+    need = int(lib().lb_siblings_workspace_bytes(tokens, n_in, len(layers), arr))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    _check(lib().lb_linear_forward_siblings(
+        x.data_ptr(), tokens, n_in, x.stride(0), len(layers), arr, workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream_handle(stream)), "lb_linear_forward_siblings")
+    return ys
 
 
 def latent_forward(x, main: PackedPath, residual: PackedPath | None = None, z=None, stream=None):

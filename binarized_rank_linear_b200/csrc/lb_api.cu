@@ -270,6 +270,82 @@ lb_status lb_linear_forward(const uint16_t *x, int64_t tokens, int64_t n_in, int
     return LB_OK;
 }
 
+// Fills g from the caller's projections; checks everything a siblings call
+// checks on the host (sizes, pointers, alignment), not the workspace.
+static lb_status build_group(const uint16_t *x, int64_t tokens, int64_t n_in, int64_t ldx, int nproj,
+                             const lb_projection *proj, bool sizes_only, lb::GroupArgs *g)
+{
+    if (tokens < 0 || n_in <= 0 || nproj < 1 || nproj > LB_MAX_SIBLINGS || !proj) return LB_ERR_INVALID_ARGUMENT;
+    if (n_in % 32 != 0 || n_in > kMaxDim || tokens > kMaxTokens) return LB_ERR_UNSUPPORTED_SHAPE;
+    if (!sizes_only) {
+        if (!x || ldx < n_in) return LB_ERR_INVALID_ARGUMENT;
+        if (ldx % 8 != 0 || !aligned16(x)) return LB_ERR_MISALIGNED;
+    }
+    *g = lb::GroupArgs{};
+    g->x = x;
+    g->ldx = ldx;
+    g->tokens = (int)tokens;
+    g->n_in = (int)n_in;
+    g->nproj = nproj;
+    for (int j = 0; j < nproj; ++j) {
+        const lb_projection &pj = proj[j];
+        lb::ProjDesc &d = g->proj[j];
+        if (pj.n_out <= 0 || !pj.main) return LB_ERR_INVALID_ARGUMENT;
+        if (pj.n_out % 32 != 0 || pj.n_out > kMaxDim) return LB_ERR_UNSUPPORTED_SHAPE;
+        d.n_out = (int)pj.n_out;
+        d.npaths = pj.residual ? 2 : 1;
+        if (sizes_only) {
+            const lb_path *ps[2] = {pj.main, pj.residual};
+            for (int q = 0; q < d.npaths; ++q) {
+                if (ps[q]->rank <= 0) return LB_ERR_INVALID_ARGUMENT;
+                if (ps[q]->rank % 32 != 0 || ps[q]->rank > kMaxRank) return LB_ERR_UNSUPPORTED_SHAPE;
+                d.path[q].rank = (int)ps[q]->rank;
+            }
+            continue;
+        }
+        if (!pj.y || pj.ldy < pj.n_out) return LB_ERR_INVALID_ARGUMENT;
+        if (pj.ldy % 8 != 0 || !aligned16(pj.y)) return LB_ERR_MISALIGNED;
+        lb_status st = check_path(pj.main, n_in, pj.n_out, &d.path[0]);
+        if (st == LB_OK && pj.residual) st = check_path(pj.residual, n_in, pj.n_out, &d.path[1]);
+        if (st != LB_OK) return st;
+        d.y = pj.y;
+        d.ldy = pj.ldy;
+    }
+    return LB_OK;
+}
+
+size_t lb_siblings_workspace_bytes(int64_t tokens, int64_t n_in, int nproj, const lb_projection *proj)
+{
+    lb::GroupArgs g;
+    if (build_group(nullptr, tokens, n_in, n_in, nproj, proj, true, &g) != LB_OK || tokens == 0) return 0;
+    return lb::group_workspace_bytes(g);
+}
+
+lb_status lb_linear_forward_siblings(const uint16_t *x, int64_t tokens, int64_t n_in, int64_t ldx, int nproj,
+                                     const lb_projection *proj, void *workspace, size_t workspace_bytes,
+                                     void *stream)
+{
+    if (tokens < 0 || n_in <= 0 || nproj < 1 || nproj > LB_MAX_SIBLINGS || !proj) return LB_ERR_INVALID_ARGUMENT;
+    if (tokens == 0) return LB_OK;
+    lb::GroupArgs g;
+    lb_status st = build_group(x, tokens, n_in, ldx, nproj, proj, false, &g);
+    if (st != LB_OK) return st;
+    const size_t need = lb::group_workspace_bytes(g);
+    if (need > 0 && !workspace) return LB_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes < need) return LB_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace && !aligned16(workspace)) return LB_ERR_MISALIGNED;
+    g.workspace = workspace;
+    g.workspace_bytes = workspace_bytes;
+    lb::DeviceInfo dev;
+    st = device_info(&dev);
+    if (st != LB_OK) return st;
+    if (lb::group_forward(g, dev, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    return LB_OK;
+}
+
 lb_status lb_latent_forward(const uint16_t *x, int64_t tokens, int64_t n_in, int64_t ldx, const lb_path *main,
                             const lb_path *residual, uint16_t *z, int64_t ldz, void *stream)
 {

@@ -1,7 +1,7 @@
 // lb_decode.cu - the forward pass for 1..128 tokens: dispatch between the
 // CUDA-core path (1..4 tokens, lb_gemv.cu) and the tcgen05 path (5..128
-// tokens, lb_mid.cu).  Also the dispatch of either contraction on
-// its own (the split latent entry points).
+// tokens, lb_mid.cu).  Also the dispatch of either contraction on its own
+// (the split latent entry points) and of sibling projections that share x.
 //
 // The layer (sesamedisk.com, "Samsung LittleBit 13B Model", section "What the
 // method actually computes", Proposition 1) is computed by a pair of
@@ -23,23 +23,99 @@ cudaError_t decode_prepare_device(const DeviceInfo &dev)
     return e;
 }
 
+GroupArgs group_of_one(const ForwardArgs &a)
+{
+    GroupArgs g{};
+    g.x = a.x;
+    g.ldx = a.ldx;
+    g.tokens = a.tokens;
+    g.n_in = a.n_in;
+    g.nproj = 1;
+    g.proj[0].n_out = a.n_out;
+    g.proj[0].npaths = a.npaths;
+    g.proj[0].path[0] = a.path[0];
+    g.proj[0].path[1] = a.path[1];
+    g.proj[0].y = a.y;
+    g.proj[0].ldy = a.ldy;
+    g.workspace = a.workspace;
+    g.workspace_bytes = a.workspace_bytes;
+    return g;
+}
+
+ForwardArgs layer_of(const GroupArgs &g, int j)
+{
+    ForwardArgs a{};
+    a.x = g.x;
+    a.ldx = g.ldx;
+    a.tokens = g.tokens;
+    a.n_in = g.n_in;
+    a.n_out = g.proj[j].n_out;
+    a.npaths = g.proj[j].npaths;
+    a.path[0] = g.proj[j].path[0];
+    a.path[1] = g.proj[j].path[1];
+    a.y = g.proj[j].y;
+    a.ldy = g.proj[j].ldy;
+    a.workspace = g.workspace;
+    a.workspace_bytes = g.workspace_bytes;
+    return a;
+}
+
+namespace {
+
+// A group of one layer with only the sizes filled in (enough for workspace sizes).
+GroupArgs sizes_only(int tokens, int n_in, int n_out, const int *ranks, int npaths)
+{
+    ForwardArgs a{};
+    a.tokens = tokens;
+    a.n_in = n_in;
+    a.n_out = n_out;
+    a.npaths = npaths;
+    a.path[0].rank = ranks[0];
+    a.path[1].rank = npaths > 1 ? ranks[1] : 0;
+    return group_of_one(a);
+}
+
+size_t layer_workspace_bytes(const ForwardArgs &a)
+{
+    const int ranks[2] = {a.path[0].rank, a.npaths > 1 ? a.path[1].rank : 0};
+    return a.tokens > kMidMaxTokens ? prefill_workspace_bytes(a.tokens, ranks, a.npaths)
+                                    : decode_workspace_bytes(a.tokens, a.n_in, a.n_out, ranks, a.npaths);
+}
+
+}  // namespace
+
 size_t decode_workspace_bytes(int tokens, int n_in, int n_out, const int *ranks, int npaths)
 {
-    (void)n_in;
-    (void)n_out;
     const int M = std::min(tokens, kMidMaxTokens);
     return std::max(mid_workspace_bytes(M, ranks, npaths),
-                    small_workspace_bytes(std::min(M, kSmallMaxTokens), ranks, npaths));
+                    small_workspace_bytes(std::min(M, kSmallMaxTokens), sizes_only(M, n_in, n_out, ranks, npaths)));
 }
 
 cudaError_t decode_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream)
 {
-    const int ranks[2] = {a.path[0].rank, a.npaths > 1 ? a.path[1].rank : 0};
+    const GroupArgs g = group_of_one(a);
     for (int m0 = 0; m0 < a.tokens; m0 += kMidMaxTokens) {
         const int M = std::min(kMidMaxTokens, a.tokens - m0);
-        const cudaError_t e = M <= kSmallMaxTokens && small_fits(M, a.n_in, a.n_out, ranks, a.npaths, dev)
-                                  ? small_forward(a, dev, stream, m0, M)
-                                  : mid_forward(a, dev, stream, m0, M);
+        const cudaError_t e = M <= kSmallMaxTokens && small_fits(M, g, dev) ? small_forward(g, dev, stream, m0, M)
+                                                                             : mid_forward(a, dev, stream, m0, M);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+size_t group_workspace_bytes(const GroupArgs &g)
+{
+    size_t need = g.tokens <= kSmallMaxTokens ? small_workspace_bytes(g.tokens, g) : 0;
+    for (int j = 0; j < g.nproj; ++j) need = std::max(need, layer_workspace_bytes(layer_of(g, j)));
+    return need;
+}
+
+cudaError_t group_forward(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream)
+{
+    if (g.tokens <= kSmallMaxTokens && small_fits(g.tokens, g, dev)) return small_forward(g, dev, stream, 0, g.tokens);
+    for (int j = 0; j < g.nproj; ++j) {
+        const ForwardArgs a = layer_of(g, j);
+        const cudaError_t e = a.tokens > kMidMaxTokens ? prefill_forward(a, dev, stream) : decode_forward(a, dev, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -70,19 +70,25 @@ __device__ __forceinline__ void load_words(uint32_t (&w)[kWW], const uint32_t *s
 }
 
 // ============================================================ contraction 1
+// One path of the group (all paths read the same x): its 32-row latent
+// blocks are blocks blk0 .. of the grid's block sequence, and its latents are
+// rows koff .. of z.
+struct S1Path {
+    const uint32_t *vt;
+    int64_t vt_ld;
+    const uint16_t *g, *l;
+    int blk0, koff;
+};
 struct Small1Params {
     const uint16_t *x;
     int64_t ldx;
     int M, W;  // tokens; words of n_in
-    const uint32_t *vt0, *vt1;
-    int64_t vt_ld0, vt_ld1;
-    const uint16_t *g0, *g1, *l0, *l1;
-    int rank0, rank1;
-    int blocks0;  // 32-row blocks of path 0 (path 1's follow)
-    int cs;       // CTAs across n_in: one cluster, whose first CTA sums the partials
-    int ww;       // words per warp (<= kWW)
-    int early;    // release the dependent launch at entry instead of after the lookups
-    float *z;     // z [R][M], l applied
+    int npaths;
+    S1Path path[2 * kMaxSiblings];  // in block order
+    int cs;     // CTAs across n_in: one cluster, whose first CTA sums the partials
+    int ww;     // words per warp (<= kWW)
+    int early;  // release the dependent launch at entry instead of after the lookups
+    float *z;   // z [R][M] over all paths, l applied
 };
 
 // CTA = 32 latent rows (one path) x (warps * ww) words of n_in.  When n_in is
@@ -91,15 +97,18 @@ struct Small1Params {
 // shared memory), and after one cluster barrier the first CTA adds them in
 // cluster-rank order.
 template <int MT>
-__global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const Small1Params p)
+__global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const __grid_constant__ Small1Params p)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nthr = blockDim.x, nwarps = nthr >> 5;
     const int M = p.M;
     const int blk = blockIdx.x / p.cs, split = blockIdx.x - blk * p.cs;
-    const bool second = blk >= p.blocks0;
-    const int row0 = (second ? blk - p.blocks0 : blk) * 32;  // within the path
+    int pi = 0;  // the path of this row block
+    for (int q = 1; q < p.npaths; ++q)
+        if (blk >= p.path[q].blk0) pi = q;
+    const S1Path &P = p.path[pi];
+    const int row0 = (blk - P.blk0) * 32;  // within the path
     const int cww = nwarps * p.ww;                           // words per CTA
     const int c0 = split * cww, c1 = min(p.W, c0 + cww);
     const int wa = c0 + warp * p.ww;
@@ -111,10 +120,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const Small1Para
     // row0 + lane, words wa ..) into registers; the CTA's slice of g and l of
     // its rows into shared memory with asynchronous copies
     uint32_t bw[kWW];
-    {
-        const int64_t ld = second ? p.vt_ld1 : p.vt_ld0;
-        load_words(bw, (second ? p.vt1 : p.vt0) + (int64_t)(row0 + lane) * ld + wa, nwd);
-    }
+    load_words(bw, P.vt + (int64_t)(row0 + lane) * P.vt_ld + wa, nwd);
     const int ntab = 8 * (c1 - c0);
     float4 *tab = reinterpret_cast<float4 *>(smem);  // [M][cww * 8][kTab / 4]
     float *red = reinterpret_cast<float *>(smem) + (size_t)M * cww * 8 * kTab;  // [warps][32][MT]
@@ -122,9 +128,9 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const Small1Para
     uint16_t *gsm = reinterpret_cast<uint16_t *>(part + kMaxCluster * 32 * MT);  // [cww * 32]
     uint16_t *lsm = gsm + cww * 32;                                              // [32]
     {
-        const uint16_t *g = (second ? p.g1 : p.g0) + 32 * c0;
+        const uint16_t *g = P.g + 32 * c0;
         for (int e = tid; e < 4 * (c1 - c0); e += nthr) cp_async16(gsm + 8 * e, g + 8 * e);
-        if (tid < 4) cp_async16(lsm + 8 * tid, (second ? p.l1 : p.l0) + row0 + 8 * tid);
+        if (tid < 4) cp_async16(lsm + 8 * tid, P.l + row0 + 8 * tid);
         cp_async_commit();
     }
     if (p.early) pdl_launch_dependents();
@@ -176,7 +182,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const Small1Para
 #pragma unroll
     for (int m = 0; m < MT; ++m) red[(warp * 32 + lane) * MT + m] = acc[m] + acc2[m];
     __syncthreads();
-    const int kg0 = (second ? p.rank0 : 0) + row0;
+    const int kg0 = P.koff + row0;
     if (p.cs > 1) cluster_wait();  // every CTA of the cluster is running
     for (int e = tid; e < 32 * M; e += nthr) {
         const int r = e / M, m = e - r * M;
@@ -199,33 +205,48 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const Small1Para
 }
 
 // ============================================================ contraction 2
-struct Small2Params {
-    const float *z;  // [R][M], l applied
-    int M, n_out;
+// One projection of the group: its rows, its paths' U and h, where its
+// latents sit in z, the first CTA of its share of the grid, and its output.
+struct S2Proj {
     const uint32_t *u0, *u1;
     int64_t u_ld0, u_ld1;
-    const uint16_t *h0, *h1;
-    int rank0, rank1;
-    int ks;     // warps per 32-row block (each takes ww words of the latent)
-    int ww;     // latent words per warp (<= kWW)
-    int early;  // release the dependent launch at entry instead of after the lookups
+    const uint16_t *h0, *h1;  // h1 null without a residual path
+    int n_out;
+    int W0, WT;  // latent words of path 0; of both paths
+    int koff;    // first latent row of the projection in z
+    int cta0;    // first CTA of the projection
     uint16_t *y;
     int64_t ldy;
 };
+struct Small2Params {
+    const float *z;  // [R][M] over all paths, l applied
+    int M;
+    int nproj;
+    S2Proj proj[kMaxSiblings];  // in CTA order
+    int ks;     // warps per 32-row block (each takes ww words of the latent)
+    int ww;     // latent words per warp (<= kWW)
+    int early;  // release the dependent launch at entry instead of after the lookups
+};
 
-// CTA = (warps / ks) blocks of 32 output rows; the ks warps of a block split
-// the latent words of both paths (path 0 first).
+// CTA = (warps / ks) blocks of 32 output rows of one projection; the ks warps
+// of a block split the latent words of the projection's paths (path 0 first).
+// Warps past the projection's latent words (a sibling may have fewer) idle.
 template <int MT>
-__global__ void __launch_bounds__(kMaxWarps * 32) small2_kernel(const Small2Params p)
+__global__ void __launch_bounds__(kMaxWarps * 32) small2_kernel(const __grid_constant__ Small2Params p)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nthr = blockDim.x, nwarps = nthr >> 5;
     const int M = p.M;
+    int qi = 0;  // the projection of this CTA
+    for (int q = 1; q < p.nproj; ++q)
+        if ((int)blockIdx.x >= p.proj[q].cta0) qi = q;
+    const S2Proj &P = p.proj[qi];
+    const int lc = blockIdx.x - P.cta0;  // CTA within the projection
     const int rb = nwarps / p.ks, rbi = warp / p.ks, kw = warp - rbi * p.ks;
-    const int o = (blockIdx.x * rb + rbi) * 32 + lane;  // output row
-    const bool rowok = o < p.n_out;                     // whole warps: n_out is a multiple of 32
-    const int R = p.rank0 + p.rank1, WT = R >> 5, W0 = p.rank0 >> 5;
+    const int o = (lc * rb + rbi) * 32 + lane;  // output row
+    const bool rowok = o < P.n_out;             // whole warps: n_out is a multiple of 32
+    const int WT = P.WT, W0 = P.W0;
     const int wa = kw * p.ww;
     const int nwd = rowok ? max(0, min(WT, wa + p.ww) - wa) : 0;
 
@@ -233,35 +254,36 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small2_kernel(const Small2Para
     uint32_t bw[kWW];
     if (wa >= W0 || wa + nwd <= W0) {  // one path
         const bool sec = wa >= W0;
-        const uint32_t *src = sec ? p.u1 + (int64_t)o * p.u_ld1 + (wa - W0) : p.u0 + (int64_t)o * p.u_ld0 + wa;
-        load_words(bw, nwd > 0 ? src : p.u0, nwd);
+        const uint32_t *src = sec ? P.u1 + (int64_t)o * P.u_ld1 + (wa - W0) : P.u0 + (int64_t)o * P.u_ld0 + wa;
+        load_words(bw, nwd > 0 ? src : P.u0, nwd);
     } else {
 #pragma unroll
         for (int j = 0; j < kWW; ++j) {
             const int w = wa + j;
-            bw[j] = j < nwd ? ldg_early_u32(w < W0 ? p.u0 + (int64_t)o * p.u_ld0 + w
-                                                   : p.u1 + (int64_t)o * p.u_ld1 + (w - W0))
+            bw[j] = j < nwd ? ldg_early_u32(w < W0 ? P.u0 + (int64_t)o * P.u_ld0 + w
+                                                   : P.u1 + (int64_t)o * P.u_ld1 + (w - W0))
                             : 0u;
         }
     }
     float h0 = 0.f, h1 = 0.f;
     if (rowok && kw == 0) {
-        h0 = f16_bits_to_float(ldg_early_u16(p.h0 + o));
-        if (p.h1) h1 = f16_bits_to_float(ldg_early_u16(p.h1 + o));
+        h0 = f16_bits_to_float(ldg_early_u16(P.h0 + o));
+        if (P.h1) h1 = f16_bits_to_float(ldg_early_u16(P.h1 + o));
     }
     if (p.early) pdl_launch_dependents();
 
-    // (2) the latent comes from the previous kernel: tables of z over both
-    // paths (path 0 first)
+    // (2) the latent comes from the previous kernel: tables of the
+    // projection's z over both its paths (path 0 first)
     pdl_wait();
     const int ntab = 8 * WT;
     float4 *tab = reinterpret_cast<float4 *>(smem);  // [M][WT * 8][kTab / 4]
+    const float *zp = p.z + (int64_t)P.koff * M;
     for (int e = tid; e < ntab * M; e += nthr) {
         const int m = e / ntab, t = e - m * ntab;
         const int k = 4 * t;
         float v[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = __ldg(p.z + (int64_t)(k + j) * M + m);
+        for (int j = 0; j < 4; ++j) v[j] = __ldg(zp + (int64_t)(k + j) * M + m);
         nibble_table(v[0], v[1], v[2], v[3], tab + (kTab / 4) * (m * ntab + t));
     }
     __syncthreads();
@@ -309,8 +331,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small2_kernel(const Small2Para
     __syncthreads();
     for (int e = tid; e < rb * 32 * M; e += nthr) {
         const int r = e & 31, rm = e >> 5, b = rm / M, m = rm - b * M;
-        const int oo = (blockIdx.x * rb + b) * 32 + r;
-        if (oo >= p.n_out) continue;
+        const int oo = (lc * rb + b) * 32 + r;
+        if (oo >= P.n_out) continue;
         float s0 = 0.f, s1 = 0.f;
         for (int w = 0; w < p.ks; ++w) {
             const int ww_ = b * p.ks + w;
@@ -318,7 +340,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small2_kernel(const Small2Para
             s1 += red[((ww_ * 32 + r) * 2 + 1) * MT + m];
         }
         const float yv = hs[(b * 32 + r) * 2 + 0] * s0 + hs[(b * 32 + r) * 2 + 1] * s1;
-        p.y[(int64_t)m * p.ldy + oo] = float_to_bf16_bits(yv);
+        P.y[(int64_t)m * P.ldy + oo] = float_to_bf16_bits(yv);
     }
 }
 
@@ -368,10 +390,14 @@ Small1Plan plan_small1(int M, int MT, int n_in, int R, const DeviceInfo &dev)
 }
 
 // Contraction 2: ks warps cover a row's latent words (8 per warp, 4 if that
-// leaves SMs idle); as many row blocks per CTA as keep one CTA per SM.
-Small2Plan plan_small2(int M, int MT, int n_out, int R, const DeviceInfo &dev)
+// leaves SMs idle; sized for the projection with the widest latent); as many
+// row blocks per CTA as keep one CTA per SM.  A CTA's row blocks belong to one
+// projection.
+Small2Plan plan_small2(int M, int MT, const GroupArgs &g, const DeviceInfo &dev)
 {
-    const int WT = R / 32, blocks = n_out / 32;
+    int WT = 0;
+    for (int j = 0; j < g.nproj; ++j)
+        WT = std::max(WT, (g.proj[j].path[0].rank + (g.proj[j].npaths > 1 ? g.proj[j].path[1].rank : 0)) / 32);
     Small2Plan best;
     for (int ww : {8, 4, 2}) {
         const int ks = (WT + ww - 1) / ww;
@@ -382,7 +408,8 @@ Small2Plan plan_small2(int M, int MT, int n_out, int R, const DeviceInfo &dev)
             pl.warps = ks * rb;
             pl.ks = ks;
             pl.ww = ww;
-            pl.ctas = (blocks + rb - 1) / rb;
+            pl.ctas = 0;
+            for (int j = 0; j < g.nproj; ++j) pl.ctas += (g.proj[j].n_out / 32 + rb - 1) / rb;
             pl.smem = small2_smem(pl.warps, WT, M, MT);
             if (pl.smem > (size_t)dev.max_smem_optin) continue;
             if (pl.ctas >= dev.sm_count) return pl;
@@ -392,52 +419,69 @@ Small2Plan plan_small2(int M, int MT, int n_out, int R, const DeviceInfo &dev)
     return best;
 }
 
-template <int MT>
-cudaError_t launch_small(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M)
+int group_rank(const GroupArgs &g)
 {
-    const int R = a.path[0].rank + (a.npaths > 1 ? a.path[1].rank : 0);
-    const Small1Plan p1 = plan_small1(M, MT, a.n_in, R, dev);
+    int R = 0;
+    for (int j = 0; j < g.nproj; ++j)
+        for (int q = 0; q < g.proj[j].npaths; ++q) R += g.proj[j].path[q].rank;
+    return R;
+}
+
+template <int MT>
+cudaError_t launch_small(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream, int m0, int M)
+{
+    const int R = group_rank(g);
+    const Small1Plan p1 = plan_small1(M, MT, g.n_in, R, dev);
     if (p1.ctas == 0) return cudaErrorInvalidConfiguration;
-    const Small2Plan p2 = plan_small2(M, MT, a.n_out, R, dev);
+    const Small2Plan p2 = plan_small2(M, MT, g, dev);
     if (p2.ctas == 0) return cudaErrorInvalidConfiguration;
 
+    // the latent of every path of every projection, in projection order
     Small1Params L{};
-    L.x = a.x + (int64_t)m0 * a.ldx;
-    L.ldx = a.ldx;
+    L.x = g.x + (int64_t)m0 * g.ldx;
+    L.ldx = g.ldx;
     L.M = M;
-    L.W = a.n_in / 32;
-    L.vt0 = a.path[0].vt_bits;
-    L.vt_ld0 = a.path[0].vt_ld;
-    L.g0 = a.path[0].g;
-    L.l0 = a.path[0].l;
-    L.rank0 = a.path[0].rank;
-    if (a.npaths > 1) {
-        L.vt1 = a.path[1].vt_bits;
-        L.vt_ld1 = a.path[1].vt_ld;
-        L.g1 = a.path[1].g;
-        L.l1 = a.path[1].l;
-        L.rank1 = a.path[1].rank;
+    L.W = g.n_in / 32;
+    Small2Params E{};
+    E.z = static_cast<const float *>(g.workspace);
+    E.M = M;
+    E.nproj = g.nproj;
+    int koff = 0, cta0 = 0;
+    const int rb = p2.warps / p2.ks;
+    for (int j = 0; j < g.nproj; ++j) {
+        const ProjDesc &pj = g.proj[j];
+        S2Proj &e = E.proj[j];
+        e.u0 = pj.path[0].u_bits;
+        e.u_ld0 = pj.path[0].u_ld;
+        e.h0 = pj.path[0].h;
+        if (pj.npaths > 1) {
+            e.u1 = pj.path[1].u_bits;
+            e.u_ld1 = pj.path[1].u_ld;
+            e.h1 = pj.path[1].h;
+        }
+        e.n_out = pj.n_out;
+        e.W0 = pj.path[0].rank / 32;
+        e.WT = e.W0 + (pj.npaths > 1 ? pj.path[1].rank / 32 : 0);
+        e.koff = koff;
+        e.cta0 = cta0;
+        e.y = pj.y + (int64_t)m0 * pj.ldy;
+        e.ldy = pj.ldy;
+        cta0 += (pj.n_out / 32 + rb - 1) / rb;
+        for (int q = 0; q < pj.npaths; ++q) {
+            S1Path &v = L.path[L.npaths++];
+            v.vt = pj.path[q].vt_bits;
+            v.vt_ld = pj.path[q].vt_ld;
+            v.g = pj.path[q].g;
+            v.l = pj.path[q].l;
+            v.blk0 = koff / 32;
+            v.koff = koff;
+            koff += pj.path[q].rank;
+        }
     }
-    L.blocks0 = a.path[0].rank / 32;
     L.cs = p1.cs;
     L.ww = p1.ww;
     L.early = 0;
-    L.z = static_cast<float *>(a.workspace);
-
-    Small2Params E{};
-    E.z = static_cast<const float *>(a.workspace);
-    E.M = M;
-    E.n_out = a.n_out;
-    E.u0 = a.path[0].u_bits;
-    E.u_ld0 = a.path[0].u_ld;
-    E.h0 = a.path[0].h;
-    E.rank0 = a.path[0].rank;
-    if (a.npaths > 1) {
-        E.u1 = a.path[1].u_bits;
-        E.u_ld1 = a.path[1].u_ld;
-        E.h1 = a.path[1].h;
-        E.rank1 = a.path[1].rank;
-    }
+    L.z = static_cast<float *>(g.workspace);
     E.ks = p2.ks;
     E.ww = p2.ww;
     // Releasing the next kernel on the stream (the next layer's contraction
@@ -445,8 +489,6 @@ cudaError_t launch_small(const ForwardArgs &a, const DeviceInfo &dev, cudaStream
     // then compete for SMs: measured faster when this grid is light (at most
     // 8 warps per SM), slower when it is not.
     E.early = (int64_t)p2.ctas * p2.warps <= 8 * (int64_t)dev.sm_count ? 1 : 0;
-    E.y = a.y + (int64_t)m0 * a.ldy;
-    E.ldy = a.ldy;
 
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -490,25 +532,23 @@ cudaError_t small_prepare_device(const DeviceInfo &dev)
     return e;
 }
 
-size_t small_workspace_bytes(int M, const int *ranks, int npaths)
+size_t small_workspace_bytes(int M, const GroupArgs &g)
 {
-    const size_t R = (size_t)ranks[0] + (npaths > 1 ? ranks[1] : 0);
-    return std::max(R * (size_t)M * 4, kMaxPartialBytes);
+    return std::max((size_t)group_rank(g) * (size_t)M * 4, kMaxPartialBytes);
 }
 
-bool small_fits(int M, int n_in, int n_out, const int *ranks, int npaths, const DeviceInfo &dev)
+bool small_fits(int M, const GroupArgs &g, const DeviceInfo &dev)
 {
-    const int R = ranks[0] + (npaths > 1 ? ranks[1] : 0);
     const int MT = M <= 1 ? 1 : (M <= 2 ? 2 : 4);
-    const Small1Plan p1 = plan_small1(M, MT, n_in, R, dev);
-    return p1.ctas > 0 && plan_small2(M, MT, n_out, R, dev).ctas > 0;
+    const Small1Plan p1 = plan_small1(M, MT, g.n_in, group_rank(g), dev);
+    return p1.ctas > 0 && plan_small2(M, MT, g, dev).ctas > 0;
 }
 
-cudaError_t small_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M)
+cudaError_t small_forward(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream, int m0, int M)
 {
-    if (M <= 1) return launch_small<1>(a, dev, stream, m0, M);
-    if (M <= 2) return launch_small<2>(a, dev, stream, m0, M);
-    return launch_small<4>(a, dev, stream, m0, M);
+    if (M <= 1) return launch_small<1>(g, dev, stream, m0, M);
+    if (M <= 2) return launch_small<2>(g, dev, stream, m0, M);
+    return launch_small<4>(g, dev, stream, m0, M);
 }
 
 }  // namespace lb

@@ -45,21 +45,51 @@ struct ForwardArgs {
     size_t workspace_bytes;
 };
 
+// Sibling projections: layers that share x (lb_linear_forward_siblings),
+// each with its own paths, output width and output buffer.
+constexpr int kMaxSiblings = LB_MAX_SIBLINGS;
+struct ProjDesc {
+    int n_out;
+    int npaths;
+    PathDesc path[2];
+    uint16_t *y;
+    int64_t ldy;
+};
+struct GroupArgs {
+    const uint16_t *x;
+    int64_t ldx;
+    int tokens;
+    int n_in;
+    int nproj;
+    ProjDesc proj[kMaxSiblings];
+    void *workspace;
+    size_t workspace_bytes;
+};
+// The single-layer call as a group of one.
+GroupArgs group_of_one(const ForwardArgs &a);
+// The layer of projection j alone, for the paths that run one layer at a time.
+ForwardArgs layer_of(const GroupArgs &g, int j);
+
 // Decode path (up to kMidMaxTokens tokens per launch pair; lb_decode.cu).
 // Up to kSmallMaxTokens tokens run on CUDA cores (nibble tables, lb_gemv.cu)
 // when the shapes fit it, the rest on tcgen05 (lb_mid.cu).  kDecodeMaxTokens
 // bounds the fixed-scratch entry point.
 constexpr int kSmallMaxTokens = 4;
-size_t small_workspace_bytes(int M, const int *ranks, int npaths);
-cudaError_t small_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M);
+size_t small_workspace_bytes(int M, const GroupArgs &g);
+// One launch pair for the whole group (a single layer is a group of one).
+cudaError_t small_forward(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream, int m0, int M);
 // False when the shapes do not fit the small path (its latent tables must fit
 // shared memory); the tensor-core decode path takes those.
-bool small_fits(int M, int n_in, int n_out, const int *ranks, int npaths, const DeviceInfo &dev);
+bool small_fits(int M, const GroupArgs &g, const DeviceInfo &dev);
 cudaError_t small_prepare_device(const DeviceInfo &dev);
 constexpr int kDecodeMaxTokens = 32;
 size_t decode_workspace_bytes(int tokens, int n_in, int n_out, const int *ranks, int npaths);
 cudaError_t decode_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 cudaError_t decode_prepare_device(const DeviceInfo &dev);
+// A group of siblings at any token count: one small-path launch pair for the
+// group when it fits, else each projection's own layer path in turn.
+size_t group_workspace_bytes(const GroupArgs &g);
+cudaError_t group_forward(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream);
 
 // Up to kMidMaxTokens tokens per launch pair on tcgen05 with the sign matrix
 // as the 128-row MMA operand and the tokens as N (lb_mid.cu).

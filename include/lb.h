@@ -211,6 +211,49 @@ LB_API lb_status lb_expand_forward(const uint16_t *z, int64_t tokens, int64_t n_
                             const lb_path *main, const lb_path *residual, uint16_t *y, int64_t ldy,
                             void *stream);
 
+/* ---------------------------------------------------------- sibling projections
+ * Several layers that read the same input x, computed together: the query,
+ * key and value projections of an attention block, or the gate and up
+ * projections of an MLP.  Each is a LittleBit layer of its own (its own
+ * factors, scales, ranks and output width; Proposition 1 of sesamedisk.com,
+ * "Samsung LittleBit 13B Model", section "What the method actually
+ * computes"); grouping them changes only how the work is launched, so that a
+ * decoder block pays the launch and dependency latency once per group
+ * instead of once per layer (littlebitllm.com, "How small": the speed claims
+ * are per layer on a memory-bound decode).
+ *
+ * lb_projection: one layer of the group.
+ *   n_out    : its output width (positive multiple of 32)
+ *   main, residual : its paths, as for lb_linear_forward (residual may be NULL)
+ *   y, ldy   : its output, device bf16 [tokens x ldy], ldy >= n_out, a multiple
+ *              of 8, 16-byte aligned; written, never read.
+ * lb_linear_forward_siblings: for every projection j,
+ *     y_j = sum over its paths p of h_p (.) sign(U_p)(l_p (.) sign(V_p)^T (g_p (.) x)),
+ *   the result of lb_linear_forward on x and that projection alone, with the
+ *   same numerics (1..4 tokens: fp32 throughout on CUDA cores; more tokens:
+ *   the tensor-core numerics of lb_linear_forward).  The output buffers must
+ *   not overlap each other, x or the workspace.
+ *   nproj: 1 .. LB_MAX_SIBLINGS.  1..4 tokens run as one pair of launches for
+ *   the whole group; more tokens run each projection's own launches in turn.
+ *   workspace: at least lb_siblings_workspace_bytes(...) bytes, 16-byte
+ *   aligned, as for lb_linear_forward.
+ * Errors as lb_linear_forward; additionally LB_ERR_INVALID_ARGUMENT for a bad
+ *   nproj or a null proj.  Nothing is launched on an error found on the host. */
+#define LB_MAX_SIBLINGS 4
+typedef struct {
+    int64_t n_out;
+    const lb_path *main;
+    const lb_path *residual;
+    uint16_t *y;
+    int64_t ldy;
+} lb_projection;
+
+/* Workspace for lb_linear_forward_siblings; 0 on a bad argument. */
+LB_API size_t lb_siblings_workspace_bytes(int64_t tokens, int64_t n_in, int nproj, const lb_projection *proj);
+LB_API lb_status lb_linear_forward_siblings(const uint16_t *x, int64_t tokens, int64_t n_in, int64_t ldx,
+                                     int nproj, const lb_projection *proj, void *workspace,
+                                     size_t workspace_bytes, void *stream);
+
 /* ---------------------------------------------------------- fixed scratch
  * lb_linear_forward_fixed_scratch: lb_linear_forward for 1..32 tokens with
  * no workspace argument.  The pages have no counterpart; this is a service of

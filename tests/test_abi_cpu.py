@@ -198,3 +198,63 @@ def test_split_halves_reject_bad_arguments_before_any_cuda_call(L):
     assert exp(n_out=48, ldy=48) == lb.LB_ERR_UNSUPPORTED_SHAPE
     assert exp(main=fake_path(h=0)) == lb.LB_ERR_INVALID_ARGUMENT  # the U half is required
     assert exp(main=fake_path(u_bits=FAKE + 4)) == lb.LB_ERR_MISALIGNED
+
+
+def siblings(L, projs=None, nproj=None, x=FAKE, tokens=1, n_in=256, ldx=256, ws=FAKE, ws_bytes=1 << 20):
+    """lb_linear_forward_siblings over fake projections [(n_out, main, residual, y, ldy), ...]."""
+    projs = [(256, fake_path(), None, FAKE, 256), (96, fake_path(64), fake_path(), FAKE, 96)] if projs is None else projs
+    arr = (lb.LbProjection * max(1, len(projs)))()
+    keep = []
+    for j, (n_out, main, res, y, ldy) in enumerate(projs):
+        keep += [main, res]
+        arr[j].n_out, arr[j].y, arr[j].ldy = n_out, y, ldy
+        arr[j].main = ctypes.pointer(main) if main is not None else None
+        arr[j].residual = ctypes.pointer(res) if res is not None else None
+    return L.lb_linear_forward_siblings(x, tokens, n_in, ldx, len(projs) if nproj is None else nproj,
+                                        arr, ws, ws_bytes, None)
+
+
+def test_siblings_reject_bad_arguments_before_any_cuda_call(L):
+    assert siblings(L, tokens=0, x=0) == lb.LB_OK                       # no-op
+    assert siblings(L, tokens=-1) == lb.LB_ERR_INVALID_ARGUMENT
+    assert siblings(L, nproj=0) == lb.LB_ERR_INVALID_ARGUMENT
+    assert siblings(L, nproj=lb.MAX_SIBLINGS + 1) == lb.LB_ERR_INVALID_ARGUMENT
+    assert siblings(L, x=0) == lb.LB_ERR_INVALID_ARGUMENT
+    assert siblings(L, x=FAKE + 2) == lb.LB_ERR_MISALIGNED
+    assert siblings(L, n_in=250, ldx=256) == lb.LB_ERR_UNSUPPORTED_SHAPE
+    bad = lambda **kw: [(256, fake_path(), None, FAKE, 256), (kw.get("n_out", 96), kw.get("main", fake_path()),
+                                                             kw.get("res", None), kw.get("y", FAKE), kw.get("ldy", 96))]
+    assert siblings(L, bad(n_out=100, ldy=104)) == lb.LB_ERR_UNSUPPORTED_SHAPE
+    assert siblings(L, bad(main=None)) == lb.LB_ERR_INVALID_ARGUMENT
+    assert siblings(L, bad(y=0)) == lb.LB_ERR_INVALID_ARGUMENT
+    assert siblings(L, bad(y=FAKE + 2)) == lb.LB_ERR_MISALIGNED
+    assert siblings(L, bad(ldy=64)) == lb.LB_ERR_INVALID_ARGUMENT
+    assert siblings(L, bad(ldy=100)) == lb.LB_ERR_MISALIGNED
+    assert siblings(L, bad(main=fake_path(rank=48))) == lb.LB_ERR_UNSUPPORTED_SHAPE
+    assert siblings(L, bad(res=fake_path(h=0))) == lb.LB_ERR_INVALID_ARGUMENT
+    assert siblings(L, ws_bytes=16) == lb.LB_ERR_WORKSPACE_TOO_SMALL
+    assert siblings(L, ws=0) == lb.LB_ERR_INVALID_ARGUMENT
+    assert siblings(L, ws=FAKE + 8) == lb.LB_ERR_MISALIGNED
+
+
+def test_siblings_workspace_covers_each_layer_and_the_group(L):
+    """The group's workspace is at least each projection's own (the paths
+    that run one layer at a time) and, for 1..4 tokens, the fp32 latent of
+    every path of the group."""
+    q, kv = synth.CONFIGS["qwen3_14b_qo"], synth.CONFIGS["qwen3_14b_kv"]
+    layers = [(q.n_out, q.rank), (kv.n_out, kv.rank), (kv.n_out, kv.rank)]
+    arr = (lb.LbProjection * 3)()
+    keep = []
+    for j, (n_out, r) in enumerate(layers):
+        m, res = fake_path(r), fake_path(r)
+        keep += [m, res]
+        arr[j].n_out, arr[j].main, arr[j].residual = n_out, ctypes.pointer(m), ctypes.pointer(res)
+    for tokens in (1, 4, 5, 40, 300):
+        need = L.lb_siblings_workspace_bytes(tokens, q.n_in, 3, arr)
+        for n_out, r in layers:
+            assert need >= lb.forward_workspace_bytes(tokens, q.n_in, n_out, r, r)
+        if tokens <= 4:
+            assert need >= 4 * tokens * sum(2 * r for _, r in layers)
+    assert L.lb_siblings_workspace_bytes(0, q.n_in, 3, arr) == 0
+    assert L.lb_siblings_workspace_bytes(1, q.n_in, 0, arr) == 0
+    assert L.lb_siblings_workspace_bytes(1, 250, 3, arr) == 0

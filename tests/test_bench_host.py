@@ -77,8 +77,10 @@ def test_blocks_are_the_models_linears():
     """--block: every entry names a workload of the table, and the linears'
     shapes chain as a decoder block does (attention in -> model width, MLP
     up -> intermediate width, down -> model width)."""
-    for name, seq in bench.BLOCKS.items():
-        linears = [synth.CONFIGS[w] for w, n in seq for _ in range(n)]
+    for name, groups in bench.BLOCKS.items():
+        linears = [synth.CONFIGS[w] for grp in groups for w in grp]
+        for grp in groups:                                        # a group shares its input
+            assert len({synth.CONFIGS[w].n_in for w in grp}) == 1 and len(grp) <= 4
         assert len(linears) == 7
         width = linears[0].n_in
         assert all(c.n_in == width for c in linears[:3])           # q, k, v read the block input
