@@ -79,12 +79,13 @@ struct S1Path {
     const uint16_t *g, *l;
     int blk0, koff;
 };
+template <int NP>  // path slots: 2 for one layer, 2 kMaxSiblings for a group
 struct Small1Params {
     const uint16_t *x;
     int64_t ldx;
     int M, W;  // tokens; words of n_in
     int npaths;
-    S1Path path[2 * kMaxSiblings];  // in block order
+    S1Path path[NP];  // in block order
     int cs;     // CTAs across n_in: one cluster, whose first CTA sums the partials
     int ww;     // words per warp (<= kWW)
     int early;  // release the dependent launch at entry instead of after the lookups
@@ -96,18 +97,21 @@ struct Small1Params {
 // each stores its partial sums into the first CTA's shared memory (distributed
 // shared memory), and after one cluster barrier the first CTA adds them in
 // cluster-rank order.
-template <int MT>
-__global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const __grid_constant__ Small1Params p)
+template <int MT, int NP>
+__global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const __grid_constant__ Small1Params<NP> p)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nthr = blockDim.x, nwarps = nthr >> 5;
     const int M = p.M;
     const int blk = blockIdx.x / p.cs, split = blockIdx.x - blk * p.cs;
-    int pi = 0;  // the path of this row block
-    for (int q = 1; q < p.npaths; ++q)
-        if (blk >= p.path[q].blk0) pi = q;
-    const S1Path &P = p.path[pi];
+    // the path of this row block, selected field by field from fixed
+    // parameter offsets: every load is independent of the block index, so
+    // none waits for another before the weight loads can start
+    S1Path P = p.path[0];
+#pragma unroll
+    for (int q = 1; q < NP; ++q)
+        if (q < p.npaths && blk >= p.path[q].blk0) P = p.path[q];
     const int row0 = (blk - P.blk0) * 32;  // within the path
     const int cww = nwarps * p.ww;                           // words per CTA
     const int c0 = split * cww, c1 = min(p.W, c0 + cww);
@@ -140,15 +144,31 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small1_kernel(const __grid_con
     pdl_wait();
     cp_async_wait_all();
     __syncthreads();
-    for (int t = tid; t < ntab; t += nthr) {
-        const uint2 gw = *reinterpret_cast<const uint2 *>(gsm + 4 * t);
-        for (int m = 0; m < M; ++m) {
-            const uint2 xq = __ldg(reinterpret_cast<const uint2 *>(p.x + (int64_t)m * p.ldx + 32 * c0 + 4 * t));
-            const float v0 = f16_bits_to_float(gw.x & 0xffff) * bf16_bits_to_float(xq.x & 0xffff);
-            const float v1 = f16_bits_to_float(gw.x >> 16) * bf16_bits_to_float(xq.x >> 16);
-            const float v2 = f16_bits_to_float(gw.y & 0xffff) * bf16_bits_to_float(xq.y & 0xffff);
-            const float v3 = f16_bits_to_float(gw.y >> 16) * bf16_bits_to_float(xq.y >> 16);
-            nibble_table(v0, v1, v2, v3, tab + (kTab / 4) * (m * cww * 8 + t));
+    // two tables per thread and pass, with every x load of the pass issued
+    // before any of them is used (one L2 round trip per pass)
+    for (int t = tid; t < ntab; t += 2 * nthr) {
+        const int tt[2] = {t, t + nthr};
+        uint2 xq[2][MT];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+                if (m < M && tt[h] < ntab)
+                    xq[h][m] = __ldg(reinterpret_cast<const uint2 *>(p.x + (int64_t)m * p.ldx + 32 * c0 + 4 * tt[h]));
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            if (tt[h] >= ntab) continue;
+            const uint2 gw = *reinterpret_cast<const uint2 *>(gsm + 4 * tt[h]);
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                if (m >= M) continue;
+                const uint2 xv = xq[h][m];
+                const float v0 = f16_bits_to_float(gw.x & 0xffff) * bf16_bits_to_float(xv.x & 0xffff);
+                const float v1 = f16_bits_to_float(gw.x >> 16) * bf16_bits_to_float(xv.x >> 16);
+                const float v2 = f16_bits_to_float(gw.y & 0xffff) * bf16_bits_to_float(xv.y & 0xffff);
+                const float v3 = f16_bits_to_float(gw.y >> 16) * bf16_bits_to_float(xv.y >> 16);
+                nibble_table(v0, v1, v2, v3, tab + (kTab / 4) * (m * cww * 8 + tt[h]));
+            }
         }
     }
     __syncthreads();
@@ -218,11 +238,12 @@ struct S2Proj {
     uint16_t *y;
     int64_t ldy;
 };
+template <int NQ>  // projection slots: 1 for one layer, kMaxSiblings for a group
 struct Small2Params {
     const float *z;  // [R][M] over all paths, l applied
     int M;
     int nproj;
-    S2Proj proj[kMaxSiblings];  // in CTA order
+    S2Proj proj[NQ];  // in CTA order
     int ks;     // warps per 32-row block (each takes ww words of the latent)
     int ww;     // latent words per warp (<= kWW)
     int early;  // release the dependent launch at entry instead of after the lookups
@@ -231,17 +252,18 @@ struct Small2Params {
 // CTA = (warps / ks) blocks of 32 output rows of one projection; the ks warps
 // of a block split the latent words of the projection's paths (path 0 first).
 // Warps past the projection's latent words (a sibling may have fewer) idle.
-template <int MT>
-__global__ void __launch_bounds__(kMaxWarps * 32) small2_kernel(const __grid_constant__ Small2Params p)
+template <int MT, int NQ>
+__global__ void __launch_bounds__(kMaxWarps * 32) small2_kernel(const __grid_constant__ Small2Params<NQ> p)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nthr = blockDim.x, nwarps = nthr >> 5;
     const int M = p.M;
-    int qi = 0;  // the projection of this CTA
-    for (int q = 1; q < p.nproj; ++q)
-        if ((int)blockIdx.x >= p.proj[q].cta0) qi = q;
-    const S2Proj &P = p.proj[qi];
+    // the projection of this CTA (selected as in contraction 1)
+    S2Proj P = p.proj[0];
+#pragma unroll
+    for (int q = 1; q < NQ; ++q)
+        if (q < p.nproj && (int)blockIdx.x >= p.proj[q].cta0) P = p.proj[q];
     const int lc = blockIdx.x - P.cta0;  // CTA within the projection
     const int rb = nwarps / p.ks, rbi = warp / p.ks, kw = warp - rbi * p.ks;
     const int o = (lc * rb + rbi) * 32 + lane;  // output row
@@ -278,13 +300,29 @@ __global__ void __launch_bounds__(kMaxWarps * 32) small2_kernel(const __grid_con
     const int ntab = 8 * WT;
     float4 *tab = reinterpret_cast<float4 *>(smem);  // [M][WT * 8][kTab / 4]
     const float *zp = p.z + (int64_t)P.koff * M;
-    for (int e = tid; e < ntab * M; e += nthr) {
-        const int m = e / ntab, t = e - m * ntab;
-        const int k = 4 * t;
-        float v[4];
+    // two tables per thread and pass, every z load of the pass issued before
+    // any is used; one token reads its 4 latents as one 16-byte load
+    for (int e = tid; e < ntab * M; e += 2 * nthr) {
+        const int ee[2] = {e, e + nthr};
+        float v[2][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = __ldg(zp + (int64_t)(k + j) * M + m);
-        nibble_table(v[0], v[1], v[2], v[3], tab + (kTab / 4) * (m * ntab + t));
+        for (int h = 0; h < 2; ++h) {
+            if (ee[h] >= ntab * M) continue;
+            const int m = ee[h] / ntab, k = 4 * (ee[h] - m * ntab);
+            if (MT == 1) {
+                const float4 q = __ldg(reinterpret_cast<const float4 *>(zp + k));
+                v[h][0] = q.x, v[h][1] = q.y, v[h][2] = q.z, v[h][3] = q.w;
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) v[h][j] = __ldg(zp + (int64_t)(k + j) * M + m);
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            if (ee[h] >= ntab * M) continue;
+            const int m = ee[h] / ntab, t = ee[h] - m * ntab;
+            nibble_table(v[h][0], v[h][1], v[h][2], v[h][3], tab + (kTab / 4) * (m * ntab + t));
+        }
     }
     __syncthreads();
 
@@ -427,7 +465,10 @@ int group_rank(const GroupArgs &g)
     return R;
 }
 
-template <int MT>
+// NP / NQ: path and projection slots of the kernels (a single layer takes the
+// kernels with 2 and 1, whose parameter blocks and selection code are the
+// smallest; a group takes 2 kMaxSiblings and kMaxSiblings).
+template <int MT, int NP, int NQ>
 cudaError_t launch_small(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream, int m0, int M)
 {
     const int R = group_rank(g);
@@ -437,12 +478,12 @@ cudaError_t launch_small(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t
     if (p2.ctas == 0) return cudaErrorInvalidConfiguration;
 
     // the latent of every path of every projection, in projection order
-    Small1Params L{};
+    Small1Params<NP> L{};
     L.x = g.x + (int64_t)m0 * g.ldx;
     L.ldx = g.ldx;
     L.M = M;
     L.W = g.n_in / 32;
-    Small2Params E{};
+    Small2Params<NQ> E{};
     E.z = static_cast<const float *>(g.workspace);
     E.M = M;
     E.nproj = g.nproj;
@@ -504,22 +545,33 @@ cudaError_t launch_small(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = p1.cs > 1 ? 2 : 1;
-    cudaError_t err = cudaLaunchKernelEx(&cfg, small1_kernel<MT>, L);
+    cudaError_t err = cudaLaunchKernelEx(&cfg, small1_kernel<MT, NP>, L);
     if (err != cudaSuccess) return err;
     cfg.gridDim = dim3((unsigned)p2.ctas);
     cfg.blockDim = dim3((unsigned)(32 * p2.warps));
     cfg.dynamicSmemBytes = p2.smem;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, small2_kernel<MT>, E);
+    return cudaLaunchKernelEx(&cfg, small2_kernel<MT, NQ>, E);
 }
 
 template <int MT>
 cudaError_t prepare_mt(const DeviceInfo &dev)
 {
-    cudaError_t e =
-        cudaFuncSetAttribute(small1_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, dev.max_smem_optin);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(small2_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, dev.max_smem_optin);
+    const int sm = dev.max_smem_optin;
+    cudaError_t e = cudaFuncSetAttribute(small1_kernel<MT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(small1_kernel<MT, 2 * kMaxSiblings>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(small2_kernel<MT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(small2_kernel<MT, kMaxSiblings>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    return e;
+}
+
+template <int MT>
+cudaError_t launch_small_mt(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream, int m0, int M)
+{
+    return g.nproj == 1 ? launch_small<MT, 2, 1>(g, dev, stream, m0, M)
+                        : launch_small<MT, 2 * kMaxSiblings, kMaxSiblings>(g, dev, stream, m0, M);
 }
 
 }  // namespace
@@ -546,9 +598,9 @@ bool small_fits(int M, const GroupArgs &g, const DeviceInfo &dev)
 
 cudaError_t small_forward(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream, int m0, int M)
 {
-    if (M <= 1) return launch_small<1>(g, dev, stream, m0, M);
-    if (M <= 2) return launch_small<2>(g, dev, stream, m0, M);
-    return launch_small<4>(g, dev, stream, m0, M);
+    if (M <= 1) return launch_small_mt<1>(g, dev, stream, m0, M);
+    if (M <= 2) return launch_small_mt<2>(g, dev, stream, m0, M);
+    return launch_small_mt<4>(g, dev, stream, m0, M);
 }
 
 }  // namespace lb
