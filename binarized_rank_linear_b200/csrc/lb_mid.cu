@@ -60,8 +60,10 @@ struct MidShape {
     // floats so that 16-byte accesses of consecutive rows cover every bank
     static constexpr int kRedStride = NT + 4;
     static constexpr uint32_t kRedBytes = (uint32_t)TM * kRedStride * 4;
-    static constexpr size_t kSmem =
-        1024 + (size_t)STAGES * (A_BYTES + kBBytes) + kRedBytes + (size_t)kProducerWarps * 2 * G_BYTES + 256;
+    // per producer warp: two g slots; per producer thread: two 8-byte slots
+    // of sign words
+    static constexpr size_t kSmem = 1024 + (size_t)STAGES * (A_BYTES + kBBytes) + kRedBytes +
+                                    (size_t)kProducerWarps * (2 * G_BYTES + 32 * 8 * 2) + 256;
     static constexpr int kCtasPerSm = 2 * kSmem <= 227 * 1024 ? 2 : 1;
 };
 
@@ -138,7 +140,8 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
     const uint32_t sA = base, sB = base + STAGES * A_BYTES;
     const uint32_t sRed = sB + STAGES * B_BYTES;  // partials received from the cluster, [cs][rpr][NT] fp32
     const uint32_t sGbf = sRed + S::kRedBytes;    // mode 1, per producer warp: g in bf16, [warp][2][path][64]
-    const uint32_t bars = sGbf + kProducerWarps * 2 * G_BYTES;
+    const uint32_t sRing = sGbf + kProducerWarps * 2 * G_BYTES;  // per producer thread: two sign-word slots
+    const uint32_t bars = sRing + kProducerWarps * 32 * 8 * 2;
     // full[STAGES], empty[STAGES], acc_full, drain, then the tmem address
     const uint32_t full0 = bars, empty0 = bars + 8 * STAGES, accf = bars + 16 * STAGES, drain = accf + 8;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem_raw + (drain + 8 - raw));
@@ -245,36 +248,45 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
             }
         }
         auto wp = [&](int w) { return (MODE == 1 || w < r0w) ? rb0 + w : rb1 + (w - r0w); };
-        struct Pref {
-            uint2 bits;  // the row's two sign words of the block (zero outside the matrix)
-            uint4 g;     // mode 1, lanes 0..15: g of path lane / 8, columns 8 (lane % 8) .. (fp16)
-        };
-        auto fetch = [&](int j) {
-            Pref f;
-            f.bits = make_uint2(0u, 0u);
-            f.g = make_uint4(0u, 0u, 0u, 0u);
-            if (j >= nkb) return f;
-            const int kb = kb0 + j, wd = 2 * kb;
-            if (row_in && wd < kwords) {
-                if (p.bits8 && wd + 1 < kwords) {
-                    f.bits = ldg_early_v2(wp(wd));
+        // A block's sign words (and, mode 1, lanes 0..15, its g in fp16) come
+        // in by cp.async into slot `slot` of the thread's two-slot ring (and
+        // of the warp's two g slots), two of the group's blocks ahead, and are
+        // waited for just before use: no register holds a load in flight
+        // across blocks (copying one would wait for it).
+        constexpr uint32_t RING_STRIDE = (uint32_t)kProducerWarps * 32 * 8;
+        const uint32_t ring = sRing + (uint32_t)(pw * 32 + lane) * 8;
+        auto copy_block = [&](int j, int slot) {
+            if (j < nkb) {
+                const int kb = kb0 + j, wd = 2 * kb;
+                const uint32_t dst = ring + (uint32_t)slot * RING_STRIDE;
+                if (row_in && wd < kwords) {
+                    if (p.bits8 && wd + 1 < kwords) {
+                        cp_async8(dst, wp(wd));
+                    } else {
+                        cp_async4(dst, wp(wd));
+                        if (wd + 1 < kwords)
+                            cp_async4(dst + 4, wp(wd + 1));
+                        else
+                            asm volatile("st.shared.u32 [%0], %1;" ::"r"(dst + 4), "r"(0u) : "memory");
+                    }
                 } else {
-                    f.bits.x = ldg_early_u32(wp(wd));
-                    if (wd + 1 < kwords) f.bits.y = ldg_early_u32(wp(wd + 1));
+                    asm volatile("st.shared.v2.u32 [%0], {%1, %1};" ::"r"(dst), "r"(0u) : "memory");
+                }
+                if (MODE == 1 && lane < 16) {
+                    const int pp = lane >> 3, k0 = kb * BK + 8 * (lane & 7);
+                    const uint16_t *gs = pp ? p.s1 : p.s0;
+                    const uint32_t gdst = gbfw + (uint32_t)slot * G_BYTES + (uint32_t)lane * 16;
+                    if (gs != nullptr && k0 < p.K)
+                        cp_async16s(gdst, gs + k0);
+                    else
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(gdst), "r"(0u) : "memory");
                 }
             }
-            if (MODE == 1 && lane < 16) {
-                const int pp = lane >> 3, k0 = kb * BK + 8 * (lane & 7);
-                const uint16_t *gs = pp ? p.s1 : p.s0;
-                if (gs != nullptr && k0 < p.K) f.g = ldg_early_v4(gs + k0);
-            }
-            return f;
+            cp_async_commit();  // one group per block (empty past the end), so the waits count blocks
         };
-        Pref f0 = fetch(grp), f1 = fetch(grp + 2);
+        copy_block(grp, 0);
+        copy_block(grp + 2, 1);
         for (int j = grp, it = 0; j < nkb; j += 2, ++it) {
-            const Pref cur = f0;
-            f0 = f1;
-            f1 = fetch(j + 4);
             const int kb = kb0 + j;
             const int s = j % STAGES;
             const uint32_t ph = (uint32_t)(j / STAGES) & 1u;
@@ -284,22 +296,28 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
                 abort_flag = 1;
                 break;
             }
+            // this block's copies have landed (at most one younger group pending)
+            cp_async_wait_group<1>();
+            const int slot = it & 1;
             uint4 sc[8];  // per chunk: the four packed scale words
             if (MODE == 1) {
-                // lanes 0..15 round this block's g to bf16 into the warp's slot
-                // it % 2 (last read two iterations ago, before a __syncwarp)
+                // lanes 0..15 round their 8 values of g to bf16 in place
+                const uint32_t gsl = gbfw + (uint32_t)slot * G_BYTES;
                 if (lane < 16) {
-                    const uint32_t w[4] = {cur.g.x, cur.g.y, cur.g.z, cur.g.w};
-                    uint32_t o[4];
+                    uint32_t w[4];
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                                 : "r"(gsl + (uint32_t)lane * 16)
+                                 : "memory");
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        o[q] = (uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[q] & 0xffffu))) |
-                               ((uint32_t)float_to_bf16_bits(f16_bits_to_float((uint16_t)(w[q] >> 16))) << 16);
-                    *reinterpret_cast<uint4 *>(smem_raw + (gbfw + (it & 1) * G_BYTES + lane * 16 - raw)) =
-                        make_uint4(o[0], o[1], o[2], o[3]);
+                        w[q] = pack_bf162(f16_bits_to_float((uint16_t)(w[q] & 0xffffu)), f16_bits_to_float((uint16_t)(w[q] >> 16)));
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(gsl + (uint32_t)lane * 16), "r"(w[0]),
+                                 "r"(w[1]), "r"(w[2]), "r"(w[3])
+                                 : "memory");
                 }
                 __syncwarp();
-                const uint8_t *gb = smem_raw + (gbfw + (it & 1) * G_BYTES + (sec_row ? BK * 2 : 0) - raw);
+                const uint8_t *gb = smem_raw + (gsl + (sec_row ? BK * 2 : 0) - raw);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) sc[q] = *reinterpret_cast<const uint4 *>(gb + 16 * q);
             } else {
@@ -310,15 +328,24 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
                     sc[q] = make_uint4(h, h, h, h);
                 }
             }
+            uint2 bits;
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                         : "=r"(bits.x), "=r"(bits.y)
+                         : "r"(ring + (uint32_t)slot * RING_STRIDE)
+                         : "memory");
             const uint32_t rowx = (sA + s * A_BYTES + row * 128) | (x7 << 4);
 #pragma unroll
             for (int q = 0; q < 8; ++q)
-                store_sign_chunk(rowx ^ (16u * q), __byte_perm(q < 4 ? cur.bits.x : cur.bits.y, 0u, 0x4440u | (uint32_t)(q & 3)),
+                store_sign_chunk(rowx ^ (16u * q), __byte_perm(q < 4 ? bits.x : bits.y, 0u, 0x4440u | (uint32_t)(q & 3)),
                                  sc[q]);
             fence_async_shared();
             __syncwarp();
             if (lane == 0) mbar_arrive(full0 + 8 * s);
+            // refill the slots (used above; every lane is past its reads after
+            // the __syncwarp) with the group's block two ahead
+            copy_block(j + 4, slot);
         }
+        cp_async_wait_all();  // no copy may land after the CTA is gone
         // warps 2..5: this thread's row 32 (warp % 4) + lane of the accumulator
         if (pw < 4) {
             bool ok = !abort_flag && mbar_wait(accf, 0);
