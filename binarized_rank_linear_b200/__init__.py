@@ -156,8 +156,12 @@ def _torch():
 
 def _stream_handle(stream) -> ctypes.c_void_p:
     torch = _torch()
-    s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+    if stream is None:
+        raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+        if raw is not None:  # the current stream of the current device, without a Stream object
+            return ctypes.c_void_p(raw(torch.cuda.current_device()))
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
 
 
 def _dtype_code(t) -> int:
@@ -186,7 +190,7 @@ def pack_signs(src, kind: str, ld_words: int | None = None, stream=None):
     return dst
 
 
-@dataclass
+@dataclass(frozen=True)
 class PackedPath:
     """One binarized path on the device: packed sign(U) [n_out, u_ld] and
     sign(V)^T [rank, vt_ld] (int32 words) and fp16 scales h [n_out], g [n_in],
@@ -208,9 +212,15 @@ class PackedPath:
                    f16(h), f16(g), f16(l), int(su.shape[1]))
 
     def as_c(self) -> LbPath:
-        return LbPath(self.u_bits.data_ptr(), self.vt_bits.data_ptr(), self.h.data_ptr(),
-                      self.g.data_ptr(), self.l.data_ptr(), self.rank, self.u_bits.shape[1],
-                      self.vt_bits.shape[1])
+        """The lb_path struct of this path, built once (the fields are frozen
+        and a tensor's storage does not move)."""
+        c = self.__dict__.get("_c")
+        if c is None:
+            c = LbPath(self.u_bits.data_ptr(), self.vt_bits.data_ptr(), self.h.data_ptr(),
+                       self.g.data_ptr(), self.l.data_ptr(), self.rank, self.u_bits.shape[1],
+                       self.vt_bits.shape[1])
+            object.__setattr__(self, "_c", c)
+        return c
 
 
 def linear_forward(x, main: PackedPath, residual: PackedPath | None = None, y=None,
@@ -223,8 +233,8 @@ def linear_forward(x, main: PackedPath, residual: PackedPath | None = None, y=No
     n_out = main.h.shape[0]
     if y is None:
         y = torch.empty((tokens, n_out), dtype=torch.bfloat16, device=x.device)
-    need = forward_workspace_bytes(tokens, n_in, n_out, main.rank, residual.rank if residual else 0)
-    if workspace is None:
+    if workspace is None:  # a caller's workspace is checked by the library itself
+        need = forward_workspace_bytes(tokens, n_in, n_out, main.rank, residual.rank if residual else 0)
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
     cm = main.as_c()
     cr = residual.as_c() if residual is not None else None

@@ -223,8 +223,8 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
     } else {
         // ---------------- producers: group grp expands blocks j = grp, grp + 2, ...
         // of this CTA's K range, one W row per thread; what a block needs from
-        // memory (the row's sign words; g in mode 1) is loaded into registers
-        // two of the group's blocks ahead
+        // memory (the row's sign words; g in mode 1) comes in by cp.async two
+        // of the group's blocks ahead (below)
         const int pw = warp - 2;  // producer warp 0 .. 7
         const int grp = pw >> 2;
         const int row = ((pw & 3) << 5) | lane;  // W row within the tile
