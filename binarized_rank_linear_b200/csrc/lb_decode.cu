@@ -105,7 +105,9 @@ cudaError_t decode_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStre
 
 size_t group_workspace_bytes(const GroupArgs &g)
 {
+    // enough for whichever path the call takes, and for each layer alone
     size_t need = g.tokens <= kSmallMaxTokens ? small_workspace_bytes(g.tokens, g) : 0;
+    if (g.tokens <= kMidMaxTokens) need = std::max(need, mid_group_workspace_bytes(g.tokens, g));
     for (int j = 0; j < g.nproj; ++j) need = std::max(need, layer_workspace_bytes(layer_of(g, j)));
     return need;
 }
@@ -113,9 +115,9 @@ size_t group_workspace_bytes(const GroupArgs &g)
 cudaError_t group_forward(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream)
 {
     if (g.tokens <= kSmallMaxTokens && small_fits(g.tokens, g, dev)) return small_forward(g, dev, stream, 0, g.tokens);
+    if (g.tokens <= kMidMaxTokens) return mid_group_forward(g, dev, stream, 0, g.tokens);
     for (int j = 0; j < g.nproj; ++j) {
-        const ForwardArgs a = layer_of(g, j);
-        const cudaError_t e = a.tokens > kMidMaxTokens ? prefill_forward(a, dev, stream) : decode_forward(a, dev, stream);
+        const cudaError_t e = prefill_forward(layer_of(g, j), dev, stream);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -86,8 +86,9 @@ constexpr int kDecodeMaxTokens = 32;
 size_t decode_workspace_bytes(int tokens, int n_in, int n_out, const int *ranks, int npaths);
 cudaError_t decode_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 cudaError_t decode_prepare_device(const DeviceInfo &dev);
-// A group of siblings at any token count: one small-path launch pair for the
-// group when it fits, else each projection's own layer path in turn.
+// A group of siblings at any token count: one launch pair for the whole group
+// up to kMidMaxTokens tokens (small path when it fits, else tcgen05), each
+// projection's own prefill launches beyond.
 size_t group_workspace_bytes(const GroupArgs &g);
 cudaError_t group_forward(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream);
 
@@ -97,6 +98,10 @@ constexpr int kMidMaxTokens = 128;
 size_t mid_workspace_bytes(int tokens, const int *ranks, int npaths);
 cudaError_t mid_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M);
 cudaError_t mid_prepare_device(const DeviceInfo &dev);
+// One launch pair for a whole group of siblings (the latent of every layer in
+// one workspace z [M][sum of ranks], fp16).
+size_t mid_group_workspace_bytes(int tokens, const GroupArgs &g);
+cudaError_t mid_group_forward(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream, int m0, int M);
 cudaError_t mid_latent(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M, uint16_t *z,
                        int64_t ldz);
 cudaError_t mid_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M,

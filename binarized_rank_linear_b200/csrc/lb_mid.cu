@@ -67,6 +67,10 @@ struct MidShape {
     static constexpr int kCtasPerSm = 2 * kSmem <= 227 * 1024 ? 2 : 1;
 };
 
+// One layer of the call (a group of sibling layers that share x has up to
+// kMaxSiblings).  Mode 1 rows are the layer's latents (path 0, then path 1),
+// which sit at rows first .. of the group's latent z; mode 2 rows are its
+// outputs, in tiles first .. of the grid, reading z columns koff ..
 struct MidParams {
     int M;       // tokens (at most NT)
     int rows;    // rows of W: mode 1 R (both paths), mode 2 n_out
@@ -82,16 +86,38 @@ struct MidParams {
     void *out;                // mode 1: z fp16 [M][ldo]; mode 2: y bf16 [M][ldo]
     int64_t ldo;
     int *status;
+    int first;  // mode 1: first row of the layer's latents in z; mode 2: first tile of the layer
+    int koff;   // mode 2: first column of the layer's latents in z
 };
+
+template <int NQ>  // layer slots: 1 for one layer, kMaxSiblings for a group
+struct MidGroup {
+    int nlayers;
+    MidParams layer[NQ];  // in row (mode 1) or tile (mode 2) order
+};
+
+// The layer that row nn (mode 1) or tile t (mode 2) belongs to, selected field
+// by field from fixed parameter offsets.
+template <int NQ>
+__device__ __forceinline__ MidParams mid_layer(const MidGroup<NQ> &g, int at)
+{
+    MidParams p = g.layer[0];
+#pragma unroll
+    for (int q = 1; q < NQ; ++q)
+        if (q < g.nlayers && at >= g.layer[q].first) p = g.layer[q];
+    return p;
+}
 
 // Finished values of row nn of the tile for the tokens c0 .. c0 + CH - 1:
 // mode 1 z[m][nn] = l_nn c (fp16; returns true if a value does not fit),
 // mode 2 y[m][nn] (bf16).  A warp's lanes take consecutive rows, so each
 // token's stores are contiguous.
 template <int MODE, int CH>
-__device__ __forceinline__ bool finish_chunk(const MidParams &p, int nn, int c0, const float (&c)[CH])
+__device__ __forceinline__ bool finish_chunk(const MidParams &p, int col, int nn, int c0, const float (&c)[CH])
 {
-    uint16_t *out = static_cast<uint16_t *>(p.out) + nn;
+    // col: the output column (mode 1: the latent's row in the group's z; mode
+    // 2: nn); nn: the row within the layer
+    uint16_t *out = static_cast<uint16_t *>(p.out) + col;
     bool overflow = false;
     if (MODE == 1) {
         const float lv = f16_bits_to_float(nn < p.r0 ? p.l0[nn] : p.l1[nn - p.r0]);
@@ -128,8 +154,9 @@ __device__ __forceinline__ void acc_chunk(uint32_t taddr, bool valid, float (&c)
     }
 }
 
-template <int MODE, int NT>
-__global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const MidParams p)
+template <int MODE, int NT, int NQ>
+__global__ void __launch_bounds__(kThreads, 2)
+    mid_gemm_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ MidGroup<NQ> g)
 {
     using S = MidShape<NT>;
     constexpr uint32_t B_BYTES = S::kBBytes;
@@ -148,8 +175,13 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
     __shared__ int abort_shared;
     volatile int &abort_flag = abort_shared;
 
-    const int cs = p.cs;
+    const int cs = g.layer[0].cs;
     const int tile = blockIdx.x / cs, split = blockIdx.x - tile * cs;  // split = rank in the cluster
+    // Mode 2: the CTA's layer and its tile within the layer.  Mode 1: the
+    // layer of the tile's first row; only the fields all layers share (M, K,
+    // kpc, z) are read from it, as a tile's rows may belong to several layers.
+    const MidParams p = mid_layer<NQ>(g, MODE == 1 ? tile * TM : tile);
+    const int ltile = MODE == 1 ? tile : tile - p.first;
     const int nk = (p.K + BK - 1) / BK;
     const int kb0 = split * p.kpc, nkb = max(0, min(nk, kb0 + p.kpc) - kb0);
     if (cs > 1) cluster_arrive_relaxed();  // waited for before partials go to other CTAs
@@ -189,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
                     break;
                 }
                 mbar_arrive_expect_tx(full0 + 8 * s, B_BYTES);
-                tma_load_2d(sB + s * B_BYTES, &tmB, (kb0 + j) * BK, 0, full0 + 8 * s);
+                tma_load_2d(sB + s * B_BYTES, &tmB, (MODE == 2 ? p.koff : 0) + (kb0 + j) * BK, 0, full0 + 8 * s);
                 ++issued;
             }
             if (abort_flag) {
@@ -228,21 +260,24 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
         const int pw = warp - 2;  // producer warp 0 .. 7
         const int grp = pw >> 2;
         const int row = ((pw & 3) << 5) | lane;  // W row within the tile
-        const int nn = tile * TM + row;
+        // the layer of this warp's 32 rows (a layer's rows start at a
+        // multiple of 32, so they are all in one) and the row within it
+        const MidParams w = MODE == 1 ? mid_layer<NQ>(g, tile * TM + 32 * (pw & 3)) : p;
+        const int nn = (MODE == 1 ? tile * TM - w.first : ltile * TM) + row;
         const uint32_t x7 = (uint32_t)(row & 7);  // the row's 128-byte swizzle
-        const bool row_in = nn < p.rows;
-        const bool sec_row = MODE == 1 && nn >= p.r0;  // mode 1: the row's path
-        const int kwords = p.K >> 5, r0w = p.r0 >> 5;
+        const bool row_in = nn < w.rows;
+        const bool sec_row = MODE == 1 && nn >= w.r0;  // mode 1: the row's path
+        const int kwords = w.K >> 5, r0w = w.r0 >> 5;
         const uint32_t gbfw = sGbf + (uint32_t)pw * 2 * G_BYTES;  // this warp's two bf16 g slots
         const uint32_t *rb0 = nullptr, *rb1 = nullptr;
         uint32_t hs0 = 0u, hs1 = 0u;  // mode 2: h of the row, both paths, both halves
         if (row_in) {
             if (MODE == 1) {
-                rb0 = sec_row ? p.bits1 + (int64_t)(nn - p.r0) * p.bld1 : p.bits0 + (int64_t)nn * p.bld0;
+                rb0 = sec_row ? w.bits1 + (int64_t)(nn - w.r0) * w.bld1 : w.bits0 + (int64_t)nn * w.bld0;
             } else {
-                rb0 = p.bits0 + (int64_t)nn * p.bld0;
-                if (p.bits1) rb1 = p.bits1 + (int64_t)nn * p.bld1;
-                const uint32_t h0 = ldg_early_u16(p.s0 + nn), h1 = p.s1 ? ldg_early_u16(p.s1 + nn) : 0u;
+                rb0 = w.bits0 + (int64_t)nn * w.bld0;
+                if (w.bits1) rb1 = w.bits1 + (int64_t)nn * w.bld1;
+                const uint32_t h0 = ldg_early_u16(w.s0 + nn), h1 = w.s1 ? ldg_early_u16(w.s1 + nn) : 0u;
                 hs0 = h0 | (h0 << 16);
                 hs1 = h1 | (h1 << 16);
             }
@@ -260,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
                 const int kb = kb0 + j, wd = 2 * kb;
                 const uint32_t dst = ring + (uint32_t)slot * RING_STRIDE;
                 if (row_in && wd < kwords) {
-                    if (p.bits8 && wd + 1 < kwords) {
+                    if (w.bits8 && wd + 1 < kwords) {
                         cp_async8(dst, wp(wd));
                     } else {
                         cp_async4(dst, wp(wd));
@@ -274,9 +309,9 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
                 }
                 if (MODE == 1 && lane < 16) {
                     const int pp = lane >> 3, k0 = kb * BK + 8 * (lane & 7);
-                    const uint16_t *gs = pp ? p.s1 : p.s0;
+                    const uint16_t *gs = pp ? w.s1 : w.s0;
                     const uint32_t gdst = gbfw + (uint32_t)slot * G_BYTES + (uint32_t)lane * 16;
-                    if (gs != nullptr && k0 < p.K)
+                    if (gs != nullptr && k0 < w.K)
                         cp_async16s(gdst, gs + k0);
                     else
                         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(gdst), "r"(0u) : "memory");
@@ -324,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const int k0 = kb * BK + 8 * q;  // first column of the chunk
-                    const uint32_t h = k0 < p.K ? (k0 >= p.r0 ? hs1 : hs0) : 0u;
+                    const uint32_t h = k0 < w.K ? (k0 >= w.r0 ? hs1 : hs0) : 0u;
                     sc[q] = make_uint4(h, h, h, h);
                 }
             }
@@ -366,11 +401,13 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
     if (cs == 1) {
         if (holder) {
             pdl_wait();  // y / z may still be in use by the previous kernel
-            const int nn = tile * TM + 32 * (warp & 3) + lane;
+            const int gr = tile * TM + 32 * (warp & 3) + lane;  // the row in the grid (mode 1: in z)
+            const MidParams L = MODE == 1 ? mid_layer<NQ>(g, gr) : p;
+            const int nn = MODE == 1 ? gr - L.first : ltile * TM + 32 * (warp & 3) + lane;  // within the layer
             for (int c0 = 0; c0 < NT; c0 += CH) {
                 float c[CH];
                 acc_chunk<CH>(ta + (uint32_t)c0, acc_ok, c);
-                if (nn < p.rows) overflow |= finish_chunk<MODE, CH>(p, nn, c0, c);
+                if (nn < L.rows) overflow |= finish_chunk<MODE, CH>(L, MODE == 1 ? gr : nn, nn, c0, c);
             }
         }
     } else {
@@ -395,7 +432,9 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
         pdl_wait();
         const float *red = reinterpret_cast<const float *>(smem_raw + (sRed - raw));
         for (int q = tid; q < rpr; q += kThreads) {  // one row per thread, every token
-            const int nn = tile * TM + split * rpr + q;
+            const int gr = tile * TM + split * rpr + q;  // the row in the grid (mode 1: in z)
+            const MidParams L = MODE == 1 ? mid_layer<NQ>(g, gr) : p;
+            const int nn = MODE == 1 ? gr - L.first : ltile * TM + split * rpr + q;  // within the layer
             for (int c0 = 0; c0 < NT; c0 += CH) {
                 float c[CH];
 #pragma unroll
@@ -411,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 2) mid_gemm_kernel(const __grid_cons
                         c[4 * j4 + 3] += v.w;
                     }
                 }
-                if (nn < p.rows) overflow |= finish_chunk<MODE, CH>(p, nn, c0, c);
+                if (nn < L.rows) overflow |= finish_chunk<MODE, CH>(L, MODE == 1 ? gr : nn, nn, c0, c);
             }
         }
     }
@@ -440,100 +479,144 @@ int pick_split(int tiles, int nk, int slots)
     return cs;
 }
 
-template <int MODE, int NT>
-cudaError_t launch_mid(MidParams p, const void *b, int64_t ldb, const DeviceInfo &dev, cudaStream_t stream)
+int layer_rank(const ProjDesc &pj) { return pj.path[0].rank + (pj.npaths > 1 ? pj.path[1].rank : 0); }
+
+// Contraction MODE for the layers of a group, tokens m0 .. m0 + M, the
+// latent z fp16 [M][ldz] (token-major, every layer's latents side by side in
+// layer order, path 0 first).  Mode 1 covers the latent rows of all layers
+// with one grid of 128-row tiles (the K range, n_in, is shared); mode 2 gives
+// each layer its own tiles of output rows, reading its columns of z.  One
+// split of the K-blocks across a cluster serves every layer; it is chosen
+// for the layer with the fewest K-blocks, and a CTA past a longer layer's
+// blocks contributes zeros.
+template <int MODE, int NT, int NQ>
+cudaError_t launch_mid(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream, int m0, int M, const uint16_t *z,
+                       int64_t ldz)
 {
-    const int tiles = (p.rows + TM - 1) / TM, nk = (p.K + BK - 1) / BK;
-    p.cs = pick_split(tiles, nk, MidShape<NT>::kCtasPerSm * dev.sm_count);
-    p.kpc = (nk + p.cs - 1) / p.cs;
+    MidGroup<NQ> G{};
+    G.nlayers = g.nproj;
+    int tiles = 0, nk = 0, koff = 0;
+    if (MODE == 1) {
+        int R = 0;
+        for (int j = 0; j < g.nproj; ++j) R += layer_rank(g.proj[j]);
+        tiles = (R + TM - 1) / TM;
+        nk = (g.n_in + BK - 1) / BK;
+    } else {
+        nk = 1 << 30;
+        for (int j = 0; j < g.nproj; ++j) {
+            tiles += (g.proj[j].n_out + TM - 1) / TM;
+            nk = std::min(nk, (layer_rank(g.proj[j]) + BK - 1) / BK);
+        }
+    }
+    const int cs = pick_split(tiles, nk, MidShape<NT>::kCtasPerSm * dev.sm_count);
+    int tile0 = 0;
+    for (int j = 0; j < g.nproj; ++j) {
+        const ProjDesc &pj = g.proj[j];
+        const PathDesc &q0 = pj.path[0], &q1 = pj.path[1];
+        const bool two = pj.npaths > 1;
+        const int R = layer_rank(pj);
+        MidParams &L = G.layer[j];
+        L.M = M;
+        L.r0 = q0.rank;
+        L.cs = cs;
+        L.status = dev.status;
+        if (MODE == 1) {
+            L.rows = R;
+            L.K = g.n_in;
+            L.bits8 = even8(q0.vt_bits, q0.vt_ld) && (!two || even8(q1.vt_bits, q1.vt_ld));
+            L.bits0 = q0.vt_bits;
+            L.bld0 = q0.vt_ld;
+            L.s0 = q0.g;
+            L.l0 = q0.l;
+            if (two) {
+                L.bits1 = q1.vt_bits;
+                L.bld1 = q1.vt_ld;
+                L.s1 = q1.g;
+                L.l1 = q1.l;
+            }
+            L.kpc = (nk + cs - 1) / cs;
+            L.out = const_cast<uint16_t *>(z);
+            L.ldo = ldz;
+            L.first = koff;
+        } else {
+            L.rows = pj.n_out;
+            L.K = R;
+            L.bits8 = even8(q0.u_bits, q0.u_ld) && (!two || (q0.rank % 64 == 0 && even8(q1.u_bits, q1.u_ld)));
+            L.bits0 = q0.u_bits;
+            L.bld0 = q0.u_ld;
+            L.s0 = q0.h;
+            if (two) {
+                L.bits1 = q1.u_bits;
+                L.bld1 = q1.u_ld;
+                L.s1 = q1.h;
+            }
+            L.kpc = ((R + BK - 1) / BK + cs - 1) / cs;
+            L.out = pj.y + (int64_t)m0 * pj.ldy;
+            L.ldo = pj.ldy;
+            L.first = tile0;
+            L.koff = koff;
+            tile0 += (pj.n_out + TM - 1) / TM;
+        }
+        koff += R;
+    }
+    // the token operand: x (mode 1) or z over every layer's latents (mode 2)
     CUtensorMap tm;
-    cudaError_t e = encode_2d(&tm, b, p.M, p.K, ldb, MODE == 1, NT);
+    const cudaError_t e = MODE == 1 ? encode_2d(&tm, g.x + (int64_t)m0 * g.ldx, M, g.n_in, g.ldx, true, NT)
+                                    : encode_2d(&tm, z, M, koff, ldz, false, NT);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = (unsigned)p.cs;
+    attr[1].val.clusterDim.x = (unsigned)cs;
     attr[1].val.clusterDim.y = 1;
     attr[1].val.clusterDim.z = 1;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)(tiles * p.cs));
+    cfg.gridDim = dim3((unsigned)(tiles * cs));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = MidShape<NT>::kSmem;
     cfg.stream = stream;
     cfg.attrs = attr;
-    cfg.numAttrs = p.cs > 1 ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, mid_gemm_kernel<MODE, NT>, tm, p);
+    cfg.numAttrs = cs > 1 ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, mid_gemm_kernel<MODE, NT, NQ>, tm, G);
 }
 
-// Contraction 1 of tokens m0 .. m0 + M: z = l (.) (W1 x^T), rows = latent
-// indices of both paths, into z fp16 [M][ldz] (token-major).
-template <int NT>
-cudaError_t mid_latent_nt(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M, uint16_t *z,
-                          int64_t ldz)
+// Dispatch on the token tile (NT) and the layer slots (a single layer takes
+// the one-slot kernels, whose parameter block and selection are smallest).
+template <int MODE>
+cudaError_t launch_mid_any(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream, int m0, int M,
+                           const uint16_t *z, int64_t ldz)
 {
-    const int r0 = a.path[0].rank, r1 = a.npaths > 1 ? a.path[1].rank : 0;
-    const int R = r0 + r1;
-    const uint16_t *x = a.x + (int64_t)m0 * a.ldx;
-    MidParams p1{};
-    p1.M = M;
-    p1.rows = R;
-    p1.K = a.n_in;
-    p1.r0 = r0;
-    p1.bits8 = even8(a.path[0].vt_bits, a.path[0].vt_ld) && (a.npaths < 2 || even8(a.path[1].vt_bits, a.path[1].vt_ld));
-    p1.bits0 = a.path[0].vt_bits;
-    p1.bld0 = a.path[0].vt_ld;
-    p1.s0 = a.path[0].g;
-    p1.l0 = a.path[0].l;
-    if (a.npaths > 1) {
-        p1.bits1 = a.path[1].vt_bits;
-        p1.bld1 = a.path[1].vt_ld;
-        p1.s1 = a.path[1].g;
-        p1.l1 = a.path[1].l;
-    }
-    p1.out = z;
-    p1.ldo = ldz;
-    p1.status = dev.status;
-    return launch_mid<1, NT>(p1, x, a.ldx, dev, stream);
+    const bool one = g.nproj == 1;
+    if (M <= 16)
+        return one ? launch_mid<MODE, 16, 1>(g, dev, stream, m0, M, z, ldz)
+                   : launch_mid<MODE, 16, kMaxSiblings>(g, dev, stream, m0, M, z, ldz);
+    if (M <= 32)
+        return one ? launch_mid<MODE, 32, 1>(g, dev, stream, m0, M, z, ldz)
+                   : launch_mid<MODE, 32, kMaxSiblings>(g, dev, stream, m0, M, z, ldz);
+    if (M <= 64)
+        return one ? launch_mid<MODE, 64, 1>(g, dev, stream, m0, M, z, ldz)
+                   : launch_mid<MODE, 64, kMaxSiblings>(g, dev, stream, m0, M, z, ldz);
+    return one ? launch_mid<MODE, 128, 1>(g, dev, stream, m0, M, z, ldz)
+               : launch_mid<MODE, 128, kMaxSiblings>(g, dev, stream, m0, M, z, ldz);
 }
 
-// Contraction 2 of tokens m0 .. m0 + M from z fp16 [M][ldz]: y = W2 z^T,
-// rows = outputs.
-template <int NT>
-cudaError_t mid_expand_nt(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M,
-                          const uint16_t *z, int64_t ldz)
+template <int NT, int NQ>
+cudaError_t prepare_slots(cudaError_t e)
 {
-    const int r0 = a.path[0].rank, r1 = a.npaths > 1 ? a.path[1].rank : 0;
-    const int R = r0 + r1;
-    MidParams p2{};
-    p2.M = M;
-    p2.rows = a.n_out;
-    p2.K = R;
-    p2.r0 = r0;
-    p2.bits8 = even8(a.path[0].u_bits, a.path[0].u_ld) && (a.npaths < 2 || (r0 % 64 == 0 && even8(a.path[1].u_bits, a.path[1].u_ld)));
-    p2.bits0 = a.path[0].u_bits;
-    p2.bld0 = a.path[0].u_ld;
-    p2.s0 = a.path[0].h;
-    if (a.npaths > 1) {
-        p2.bits1 = a.path[1].u_bits;
-        p2.bld1 = a.path[1].u_ld;
-        p2.s1 = a.path[1].h;
-    }
-    p2.out = a.y + (int64_t)m0 * a.ldy;
-    p2.ldo = a.ldy;
-    p2.status = dev.status;
-    return launch_mid<2, NT>(p2, z, ldz, dev, stream);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(mid_gemm_kernel<1, NT, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)MidShape<NT>::kSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(mid_gemm_kernel<2, NT, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)MidShape<NT>::kSmem);
+    return e;
 }
-
 
 template <int NT>
 cudaError_t prepare_nt(cudaError_t e)
 {
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(mid_gemm_kernel<1, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MidShape<NT>::kSmem);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(mid_gemm_kernel<2, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MidShape<NT>::kSmem);
-    return e;
+    return prepare_slots<NT, kMaxSiblings>(prepare_slots<NT, 1>(e));
 }
 
 }  // namespace
@@ -554,30 +637,37 @@ size_t mid_workspace_bytes(int tokens, const int *ranks, int npaths)
     return (size_t)std::min(tokens, kMidMaxTokens) * R * 2;
 }
 
+size_t mid_group_workspace_bytes(int tokens, const GroupArgs &g)
+{
+    size_t R = 0;
+    for (int j = 0; j < g.nproj; ++j) R += (size_t)layer_rank(g.proj[j]);
+    return (size_t)std::min(tokens, kMidMaxTokens) * R * 2;
+}
+
 cudaError_t mid_latent(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M, uint16_t *z,
                        int64_t ldz)
 {
-    if (M <= 16) return mid_latent_nt<16>(a, dev, stream, m0, M, z, ldz);
-    if (M <= 32) return mid_latent_nt<32>(a, dev, stream, m0, M, z, ldz);
-    if (M <= 64) return mid_latent_nt<64>(a, dev, stream, m0, M, z, ldz);
-    return mid_latent_nt<128>(a, dev, stream, m0, M, z, ldz);
+    return launch_mid_any<1>(group_of_one(a), dev, stream, m0, M, z, ldz);
 }
 
 cudaError_t mid_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M,
                        const uint16_t *z, int64_t ldz)
 {
-    if (M <= 16) return mid_expand_nt<16>(a, dev, stream, m0, M, z, ldz);
-    if (M <= 32) return mid_expand_nt<32>(a, dev, stream, m0, M, z, ldz);
-    if (M <= 64) return mid_expand_nt<64>(a, dev, stream, m0, M, z, ldz);
-    return mid_expand_nt<128>(a, dev, stream, m0, M, z, ldz);
+    return launch_mid_any<2>(group_of_one(a), dev, stream, m0, M, z, ldz);
+}
+
+cudaError_t mid_group_forward(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream, int m0, int M)
+{
+    int R = 0;
+    for (int j = 0; j < g.nproj; ++j) R += layer_rank(g.proj[j]);
+    uint16_t *z = static_cast<uint16_t *>(g.workspace);  // [M][R] fp16, every layer's latents
+    const cudaError_t e = launch_mid_any<1>(g, dev, stream, m0, M, z, R);
+    return e != cudaSuccess ? e : launch_mid_any<2>(g, dev, stream, m0, M, z, R);
 }
 
 cudaError_t mid_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, int m0, int M)
 {
-    const int R = a.path[0].rank + (a.npaths > 1 ? a.path[1].rank : 0);
-    uint16_t *z = static_cast<uint16_t *>(a.workspace);  // [M][R] fp16
-    const cudaError_t e = mid_latent(a, dev, stream, m0, M, z, R);
-    return e != cudaSuccess ? e : mid_expand(a, dev, stream, m0, M, z, R);
+    return mid_group_forward(group_of_one(a), dev, stream, m0, M);
 }
 
 }  // namespace lb

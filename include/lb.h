@@ -233,8 +233,8 @@ LB_API lb_status lb_expand_forward(const uint16_t *z, int64_t tokens, int64_t n_
  *   same numerics (1..4 tokens: fp32 throughout on CUDA cores; more tokens:
  *   the tensor-core numerics of lb_linear_forward).  The output buffers must
  *   not overlap each other, x or the workspace.
- *   nproj: 1 .. LB_MAX_SIBLINGS.  1..4 tokens run as one pair of launches for
- *   the whole group; more tokens run each projection's own launches in turn.
+ *   nproj: 1 .. LB_MAX_SIBLINGS.  Up to 128 tokens the whole group runs as one
+ *   pair of launches; more tokens run each projection's own launches in turn.
  *   workspace: at least lb_siblings_workspace_bytes(...) bytes, 16-byte
  *   aligned, as for lb_linear_forward.
  * Errors as lb_linear_forward; additionally LB_ERR_INVALID_ARGUMENT for a bad
