@@ -13,8 +13,9 @@ the calls run back to back from CUDA graphs (the chained, per-layer number).
 Printed on rank 0, one JSON line:
   value       whole-job algorithmic HBM GB/s (prefill workloads: TFLOP/s),
               device-timed with CUDA events, max over ranks
-  e2e         the same metric through the public Python API with pinned host
-              x copied in and y copied out every step
+  e2e         the same metric through the C ABI with host buffers
+              (lb_linear_forward_host: pinned x copied in, y copied out,
+              every step)
   roofline    achieved GB/s of the forward call against the measured HBM peak
   cpu_baseline the fp64 oracle on this host's cores (bounded sample)
   clocks      SM clocks and throttle reasons sampled during the timed region
@@ -604,23 +605,26 @@ def run_lb(args, world, rank, local):
     iso_us = statistics.median(iso)
     del flush
 
-    # end to end through the public API: pinned x in, y out, every step
+    # end to end through the C ABI with host buffers (lb_linear_forward_host):
+    # every step copies x in from pinned host memory, runs the layer and
+    # copies y back to pinned host memory, all inside the one call
     x_host = torch.empty_like(x, device="cpu").pin_memory()
     x_host.copy_(x.cpu())
     y_host = torch.empty((tokens, c.n_out), dtype=torch.bfloat16).pin_memory()
     e2e_steps = min(args.steps, max(50, args.e2e_steps))
+
+    def call_host(i):
+        s = sets[i % nsets]
+        lb.linear_forward_host(x_host, s[0], s[1] if len(s) > 1 else None, y_host, x, y, ws)
+
     for i in range(min(20, e2e_steps)):
-        x.copy_(x_host, non_blocking=True)
-        call(i)
-        y_host.copy_(y, non_blocking=True)
+        call_host(i)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(e2e_steps):
-        x.copy_(x_host, non_blocking=True)
-        call(i)
-        y_host.copy_(y, non_blocking=True)
+        call_host(i)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -681,7 +685,7 @@ def run_lb(args, world, rank, local):
            "clocks": clk.summary(),
            "e2e": {"value": e2e_value, "unit": "GB/s" if decode else "TFLOP/s",
                    "h2d_bytes_per_step": 2 * tokens * c.n_in, "d2h_bytes_per_step": 2 * tokens * c.n_out,
-                   "steps": e2e_steps},
+                   "steps": e2e_steps, "call": "lb_linear_forward_host (pinned host x and y, copies inside the call)"},
            "gpu_launches": 2 * args.steps,  # contraction 1 + contraction 2 per call, decode and prefill
            "impl": "lb"}
     if dense is not None:

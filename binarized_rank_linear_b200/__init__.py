@@ -109,6 +109,9 @@ def lib() -> ctypes.CDLL:
             L.lb_siblings_workspace_bytes.argtypes = [i64, i64, i32, ctypes.POINTER(LbProjection)]
             L.lb_linear_forward_siblings.restype = i32
             L.lb_linear_forward_siblings.argtypes = [vp, i64, i64, i64, i32, ctypes.POINTER(LbProjection), vp, sz, vp]
+            L.lb_linear_forward_host.restype = i32
+            L.lb_linear_forward_host.argtypes = [vp, i64, i64, i64, ctypes.POINTER(LbPath), ctypes.POINTER(LbPath),
+                                                 vp, vp, vp, vp, sz, vp]
             L.lb_device_status.restype = i32
             L.lb_device_status.argtypes = [vp, ctypes.POINTER(i32)]
             _lib = L
@@ -284,6 +287,23 @@ def linear_forward_siblings(x, layers, ys=None, workspace=None, stream=None):
         x.data_ptr(), tokens, n_in, x.stride(0), len(layers), arr, workspace.data_ptr(),
         workspace.numel() * workspace.element_size(), _stream_handle(stream)), "lb_linear_forward_siblings")
     return ys
+
+
+def linear_forward_host(x_host, main: PackedPath, residual: PackedPath | None, y_host, x_dev, y_dev, workspace,
+                        stream=None):
+    """``lb_linear_forward_host``: x from pinned host memory (bf16 [tokens,
+    n_in], contiguous) through the caller's device buffers x_dev and y_dev to
+    y in pinned host memory (bf16 [tokens, n_out]), all on one stream; y_host
+    is valid once the stream is synchronised."""
+    tokens, n_in = x_host.shape
+    n_out = main.h.shape[0]
+    cm = main.as_c()
+    cr = residual.as_c() if residual is not None else None
+    _check(lib().lb_linear_forward_host(
+        x_host.data_ptr(), tokens, n_in, n_out, ctypes.byref(cm), ctypes.byref(cr) if cr is not None else None,
+        y_host.data_ptr(), x_dev.data_ptr(), y_dev.data_ptr(), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream_handle(stream)), "lb_linear_forward_host")
+    return y_host
 
 
 def latent_forward(x, main: PackedPath, residual: PackedPath | None = None, z=None, stream=None):

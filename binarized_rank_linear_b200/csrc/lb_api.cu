@@ -221,6 +221,28 @@ size_t lb_forward_workspace_bytes(int64_t tokens, int64_t n_in, int64_t n_out, i
     return workspace_for(tokens, n_in, n_out, ranks, rank_residual > 0 ? 2 : 1);
 }
 
+// Every host-side check of lb_linear_forward (tokens > 0).
+static lb_status check_forward(const uint16_t *x, int64_t tokens, int64_t n_in, int64_t n_out, int64_t ldx,
+                               const lb_path *main, const lb_path *residual, const uint16_t *y, int64_t ldy,
+                               const void *workspace, size_t workspace_bytes)
+{
+    if (!x || !y || !main) return LB_ERR_INVALID_ARGUMENT;
+    if (ldx < n_in || ldy < n_out) return LB_ERR_INVALID_ARGUMENT;
+    if (n_in % 32 != 0 || n_out % 32 != 0 || n_in > kMaxDim || n_out > kMaxDim || tokens > kMaxTokens)
+        return LB_ERR_UNSUPPORTED_SHAPE;
+    if (ldx % 8 != 0 || ldy % 8 != 0 || !aligned16(x) || !aligned16(y)) return LB_ERR_MISALIGNED;
+    lb::PathDesc d[2];
+    lb_status st = check_path(main, n_in, n_out, &d[0]);
+    if (st == LB_OK && residual) st = check_path(residual, n_in, n_out, &d[1]);
+    if (st != LB_OK) return st;
+    const int ranks[2] = {d[0].rank, residual ? d[1].rank : 0};
+    const size_t need = workspace_for(tokens, n_in, n_out, ranks, residual ? 2 : 1);
+    if (need > 0 && !workspace) return LB_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes < need) return LB_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace && !aligned16(workspace)) return LB_ERR_MISALIGNED;
+    return LB_OK;
+}
+
 lb_status lb_linear_forward(const uint16_t *x, int64_t tokens, int64_t n_in, int64_t n_out, int64_t ldx,
                             const lb_path *main, const lb_path *residual, uint16_t *y, int64_t ldy,
                             void *workspace, size_t workspace_bytes, void *stream)
@@ -340,6 +362,32 @@ lb_status lb_linear_forward_siblings(const uint16_t *x, int64_t tokens, int64_t 
     st = device_info(&dev);
     if (st != LB_OK) return st;
     if (lb::group_forward(g, dev, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    return LB_OK;
+}
+
+lb_status lb_linear_forward_host(const uint16_t *x_host, int64_t tokens, int64_t n_in, int64_t n_out,
+                                 const lb_path *main, const lb_path *residual, uint16_t *y_host, uint16_t *x_dev,
+                                 uint16_t *y_dev, void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (tokens < 0 || n_in <= 0 || n_out <= 0) return LB_ERR_INVALID_ARGUMENT;
+    if (tokens == 0) return LB_OK;
+    if (!x_host || !y_host) return LB_ERR_INVALID_ARGUMENT;
+    // every check on the device side first: nothing is copied when the call is refused
+    lb_status st = check_forward(x_dev, tokens, n_in, n_out, n_in, main, residual, y_dev, n_out, workspace,
+                                 workspace_bytes);
+    if (st != LB_OK) return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(x_dev, x_host, (size_t)tokens * (size_t)n_in * 2, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    st = lb_linear_forward(x_dev, tokens, n_in, n_out, n_in, main, residual, y_dev, n_out, workspace, workspace_bytes,
+                           stream);
+    if (st != LB_OK) return st;
+    if (cudaMemcpyAsync(y_host, y_dev, (size_t)tokens * (size_t)n_out * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
         cudaGetLastError();
         return LB_ERR_CUDA;
     }

@@ -211,6 +211,28 @@ LB_API lb_status lb_expand_forward(const uint16_t *z, int64_t tokens, int64_t n_
                             const lb_path *main, const lb_path *residual, uint16_t *y, int64_t ldy,
                             void *stream);
 
+/* ---------------------------------------------------------- host buffers
+ * lb_linear_forward_host: the layer on x in host memory, y back to host
+ * memory, in one call on `stream`: an asynchronous copy of x into x_dev, the
+ * forward pass of lb_linear_forward on x_dev into y_dev, an asynchronous copy
+ * of y_dev into y_host (one cudaMemcpyAsync each way).  For callers whose
+ * activations live on the host; the library allocates nothing, so the device
+ * buffers are the caller's.
+ *   x_host : bf16 [tokens x n_in], rows contiguous (row stride n_in); pinned
+ *            (page-locked) memory for the copy to be asynchronous
+ *   y_host : bf16 [tokens x n_out], rows contiguous; pinned likewise.  Valid
+ *            once the stream has reached the end of the call.
+ *   x_dev, y_dev : device scratch of tokens x n_in and tokens x n_out bf16,
+ *            16-byte aligned; their contents on entry do not matter
+ *   the rest as lb_linear_forward (x_dev and y_dev take the roles of x and y,
+ *   with ldx = n_in and ldy = n_out).
+ * Errors as lb_linear_forward; LB_ERR_INVALID_ARGUMENT for a null host
+ *   pointer.  A copy that fails to start returns LB_ERR_CUDA. */
+LB_API lb_status lb_linear_forward_host(const uint16_t *x_host, int64_t tokens, int64_t n_in, int64_t n_out,
+                                 const lb_path *main, const lb_path *residual, uint16_t *y_host,
+                                 uint16_t *x_dev, uint16_t *y_dev, void *workspace, size_t workspace_bytes,
+                                 void *stream);
+
 /* ---------------------------------------------------------- sibling projections
  * Several layers that read the same input x, computed together: the query,
  * key and value projections of an attention block, or the gate and up

@@ -258,3 +258,19 @@ def test_siblings_workspace_covers_each_layer_and_the_group(L):
     assert L.lb_siblings_workspace_bytes(0, q.n_in, 3, arr) == 0
     assert L.lb_siblings_workspace_bytes(1, q.n_in, 0, arr) == 0
     assert L.lb_siblings_workspace_bytes(1, 250, 3, arr) == 0
+
+
+def test_host_buffer_call_rejects_before_any_cuda_call(L):
+    host = lambda **kw: L.lb_linear_forward_host(
+        kw.get("xh", FAKE), kw.get("tokens", 1), kw.get("n_in", 256), kw.get("n_out", 256),
+        ctypes.byref(kw.get("main", fake_path())), None, kw.get("yh", FAKE), kw.get("xd", FAKE), kw.get("yd", FAKE),
+        kw.get("ws", FAKE), kw.get("ws_bytes", 1 << 20), None)
+    assert host(tokens=0, xh=0, yh=0) == lb.LB_OK            # no-op
+    assert host(tokens=-1) == lb.LB_ERR_INVALID_ARGUMENT
+    assert host(xh=0) == lb.LB_ERR_INVALID_ARGUMENT
+    assert host(yh=0) == lb.LB_ERR_INVALID_ARGUMENT
+    assert host(xd=0) == lb.LB_ERR_INVALID_ARGUMENT
+    assert host(yd=FAKE + 2) == lb.LB_ERR_MISALIGNED
+    assert host(n_in=250) == lb.LB_ERR_UNSUPPORTED_SHAPE
+    assert host(main=fake_path(rank=48)) == lb.LB_ERR_UNSUPPORTED_SHAPE
+    assert host(ws_bytes=16) == lb.LB_ERR_WORKSPACE_TOO_SMALL

@@ -243,3 +243,26 @@ def test_layer_object():
     mod = lb.LittleBitLinear.from_factors(layer["paths"])
     y = mod(gu.bf16_tensor(layer["x"]))
     gu.assert_close(gu.bf16_to_f64(y), gu.oracle_y(layer), "module")
+
+
+@pytest.mark.parametrize("tokens", [1, 8, 300])
+def test_host_buffer_call_equals_device_call(tokens):
+    """lb_linear_forward_host: x from pinned host memory and y back to it,
+    through the caller's device buffers; the same kernels as the device call,
+    so the same bits."""
+    import torch
+    layer = synth.make_layer(512, 224, [64, 32], tokens, config_id=880)
+    paths = gu.device_paths(layer)
+    res = paths[1] if len(paths) > 1 else None
+    x = gu.bf16_tensor(layer["x"])
+    ref = lb.linear_forward(x, paths[0], res)
+    x_host = x.cpu().pin_memory()
+    y_host = torch.full((tokens, 224), 3.0, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    y_dev = torch.empty((tokens, 224), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(max(16, lb.forward_workspace_bytes(tokens, 512, 224, 64, 32)), dtype=torch.uint8, device="cuda")
+    lb.linear_forward_host(x_host, paths[0], res, y_host, x_dev, y_dev, ws)
+    torch.cuda.synchronize()
+    assert lb.device_status() == lb.LB_OK
+    assert np.array_equal(gu.bf16_bits(y_host), gu.bf16_bits(ref))
+    gu.assert_close(gu.bf16_to_f64(y_host), gu.oracle_y(layer), f"host buffers M={tokens}")
