@@ -16,6 +16,7 @@ struct DeviceInfo {
     int sm_count = 0;
     int max_smem_optin = 0;  // bytes of dynamic shared memory a block may opt into
     int *status = nullptr;   // device address of this device's status word
+    int pair_slots = 0;      // CTA pairs of the prefill pair kernels resident at once
 };
 
 // ----------------------------------------------------------------- packing
@@ -111,7 +112,7 @@ cudaError_t mid_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t
 // binary operand expanded in shared memory (lb_prefill.cu).
 size_t prefill_workspace_bytes(int tokens, const int *ranks, int npaths);
 cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream);
-cudaError_t prefill_prepare_device(const DeviceInfo &dev);
+cudaError_t prefill_prepare_device(DeviceInfo &dev);  // also fills dev.pair_slots
 cudaError_t prefill_latent(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, uint16_t *z, int64_t ldz);
 cudaError_t prefill_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, const uint16_t *z,
                            int64_t ldz);

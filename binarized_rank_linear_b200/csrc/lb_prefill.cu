@@ -15,7 +15,7 @@
 // Accumulation is fp32 in tensor memory.
 //
 // A persistent grid (one CTA per SM) walks the 128 x bn tiles of C = A . B^T,
-// bn a multiple of 32 up to 256 chosen per call (see launch_sign_gemm).
+// bn a multiple of 32 up to 256 chosen per call (see plan_tiles).
 // In each CTA:
 //   warp 0       allocates tensor memory (two 256-column accumulators) and
 //                streams A tiles with TMA (128-byte swizzle, no multicast)
@@ -25,10 +25,23 @@
 //                bits into +-scale values in the same swizzled layout
 //   warps 18..21 read a finished accumulator out of tensor memory and store
 //                the tile, while the MMA fills the other accumulator
-// Stages are handed over with mbarriers (4-deep ring).  Every wait is bounded
-// in time: a wait that gives up sets LB_ERR_DEVICE_TIMEOUT on the status word
-// and the CTA winds down (drains its copies, frees tensor memory) instead of
-// hanging.
+// Stages are handed over with mbarriers (3- to 6-deep rings).  Every
+// mbarrier wait is bounded in time: a wait that gives up sets
+// LB_ERR_DEVICE_TIMEOUT on the status word and the CTA winds down (drains its
+// copies, frees tensor memory) instead of hanging.  The other waits are the
+// hardware's own (tensor-memory allocation, which the one CTA per SM always
+// gets, and the pair's cluster barriers, which every thread of both CTAs
+// reaches once its mbarrier waits have ended).
+//
+// Larger problems run on CTA pairs (clusters of two, cta_group::2): one MMA
+// of M = 256 spans both SMs, each CTA stages its own 128 rows of A and half
+// of the B tile, and the MMA reads each half of B once for both SMs.  Per
+// flop, each CTA then expands half as many sign rows and its shared memory
+// serves a third fewer operand bytes, which is what bounds the one-CTA tiles
+// (MMA operand reads plus the producers' and TMA's writes come close to the
+// shared-memory bandwidth).  CTA 0 issues the MMAs and its tcgen05.commit
+// arrives on the barriers of both CTAs; the TMA loads and producer arrivals
+// of CTA 1 count on CTA 0's stage barriers.
 #include <algorithm>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -44,7 +57,7 @@ using namespace tc;
 
 constexpr int BM = 128, BN = 256, BK = 64;  // one MMA: M = 128, N = bn <= 256; K-blocks of 64
 constexpr int kGroupWarps = 8;                // producer warps per K-block: one B row per thread
-constexpr uint32_t B_BYTES = BN * BK * 2;     // 32 KB
+constexpr uint32_t B_BYTES = BN * BK * 2;     // 32 KB: a whole B tile
 constexpr uint32_t TMEM_COLS = 2 * BN;        // two 256-column accumulators
 constexpr uint32_t G_BYTES = 2 * BK * 2;      // a K-block of g for both paths
 constexpr uint32_t OUT_BYTES = 32 * 64;       // an output box: 32 rows x 32 two-byte columns
@@ -55,21 +68,28 @@ constexpr uint32_t OUT_BYTES = 32 * 64;       // an output box: 32 rows x 32 two
 // each expanded B tile (half the sign expansion per flop); the two
 // accumulators hold the halves of one tile, and one producer group has twice
 // as long per K-block.
-template <int H>
+//
+// P = 2: a CTA pair (cluster of two) shares each MMA (cta_group::2, M = 256):
+// CTA r of the pair holds rows 128 H r .. of the pair's 256 H-row tile of A
+// and expands B rows bn r / 2 .. of the tile's bn, so each CTA stages and
+// expands half of B, and the MMA reads each half of B from shared memory once
+// for both SMs.  Stages are then smaller and the ring deeper.
+template <int H, int P>
 struct Shape {
-    static constexpr int kStages = H == 1 ? 4 : 3;
+    static constexpr int kStages = P == 1 ? (H == 1 ? 4 : 3) : (H == 1 ? 6 : 4);
     static constexpr int kGroups = H == 1 ? 2 : 1;
     static constexpr int kProducerWarps = kGroupWarps * kGroups;
     static constexpr int kEpiWarps = 4 * H;  // per accumulator in use, one per tensor-memory lane quadrant
     static constexpr int kThreads = 32 * (2 + kProducerWarps + kEpiWarps);
     static constexpr int kTileM = BM * H;
     static constexpr uint32_t kABytes = (uint32_t)kTileM * BK * 2;  // 16 or 32 KB
+    static constexpr uint32_t kBBytes = B_BYTES / P;                 // this CTA's rows of a B tile
     static constexpr int kOutBufs = 1;  // output boxes per epilogue warp
     static constexpr int kRing = 2;     // sign-word slots per producer thread
     // per stage: A tile, B tile; per epilogue warp: its output boxes and the
     // tile's latent scale in fp32 (mode 1); per producer warp: two slots of g
     // rounded to bf16; per producer thread: kRing slots of sign words
-    static constexpr size_t kSmem = 1024 + (size_t)kStages * (kABytes + B_BYTES) +
+    static constexpr size_t kSmem = 1024 + (size_t)kStages * (kABytes + kBBytes) +
                                     (size_t)kEpiWarps * (kOutBufs * OUT_BYTES + BN * 4) +
                                     (size_t)kProducerWarps * (2 * G_BYTES + 32 * 8 * kRing) + 256;
     static_assert(kSmem <= 232448, "shared memory per CTA");
@@ -99,21 +119,22 @@ struct SignGemmParams {
 // one sequence over all its tiles, so stages, phases and the producer groups'
 // alternation run on across tile boundaries.  Two accumulators in tensor
 // memory let the epilogue warps drain tile i while the MMA runs tile i + 1.
-template <int MODE, int H>
-__global__ void __launch_bounds__(Shape<H>::kThreads, 1)
+template <int MODE, int H, int P>
+__global__ void __launch_bounds__(Shape<H, P>::kThreads, 1)
     sign_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmOut,
                      const SignGemmParams p)
 {
-    using S = Shape<H>;
+    using S = Shape<H, P>;
     constexpr int STAGES = S::kStages;
     constexpr uint32_t A_BYTES = S::kABytes;
+    constexpr uint32_t B_STAGE = S::kBBytes;
     constexpr int kProducerWarps = S::kProducerWarps;
     extern __shared__ uint8_t smem_raw[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;  // SW128 tiles need 1024-byte alignment
     const uint32_t sA = base, sB = base + STAGES * A_BYTES;
-    const uint32_t sOut = sB + STAGES * B_BYTES;  // per epilogue warp: kOutBufs output boxes
+    const uint32_t sOut = sB + STAGES * B_STAGE;  // per epilogue warp: kOutBufs output boxes
     const uint32_t sGbf = sOut + S::kEpiWarps * S::kOutBufs * OUT_BYTES;  // mode 1, per producer warp: g in bf16, [warp][2][path][64]
     const uint32_t sLf = sGbf + kProducerWarps * 2 * G_BYTES;  // mode 1, per epilogue warp: l of the tile in fp32
     const uint32_t sRing = sLf + S::kEpiWarps * BN * 4;  // per producer thread: kRing 8-byte sign-word slots
@@ -125,10 +146,13 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
     __shared__ int abort_shared;
     volatile int &abort_flag = abort_shared;  // set by whichever role gives up; read by all
 
-    const int tiles_m = (p.M + S::kTileM - 1) / S::kTileM;
+    // P = 2: this CTA's rank in its pair; the pair's tiles are 256 H x bn
+    const int rank = P == 2 ? (int)cluster_rank() : 0;
+    const int tiles_m = (p.M + P * S::kTileM - 1) / (P * S::kTileM);
     const int ntiles = tiles_m * ((p.N + p.bn - 1) / p.bn);
-    const int busy_warps = (p.bn + 31) >> 5;  // producer warps per group with rows in the tile
-    const int G = gridDim.x, c = blockIdx.x;
+    const int rows_b = p.bn / P;                // B rows this CTA expands per tile
+    const int busy_warps = (rows_b + 31) >> 5;  // producer warps per group with rows in the tile
+    const int G = gridDim.x / P, c = blockIdx.x / P;  // persistent units: CTAs, or pairs
     const int my_tiles = c < ntiles ? (ntiles - c + G - 1) / G : 0;
     const int nk = (p.K + BK - 1) / BK;
     const int nblocks = my_tiles * nk;  // this CTA's K-blocks, all tiles
@@ -136,24 +160,35 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             for (int s = 0; s < STAGES; ++s) {
-                mbar_init(full0 + 8 * s, 1 + busy_warps);  // TMA arrive.expect_tx + one group's busy warps
+                // TMA arrive.expect_tx + one group's busy warps (P = 2: of both
+                // CTAs; only CTA 0's full barriers are used)
+                mbar_init(full0 + 8 * s, 1 + P * busy_warps);
                 mbar_init(empty0 + 8 * s, 1);               // one tcgen05.commit
             }
             for (int b = 0; b < 2; ++b) {
                 mbar_init(accf0 + 8 * b, 1);          // one tcgen05.commit
-                mbar_init(acce0 + 8 * b, S::kEpiWarps);  // every epilogue warp
+                mbar_init(acce0 + 8 * b, P * S::kEpiWarps);  // every epilogue warp (of the pair)
             }
             mbar_init(drain, 1);
             abort_flag = 0;
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         }
         __syncwarp();
-        tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+        if constexpr (P == 2)
+            tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+        else
+            tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
         tc_fence_before();
     }
-    __syncthreads();
+    if (P == 2)
+        cluster_sync();  // both CTAs' barriers are initialised before either arrives on the other's
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // P = 2: CTA 0's full and acc-empty barriers, as this CTA reaches them
+    const uint32_t full_lead = P == 2 ? map_shared_addr(full0, 0) : full0;
+    const uint32_t acce_lead = P == 2 ? map_shared_addr(acce0, 0) : acce0;
 
     if (warp == 0) {
         // ---------------- A producer (TMA)
@@ -168,11 +203,24 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
                     abort_flag = 1;
                     break;
                 }
-                mbar_arrive_expect_tx(full0 + 8 * s, A_BYTES);
-                tma_load_2d(sA + s * A_BYTES, &tmA, kb * BK, (t % tiles_m) * S::kTileM, full0 + 8 * s);
+                const int row0 = (t % tiles_m) * (P * S::kTileM);  // the (pair's) tile
+                if (P == 1) {
+                    mbar_arrive_expect_tx(full0 + 8 * s, A_BYTES);
+                    tma_load_2d(sA + s * A_BYTES, &tmA, kb * BK, row0, full0 + 8 * s);
+                } else {
+                    // both CTAs' A bytes complete on CTA 0's barrier, which CTA 0 arms
+                    if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * s, 2 * A_BYTES);
+                    tma_load_2d_pair(sA + s * A_BYTES, &tmA, kb * BK, row0 + rank * S::kTileM, full_lead + 8 * s);
+                }
                 ++issued;
             }
-            if (abort_flag) {
+            if (abort_flag && P == 2 && rank == 1) {
+                // this CTA cannot wait on CTA 0's barriers: give copies in
+                // flight time to land (they take microseconds)
+                const unsigned long long t0 = globaltimer();
+                while (globaltimer() - t0 < 200000ull) {
+                }
+            } else if (abort_flag) {
                 // let copies already in flight land before the CTA goes away
                 for (int gb = (issued > STAGES ? issued - STAGES : 0); gb < issued; ++gb)
                     mbar_wait(full0 + 8 * (gb % STAGES), (uint32_t)(gb / STAGES) & 1u);
@@ -181,8 +229,18 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
     } else if (warp == 1) {
         // ---------------- MMA issuer.  H = 1: tile i accumulates in columns
         // 256 (i % 2) ..; H = 2: half h of every tile accumulates in columns 256 h ..
-        if (lane == 0) {
-            const uint32_t idesc = instr_desc(MODE == 1 ? 1u : 0u, BM, p.bn);
+        // P = 2: CTA 0 issues the pair's MMAs and signals both CTAs; CTA 1
+        // only waits for the last of them before it may free tensor memory.
+        if (lane == 0 && P == 2 && rank == 1) {
+            if (!mbar_wait(drain, 0)) abort_flag = 1;
+        } else if (lane == 0) {
+            const uint32_t idesc = instr_desc(MODE == 1 ? 1u : 0u, BM * P, p.bn);
+            auto commit = [&](uint32_t bar) {
+                if constexpr (P == 2)
+                    umma_commit_pair(bar);
+                else
+                    umma_commit(bar);
+            };
             int gb = 0;
             for (int i = 0; i < my_tiles && !abort_flag; ++i) {
                 const int b = H == 1 ? (i & 1) : 0;  // hand-over barriers of the accumulator(s)
@@ -202,22 +260,26 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t bd = smem_desc(sB + s * B_BYTES);
+                    const uint64_t bd = smem_desc(sB + s * B_STAGE);
 #pragma unroll
                     for (int h = 0; h < H; ++h) {
                         // half h: A rows 128 h .. (16 KB further on, a whole number of 8-row atoms)
                         const uint64_t ad = smem_desc(sA + s * A_BYTES + (uint32_t)h * (BM * BK * 2));
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk)  // +32 bytes along K per step of 16
-                            umma(acc + (uint32_t)(h * BN), ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                        for (int kk = 0; kk < BK / 16; ++kk) {  // +32 bytes along K per step of 16
+                            if constexpr (P == 2)
+                                umma_pair(acc + (uint32_t)(h * BN), ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                            else
+                                umma(acc + (uint32_t)(h * BN), ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
+                        }
                     }
-                    umma_commit(empty0 + 8 * s);
+                    commit(empty0 + 8 * s);
                 }
                 if (abort_flag) break;
-                umma_commit(accf0 + 8 * b);
+                commit(accf0 + 8 * b);
             }
-            // every MMA issued has finished before the CTA frees tensor memory
-            umma_commit(drain);
+            // every MMA issued has finished before the CTA (and its pair) frees tensor memory
+            commit(drain);
             if (!mbar_wait(drain, 0)) abort_flag = 1;
         }
     } else if (warp < 2 + kProducerWarps) {
@@ -244,7 +306,8 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
         static_assert(RING == 2, "the warp's two g slots double as the g ring");
         constexpr uint32_t RING_STRIDE = (uint32_t)kProducerWarps * 32 * 8;  // bytes between ring slots
         const int grp = pt >> 8;        // 0 .. NG - 1
-        const int row = pt & (BN - 1);  // B row within the tile
+        const int row = pt & (BN - 1);  // B row within this CTA's rows of the tile (valid below rows_b)
+        const int nrow = rank * rows_b + row;  // ... within the tile
         const int wl = warp - 2;        // producer warp 0 .. 15
         const uint32_t x7 = (uint32_t)(row & 7);  // the row's 128-byte swizzle: logical chunk j sits at chunk j ^ x7
         const int kwords = p.K >> 5, r0w = p.r0 >> 5;
@@ -263,7 +326,7 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
             u.gb = gb;
             u.i = gb / nk;
             u.kb = gb - u.i * nk;
-            u.nn = ((c + u.i * G) / tiles_m) * p.bn + row;
+            u.nn = ((c + u.i * G) / tiles_m) * p.bn + nrow;
             return u;
         };
         auto advance = [&](Cursor &u) {
@@ -274,7 +337,7 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
                     u.kb -= nk;
                     ++u.i;
                 }
-                u.nn = ((c + u.i * G) / tiles_m) * p.bn + row;
+                u.nn = ((c + u.i * G) / tiles_m) * p.bn + nrow;
             }
         };
         // Start the copies of block u's two sign words into ring slot `slot`
@@ -293,7 +356,7 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
             }
             const uint32_t dst = ring + (uint32_t)slot * RING_STRIDE;
             const int wd = 2 * u.kb;  // first word of the block in the (concatenated) row
-            if (u.gb < my_blocks && row < p.bn && u.nn < p.N && wd < kwords) {
+            if (u.gb < my_blocks && row < rows_b && u.nn < p.N && wd < kwords) {
                 const int nn = u.nn;
                 const uint32_t *rb0, *rb1 = nullptr;
                 if (MODE == 1) {
@@ -321,8 +384,8 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
         // mode 2: h of this thread's row in tile iteration i, both paths (fp16 pair)
         auto fetch_h = [&](int i) {
             uint32_t hv = 0u;
-            const int nn = ((c + i * G) / tiles_m) * p.bn + row;
-            if (MODE == 2 && i < my_tiles && row < p.bn && nn < p.N) {
+            const int nn = ((c + i * G) / tiles_m) * p.bn + nrow;
+            if (MODE == 2 && i < my_tiles && row < rows_b && nn < p.N) {
                 hv = ldg_early_u16(p.s0 + nn);
                 if (p.s1) hv |= (uint32_t)ldg_early_u16(p.s1 + nn) << 16;
             }
@@ -395,8 +458,8 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
             // chunk q of the row goes to chunk position q ^ x7 (the tile is
             // 1024-byte aligned, so the XOR acts on address bits 4..6 alone);
             // the 8 rows of a store phase then cover all 32 banks
-            const uint32_t rowx = (sB + s * B_BYTES + row * 128) | (x7 << 4);
-            if (row < p.bn) {
+            const uint32_t rowx = (sB + s * B_STAGE + row * 128) | (x7 << 4);
+            if (row < rows_b) {
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     store_sign_chunk(rowx ^ (16u * q), __byte_perm(q < 4 ? bits.x : bits.y, 0u, 0x4440u | (uint32_t)(q & 3)),
@@ -405,7 +468,12 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
             }
             fence_async_shared();
             __syncwarp();
-            if (lane == 0) mbar_arrive(full0 + 8 * s);
+            if (lane == 0) {
+                if (P == 2 && rank == 1)
+                    mbar_arrive_remote(full_lead + 8 * s);
+                else
+                    mbar_arrive(full0 + 8 * s);
+            }
             // refill the slots (their contents are used above, and every lane
             // is past its reads after the __syncwarp) with the group's block
             // RING ahead
@@ -432,7 +500,8 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
             const int b = H == 1 ? (i & 1) : 0;
             const int use = H == 1 ? (i >> 1) : i;
             const int t = c + i * G;
-            const int m0 = (t % tiles_m) * S::kTileM + eh * BM + 32 * quad;  // the warp's first row
+            // the warp's first row (P = 2: this CTA's rows of the pair's tile)
+            const int m0 = (t % tiles_m) * (P * S::kTileM) + rank * S::kTileM + eh * BM + 32 * quad;
             const bool row_in = m0 + lane < p.M;
             const int n0 = (t / tiles_m) * p.bn;
             if (MODE == 1) {
@@ -497,7 +566,12 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acce0 + 8 * b);
+            if (lane == 0) {
+                if (P == 2 && rank == 1)
+                    mbar_arrive_remote(acce_lead + 8 * b);
+                else
+                    mbar_arrive(acce0 + 8 * b);
+            }
         }
         if (lane == 0) bulk_wait_all();
         if (overflow) set_status(p.status, LB_ERR_RANGE);
@@ -505,61 +579,101 @@ __global__ void __launch_bounds__(Shape<H>::kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    // P = 2: neither CTA leaves (or frees its half of tensor memory) while
+    // the other may still arrive on its barriers or read its shared memory
+    if (P == 2) cluster_sync();
     if (abort_flag && tid == 0) set_status(p.status, LB_ERR_DEVICE_TIMEOUT);
     if (warp == 0) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        if constexpr (P == 2)
+            tmem_dealloc_pair(tmem, TMEM_COLS);
+        else
+            tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
 // ---------------------------------------------------------------- host side
 // The tile shape of one contraction, from a makespan model fitted to timings
-// of this kernel on B200 (Qwen3-14B and Llama-2-7B shapes, 256 to 8192
-// tokens).  A CTA spends per K-block of a tile, in tenths of a nanosecond,
-//   H = 1:  max(4800, 2000 + 20 bn)    (two producer groups alternate)
-//   H = 2:  max(8000, 5500 + 18 bn)    (one group feeds both halves)
-// where the constant floors are the producers' latency per block and the
-// slopes the sign expansion and MMA, plus per tile 500 ns (H = 1: its
-// epilogue overlaps the next tile) or 3000 ns (H = 2: both accumulators hold
-// the one tile, so the MMA waits for its epilogue).  The makespan is
-// ceil(tiles / SMs) tiles.  Of the widths giving each column-tile count only
-// the narrowest (rounded up to 32, the output box width) is worth trying;
-// ties (widths whose blocks all sit at the floor) go to more tiles, i.e. less
-// work per CTA.
+// of this kernel on B200 (Qwen3-14B and Llama-2-7B shapes, 129 to 8192
+// tokens).  A CTA (or each CTA of a pair) spends per K-block of a tile, in
+// tenths of a nanosecond,
+//   P = 1, H = 1:  max(4800, 2000 + 20 bn)    (two producer groups alternate)
+//   P = 1, H = 2:  max(8000, 5500 + 18 bn)    (one group feeds both halves)
+//   P = 2, H = 1:  max(5000, 2000 + 11 bn)    (each CTA expands bn / 2 rows)
+//   P = 2, H = 2:  max(6000, 3900 + 14 bn)
+// where the constant floors are the producers' latency per block (a little
+// longer for a pair, whose stages also wait on the other CTA) and the slopes
+// the sign expansion and MMA, plus per tile 500 ns (H = 1: its epilogue
+// overlaps the next tile) or 3000 ns (H = 2: both accumulators hold the one
+// tile, so the MMA waits for its epilogue).  The makespan is ceil(tiles /
+// units) tiles, units being SMs (P = 1) or the pairs resident at once
+// (P = 2).  Of the widths giving each column-tile count only the narrowest
+// (rounded up to 32, the output box width) is worth trying; ties (plans whose
+// blocks all sit at a floor) go to more tiles, i.e. less work per unit.
 struct TilePlan {
     int H, bn, tiles;
+    int P;  // CTAs per MMA
 };
 
-TilePlan plan_tiles(int M, int N, int K, int sms)
+TilePlan plan_tiles(int M, int N, int K, int sms, int pairs)
 {
     const long nk = (K + BK - 1) / BK;
-    TilePlan best{1, BN, 0};
+    TilePlan best{1, BN, 0, 1};
     long best_cost = -1;
-    for (int H = 1; H <= 2; ++H) {
-        const int tm = (M + BM * H - 1) / (BM * H);
-        for (int tn = (N + BN - 1) / BN; tn <= (N + 31) / 32; ++tn) {
-            const int bn = ((N + tn - 1) / tn + 31) & ~31;
-            if ((N + bn - 1) / bn != tn) continue;
-            const int tiles = tm * tn, waves = (tiles + sms - 1) / sms;
-            const long per_block = H == 1 ? std::max(4800, 2000 + 20 * bn) : std::max(8000, 5500 + 18 * bn);
-            const long cost = (long)waves * (nk * per_block + (H == 1 ? 5000 : 30000));
-            if (best_cost < 0 || cost < best_cost || (cost == best_cost && tiles > best.tiles)) {
-                best_cost = cost;
-                best = TilePlan{H, bn, tiles};
+    for (int P = 1; P <= 2; ++P) {
+        const int units = P == 1 ? sms : pairs;
+        if (units <= 0) continue;
+        for (int H = 1; H <= 2; ++H) {
+            const int tm = (M + BM * H * P - 1) / (BM * H * P);
+            for (int tn = (N + BN - 1) / BN; tn <= (N + 31) / 32; ++tn) {
+                const int bn = ((N + tn - 1) / tn + 31) & ~31;
+                if ((N + bn - 1) / bn != tn) continue;
+                const int tiles = tm * tn, waves = (tiles + units - 1) / units;
+                long per_block;
+                if (P == 1)
+                    per_block = H == 1 ? std::max(4800, 2000 + 20 * bn) : std::max(8000, 5500 + 18 * bn);
+                else
+                    per_block = H == 1 ? std::max(5000, 2000 + 11 * bn) : std::max(6000, 3900 + 14 * bn);
+                const long cost = (long)waves * (nk * per_block + (H == 1 ? 5000 : 30000));
+                if (best_cost < 0 || cost < best_cost || (cost == best_cost && tiles > best.tiles)) {
+                    best_cost = cost;
+                    best = TilePlan{H, bn, tiles, P};
+                }
             }
         }
     }
     return best;
 }
 
-// One contraction on a persistent grid of min(tiles, SMs) CTAs.
+// A persistent grid of `units` CTAs (P = 1) or CTA pairs (P = 2, clusters of two).
+template <int MODE, int H, int P>
+cudaError_t launch_units(const CUtensorMap &tm, const CUtensorMap &tmo, const SignGemmParams &p, int units,
+                         cudaStream_t stream)
+{
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)P;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(units * P));
+    cfg.blockDim = dim3(Shape<H, P>::kThreads);
+    cfg.dynamicSmemBytes = Shape<H, P>::kSmem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = P == 2 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, sign_gemm_kernel<MODE, H, P>, tm, tmo, p);
+}
+
+// One contraction on a persistent grid: min(tiles, SMs) CTAs, or
+// min(tiles, resident pairs) CTA pairs.
 // A is x (mode 1, bf16) or z (mode 2, fp16), row-major with stride lda.
 template <int MODE>
 cudaError_t launch_sign_gemm(SignGemmParams p, const void *a, int64_t lda, const DeviceInfo &dev,
                              cudaStream_t stream)
 {
-    const TilePlan tp = plan_tiles(p.M, p.N, p.K, dev.sm_count);
+    const TilePlan tp = plan_tiles(p.M, p.N, p.K, dev.sm_count, dev.pair_slots);
     const int H = tp.H;
     p.bn = tp.bn;
     CUtensorMap tm, tmo;
@@ -567,28 +681,60 @@ cudaError_t launch_sign_gemm(SignGemmParams p, const void *a, int64_t lda, const
     // the output: z fp16 (mode 1) or y bf16 (mode 2), [M x N] with stride ldo
     if (e == cudaSuccess) e = encode_store_2d(&tmo, p.out, p.M, p.N, p.ldo, MODE == 2);
     if (e != cudaSuccess) return e;
-    const int grid = std::min(tp.tiles, dev.sm_count);
-    if (H == 2)
-        sign_gemm_kernel<MODE, 2><<<grid, Shape<2>::kThreads, Shape<2>::kSmem, stream>>>(tm, tmo, p);
-    else
-        sign_gemm_kernel<MODE, 1><<<grid, Shape<1>::kThreads, Shape<1>::kSmem, stream>>>(tm, tmo, p);
-    return cudaGetLastError();
+    if (tp.P == 2) {
+        const int units = std::min(tp.tiles, dev.pair_slots);
+        return H == 2 ? launch_units<MODE, 2, 2>(tm, tmo, p, units, stream)
+                      : launch_units<MODE, 1, 2>(tm, tmo, p, units, stream);
+    }
+    const int units = std::min(tp.tiles, dev.sm_count);
+    return H == 2 ? launch_units<MODE, 2, 1>(tm, tmo, p, units, stream)
+                  : launch_units<MODE, 1, 1>(tm, tmo, p, units, stream);
 }
 
 }  // namespace
 
-cudaError_t prefill_prepare_device(const DeviceInfo &dev)
+namespace {
+
+// Opts a kernel into its shared memory; for pair kernels also counts the
+// clusters of two that fit on the device at once (the fewest of any kernel).
+template <int MODE, int H, int P>
+cudaError_t prepare_kernel(DeviceInfo &dev)
 {
-    (void)dev;
+    cudaError_t e = cudaFuncSetAttribute(sign_gemm_kernel<MODE, H, P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Shape<H, P>::kSmem);
+    if (e != cudaSuccess || P == 1) return e;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)dev.sm_count);
+    cfg.blockDim = dim3(Shape<H, P>::kThreads);
+    cfg.dynamicSmemBytes = Shape<H, P>::kSmem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, sign_gemm_kernel<MODE, H, P>, &cfg);
+    if (e != cudaSuccess) return e;
+    dev.pair_slots = dev.pair_slots == 0 ? clusters : std::min(dev.pair_slots, clusters);
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t prefill_prepare_device(DeviceInfo &dev)
+{
     cudaError_t e = get_encoder();
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(sign_gemm_kernel<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Shape<1>::kSmem);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(sign_gemm_kernel<2, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Shape<1>::kSmem);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(sign_gemm_kernel<1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Shape<2>::kSmem);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(sign_gemm_kernel<2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Shape<2>::kSmem);
+    dev.pair_slots = 0;
+    if (e == cudaSuccess) e = prepare_kernel<1, 1, 1>(dev);
+    if (e == cudaSuccess) e = prepare_kernel<2, 1, 1>(dev);
+    if (e == cudaSuccess) e = prepare_kernel<1, 2, 1>(dev);
+    if (e == cudaSuccess) e = prepare_kernel<2, 2, 1>(dev);
+    if (e == cudaSuccess) e = prepare_kernel<1, 1, 2>(dev);
+    if (e == cudaSuccess) e = prepare_kernel<2, 1, 2>(dev);
+    if (e == cudaSuccess) e = prepare_kernel<1, 2, 2>(dev);
+    if (e == cudaSuccess) e = prepare_kernel<2, 2, 2>(dev);
     return e;
 }
 

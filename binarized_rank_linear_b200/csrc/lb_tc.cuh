@@ -111,6 +111,68 @@ __device__ __forceinline__ void umma_commit(uint32_t bar)
 {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
+// ---------------------------------------------------------------- CTA pairs
+// A pair of CTAs (a cluster of two) sharing each MMA (cta_group::2): the
+// instruction, issued by CTA 0, takes rows 0..127 of A and columns 0..N/2-1
+// of B from CTA 0's shared memory and the rest from CTA 1's (same offsets),
+// and writes rows 0..127 of D into CTA 0's tensor memory, rows 128..255 into
+// CTA 1's.  Barriers that both CTAs feed live in CTA 0.
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Arrive on an mbarrier given by its shared::cluster address (possibly in
+// the peer CTA).  What the arrival hands over is shared memory that the
+// pair's MMA reads through the async proxy, so the writer's
+// fence.proxy.async before it is the ordering that matters; a cluster-scope
+// release here would also wait for the thread's own copies still in flight.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster)
+{
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+// TMA tile load into this CTA's shared memory whose completion (bytes) is
+// counted on an mbarrier of CTA 0 of the pair (`bar_cluster`: its
+// shared::cluster address).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *tm, int x, int y, uint32_t bar_cluster)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(dst),
+        "l"(tm), "r"(x), "r"(y), "r"(bar_cluster)
+        : "memory");
+}
+// Tensor memory for a pair: one warp of each CTA (the same warp) allocates
+// together; the columns are the same in both CTAs.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t cols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t cols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+// One pair MMA (M = 256), issued by CTA 0.
+__device__ __forceinline__ void umma_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// When the pair MMAs issued so far have finished, arrive once on the
+// mbarrier at offset `bar` in each CTA of the pair.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+        "h"((unsigned short)3)
+        : "memory");
+}
 // 16 consecutive fp32 columns of this warp's 32 lanes, one register each,
 // then wait for them.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16])

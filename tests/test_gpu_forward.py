@@ -43,7 +43,9 @@ def test_prefill_configs_sampled(name):
     M = layer["x"].shape[0]
     y = gu.bf16_to_f64(gu.run_gpu(layer))
     rng = np.random.default_rng(1)
-    rows = np.unique(np.concatenate([[0, 1, 127, 128, M - 1], rng.choice(M, 27, replace=False)]))
+    # rows of each 128-row quarter of a 512-row pair tile (both CTAs, both halves)
+    edges = [0, 1, 127, 128, 255, 256, 383, 384, 511, 512, M - 1]
+    rows = np.unique(np.concatenate([edges, rng.choice(M, 27, replace=False)]))
     gu.assert_close(y[rows], gu.oracle_y(layer, rows), f"{name} sampled rows")
     assert np.all(np.isfinite(y))
 
@@ -71,14 +73,21 @@ def test_prefill_tile_shapes_ragged(n_in, n_out, ranks):
 # 256-row tiles at 2100 tokens), each checked whole against the oracle.  The
 # plan is the library's choice; the ids record which one each shape took when
 # the cases were picked.
+# Shapes whose planned tiles cover the kernel's variants (ids: the contraction
+# and its plan; "pair" = CTA pairs sharing each MMA, "h2" = two 128-row halves
+# per CTA).
 TILE_PLAN_CASES = [
     pytest.param(129, 256, 256, [32, 32], id="m129-c1-w32"),
     pytest.param(129, 256, 4096, [32, 32], id="m129-c2-w64"),
     pytest.param(520, 256, 2048, [32, 32], id="m520-c2-w96"),
     pytest.param(1000, 256, 2048, [32, 32], id="m1000-c2-w128"),
-    pytest.param(700, 256, 4096, [32, 32], id="m700-c2-w192"),
-    pytest.param(2600, 256, 2048, [32, 32], id="m2600-c2-w160-2waves"),
-    pytest.param(2100, 256, 4096, [160, 160], id="m2100-c2-h2-w256"),
+    pytest.param(700, 256, 4096, [32, 32], id="m700-c2-pair-w192"),
+    pytest.param(2600, 256, 2048, [32, 32], id="m2600-c2-pair-w160-2waves"),
+    pytest.param(2100, 256, 4096, [160, 160], id="m2100-c2-pair-w256"),
+    pytest.param(2600, 256, 256, [512, 512], id="m2600-c1-pair-w192"),
+    pytest.param(3000, 256, 416, [512, 512], id="m3000-c1-pair-w192-ragged-m"),
+    pytest.param(520, 256, 8192, [256, 256], id="m520-c2-pair-h2-w224"),
+    pytest.param(900, 512, 6016, [256, 224], id="m900-c2-pair-h2-w192-ragged-n"),
 ]
 
 
@@ -125,6 +134,19 @@ def test_integer_exact_is_bitwise(tokens):
     layer = integer_layer(512, 224, [64, 32], tokens, tokens, 0.9 if tokens < 100 else 0.97)
     ref = gu.oracle_y(layer)
     assert np.abs(ref).max() <= 256 and np.array_equal(ref, np.rint(ref))
+    got = gu.bf16_bits(gu.run_gpu(layer))
+    assert np.array_equal(got, bf16_rne(ref))
+
+
+@pytest.mark.parametrize("n_in,n_out,ranks,tokens", [(256, 8192, [256, 256], 520), (256, 256, [512, 512], 2600)],
+                         ids=["c2-pair-h2", "c1-pair"])
+def test_integer_exact_pair_plans_are_bitwise(n_in, n_out, ranks, tokens):
+    """The integer-exact case on shapes planned as CTA pairs.  Every value is
+    an integer well inside fp32's exact range and z inside fp16's, so the GPU
+    equals the oracle rounded to bf16 (round to nearest even) bit for bit."""
+    layer = integer_layer(n_in, n_out, ranks, tokens, 31 + tokens, 0.95)
+    ref = gu.oracle_y(layer)
+    assert np.abs(ref).max() < 2 ** 24 and np.array_equal(ref, np.rint(ref))
     got = gu.bf16_bits(gu.run_gpu(layer))
     assert np.array_equal(got, bf16_rne(ref))
 
