@@ -114,6 +114,8 @@ def lib() -> ctypes.CDLL:
                                                  vp, vp, vp, vp, sz, vp]
             L.lb_device_status.restype = i32
             L.lb_device_status.argtypes = [vp, ctypes.POINTER(i32)]
+            L.lb_set_prefill_pairs.restype = i32
+            L.lb_set_prefill_pairs.argtypes = [i32]
             _lib = L
     return _lib
 
@@ -365,6 +367,12 @@ def device_status(stream=None) -> int:
     out = ctypes.c_int(0)
     _check(lib().lb_device_status(_stream_handle(stream), ctypes.byref(out)), "lb_device_status")
     return int(out.value)
+
+
+def set_prefill_pairs(enable: bool) -> None:
+    """``lb_set_prefill_pairs``: let prefill contractions run on CTA pairs
+    (the default) or keep them on single-CTA tiles."""
+    _check(lib().lb_set_prefill_pairs(1 if enable else 0), "lb_set_prefill_pairs")
 
 
 class LittleBitLinear:

@@ -1,6 +1,7 @@
 // lb_api.cu - the C ABI (include/lb.h): argument checks, per-device set-up,
 // dispatch by token count, and the device status word.
 #include <array>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -22,6 +23,7 @@ constexpr int64_t kMaxRank = 32768;
 constexpr int64_t kMaxTokens = int64_t(1) << 24;
 
 std::mutex g_mutex;
+std::atomic<int> g_prefill_pairs{1};  // lb_set_prefill_pairs
 std::array<lb::DeviceInfo, kMaxDevices> g_dev;
 std::array<bool, kMaxDevices> g_ready{};
 
@@ -133,6 +135,8 @@ size_t workspace_for(int64_t tokens, int64_t n_in, int64_t n_out, const int *ran
 }
 
 }  // namespace
+
+bool lb::prefill_pairs_enabled() { return g_prefill_pairs.load(std::memory_order_relaxed) != 0; }
 
 extern "C" {
 
@@ -478,6 +482,13 @@ lb_status lb_device_status(void *stream, lb_status *out)
         }
     }
     *out = static_cast<lb_status>(v);
+    return LB_OK;
+}
+
+lb_status lb_set_prefill_pairs(int enable)
+{
+    if (enable != 0 && enable != 1) return LB_ERR_INVALID_ARGUMENT;
+    g_prefill_pairs.store(enable, std::memory_order_relaxed);
     return LB_OK;
 }
 

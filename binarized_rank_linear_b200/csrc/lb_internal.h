@@ -113,6 +113,7 @@ cudaError_t mid_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t
 size_t prefill_workspace_bytes(int tokens, const int *ranks, int npaths);
 cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 cudaError_t prefill_prepare_device(DeviceInfo &dev);  // also fills dev.pair_slots
+bool prefill_pairs_enabled();                          // lb_set_prefill_pairs
 cudaError_t prefill_latent(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, uint16_t *z, int64_t ldz);
 cudaError_t prefill_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, const uint16_t *z,
                            int64_t ldz);

@@ -56,7 +56,7 @@ namespace {
 using namespace tc;
 
 constexpr int BM = 128, BN = 256, BK = 64;  // one MMA: M = 128, N = bn <= 256; K-blocks of 64
-constexpr int kGroupWarps = 8;                // producer warps per K-block: one B row per thread
+constexpr int kRowWarps = 8;                  // warps for the 256 rows of a whole B tile, one row per thread
 constexpr uint32_t B_BYTES = BN * BK * 2;     // 32 KB: a whole B tile
 constexpr uint32_t TMEM_COLS = 2 * BN;        // two 256-column accumulators
 constexpr uint32_t G_BYTES = 2 * BK * 2;      // a K-block of g for both paths
@@ -77,8 +77,11 @@ constexpr uint32_t OUT_BYTES = 32 * 64;       // an output box: 32 rows x 32 two
 template <int H, int P>
 struct Shape {
     static constexpr int kStages = P == 1 ? (H == 1 ? 4 : 3) : (H == 1 ? 6 : 4);
-    static constexpr int kGroups = H == 1 ? 2 : 1;
-    static constexpr int kProducerWarps = kGroupWarps * kGroups;
+    // producer groups: one B row per thread, a group per K-block in turn
+    // (P = 2: a CTA's B rows take half a group's warps, so twice the groups)
+    static constexpr int kGroupWarps = kRowWarps / P;
+    static constexpr int kGroups = (H == 1 ? 2 : 1) * P;
+    static constexpr int kProducerWarps = kGroupWarps * kGroups;  // 16 (H = 1) or 8 (H = 2)
     static constexpr int kEpiWarps = 4 * H;  // per accumulator in use, one per tensor-memory lane quadrant
     static constexpr int kThreads = 32 * (2 + kProducerWarps + kEpiWarps);
     static constexpr int kTileM = BM * H;
@@ -283,12 +286,15 @@ __global__ void __launch_bounds__(Shape<H, P>::kThreads, 1)
             if (!mbar_wait(drain, 0)) abort_flag = 1;
         }
     } else if (warp < 2 + kProducerWarps) {
-        // ---------------- B producers: groups of 8 warps, one B row per thread.
-        // H = 1: two groups; group q expands the blocks gb = q, q + 2, ... of
-        // the CTA's K-block sequence, so every warp has two MMA periods for
-        // each of its blocks and its latency (barrier wait, expansion, arrive)
-        // hides behind the other group's block.  H = 2: one group; a block
-        // feeds two MMA halves, so it has two MMA periods as well.
+        // ---------------- B producers: groups of kGroupWarps warps, one B row
+        // per thread.  P = 1, H = 1: two groups of 8; group q expands the
+        // blocks gb = q, q + 2, ... of the CTA's K-block sequence, so every
+        // warp has two MMA periods for each of its blocks and its latency
+        // (barrier wait, expansion, arrive) hides behind the other group's
+        // block.  P = 1, H = 2: one group; a block feeds two MMA halves, so it
+        // has two MMA periods as well.  P = 2: a CTA expands at most 128 rows
+        // of a block, so groups of 4 warps and twice as many of them: four
+        // (or two) MMA periods per block.
         // What a block needs from memory arrives without a register holding a
         // load in flight across blocks (copying such a register would wait
         // for the load):
@@ -305,8 +311,9 @@ __global__ void __launch_bounds__(Shape<H, P>::kThreads, 1)
         constexpr int RING = S::kRing;
         static_assert(RING == 2, "the warp's two g slots double as the g ring");
         constexpr uint32_t RING_STRIDE = (uint32_t)kProducerWarps * 32 * 8;  // bytes between ring slots
-        const int grp = pt >> 8;        // 0 .. NG - 1
-        const int row = pt & (BN - 1);  // B row within this CTA's rows of the tile (valid below rows_b)
+        constexpr int GT = S::kGroupWarps * 32;  // threads (rows) of a group
+        const int grp = pt / GT;                // 0 .. NG - 1
+        const int row = pt & (GT - 1);          // B row within this CTA's rows of the tile (valid below rows_b)
         const int nrow = rank * rows_b + row;  // ... within the tile
         const int wl = warp - 2;        // producer warp 0 .. 15
         const uint32_t x7 = (uint32_t)(row & 7);  // the row's 128-byte swizzle: logical chunk j sits at chunk j ^ x7
@@ -315,7 +322,7 @@ __global__ void __launch_bounds__(Shape<H, P>::kThreads, 1)
         const uint32_t ring = sRing + (uint32_t)pt * 8;           // this thread's slot 0 (8 bytes)
         // a warp whose rows all lie past bn takes no part (the stage barriers
         // count only the busy warps)
-        const int my_blocks = (wl & (kGroupWarps - 1)) < busy_warps ? nblocks : 0;
+        const int my_blocks = (wl & (S::kGroupWarps - 1)) < busy_warps ? nblocks : 0;
         // Position of a block in the sequence, advanced without divisions:
         // tile iteration, K-block, and this thread's B row in that tile.
         struct Cursor {
@@ -600,15 +607,16 @@ __global__ void __launch_bounds__(Shape<H, P>::kThreads, 1)
 // tenths of a nanosecond,
 //   P = 1, H = 1:  max(4800, 2000 + 20 bn)    (two producer groups alternate)
 //   P = 1, H = 2:  max(8000, 5500 + 18 bn)    (one group feeds both halves)
-//   P = 2, H = 1:  max(5000, 2000 + 11 bn)    (each CTA expands bn / 2 rows)
-//   P = 2, H = 2:  max(6000, 3900 + 14 bn)
-// where the constant floors are the producers' latency per block (a little
-// longer for a pair, whose stages also wait on the other CTA) and the slopes
-// the sign expansion and MMA, plus per tile 500 ns (H = 1: its epilogue
-// overlaps the next tile) or 3000 ns (H = 2: both accumulators hold the one
-// tile, so the MMA waits for its epilogue).  The makespan is ceil(tiles /
-// units) tiles, units being SMs (P = 1) or the pairs resident at once
-// (P = 2).  Of the widths giving each column-tile count only the narrowest
+//   P = 2, H = 1:  max(4300, 2000 + 11 bn)    (each CTA expands bn / 2 rows)
+//   P = 2, H = 2:  max(5000, 24.5 bn)
+// where the constant floors are the latency of a stage's round trip (shorter
+// for a pair, whose four producer groups each have four MMA periods per
+// block) and the slopes the sign expansion and MMA, plus per tile 500 ns (H = 1: its
+// epilogue overlaps the next tile), 3000 ns (P = 1, H = 2: both accumulators
+// hold the one tile, so the MMA waits for its epilogue) or 5600 ns (P = 2,
+// H = 2: the same for a 512-row tile, whose stores leave all SMs at once).
+// The makespan is ceil(tiles / units) tiles, units being SMs (P = 1) or the
+// pairs resident at once (P = 2).  Of the widths giving each column-tile count only the narrowest
 // (rounded up to 32, the output box width) is worth trying; ties (plans whose
 // blocks all sit at a floor) go to more tiles, i.e. less work per unit.
 struct TilePlan {
@@ -630,12 +638,15 @@ TilePlan plan_tiles(int M, int N, int K, int sms, int pairs)
                 const int bn = ((N + tn - 1) / tn + 31) & ~31;
                 if ((N + bn - 1) / bn != tn) continue;
                 const int tiles = tm * tn, waves = (tiles + units - 1) / units;
-                long per_block;
-                if (P == 1)
+                long per_block, per_tile;
+                if (P == 1) {
                     per_block = H == 1 ? std::max(4800, 2000 + 20 * bn) : std::max(8000, 5500 + 18 * bn);
-                else
-                    per_block = H == 1 ? std::max(5000, 2000 + 11 * bn) : std::max(6000, 3900 + 14 * bn);
-                const long cost = (long)waves * (nk * per_block + (H == 1 ? 5000 : 30000));
+                    per_tile = H == 1 ? 5000 : 30000;
+                } else {
+                    per_block = H == 1 ? std::max(4300, 2000 + 11 * bn) : std::max(5000, 49 * bn / 2);
+                    per_tile = H == 1 ? 5000 : 56000;
+                }
+                const long cost = (long)waves * (nk * per_block + per_tile);
                 if (best_cost < 0 || cost < best_cost || (cost == best_cost && tiles > best.tiles)) {
                     best_cost = cost;
                     best = TilePlan{H, bn, tiles, P};
@@ -673,7 +684,7 @@ template <int MODE>
 cudaError_t launch_sign_gemm(SignGemmParams p, const void *a, int64_t lda, const DeviceInfo &dev,
                              cudaStream_t stream)
 {
-    const TilePlan tp = plan_tiles(p.M, p.N, p.K, dev.sm_count, dev.pair_slots);
+    const TilePlan tp = plan_tiles(p.M, p.N, p.K, dev.sm_count, prefill_pairs_enabled() ? dev.pair_slots : 0);
     const int H = tp.H;
     p.bn = tp.bn;
     CUtensorMap tm, tmo;

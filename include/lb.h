@@ -316,6 +316,15 @@ LB_API lb_status lb_linear_forward_fixed_scratch(const uint16_t *x, int64_t toke
  * condition.  Returns LB_ERR_CUDA if the synchronisation itself fails. */
 LB_API lb_status lb_device_status(void *stream, lb_status *out);
 
+/* Whether the prefill contractions (more than 128 tokens) may run on CTA
+ * pairs: thread-block clusters of two SMs that share each tensor-core MMA
+ * (the default, 1), or only on single-CTA tiles (0).  Both give the same
+ * results to the bit; pairs are faster wherever the device can co-schedule
+ * them.  The setting is process-wide and applies to calls made after it
+ * returns; a call already enqueued keeps the kernels it was given.  Returns
+ * LB_ERR_INVALID_ARGUMENT unless `enable` is 0 or 1. */
+LB_API lb_status lb_set_prefill_pairs(int enable);
+
 #ifdef __cplusplus
 }
 #endif

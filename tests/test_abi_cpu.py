@@ -274,3 +274,11 @@ def test_host_buffer_call_rejects_before_any_cuda_call(L):
     assert host(n_in=250) == lb.LB_ERR_UNSUPPORTED_SHAPE
     assert host(main=fake_path(rank=48)) == lb.LB_ERR_UNSUPPORTED_SHAPE
     assert host(ws_bytes=16) == lb.LB_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_prefill_pairs_switch_takes_only_zero_or_one(L):
+    # host-only: the setting is a process-wide flag read when a call plans its tiles
+    for bad in (-1, 2, 7):
+        assert L.lb_set_prefill_pairs(bad) == lb.LB_ERR_INVALID_ARGUMENT
+    assert L.lb_set_prefill_pairs(0) == lb.LB_OK
+    assert L.lb_set_prefill_pairs(1) == lb.LB_OK

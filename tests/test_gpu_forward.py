@@ -86,16 +86,26 @@ TILE_PLAN_CASES = [
     pytest.param(2100, 256, 4096, [160, 160], id="m2100-c2-pair-w256"),
     pytest.param(2600, 256, 256, [512, 512], id="m2600-c1-pair-w192"),
     pytest.param(3000, 256, 416, [512, 512], id="m3000-c1-pair-w192-ragged-m"),
-    pytest.param(520, 256, 8192, [256, 256], id="m520-c2-pair-h2-w224"),
-    pytest.param(900, 512, 6016, [256, 224], id="m900-c2-pair-h2-w192-ragged-n"),
+    pytest.param(900, 512, 6016, [256, 224], id="m900-c2-pair-w192-ragged-n"),
+    pytest.param(520, 256, 8192, [512, 512], id="m520-c2-pair-h2-w224-ragged"),
+    pytest.param(5000, 1024, 256, [512, 512], id="m5000-c1-pair-h2-w160-ragged"),
 ]
 
 
+@pytest.fixture(params=[True, False], ids=["pairs", "single-cta"])
+def prefill_pairs(request):
+    """Runs a test with CTA-pair prefill tiles allowed (the default) and with
+    single-CTA tiles only (lb_set_prefill_pairs), restoring the default."""
+    lb.set_prefill_pairs(request.param)
+    yield request.param
+    lb.set_prefill_pairs(True)
+
+
 @pytest.mark.parametrize("tokens,n_in,n_out,ranks", TILE_PLAN_CASES)
-def test_prefill_tile_plans(tokens, n_in, n_out, ranks):
+def test_prefill_tile_plans(tokens, n_in, n_out, ranks, prefill_pairs):
     layer = synth.make_layer(n_in, n_out, ranks, tokens, config_id=900 + n_out + sum(ranks))
     y = gu.bf16_to_f64(gu.run_gpu(layer))
-    gu.assert_close(y, gu.oracle_y(layer), f"{n_in}x{n_out} r={ranks} M={tokens}")
+    gu.assert_close(y, gu.oracle_y(layer), f"{n_in}x{n_out} r={ranks} M={tokens} pairs={prefill_pairs}")
 
 
 @pytest.mark.parametrize("n_in,n_out,ranks", [(32, 32, [32]), (96, 64, [32]), (64, 800, [32, 64]),
@@ -138,17 +148,37 @@ def test_integer_exact_is_bitwise(tokens):
     assert np.array_equal(got, bf16_rne(ref))
 
 
-@pytest.mark.parametrize("n_in,n_out,ranks,tokens", [(256, 8192, [256, 256], 520), (256, 256, [512, 512], 2600)],
-                         ids=["c2-pair-h2", "c1-pair"])
-def test_integer_exact_pair_plans_are_bitwise(n_in, n_out, ranks, tokens):
-    """The integer-exact case on shapes planned as CTA pairs.  Every value is
-    an integer well inside fp32's exact range and z inside fp16's, so the GPU
-    equals the oracle rounded to bf16 (round to nearest even) bit for bit."""
+@pytest.mark.parametrize("n_in,n_out,ranks,tokens", [(256, 8192, [512, 512], 520), (256, 256, [512, 512], 2600),
+                                                     (512, 224, [64, 32], 300), (512, 224, [64, 32], 1000)],
+                         ids=["c2-h2", "c1-wide", "m300", "m1000"])
+def test_integer_exact_prefill_tiles_are_bitwise(n_in, n_out, ranks, tokens, prefill_pairs):
+    """The integer-exact case on prefill shapes, on CTA pairs and on single
+    CTAs.  Every value is an integer well inside fp32's exact range and z
+    inside fp16's, so the GPU equals the oracle rounded to bf16 (round to
+    nearest even) bit for bit."""
     layer = integer_layer(n_in, n_out, ranks, tokens, 31 + tokens, 0.95)
     ref = gu.oracle_y(layer)
     assert np.abs(ref).max() < 2 ** 24 and np.array_equal(ref, np.rint(ref))
     got = gu.bf16_bits(gu.run_gpu(layer))
     assert np.array_equal(got, bf16_rne(ref))
+
+
+@pytest.mark.parametrize("tokens,n_in,n_out,ranks", [(700, 256, 4096, [32, 32]), (2100, 256, 4096, [160, 160]),
+                                                     (520, 256, 8192, [512, 512])])
+def test_pair_and_single_cta_tiles_agree_bitwise(tokens, n_in, n_out, ranks):
+    """Every output element sums the same K-steps in the same order whether
+    its row sits in a single-CTA tile or in a CTA pair's, and the epilogue
+    rounds it the same way, so the two give the same bits."""
+    layer = synth.make_layer(n_in, n_out, ranks, tokens, config_id=1900 + n_out + sum(ranks))
+    paths = gu.device_paths(layer)
+    try:
+        lb.set_prefill_pairs(True)
+        a = gu.bf16_bits(gu.run_gpu(layer, paths=paths))
+        lb.set_prefill_pairs(False)
+        b = gu.bf16_bits(gu.run_gpu(layer, paths=paths))
+    finally:
+        lb.set_prefill_pairs(True)
+    assert np.array_equal(a, b)
 
 
 @pytest.mark.parametrize("tokens", [1, 8, 300])
