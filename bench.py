@@ -88,8 +88,10 @@ def load_peaks():
 
 
 def load_traffic(config, tokens):
-    """dram bytes per call from a committed ncu summary, only if it was taken
-    on the current kernel sources."""
+    """DRAM bytes from a committed ncu summary, only if it was taken on the
+    current kernel sources: per launch of the dominant kernel where the
+    roofline is that kernel's (prefill), else per call (decode, whose
+    roofline is the whole call)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -98,7 +100,7 @@ def load_traffic(config, tokens):
     e = d.get(f"{config}/M{tokens}")
     if not e or e.get("source_hash") != source_hash():
         return None
-    return e.get("dram_bytes_per_call")
+    return e.get("dram_bytes_per_launch", e.get("dram_bytes_per_call"))
 
 
 # ---------------------------------------------------------------- clocks
@@ -474,8 +476,8 @@ def time_contractions(sets, x, tokens, c, stream, device, n):
     out = {}
     cap = torch.cuda.Stream(device)
     flops = {"contraction_1": 2 * tokens * R * c.n_in, "contraction_2": 2 * tokens * R * c.n_out}
-    names = {"contraction_1": "sign_gemm_kernel<1, H> (contraction 1, tcgen05)",
-             "contraction_2": "sign_gemm_kernel<2, H> (contraction 2, tcgen05)"}
+    names = {"contraction_1": "sign_gemm_kernel<1, H, P> (contraction 1, tcgen05)",
+             "contraction_2": "sign_gemm_kernel<2, H, P> (contraction 2, tcgen05)"}
     lat(0)
     torch.cuda.synchronize()
     for key, fn in (("contraction_1", lat), ("contraction_2", exp)):
