@@ -226,24 +226,47 @@ size_t lb_forward_workspace_bytes(int64_t tokens, int64_t n_in, int64_t n_out, i
 }
 
 // Every host-side check of lb_linear_forward (tokens > 0).
-static lb_status check_forward(const uint16_t *x, int64_t tokens, int64_t n_in, int64_t n_out, int64_t ldx,
-                               const lb_path *main, const lb_path *residual, const uint16_t *y, int64_t ldy,
-                               const void *workspace, size_t workspace_bytes)
+// Every host-side check of a forward call (sizes, pointers, alignment,
+// workspace); on success fills `a`.  Launches nothing.
+static lb_status make_forward(const uint16_t *x, int64_t tokens, int64_t n_in, int64_t n_out, int64_t ldx,
+                              const lb_path *main, const lb_path *residual, uint16_t *y, int64_t ldy,
+                              void *workspace, size_t workspace_bytes, lb::ForwardArgs *a)
 {
     if (!x || !y || !main) return LB_ERR_INVALID_ARGUMENT;
     if (ldx < n_in || ldy < n_out) return LB_ERR_INVALID_ARGUMENT;
     if (n_in % 32 != 0 || n_out % 32 != 0 || n_in > kMaxDim || n_out > kMaxDim || tokens > kMaxTokens)
         return LB_ERR_UNSUPPORTED_SHAPE;
     if (ldx % 8 != 0 || ldy % 8 != 0 || !aligned16(x) || !aligned16(y)) return LB_ERR_MISALIGNED;
-    lb::PathDesc d[2];
-    lb_status st = check_path(main, n_in, n_out, &d[0]);
-    if (st == LB_OK && residual) st = check_path(residual, n_in, n_out, &d[1]);
+    *a = lb::ForwardArgs{};
+    a->npaths = residual ? 2 : 1;
+    lb_status st = check_path(main, n_in, n_out, &a->path[0]);
+    if (st == LB_OK && residual) st = check_path(residual, n_in, n_out, &a->path[1]);
     if (st != LB_OK) return st;
-    const int ranks[2] = {d[0].rank, residual ? d[1].rank : 0};
-    const size_t need = workspace_for(tokens, n_in, n_out, ranks, residual ? 2 : 1);
+    const int ranks[2] = {a->path[0].rank, a->npaths > 1 ? a->path[1].rank : 0};
+    const size_t need = workspace_for(tokens, n_in, n_out, ranks, a->npaths);
     if (need > 0 && !workspace) return LB_ERR_INVALID_ARGUMENT;
     if (workspace_bytes < need) return LB_ERR_WORKSPACE_TOO_SMALL;
     if (workspace && !aligned16(workspace)) return LB_ERR_MISALIGNED;
+    a->x = x;
+    a->ldx = ldx;
+    a->tokens = (int)tokens;
+    a->n_in = (int)n_in;
+    a->n_out = (int)n_out;
+    a->y = y;
+    a->ldy = ldy;
+    a->workspace = workspace;
+    a->workspace_bytes = workspace_bytes;
+    return LB_OK;
+}
+
+static lb_status run_forward(const lb::ForwardArgs &a, const lb::DeviceInfo &dev, void *stream)
+{
+    const cudaError_t e = a.tokens > lb::kMidMaxTokens ? lb::prefill_forward(a, dev, static_cast<cudaStream_t>(stream))
+                                                       : lb::decode_forward(a, dev, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
     return LB_OK;
 }
 
@@ -253,47 +276,13 @@ lb_status lb_linear_forward(const uint16_t *x, int64_t tokens, int64_t n_in, int
 {
     if (tokens < 0 || n_in <= 0 || n_out <= 0) return LB_ERR_INVALID_ARGUMENT;
     if (tokens == 0) return LB_OK;
-    if (!x || !y || !main) return LB_ERR_INVALID_ARGUMENT;
-    if (ldx < n_in || ldy < n_out) return LB_ERR_INVALID_ARGUMENT;
-    if (n_in % 32 != 0 || n_out % 32 != 0 || n_in > kMaxDim || n_out > kMaxDim || tokens > kMaxTokens)
-        return LB_ERR_UNSUPPORTED_SHAPE;
-    if (ldx % 8 != 0 || ldy % 8 != 0 || !aligned16(x) || !aligned16(y)) return LB_ERR_MISALIGNED;
-
-    lb::ForwardArgs a{};
-    a.npaths = residual ? 2 : 1;
-    lb_status st = check_path(main, n_in, n_out, &a.path[0]);
+    lb::ForwardArgs a;
+    lb_status st = make_forward(x, tokens, n_in, n_out, ldx, main, residual, y, ldy, workspace, workspace_bytes, &a);
     if (st != LB_OK) return st;
-    if (residual) {
-        st = check_path(residual, n_in, n_out, &a.path[1]);
-        if (st != LB_OK) return st;
-    }
-    const int ranks[2] = {a.path[0].rank, a.npaths > 1 ? a.path[1].rank : 0};
-    const size_t need = workspace_for(tokens, n_in, n_out, ranks, a.npaths);
-    if (need > 0 && !workspace) return LB_ERR_INVALID_ARGUMENT;
-    if (workspace_bytes < need) return LB_ERR_WORKSPACE_TOO_SMALL;
-    if (workspace && !aligned16(workspace)) return LB_ERR_MISALIGNED;
-
-    a.x = x;
-    a.ldx = ldx;
-    a.tokens = (int)tokens;
-    a.n_in = (int)n_in;
-    a.n_out = (int)n_out;
-    a.y = y;
-    a.ldy = ldy;
-    a.workspace = workspace;
-    a.workspace_bytes = workspace_bytes;
-
     lb::DeviceInfo dev;
     st = device_info(&dev);
     if (st != LB_OK) return st;
-    const cudaError_t e = a.tokens > lb::kMidMaxTokens
-                              ? lb::prefill_forward(a, dev, static_cast<cudaStream_t>(stream))
-                              : lb::decode_forward(a, dev, static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        return LB_ERR_CUDA;
-    }
-    return LB_OK;
+    return run_forward(a, dev, stream);
 }
 
 // Fills g from the caller's projections; checks everything a siblings call
@@ -372,6 +361,20 @@ lb_status lb_linear_forward_siblings(const uint16_t *x, int64_t tokens, int64_t 
     return LB_OK;
 }
 
+// The device's view of host memory: the address under which kernels reach
+// `p` when it lies in pinned host memory mapped into the device's address
+// space (as page-locked allocations are with unified addressing); null
+// otherwise (pageable memory, device memory, an unknown pointer).
+static void *device_view(const void *p)
+{
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+}
+
 lb_status lb_linear_forward_host(const uint16_t *x_host, int64_t tokens, int64_t n_in, int64_t n_out,
                                  const lb_path *main, const lb_path *residual, uint16_t *y_host, uint16_t *x_dev,
                                  uint16_t *y_dev, void *workspace, size_t workspace_bytes, void *stream)
@@ -379,17 +382,41 @@ lb_status lb_linear_forward_host(const uint16_t *x_host, int64_t tokens, int64_t
     if (tokens < 0 || n_in <= 0 || n_out <= 0) return LB_ERR_INVALID_ARGUMENT;
     if (tokens == 0) return LB_OK;
     if (!x_host || !y_host) return LB_ERR_INVALID_ARGUMENT;
-    // every check on the device side first: nothing is copied when the call is refused
-    lb_status st = check_forward(x_dev, tokens, n_in, n_out, n_in, main, residual, y_dev, n_out, workspace,
-                                 workspace_bytes);
+    // every check on the device side first: nothing moves when the call is refused
+    lb::ForwardArgs a;
+    lb_status st = make_forward(x_dev, tokens, n_in, n_out, n_in, main, residual, y_dev, n_out, workspace,
+                                workspace_bytes, &a);
     if (st != LB_OK) return st;
+    lb::DeviceInfo dev;
+    st = device_info(&dev);
+    if (st != LB_OK) return st;
+    // 1-4 tokens on the CUDA-core kernels, with both host buffers pinned and
+    // mapped: x reaches x_dev through one gather kernel (a single round trip
+    // over the host link, chained into the forward kernels, where a DMA copy
+    // and the switch from copy engine to kernels cost several times that),
+    // and the last kernel writes y straight into y_host with plain stores
+    if (tokens <= lb::kSmallMaxTokens) {
+        const void *xd = device_view(x_host);
+        void *yd = device_view(y_host);
+        if (xd && yd && aligned16(xd) && aligned16(yd)) {
+            lb::ForwardArgs h = a;
+            h.y = static_cast<uint16_t *>(yd);
+            if (lb::small_fits(h.tokens, lb::group_of_one(h), dev)) {
+                if (lb::host_gather_launch(xd, x_dev, (size_t)tokens * (size_t)n_in * 2,
+                                           static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+                    cudaGetLastError();
+                    return LB_ERR_CUDA;
+                }
+                return run_forward(h, dev, stream);
+            }
+        }
+    }
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaMemcpyAsync(x_dev, x_host, (size_t)tokens * (size_t)n_in * 2, cudaMemcpyHostToDevice, s) != cudaSuccess) {
         cudaGetLastError();
         return LB_ERR_CUDA;
     }
-    st = lb_linear_forward(x_dev, tokens, n_in, n_out, n_in, main, residual, y_dev, n_out, workspace, workspace_bytes,
-                           stream);
+    st = run_forward(a, dev, stream);
     if (st != LB_OK) return st;
     if (cudaMemcpyAsync(y_host, y_dev, (size_t)tokens * (size_t)n_out * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
         cudaGetLastError();

@@ -114,6 +114,12 @@ size_t prefill_workspace_bytes(int tokens, const int *ranks, int npaths);
 cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream);
 cudaError_t prefill_prepare_device(DeviceInfo &dev);  // also fills dev.pair_slots
 bool prefill_pairs_enabled();                          // lb_set_prefill_pairs
+
+// ----------------------------------------------------------------- host buffers (lb_host_io.cu)
+// Copies `bytes` (a multiple of 16) from pinned host memory, given by its
+// device mapping, to device memory with one kernel on `stream`, chained to
+// the kernels before and after it by programmatic dependent launch.
+cudaError_t host_gather_launch(const void *src, void *dst, size_t bytes, cudaStream_t stream);
 cudaError_t prefill_latent(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, uint16_t *z, int64_t ldz);
 cudaError_t prefill_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, const uint16_t *z,
                            int64_t ldz);

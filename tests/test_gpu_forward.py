@@ -297,6 +297,50 @@ def test_layer_object():
     gu.assert_close(gu.bf16_to_f64(y), gu.oracle_y(layer), "module")
 
 
+@pytest.mark.parametrize("tokens", [1, 3, 4])
+def test_host_call_on_pinned_buffers_writes_y_in_place(tokens):
+    """1-4 tokens on pinned host buffers: x reaches x_dev through the gather
+    kernel and the last kernel writes y to host memory directly, so y_dev
+    keeps its sentinel, x_dev holds x, and y_host has the device call's bits."""
+    import torch
+    layer = synth.make_layer(512, 224, [64, 32], tokens, config_id=881)
+    paths = gu.device_paths(layer)
+    x = gu.bf16_tensor(layer["x"])
+    ref = lb.linear_forward(x, paths[0], paths[1])
+    x_host = x.cpu().pin_memory()
+    y_host = torch.full((tokens, 224), 3.0, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.full_like(x, 5.0)
+    y_dev = torch.full((tokens, 224), 7.0, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(max(16, lb.forward_workspace_bytes(tokens, 512, 224, 64, 32)), dtype=torch.uint8, device="cuda")
+    lb.linear_forward_host(x_host, paths[0], paths[1], y_host, x_dev, y_dev, ws)
+    torch.cuda.synchronize()
+    assert lb.device_status() == lb.LB_OK
+    assert np.array_equal(gu.bf16_bits(y_host), gu.bf16_bits(ref))
+    assert np.array_equal(gu.bf16_bits(x_dev), gu.bf16_bits(x)) and bool((y_dev == 7.0).all())
+
+
+def test_host_call_on_pageable_buffers_copies():
+    """Pageable host memory is not visible to the kernels: the call copies x
+    into x_dev and y out of y_dev, with the same bits."""
+    import torch
+    tokens = 2
+    layer = synth.make_layer(512, 224, [64, 32], tokens, config_id=882)
+    paths = gu.device_paths(layer)
+    x = gu.bf16_tensor(layer["x"])
+    ref = lb.linear_forward(x, paths[0], paths[1])
+    x_host = x.cpu().clone()
+    y_host = torch.full((tokens, 224), 3.0, dtype=torch.bfloat16)
+    assert not x_host.is_pinned() and not y_host.is_pinned()
+    x_dev = torch.full_like(x, 5.0)
+    y_dev = torch.full((tokens, 224), 7.0, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(max(16, lb.forward_workspace_bytes(tokens, 512, 224, 64, 32)), dtype=torch.uint8, device="cuda")
+    lb.linear_forward_host(x_host, paths[0], paths[1], y_host, x_dev, y_dev, ws)
+    torch.cuda.synchronize()
+    assert lb.device_status() == lb.LB_OK
+    assert np.array_equal(gu.bf16_bits(y_host), gu.bf16_bits(ref))
+    assert np.array_equal(gu.bf16_bits(x_dev), gu.bf16_bits(x)) and np.array_equal(gu.bf16_bits(y_dev), gu.bf16_bits(ref))
+
+
 @pytest.mark.parametrize("tokens", [1, 8, 300])
 def test_host_buffer_call_equals_device_call(tokens):
     """lb_linear_forward_host: x from pinned host memory and y back to it,
