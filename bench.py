@@ -700,7 +700,7 @@ def run_lb(args, world, rank, local):
            "e2e": {"value": e2e_value, "unit": "GB/s" if decode else "TFLOP/s",
                    "h2d_bytes_per_step": 2 * tokens * c.n_in, "d2h_bytes_per_step": 2 * tokens * c.n_out,
                    "steps": e2e_steps, "call": "lb_linear_forward_host (pinned host x and y; " + (
-                       "x gathered by a kernel in one pass, y written in place by the last kernel)" if tokens <= 4 else
+                       "x gathered by a kernel in one pass, y written in place by the last kernel)" if tokens <= 128 else
                        "copied through device buffers inside the call)")},
            "gpu_launches": 2 * args.steps,  # contraction 1 + contraction 2 per call, decode and prefill
            "impl": "lb"}

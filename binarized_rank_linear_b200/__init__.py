@@ -296,7 +296,7 @@ def linear_forward_host(x_host, main: PackedPath, residual: PackedPath | None, y
     """``lb_linear_forward_host``: x from pinned host memory (bf16 [tokens,
     n_in], contiguous) through the caller's device buffers x_dev and y_dev to
     y in pinned host memory (bf16 [tokens, n_out]), all on one stream; y_host
-    is valid once the stream is synchronised.  For 1-4 tokens on pinned
+    is valid once the stream is synchronised.  For 1-128 tokens on pinned
     buffers x comes in through a gather kernel and y is written to y_host by
     the last kernel (y_dev is then not touched)."""
     tokens, n_in = x_host.shape

@@ -390,25 +390,24 @@ lb_status lb_linear_forward_host(const uint16_t *x_host, int64_t tokens, int64_t
     lb::DeviceInfo dev;
     st = device_info(&dev);
     if (st != LB_OK) return st;
-    // 1-4 tokens on the CUDA-core kernels, with both host buffers pinned and
-    // mapped: x reaches x_dev through one gather kernel (a single round trip
-    // over the host link, chained into the forward kernels, where a DMA copy
-    // and the switch from copy engine to kernels cost several times that),
-    // and the last kernel writes y straight into y_host with plain stores
-    if (tokens <= lb::kSmallMaxTokens) {
+    // Up to 128 tokens (the decode kernels, whose last kernel stores y with
+    // plain coalesced stores), with both host buffers pinned and mapped: x
+    // reaches x_dev through one gather kernel (a single round trip over the
+    // host link, chained into the forward kernels, where a DMA copy and the
+    // switch from copy engine to kernels cost several times that), and the
+    // last kernel writes y straight into y_host
+    if (tokens <= lb::kMidMaxTokens) {
         const void *xd = device_view(x_host);
         void *yd = device_view(y_host);
         if (xd && yd && aligned16(xd) && aligned16(yd)) {
             lb::ForwardArgs h = a;
             h.y = static_cast<uint16_t *>(yd);
-            if (lb::small_fits(h.tokens, lb::group_of_one(h), dev)) {
-                if (lb::host_gather_launch(xd, x_dev, (size_t)tokens * (size_t)n_in * 2,
-                                           static_cast<cudaStream_t>(stream)) != cudaSuccess) {
-                    cudaGetLastError();
-                    return LB_ERR_CUDA;
-                }
-                return run_forward(h, dev, stream);
+            if (lb::host_gather_launch(xd, x_dev, (size_t)tokens * (size_t)n_in * 2,
+                                       static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+                cudaGetLastError();
+                return LB_ERR_CUDA;
             }
+            return run_forward(h, dev, stream);
         }
     }
     const cudaStream_t s = static_cast<cudaStream_t>(stream);

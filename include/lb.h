@@ -218,13 +218,12 @@ LB_API lb_status lb_expand_forward(const uint16_t *z, int64_t tokens, int64_t n_
  * of y_dev into y_host (one cudaMemcpyAsync each way).  For callers whose
  * activations live on the host; the library allocates nothing, so the device
  * buffers are the caller's.
- * For 1-4 tokens, when both host buffers are pinned memory mapped into the
+ * For 1-128 tokens, when both host buffers are pinned memory mapped into the
  * device's address space (page-locked allocations are, with unified
- * addressing) and the call runs on the CUDA-core kernels, x reaches x_dev
- * through a kernel that reads it from host memory in one pass instead of a
- * copy, and the last kernel writes y into y_host directly, leaving y_dev
- * untouched: the same bytes cross the host link, inside the kernel chain.
- * The result is the same to the bit.
+ * addressing), x reaches x_dev through a kernel that reads it from host
+ * memory in one pass instead of a copy, and the last kernel writes y into
+ * y_host directly, leaving y_dev untouched: the same bytes cross the host
+ * link, inside the kernel chain.  The result is the same to the bit.
  *   x_host : bf16 [tokens x n_in], rows contiguous (row stride n_in); pinned
  *            (page-locked) memory for the copy to be asynchronous
  *   y_host : bf16 [tokens x n_out], rows contiguous; pinned likewise.  Valid
