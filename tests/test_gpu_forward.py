@@ -319,6 +319,31 @@ def test_host_call_on_pinned_buffers_writes_y_in_place(tokens):
     assert np.array_equal(gu.bf16_bits(x_dev), gu.bf16_bits(x)) and bool((y_dev == 7.0).all())
 
 
+@pytest.mark.parametrize("tokens", [1, 37])
+def test_back_to_back_host_calls_share_device_buffers(tokens):
+    """Several host-buffer calls queued on one stream without a sync, all
+    through the same x_dev: each call's gather kernel must wait for the
+    previous call's kernels before it overwrites x_dev, so every y_host holds
+    its own input's result."""
+    import torch
+    layers = [synth.make_layer(512, 224, [64, 32], tokens, config_id=890 + i) for i in range(4)]
+    paths = gu.device_paths(layers[0])
+    x_dev = torch.empty((tokens, 512), dtype=torch.bfloat16, device="cuda")
+    y_dev = torch.empty((tokens, 224), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(max(16, lb.forward_workspace_bytes(tokens, 512, 224, 64, 32)), dtype=torch.uint8, device="cuda")
+    xs = [gu.bf16_tensor(L["x"]).cpu().pin_memory() for L in layers]
+    ys = [torch.zeros((tokens, 224), dtype=torch.bfloat16).pin_memory() for _ in layers]
+    torch.cuda.synchronize()
+    for _ in range(3):
+        for xh, yh in zip(xs, ys):
+            lb.linear_forward_host(xh, paths[0], paths[1], yh, x_dev, y_dev, ws)
+    torch.cuda.synchronize()
+    assert lb.device_status() == lb.LB_OK
+    for xh, yh in zip(xs, ys):
+        ref = lb.linear_forward(xh.cuda(), paths[0], paths[1])
+        assert np.array_equal(gu.bf16_bits(yh), gu.bf16_bits(ref))
+
+
 def test_host_call_on_pageable_buffers_copies():
     """Pageable host memory is not visible to the kernels: the call copies x
     into x_dev and y out of y_dev, with the same bits."""
