@@ -29,6 +29,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -67,13 +68,22 @@ def workload_name(c, tokens):
             f"{c.paths} path(s) x rank {c.rank}, {tokens} token(s)")
 
 
+def source_code(text):
+    """A C/CUDA source with its comments removed and whitespace collapsed: what
+    the compiler sees (the kernel sources hold no "//" or "/*" in a string)."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def source_hash():
-    """Hash of every kernel source: a traffic figure taken on other sources is stale."""
+    """Hash of every kernel source's code: a traffic figure taken on other code
+    is stale (comments and layout do not count)."""
     h = hashlib.sha256()
     for f in sorted(os.listdir(CSRC)):
         if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(CSRC, f), "rb") as fh:
-                h.update(f.encode() + b"\0" + fh.read())
+            with open(os.path.join(CSRC, f)) as fh:
+                h.update(f.encode() + b"\0" + source_code(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -14,9 +14,10 @@
 // to bf16); contraction 2 runs fp16 x fp16 (z rounded to fp16; h exact).
 // Accumulation is fp32 in tensor memory.
 //
-// A persistent grid (one CTA per SM) walks the 128 x bn tiles of C = A . B^T,
-// bn a multiple of 32 up to 256 chosen per call (see plan_tiles).
-// In each CTA:
+// A persistent grid (one CTA per SM, or one CTA pair per two SMs) walks the
+// tiles of C = A . B^T, 128 or 256 rows per CTA by bn columns, bn a multiple
+// of 32 up to 256, the shape chosen per call (see plan_tiles).  In each CTA
+// (here for single-CTA tiles of 128 rows):
 //   warp 0       allocates tensor memory (two 256-column accumulators) and
 //                streams A tiles with TMA (128-byte swizzle, no multicast)
 //   warp 1       one thread issues tcgen05.mma (M = 128, N = bn, K = 16)
@@ -62,12 +63,12 @@ constexpr uint32_t TMEM_COLS = 2 * BN;        // two 256-column accumulators
 constexpr uint32_t G_BYTES = 2 * BK * 2;      // a K-block of g for both paths
 constexpr uint32_t OUT_BYTES = 32 * 64;       // an output box: 32 rows x 32 two-byte columns
 
-// Two tile shapes.  H = 1: a CTA tile is 128 x 256; the two accumulators
-// double-buffer consecutive tiles, and two producer groups take alternate
-// K-blocks.  H = 2: a CTA tile is 256 x 256, two M = 128 halves that share
-// each expanded B tile (half the sign expansion per flop); the two
-// accumulators hold the halves of one tile, and one producer group has twice
-// as long per K-block.
+// Two tile heights.  H = 1: a CTA holds 128 rows of a tile; the two
+// accumulators double-buffer consecutive tiles, and (P = 1) two producer
+// groups take alternate K-blocks.  H = 2: a CTA holds 256 rows, two M = 128
+// halves that share each expanded B tile (half the sign expansion per flop);
+// the two accumulators hold the halves of one tile, and (P = 1) one producer
+// group has twice as long per K-block.
 //
 // P = 2: a CTA pair (cluster of two) shares each MMA (cta_group::2, M = 256):
 // CTA r of the pair holds rows 128 H r .. of the pair's 256 H-row tile of A

@@ -107,3 +107,14 @@ def test_tensor_peak_follows_the_sampled_clocks():
     slow = dict(at_max, sm_mhz=1365.0)
     assert bench.tensor_peak(peaks, slow) == (1401.9, "measured (sustained)")
     assert bench.tensor_peak(peaks, {"error": "nvml unavailable"}) == (1651.4, "measured (burst)")
+
+
+def test_source_hash_sees_code_not_comments():
+    """Traffic figures stay valid across comment edits and go stale on any
+    change to the code itself."""
+    a = "int f(int x) { return x + 1; }  // one\n/* two */\n"
+    b = "// one, reworded\nint f(int x)\n{\n    return x + 1; /* three */\n}\n"
+    c = "int f(int x) { return x + 2; }\n"
+    assert bench.source_code(a) == bench.source_code(b)
+    assert bench.source_code(a) != bench.source_code(c)
+    assert "one" not in bench.source_code(a) and "two" not in bench.source_code(a)
