@@ -295,8 +295,10 @@ def run_reference(args, world, rank):
 
 # ---------------------------------------------------------------- the GPU arm
 
-def kernel_label(tokens):
-    if tokens <= 4:
+def kernel_label(tokens, sign_bits=0):
+    """The kernels a call runs, as the library dispatches: 1-4 tokens on CUDA
+    cores unless 3-4 tokens x sign bits (sum of r (in + out)) pass 80 M."""
+    if tokens <= 2 or (tokens <= 4 and tokens * sign_bits <= 80_000_000):
         return "lb_linear_forward call: small1_kernel + small2_kernel (CUDA cores, PDL-chained)"
     if tokens <= 128:
         return ("lb_linear_forward call: mid_gemm_kernel<1> + mid_gemm_kernel<2> "
@@ -666,7 +668,7 @@ def run_lb(args, world, rank, local):
         achieved = nbytes / per_call_s / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm"], "traffic": load_traffic(args.config, tokens),
-                "kernel": kernel_label(tokens),
+                "kernel": kernel_label(tokens, c.rank * c.paths * (c.n_in + c.n_out)),
                 "peak_source": peaks["source"]}
     else:
         pk, pk_source = tensor_peak(peaks, clk.summary())
@@ -686,7 +688,7 @@ def run_lb(args, world, rank, local):
             achieved = nflops / per_call_s / 1e12
             roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
                     "frac": achieved / pk, "traffic": load_traffic(args.config, tokens),
-                    "kernel": kernel_label(tokens),
+                    "kernel": kernel_label(tokens, c.rank * c.paths * (c.n_in + c.n_out)),
                     "peak_source": pk_source}
     cpu = None
     if world == 1 and not args.no_cpu:

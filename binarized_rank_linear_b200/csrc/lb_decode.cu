@@ -75,6 +75,23 @@ GroupArgs sizes_only(int tokens, int n_in, int n_out, const int *ranks, int npat
     return group_of_one(a);
 }
 
+// 1-4 tokens go to the CUDA-core kernels when they fit, except 3-4 tokens on
+// wide layers: their tables and lookups grow with the tokens while the
+// tcgen05 kernels cost about the same at 1-16 tokens (B200, Llama-2-7B
+// gate/up: 6.9, 9.6, 14.9, 19.4 us at 1-4 tokens against 15.2 on tcgen05;
+// q_proj 12.3 against 14.8 at 4 tokens).  The switch is at tokens x sign
+// bits (sum of r (n_in + n_out) over the group's paths) above 80 M.
+bool small_preferred(int M, const GroupArgs &g, const DeviceInfo &dev)
+{
+    if (M > kSmallMaxTokens || !small_fits(M, g, dev)) return false;
+    if (M <= 2) return true;
+    int64_t bits = 0;
+    for (int j = 0; j < g.nproj; ++j)
+        for (int q = 0; q < g.proj[j].npaths; ++q)
+            bits += (int64_t)g.proj[j].path[q].rank * (g.n_in + g.proj[j].n_out);
+    return (int64_t)M * bits <= 80000000;
+}
+
 size_t layer_workspace_bytes(const ForwardArgs &a)
 {
     const int ranks[2] = {a.path[0].rank, a.npaths > 1 ? a.path[1].rank : 0};
@@ -96,7 +113,7 @@ cudaError_t decode_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStre
     const GroupArgs g = group_of_one(a);
     for (int m0 = 0; m0 < a.tokens; m0 += kMidMaxTokens) {
         const int M = std::min(kMidMaxTokens, a.tokens - m0);
-        const cudaError_t e = M <= kSmallMaxTokens && small_fits(M, g, dev) ? small_forward(g, dev, stream, m0, M)
+        const cudaError_t e = small_preferred(M, g, dev) ? small_forward(g, dev, stream, m0, M)
                                                                              : mid_forward(a, dev, stream, m0, M);
         if (e != cudaSuccess) return e;
     }
@@ -114,7 +131,7 @@ size_t group_workspace_bytes(const GroupArgs &g)
 
 cudaError_t group_forward(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream)
 {
-    if (g.tokens <= kSmallMaxTokens && small_fits(g.tokens, g, dev)) return small_forward(g, dev, stream, 0, g.tokens);
+    if (small_preferred(g.tokens, g, dev)) return small_forward(g, dev, stream, 0, g.tokens);
     if (g.tokens <= kMidMaxTokens) return mid_group_forward(g, dev, stream, 0, g.tokens);
     for (int j = 0; j < g.nproj; ++j) {
         const cudaError_t e = prefill_forward(layer_of(g, j), dev, stream);

@@ -91,7 +91,11 @@ def test_blocks_are_the_models_linears():
 
 
 def test_kernel_labels_follow_the_dispatch():
-    assert "small1_kernel" in bench.kernel_label(1) and "small1_kernel" in bench.kernel_label(4)
+    q7 = 2 * 1024 * (4096 + 4096)      # Llama-2-7B q_proj sign bits
+    gate7 = 2 * 800 * (4096 + 11008)   # Llama-2-7B gate/up
+    assert "small1_kernel" in bench.kernel_label(1, gate7) and "small1_kernel" in bench.kernel_label(2, gate7)
+    assert "small1_kernel" in bench.kernel_label(4, q7) and "small1_kernel" in bench.kernel_label(3, gate7)
+    assert "mid_gemm_kernel" in bench.kernel_label(4, gate7)
     assert "mid_gemm_kernel" in bench.kernel_label(5) and "mid_gemm_kernel" in bench.kernel_label(128)
     assert "sign_gemm_kernel" in bench.kernel_label(129)
 
