@@ -89,6 +89,11 @@ TILE_PLAN_CASES = [
     pytest.param(900, 512, 6016, [256, 224], id="m900-c2-pair-w192-ragged-n"),
     pytest.param(520, 256, 8192, [512, 512], id="m520-c2-pair-h2-w224-ragged"),
     pytest.param(5000, 1024, 256, [512, 512], id="m5000-c1-pair-h2-w160-ragged"),
+    # K not a multiple of the 64-column K-block in both contractions, and the
+    # two paths meeting inside a K-block of contraction 2 (r0 = 480)
+    pytest.param(5000, 1056, 288, [480, 512], id="m5000-c1-pair-h2-ragged-k"),
+    pytest.param(520, 288, 8192, [480, 512], id="m520-c2-pair-h2-ragged-k-mid-block-paths"),
+    pytest.param(3000, 1056, 2048, [480, 512], id="m3000-pair-both-ragged-k"),
 ]
 
 
@@ -149,8 +154,9 @@ def test_integer_exact_is_bitwise(tokens):
 
 
 @pytest.mark.parametrize("n_in,n_out,ranks,tokens", [(256, 8192, [512, 512], 520), (256, 256, [512, 512], 2600),
-                                                     (512, 224, [64, 32], 300), (512, 224, [64, 32], 1000)],
-                         ids=["c2-h2", "c1-wide", "m300", "m1000"])
+                                                     (512, 224, [64, 32], 300), (512, 224, [64, 32], 1000),
+                                                     (288, 8192, [480, 512], 520)],
+                         ids=["c2-h2", "c1-wide", "m300", "m1000", "ragged-k"])
 def test_integer_exact_prefill_tiles_are_bitwise(n_in, n_out, ranks, tokens, prefill_pairs):
     """The integer-exact case on prefill shapes, on CTA pairs and on single
     CTAs.  Every value is an integer well inside fp32's exact range and z
