@@ -214,18 +214,22 @@ def test_deterministic_and_workspace_independent():
     assert all(np.array_equal(outs[0], o) for o in outs[1:])
 
 
-def test_strided_io_and_canaries():
+@pytest.mark.parametrize("tokens", [2, 5, 300, 1000])
+def test_strided_io_and_canaries(tokens, prefill_pairs):
+    """x and y with row strides past their widths, on every kernel family
+    (the prefill ones on CTA pairs and on single CTAs): y right, and nothing
+    written past its columns or rows."""
     t = torch()
-    layer = synth.make_layer(256, 128, [32, 64], 5, config_id=800)
+    layer = synth.make_layer(256, 128, [32, 64], tokens, config_id=800)
     paths = gu.device_paths(layer)
-    xb = t.zeros((5, 264), dtype=t.bfloat16, device="cuda")
+    xb = t.zeros((tokens, 264), dtype=t.bfloat16, device="cuda")
     xb[:, :256] = gu.bf16_tensor(layer["x"])
-    ybig = t.full((7, 136), 12345.0, dtype=t.bfloat16, device="cuda")
-    y = ybig[:5, :128]
+    ybig = t.full((tokens + 2, 136), 12345.0, dtype=t.bfloat16, device="cuda")
+    y = ybig[:tokens, :128]
     lb.linear_forward(xb[:, :256], paths[0], paths[1], y=y)
     t.cuda.synchronize()
-    gu.assert_close(gu.bf16_to_f64(y.contiguous()), gu.oracle_y(layer), "strided")
-    assert bool((ybig[:, 128:] == 12345.0).all()) and bool((ybig[5:] == 12345.0).all())
+    gu.assert_close(gu.bf16_to_f64(y.contiguous()), gu.oracle_y(layer), f"strided M={tokens}")
+    assert bool((ybig[:, 128:] == 12345.0).all()) and bool((ybig[tokens:] == 12345.0).all())
 
 
 def test_bad_arguments_write_nothing():

@@ -53,7 +53,7 @@ def test_halves_against_the_oracle(name, tokens):
     assert lb.device_status() == lb.LB_OK
 
 
-@pytest.mark.parametrize("tokens", [7, 40])
+@pytest.mark.parametrize("tokens", [7, 40, 300])
 def test_strided_latent_and_unread_halves(tokens):
     """A latent with row stride r + 24 (the padding is never written), and
     each call given only the half of a path it reads (the rest null)."""
