@@ -200,13 +200,16 @@ def test_sign_flip_invariance_is_bitwise(tokens):
     assert np.array_equal(y0, y1)
 
 
-def test_deterministic_and_workspace_independent():
+@pytest.mark.parametrize("tokens", [1, 16, 300])
+def test_deterministic_and_workspace_independent(tokens):
+    """Repeated calls give the same bits whatever the workspace held before
+    (CUDA-core, tcgen05 decode and prefill pair kernels)."""
     t = torch()
-    layer = synth.make_config("llama2_7b_gate", 16)
+    layer = synth.make_config("llama2_7b_gate", tokens)
     paths = gu.device_paths(layer)
     x = gu.bf16_tensor(layer["x"])
     c = synth.CONFIGS["llama2_7b_gate"]
-    need = lb.forward_workspace_bytes(16, c.n_in, c.n_out, c.rank, c.rank)
+    need = lb.forward_workspace_bytes(tokens, c.n_in, c.n_out, c.rank, c.rank)
     outs = []
     for fill in (0, 0xFF, 0x7C):
         ws = t.full((need,), fill, dtype=t.uint8, device="cuda")
