@@ -1,24 +1,31 @@
 """Benchmark of the LittleBit factored layer's forward pass on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {lb,reference}]
-                    [--config NAME] [--tokens M]
+                    [--config NAME] [--tokens M] [--no-extras]
 
-One step is one ``lb_linear_forward`` call (both contractions, both paths)
-over one batch of synthetic input.  Default workload: the Llama-2-7B q_proj
-shape (4096 -> 4096, eff_bit 1.0, residual on: two paths of rank 1024) at
-batch 1.  Steps rotate over enough copies of the weights that the set is
-larger than twice the L2 cache, so every call streams its sign bits from HBM;
-the calls run back to back from CUDA graphs (the chained, per-layer number).
+Default workload: the Llama-2-7B q_proj shape (4096 -> 4096, eff_bit 1.0,
+residual on: two paths of rank 1024) at batch 1.  One step is one pass over
+a rotation of distinct copies of the layer's weights (1024 copies, 2.2 GB:
+a chain of 1024 layers of this shape), every copy one ``lb_linear_forward``
+call (both contractions, both paths), chained on one stream from one CUDA
+graph.  The copies span far more than twice the L2 cache and the warm-up
+passes over all of them, so every timed call streams its sign bits from HBM.
 
 Printed on rank 0, one JSON line:
   value       whole-job algorithmic HBM GB/s (prefill workloads: TFLOP/s),
-              device-timed with CUDA events, max over ranks
+              device-timed with CUDA events, max over ranks; us_per_call is
+              the timed region over the calls in it
   e2e         the same metric through the C ABI with host buffers
-              (lb_linear_forward_host: pinned x copied in, y copied out,
-              every step)
+              (lb_linear_forward_host: pinned x in, y out, every call)
   roofline    achieved GB/s of the forward call against the measured HBM peak
   cpu_baseline the fp64 oracle on this host's cores (bounded sample)
   clocks      SM clocks and throttle reasons sampled during the timed region
+  prefill     Qwen3-14B gate/up and k/v at 8192 tokens: TFLOP/s, the dominant
+              kernel's roofline against the measured bf16 peak, clocks
+  decode_block_fused  a Llama-2-7B decoder block's seven linears at 1 token as
+              four sibling calls, chained
+  dense_baseline      Llama-2-70B gate/up at 1 token against one cuBLAS bf16
+              GEMM on the same layer as a dense matrix
 With ``--impl reference`` the fp64 CPU oracle is timed instead (rank 0 only).
 Multi-GPU runs are independent replicas (the layer needs no exchange at this
 scale): every rank runs the same workload on its own GPU.
@@ -306,46 +313,268 @@ def kernel_label(tokens, sign_bits=0):
     return "lb_linear_forward call: sign_gemm_kernel<1> + sign_gemm_kernel<2> (tcgen05, persistent)"
 
 
-def dense_baseline(layer, x, steps, stream, device):
-    """The layer as the dense bf16 matrix W = sum_p diag(h_p) S_U diag(l_p)
-    S_V^T diag(g_p), applied with one cuBLAS GEMM per call (torch.matmul): the comparison the pages' kernel speedup
-    figure makes (littlebitllm.com, "How small"; the single-kernel speedup
-    quoted for a Llama2-70B layer).  W is built with plain PyTorch ops on the
-    GPU; copies rotate past twice the L2 cache, as the packed weights do."""
+def rotation_size(set_bytes, min_sets=1, cap_bytes=4 << 30, max_sets=4096):
+    """Weight copies to rotate over: enough that the copies span more than
+    twice the L2 cache (every call then finds its weights evicted: between two
+    uses of a copy, more than the cache's capacity of other copies is read),
+    at least `min_sets`, at most `max_sets` and `cap_bytes` of weights."""
+    n = max(-(-2 * L2_BYTES // max(1, set_bytes)) + 1, min_sets)
+    return max(1, min(n, max_sets, max(1, cap_bytes // max(1, set_bytes))))
+
+
+def dense_weight_torch(layer, device):
+    """The layer as one dense fp32 matrix W [n_out, n_in] built with plain
+    PyTorch ops: W = sum_p diag(h_p) S_U,p diag(l_p) S_V,p^T diag(g_p)
+    (sesamedisk.com, "Samsung LittleBit 13B Model", "How low-rank binarization
+    works": h scales rows, g columns, l the latent dimension).  The comparison
+    arm of the dense baseline; tests check it against the oracle's dense W."""
     import torch
     W = None
     for p in layer["paths"]:
         t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
         su, sv = t(p["su"]).float(), t(p["sv"]).float()
-        h, g, l = (t(p[k].view(np.int16)).view(torch.float16).float() for k in ("h", "g", "l"))
+        h, g, l = (t(np.asarray(p[k], dtype=np.float16).view(np.int16)).view(torch.float16).float()
+                   for k in ("h", "g", "l"))
         term = (h[:, None] * su * l[None, :]) @ (sv * g[:, None]).t()
         W = term if W is None else W + term
-    W = W.to(torch.bfloat16)
-    w_bytes = W.numel() * 2
-    nsets = max(1, min(64, -(-2 * L2_BYTES // w_bytes) + 1))
-    Ws = [W] + [W.clone() for _ in range(nsets - 1)]
-    y = torch.empty((x.shape[0], W.shape[0]), dtype=torch.bfloat16, device=device)
-    per_graph = max(nsets, 32)
-    cap = torch.cuda.Stream(device)
-    torch.matmul(x, Ws[0].t(), out=y)  # warm the cuBLAS handle before capture
+    return W
+
+
+def time_graph(graph, reps, stream, local, world, device):
+    """Replays `graph` `reps` times between CUDA events on `stream`, with a
+    barrier and a synchronise on both sides, sampling clocks meanwhile.
+    Returns (max-over-ranks ms, clock summary)."""
+    import torch
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(local)
+    barrier(world)
     torch.cuda.synchronize()
+    with clk:
+        start.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        stop.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(start.elapsed_time(stop), world, device), clk.summary()
+
+
+class DeviceLayer:
+    """One synthetic workload on the device: its packed paths (and copies of
+    them to rotate over), x, y and the workspace."""
+
+    def __init__(self, layer, device, tokens):
+        import torch
+        import binarized_rank_linear_b200 as lb
+        self.lb = lb
+        self.layer, self.device, self.tokens = layer, device, tokens
+        self.base = []
+        for p in layer["paths"]:
+            dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+            self.base.append(lb.PackedPath.from_factors(dev(p["su"]), dev(p["sv"]), dev(p["h"]), dev(p["g"]),
+                                                        dev(p["l"])))
+        self.n_in, self.n_out = layer["n_in"], layer["n_out"]
+        self.ranks = [p.rank for p in self.base]
+        self.set_bytes = sum(p.u_bits.numel() * 4 + p.vt_bits.numel() * 4 for p in self.base)
+        self.nbytes = algorithmic_bytes(self.n_in, self.n_out, self.ranks, tokens)
+        self.nflops = algorithmic_flops(self.n_in, self.n_out, self.ranks, tokens)
+        self.x = torch.from_numpy(layer["x"].view(np.int16)).to(device).view(torch.bfloat16)
+        self.y = torch.empty((tokens, self.n_out), dtype=torch.bfloat16, device=device)
+        self.ws = torch.empty(max(16, lb.forward_workspace_bytes(tokens, self.n_in, self.n_out, self.ranks[0],
+                                                                 self.ranks[1] if len(self.ranks) > 1 else 0)),
+                              dtype=torch.uint8, device=device)
+        self.sets = [self.base]
+
+    def rotate(self, nsets):
+        lb = self.lb
+        clone = lambda p: lb.PackedPath(p.u_bits.clone(), p.vt_bits.clone(), p.h.clone(), p.g.clone(),
+                                        p.l.clone(), p.rank)
+        self.sets = [self.base] + [[clone(p) for p in self.base] for _ in range(nsets - 1)]
+
+    def call(self, i, x=None, stream=None):
+        s = self.sets[i % len(self.sets)]
+        self.lb.linear_forward(self.x if x is None else x, s[0], s[1] if len(s) > 1 else None, y=self.y,
+                               workspace=self.ws, stream=stream)
+
+    def parity(self, rows):
+        """Sampled rows of the last call's y against the fp64 oracle."""
+        import torch
+        import oracle
+        L = self.layer
+        ref = oracle.forward(oracle.bf16_bits_to_f64(L["x"][rows]),
+                             [dict(su=p["su"], sv=p["sv"], h=oracle.f16_to_f64(p["h"]), g=oracle.f16_to_f64(p["g"]),
+                                   l=oracle.f16_to_f64(p["l"])) for p in L["paths"]])
+        got = oracle.bf16_bits_to_f64(self.y[torch.from_numpy(rows).to(self.device)].view(torch.int16).cpu()
+                                      .numpy().view(np.uint16))
+        out = {"rows": int(len(rows)), "rel_l2": float(np.linalg.norm(got - ref) / np.linalg.norm(ref)),
+               "max_err_over_max_y": float(np.abs(got - ref).max() / np.abs(ref).max())}
+        assert out["rel_l2"] <= 5e-3 and out["max_err_over_max_y"] <= 1e-2, out
+        return out
+
+
+def capture(fn, n, device):
+    """A CUDA graph of fn(0), ..., fn(n - 1)."""
+    import torch
+    cap = torch.cuda.Stream(device)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=cap):
-        for i in range(per_graph):
-            torch.matmul(x, Ws[i % nsets].t(), out=y)
+        for i in range(n):
+            fn(i)
+    return g
+
+
+def time_contractions(d, xs, stream, device, n):
+    """Each contraction of the prefill path on its own: lb_latent_forward and
+    lb_expand_forward run the same two kernels as lb_linear_forward at these
+    token counts.  CUDA graphs of n calls each, over the rotating inputs,
+    timed with events on `stream`; flops per contraction from the workload
+    table (2 M R n_in and 2 M R n_out)."""
+    import torch
+    import binarized_rank_linear_b200 as lb
+    tokens = d.tokens
+    R = sum(d.ranks)
+    z = torch.empty((tokens, R), dtype=torch.float16, device=device)
+    y = torch.empty((tokens, d.n_out), dtype=torch.bfloat16, device=device)
+    two = lambda s: (s[0], s[1] if len(s) > 1 else None)
+    lat = lambda i: lb.latent_forward(xs[i % len(xs)], *two(d.sets[i % len(d.sets)]), z=z)
+    exp = lambda i: lb.expand_forward(z, *two(d.sets[i % len(d.sets)]), y=y)
+    out = {}
+    flops = {"contraction_1": 2 * tokens * R * d.n_in, "contraction_2": 2 * tokens * R * d.n_out}
+    names = {"contraction_1": "sign_gemm_kernel<1, H, P> (contraction 1, tcgen05)",
+             "contraction_2": "sign_gemm_kernel<2, H, P> (contraction 2, tcgen05)"}
+    lat(0)
+    torch.cuda.synchronize()
+    for key, fn in (("contraction_1", lat), ("contraction_2", exp)):
+        g = capture(fn, n, device)
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / n
+        out[key] = {"kernel": names[key], "flop": flops[key], "us_alone": us, "TFLOP/s_alone": flops[key] / us / 1e6}
+        del g
+    total = sum(v["us_alone"] for v in out.values())
+    for v in out.values():
+        v["share"] = v["us_alone"] / total
+    return out
+
+
+def measure_prefill(name, args, world, local, device, peaks, tokens=None):
+    """One prefill workload (Qwen3-14B linears at 8192 tokens by default):
+    the call chained from a CUDA graph, inputs larger than L2 (x rotated over
+    copies where x and y together are not), at least `--prefill-seconds` of
+    timed calls with the clocks sampled meanwhile; the dominant kernel's
+    roofline from its share of the call."""
+    import torch
+    c = synth.CONFIGS[name]
+    tokens = tokens or c.tokens[0]
+    d = DeviceLayer(synth.make_config(name, tokens), device, tokens)
+    io = 2 * tokens * (d.n_in + d.n_out)
+    nx = max(1, min(4, -(-2 * L2_BYTES // io) + 1)) if io <= 2 * L2_BYTES else 1
+    xs = [d.x] + [d.x.clone() for _ in range(nx - 1)]
+    d.call(0)
+    torch.cuda.synchronize()
+    assert d.lb.device_status() == d.lb.LB_OK
+    rng = np.random.default_rng(2)
+    rows = np.unique(np.concatenate([[0, 127, 128, 255, 256, 511, tokens - 1], rng.choice(tokens, 9, replace=False)]))
+    parity = d.parity(rows) if not args.no_parity else None
+    g = capture(lambda i: d.call(i, x=xs[i % nx]), nx, device)
+    for _ in range(max(3, args.warmup)):
+        g.replay()
+    torch.cuda.synchronize()
+    # size the region from one timed replay
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream(device)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    reps = max(3, int(args.prefill_seconds / max(1e-6, e0.elapsed_time(e1) / 1e3)))
+    ms, clocks = time_graph(g, reps, stream, local, world, device)
+    assert d.lb.device_status() == d.lb.LB_OK
+    calls = reps * nx
+    per_call_s = ms / 1e3 / calls
+    per_kernel = time_contractions(d, xs, stream, device, max(3, min(50, calls)))
+    dom = max(per_kernel.values(), key=lambda k: k["share"])
+    pk, pk_source = tensor_peak(peaks, clocks)
+    achieved = dom["flop"] / (per_call_s * dom["share"]) / 1e12
+    return {"workload": workload_name(c, tokens), "tokens": tokens, "calls": calls,
+            "l2": "inputs larger than L2" + (" (x rotated over %d copies)" % nx if nx > 1 else ""),
+            "us_per_call": per_call_s * 1e6, "value": aggregate(d.nflops / 1e12 * calls, ms / 1e3, world),
+            "unit": "TFLOP/s", "algorithmic_flops_per_call": d.nflops,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
+                         "frac": achieved / pk, "traffic": load_traffic(name, tokens), "kernel": dom["kernel"],
+                         "share_of_call": dom["share"], "call_TFLOP/s": d.nflops / per_call_s / 1e12,
+                         "peak_source": pk_source},
+            "per_kernel": per_kernel, "parity": parity, "clocks": clocks, "gpu_launches": 2 * calls}
+
+
+def dense_baseline(d, device, seconds, stream, local, world):
+    """The layer as the dense bf16 matrix of dense_weight_torch, applied with
+    one cuBLAS GEMM per call (torch.matmul): the comparison behind the pages'
+    kernel speedup figure (sesamedisk.com, "Samsung LittleBit 13B Model", "The
+    speedup number": a single-kernel speedup over FP16 for one Llama2-70B MLP
+    layer).  Copies of W rotate past twice the L2 cache, as the packed weights
+    do; calls are chained from a CUDA graph."""
+    import torch
+    W = dense_weight_torch(d.layer, device).to(torch.bfloat16)
+    w_bytes = W.numel() * 2
+    nsets = rotation_size(w_bytes, max_sets=64)
+    Ws = [W] + [W.clone() for _ in range(nsets - 1)]
+    y = torch.empty((d.tokens, W.shape[0]), dtype=torch.bfloat16, device=device)
+    n = max(nsets, 32)
+    torch.matmul(d.x, Ws[0].t(), out=y)  # warm the cuBLAS handle before capture
+    torch.cuda.synchronize()
+    g = capture(lambda i: torch.matmul(d.x, Ws[i % nsets].t(), out=y), n, device)
     for _ in range(3):
         g.replay()
     torch.cuda.synchronize()
-    reps = max(1, min(200, steps // per_graph))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(reps):
-        g.replay()
+    g.replay()
     e1.record(stream)
     torch.cuda.synchronize()
-    us = e0.elapsed_time(e1) * 1e3 / (reps * per_graph)
-    return {"us_per_call": us, "kind": "cuBLAS bf16 GEMM (torch.matmul) on the dense weight, CUDA graphs",
-            "dense_weight_bytes": w_bytes, "weight_sets": nsets}
+    reps = max(3, int(seconds / max(1e-6, e0.elapsed_time(e1) / 1e3)))
+    ms, clocks = time_graph(g, reps, stream, local, world, device)
+    del Ws, W
+    return {"us_per_call": ms * 1e3 / (reps * n), "kind": "cuBLAS bf16 GEMM (torch.matmul) on the dense weight, "
+            "CUDA graphs", "dense_weight_bytes": w_bytes, "weight_sets": nsets, "clocks": clocks}
+
+
+def time_chained(d, nsets, steps, warmup, device, local, world):
+    """Calls chained on one stream from one CUDA graph per pass over `nsets`
+    rotating weight copies: `warmup` untimed passes, then `steps` timed
+    passes.  Returns (max-over-ranks ms of the timed passes, clocks)."""
+    import torch
+    d.rotate(nsets)
+    g = capture(d.call, nsets, device)
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    ms, clocks = time_graph(g, steps, torch.cuda.current_stream(device), local, world, device)
+    del g
+    return ms, clocks
+
+
+def dense_comparison(name, args, world, local, device):
+    """The dense baseline beside the LittleBit call on one workload, both
+    chained over weights rotated past L2 (Llama-2-70B gate/up at 1 token by
+    default: the pages' own kernel comparison)."""
+    import torch
+    c = synth.CONFIGS[name]
+    d = DeviceLayer(synth.make_config(name, c.tokens[0]), device, c.tokens[0])
+    nsets = rotation_size(d.set_bytes, min_sets=256)
+    ms, _ = time_chained(d, nsets, max(3, args.steps), 3, device, local, world)
+    lb_us = ms * 1e3 / (max(3, args.steps) * nsets)
+    dense = dense_baseline(d, device, 0.2, torch.cuda.current_stream(device), local, world)
+    dense.update(workload=workload_name(c, c.tokens[0]), littlebit_us_per_call=lb_us,
+                 speedup=dense["us_per_call"] / lb_us)
+    d.sets = [d.base]
+    return dense
 
 
 # A decoder block's linears in the order a forward pass runs them, grouped by
@@ -358,19 +587,18 @@ BLOCKS = {
 }
 
 
-def run_block(args, world, rank, local):
-    """One step is a whole decoder block's linears at `tokens` tokens, called
-    back to back on one stream (each call's launches PDL-chained to the
-    previous one) from CUDA graphs; weights rotate past twice the L2 cache.
-    With --fused the linears that read the same input (q k v; gate up) run
-    as one lb_linear_forward_siblings call."""
+def measure_block(block, tokens, fused, steps, warmup, world, local, device, seconds=0.0):
+    """A whole decoder block's linears at `tokens` tokens, called back to back
+    on one stream (each call's launches PDL-chained to the previous one) from
+    CUDA graphs; weights rotate past twice the L2 cache.  With `fused` the
+    linears that read the same input (q k v; gate up) run as one
+    lb_linear_forward_siblings call.  One step is one pass over the block
+    copies of a graph; at least `steps` of them are timed (more if needed to
+    fill `seconds`)."""
     import torch
     import binarized_rank_linear_b200 as lb
 
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    tokens = args.tokens or 1
-    groups = BLOCKS[args.block]
+    groups = BLOCKS[block]
     seq = [name for grp in groups for name in grp]
     layers, nbytes, nflops = [], 0, 0
     for j, name in enumerate(seq):
@@ -390,7 +618,7 @@ def run_block(args, world, rank, local):
                          dtype=torch.uint8, device=device)
         layers.append((paths, x, y, ws))
     set_bytes = sum(p.u_bits.numel() * 4 + p.vt_bits.numel() * 4 for lay in layers for p in lay[0])
-    nsets = max(1, min(64, -(-2 * L2_BYTES // set_bytes) + 1))
+    nsets = rotation_size(set_bytes, max_sets=64)
 
     def clone(p):
         return lb.PackedPath(p.u_bits.clone(), p.vt_bits.clone(), p.h.clone(), p.g.clone(), p.l.clone(), p.rank)
@@ -406,9 +634,9 @@ def run_block(args, world, rank, local):
         gws.append(torch.empty(max(16, lb.siblings_workspace_bytes(tokens, gx[-1].shape[1], spec)),
                                dtype=torch.uint8, device=device))
 
-    def block(i):
+    def run(i):
         s = sets[i % nsets]
-        if not args.fused:
+        if not fused:
             for (paths0, x, y, ws), paths in zip(layers, s):
                 lb.linear_forward(x, paths[0], paths[1] if len(paths) > 1 else None, y=y, workspace=ws)
             return
@@ -416,102 +644,69 @@ def run_block(args, world, rank, local):
             lb.linear_forward_siblings(gx[gi], [(s[k][0], s[k][1] if len(s[k]) > 1 else None) for k in range(a, b)],
                                        ys=[layers[k][2] for k in range(a, b)], workspace=gws[gi])
 
-    block(0)
+    run(0)
     torch.cuda.synchronize()
     assert lb.device_status() == lb.LB_OK
     per_graph = max(1, min(2 * nsets, 64))
-    cap = torch.cuda.Stream(device)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=cap):
-        for i in range(per_graph):
-            block(i)
-    for _ in range(max(1, args.warmup // per_graph)):
+    g = capture(run, per_graph, device)
+    for _ in range(max(1, warmup)):
         g.replay()
     torch.cuda.synchronize()
-    reps = max(1, args.steps // per_graph)
     stream = torch.cuda.current_stream(device)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clk = ClockSampler(local)
-    barrier(world)
-    torch.cuda.synchronize()
-    with clk:
-        e0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    ms = max_over_ranks(e0.elapsed_time(e1), world, device)
-    steps = reps * per_graph
-    per_block_s = ms / 1e3 / steps
-    assert lb.device_status() == lb.LB_OK
-    if rank != 0:
-        return
-    decode = tokens <= DECODE_MAX_TOKENS
-    peaks = load_peaks()
-    achieved = (nbytes / per_block_s / 1e9) if decode else (nflops / per_block_s / 1e12)
-    pk, pk_source = (peaks["hbm"], peaks["source"]) if decode else tensor_peak(peaks, clk.summary())
-    out = {"metric": "decoder block of LittleBit linears: us/block, " + ("HBM GB/s" if decode else "TFLOP/s"),
-           "value": aggregate(((nbytes / 1e9) if decode else (nflops / 1e12)) * steps, ms / 1e3, world),
-           "unit": "GB/s" if decode else "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
-           "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-           "dtype": "f16", "data": "synthetic",
-           "config": {"workload": "%s block (%s) at %d tokens" % (args.block, ", ".join(seq), tokens),
-                      "tokens": tokens, "linears": len(seq), "weight_sets": nsets,
-                      "calls": ("one lb_linear_forward_siblings call per input group (%d)" % len(groups))
-                      if args.fused else "one lb_linear_forward call per linear",
-                      "launch": "CUDA graphs of %d blocks" % per_graph},
-           "us_per_block": per_block_s * 1e6, "algorithmic_bytes_per_block": nbytes,
-           "algorithmic_flops_per_block": nflops,
-           "roofline": {"bound": "hbm" if decode else "tensor", "achieved": achieved, "peak": pk,
-                        "unit": "GB/s" if decode else "TFLOP/s", "frac": achieved / pk, "traffic": None,
-                        "peak_source": pk_source},
-           "clocks": clk.summary(),
-           "gpu_launches": 2 * (len(groups) if args.fused and tokens <= 4 else len(seq)) * steps, "impl": "lb"}
-    print(json.dumps(out), flush=True)
-
-
-def time_contractions(sets, x, tokens, c, stream, device, n):
-    """Each contraction of the prefill path on its own: lb_latent_forward and
-    lb_expand_forward run the same two kernels as lb_linear_forward at these
-    token counts.  CUDA graphs of n calls each, over the rotating weights,
-    timed with events on `stream`; flops per contraction from the workload
-    table (2 M R n_in and 2 M R n_out)."""
-    import torch
-    import binarized_rank_linear_b200 as lb
-    R = sum(p.rank for p in sets[0])
-    z = torch.empty((tokens, R), dtype=torch.float16, device=device)
-    y = torch.empty((tokens, c.n_out), dtype=torch.bfloat16, device=device)
-    two = lambda s: (s[0], s[1] if len(s) > 1 else None)
-    lat = lambda i: lb.latent_forward(x, *two(sets[i % len(sets)]), z=z)
-    exp = lambda i: lb.expand_forward(z, *two(sets[i % len(sets)]), y=y)
-    out = {}
-    cap = torch.cuda.Stream(device)
-    flops = {"contraction_1": 2 * tokens * R * c.n_in, "contraction_2": 2 * tokens * R * c.n_out}
-    names = {"contraction_1": "sign_gemm_kernel<1, H, P> (contraction 1, tcgen05)",
-             "contraction_2": "sign_gemm_kernel<2, H, P> (contraction 2, tcgen05)"}
-    lat(0)
-    torch.cuda.synchronize()
-    for key, fn in (("contraction_1", lat), ("contraction_2", exp)):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=cap):
-            for i in range(n):
-                fn(i)
-        for _ in range(2):
-            g.replay()
-        torch.cuda.synchronize()
+    reps = max(1, steps)
+    if seconds > 0:
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         g.replay()
         e1.record(stream)
         torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / n
-        out[key] = {"kernel": names[key], "flop": flops[key], "us_alone": us, "TFLOP/s_alone": flops[key] / us / 1e6}
-        del g
-    total = sum(v["us_alone"] for v in out.values())
-    for v in out.values():
-        v["share"] = v["us_alone"] / total
-    return out
+        reps = max(reps, int(seconds / max(1e-6, e0.elapsed_time(e1) / 1e3)))
+    ms, clocks = time_graph(g, reps, stream, local, world, device)
+    assert lb.device_status() == lb.LB_OK
+    blocks = reps * per_graph
+    per_block_s = ms / 1e3 / blocks
+    decode = tokens <= DECODE_MAX_TOKENS
+    peaks = load_peaks()
+    achieved = (nbytes / per_block_s / 1e9) if decode else (nflops / per_block_s / 1e12)
+    pk, pk_source = (peaks["hbm"], peaks["source"]) if decode else tensor_peak(peaks, clocks)
+    launches_per_block = 2 * (len(groups) if fused and tokens <= 128 else len(seq))
+    return {"workload": "%s block (%s) at %d tokens" % (block, ", ".join(seq), tokens), "tokens": tokens,
+            "linears": len(seq), "weight_sets": nsets, "blocks": blocks, "ms": ms,
+            "calls": ("one lb_linear_forward_siblings call per input group (%d)" % len(groups))
+            if fused else "one lb_linear_forward call per linear",
+            "launch": "CUDA graphs of %d blocks" % per_graph,
+            "us_per_block": per_block_s * 1e6, "algorithmic_bytes_per_block": nbytes,
+            "algorithmic_flops_per_block": nflops,
+            "value": aggregate(((nbytes / 1e9) if decode else (nflops / 1e12)) * blocks, ms / 1e3, world),
+            "unit": "GB/s" if decode else "TFLOP/s",
+            "roofline": {"bound": "hbm" if decode else "tensor", "achieved": achieved, "peak": pk,
+                         "unit": "GB/s" if decode else "TFLOP/s", "frac": achieved / pk, "traffic": None,
+                         "peak_source": pk_source},
+            "clocks": clocks, "gpu_launches": launches_per_block * blocks}
+
+
+def run_block(args, world, rank, local):
+    """--block: one step is one pass of a whole decoder block's linears."""
+    import torch
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    tokens = args.tokens or 1
+    r = measure_block(args.block, tokens, args.fused, args.steps, args.warmup, world, local, device)
+    if rank != 0:
+        return
+    out = {"metric": "decoder block of LittleBit linears: us/block, " + r["unit"], "value": r["value"],
+           "unit": r["unit"], "n_gpus": world, "steps": r["blocks"], "warmup": args.warmup,
+           "ms_per_step": r["ms"] / r["blocks"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "bf16", "data": "synthetic",
+           "config": {k: r[k] for k in ("workload", "tokens", "linears", "weight_sets", "calls", "launch")},
+           "us_per_block": r["us_per_block"], "algorithmic_bytes_per_block": r["algorithmic_bytes_per_block"],
+           "algorithmic_flops_per_block": r["algorithmic_flops_per_block"], "roofline": r["roofline"],
+           "clocks": r["clocks"], "gpu_launches": r["gpu_launches"], "impl": "lb"}
+    print(json.dumps(out), flush=True)
+
+
+NUMERICS = ("bf16 x and y, fp16 scales, fp32 accumulation (1-4 tokens: fp32 throughout; more tokens: tensor-core "
+            "operands bf16 in contraction 1, fp16 in contraction 2)")
 
 
 def run_lb(args, world, rank, local):
@@ -522,99 +717,32 @@ def run_lb(args, world, rank, local):
     torch.cuda.set_device(device)
     c = synth.CONFIGS[args.config]
     tokens = args.tokens or c.tokens[0]
-    ranks = [c.rank] * c.paths
     decode = tokens <= DECODE_MAX_TOKENS
-    nbytes = algorithmic_bytes(c.n_in, c.n_out, ranks, tokens)
-    nflops = algorithmic_flops(c.n_in, c.n_out, ranks, tokens)
-    layer = synth.make_config(args.config, tokens)
-
-    # weights: one packed set through the C ABI, then copies so the rotation
-    # covers more than twice the L2 cache
-    base = []
-    for p in layer["paths"]:
-        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
-        base.append(lb.PackedPath.from_factors(dev(p["su"]), dev(p["sv"]), dev(p["h"]), dev(p["g"]), dev(p["l"])))
-    set_bytes = sum(p.u_bits.numel() * 4 + p.vt_bits.numel() * 4 for p in base)
-    io_bytes = 2 * tokens * (c.n_in + c.n_out)
-    nsets = 1 if io_bytes > 2 * L2_BYTES else max(1, min(512, -(-2 * L2_BYTES // set_bytes) + 1))
-
-    def clone(p):
-        return lb.PackedPath(p.u_bits.clone(), p.vt_bits.clone(), p.h.clone(), p.g.clone(), p.l.clone(), p.rank)
-
-    sets = [base] + [[clone(p) for p in base] for _ in range(nsets - 1)]
-    x = torch.from_numpy(layer["x"].view(np.int16)).to(device).view(torch.bfloat16)
-    y = torch.empty((tokens, c.n_out), dtype=torch.bfloat16, device=device)
-    ws = torch.empty(max(16, lb.forward_workspace_bytes(tokens, c.n_in, c.n_out, c.rank,
-                                                        c.rank if c.paths > 1 else 0)),
-                     dtype=torch.uint8, device=device)
-
-    def call(i, stream=None):
-        s = sets[i % nsets]
-        lb.linear_forward(x, s[0], s[1] if len(s) > 1 else None, y=y, workspace=ws, stream=stream)
+    peaks = load_peaks()
+    d = DeviceLayer(synth.make_config(args.config, tokens), device, tokens)
+    nbytes, nflops = d.nbytes, d.nflops
+    stream = torch.cuda.current_stream(device)
 
     # parity of the benchmarked configuration against the oracle (sampled rows)
-    call(0)
+    d.call(0)
     torch.cuda.synchronize()
     assert lb.device_status() == lb.LB_OK
     parity = None
     if rank == 0 and not args.no_parity:
-        import oracle
-        rows = np.arange(tokens) if tokens <= 8 else np.linspace(0, tokens - 1, 8).astype(int)
-        ref = oracle.forward(oracle.bf16_bits_to_f64(layer["x"][rows]),
-                             [dict(su=p["su"], sv=p["sv"], h=oracle.f16_to_f64(p["h"]),
-                                   g=oracle.f16_to_f64(p["g"]), l=oracle.f16_to_f64(p["l"]))
-                              for p in layer["paths"]])
-        got = oracle.bf16_bits_to_f64(y[torch.from_numpy(rows).to(device)].view(torch.int16).cpu().numpy()
-                                      .view(np.uint16))
-        parity = {"rows": int(len(rows)),
-                  "rel_l2": float(np.linalg.norm(got - ref) / np.linalg.norm(ref)),
-                  "max_err_over_max_y": float(np.abs(got - ref).max() / np.abs(ref).max())}
-        assert parity["rel_l2"] <= 5e-3 and parity["max_err_over_max_y"] <= 1e-2, parity
+        parity = d.parity(np.arange(tokens) if tokens <= 8 else np.linspace(0, tokens - 1, 8).astype(int))
 
-    # CUDA graphs of consecutive calls over the rotating weight sets
-    per_graph = max(1, min(nsets * (2 if nsets < 64 else 1), 512)) if decode else 1
-    cap_stream = torch.cuda.Stream(device)
-
-    def capture(n, start):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=cap_stream):
-            for i in range(n):
-                call(start + i)
-        return g
-
-    graph = capture(per_graph, 0)
-    tail_n = args.steps % per_graph
-    tail = capture(tail_n, 0) if tail_n else None
-    full_graphs = args.steps // per_graph
-
-    def run_steps(n_full, tail_graph):
-        for _ in range(n_full):
-            graph.replay()
-        if tail_graph is not None:
-            tail_graph.replay()
-
-    # warm-up
-    wf, wt = divmod(args.warmup, per_graph)
-    run_steps(wf, capture(wt, 0) if wt else None)
-    torch.cuda.synchronize()
-
-    # timed region
-    stream = torch.cuda.current_stream(device)
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clk = ClockSampler(local)
-    barrier(world)
-    torch.cuda.synchronize()
-    with clk:
-        start.record(stream)
-        run_steps(full_graphs, tail)
-        stop.record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    ms = start.elapsed_time(stop)
-    ms_max = max_over_ranks(ms, world, device)
-    per_call_s = ms_max / 1e3 / args.steps
+    # One step is one pass over `nsets` distinct copies of the layer's weights
+    # (a chain of nsets layers of this shape), chained on one stream from one
+    # CUDA graph.  The copies span more than twice the L2 cache, and the
+    # warm-up passes over all of them, so no call of the timed region finds
+    # its weights in L2.
+    io_bytes = 2 * tokens * (d.n_in + d.n_out)
+    nsets = 1 if io_bytes > 2 * L2_BYTES else rotation_size(d.set_bytes, min_sets=args.min_sets)
+    ms_max, clocks = time_chained(d, nsets, args.steps, args.warmup, device, local, world)
+    calls = args.steps * nsets
+    per_call_s = ms_max / 1e3 / calls
     units = nbytes / 1e9 if decode else nflops / 1e12
-    value = aggregate(units * args.steps, ms_max / 1e3, world)
+    value = aggregate(units * calls, ms_max / 1e3, world)
     assert lb.device_status() == lb.LB_OK
 
     # isolated calls: cold L2 before each
@@ -624,7 +752,7 @@ def run_lb(args, world, rank, local):
         flush.fill_(i & 0xFF)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        call(i)
+        d.call(i)
         e1.record(stream)
         torch.cuda.synchronize()
         iso.append(e0.elapsed_time(e1) * 1e3)
@@ -632,92 +760,99 @@ def run_lb(args, world, rank, local):
     del flush
 
     # end to end through the C ABI with host buffers (lb_linear_forward_host):
-    # every step copies x in from pinned host memory, runs the layer and
-    # copies y back to pinned host memory, all inside the one call
-    x_host = torch.empty_like(x, device="cpu").pin_memory()
-    x_host.copy_(x.cpu())
-    y_host = torch.empty((tokens, c.n_out), dtype=torch.bfloat16).pin_memory()
-    e2e_steps = min(args.steps, max(50, args.e2e_steps))
+    # the same steps (passes over the weight copies), every call copying its x
+    # in from pinned host memory and its y back to pinned host memory inside
+    # the one call, issued eagerly from Python
+    x_host = torch.empty_like(d.x, device="cpu").pin_memory()
+    x_host.copy_(d.x.cpu())
+    y_host = torch.empty((tokens, d.n_out), dtype=torch.bfloat16).pin_memory()
 
     def call_host(i):
-        s = sets[i % nsets]
-        lb.linear_forward_host(x_host, s[0], s[1] if len(s) > 1 else None, y_host, x, y, ws)
+        s = d.sets[i % nsets]
+        lb.linear_forward_host(x_host, s[0], s[1] if len(s) > 1 else None, y_host, d.x, d.y, d.ws)
 
-    for i in range(min(20, e2e_steps)):
+    for i in range(nsets):
         call_host(i)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(e2e_steps):
+    for i in range(calls):
         call_host(i)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
-    e2e_value = aggregate(units * e2e_steps, e2e_ms / 1e3, world)
+    e2e_value = aggregate(units * calls, e2e_ms / 1e3, world)
+    d.sets = [d.base]
+    torch.cuda.empty_cache()
 
-    dense = dense_baseline(layer, x, args.steps, stream, device) if args.dense_baseline else None
-    per_kernel = (time_contractions(sets, x, tokens, c, stream, device, max(3, min(args.steps, 50)))
-                  if not decode and tokens > 128 else None)
+    # the default run also measures prefill (the metric's TFLOP/s half), a
+    # whole decoder block of fused sibling calls at batch 1, and the dense
+    # baseline of the pages' kernel comparison
+    prefill = block = dense = None
+    if not args.no_extras:
+        prefill = {}
+        for name in args.prefill.split(",") if args.prefill else []:
+            prefill[name] = measure_prefill(name, args, world, local, device, peaks)
+            torch.cuda.empty_cache()
+        block = measure_block("llama2_7b", 1, True, args.steps, args.warmup, world, local, device, seconds=0.1)
+        torch.cuda.empty_cache()
+        dense = dense_comparison("llama2_70b_gate", args, world, local, device)
+        torch.cuda.empty_cache()
+    if args.dense_baseline and dense is None:
+        dense = dense_comparison(args.config, args, world, local, device)
 
     if rank != 0:
         return
-    peaks = load_peaks()
-    if decode:
+    if decode or tokens <= 128:
         achieved = nbytes / per_call_s / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm"], "traffic": load_traffic(args.config, tokens),
                 "kernel": kernel_label(tokens, c.rank * c.paths * (c.n_in + c.n_out)),
                 "peak_source": peaks["source"]}
     else:
-        pk, pk_source = tensor_peak(peaks, clk.summary())
-        if per_kernel is not None:
-            # the dominant kernel: its share of the call comes from timing each
-            # contraction alone (after the timed region, where the clocks under
-            # the power cap have settled lower, so only the ratio is used); its
-            # duration is that share of the live per-call time
-            dom = max(per_kernel.values(), key=lambda k: k["share"])
-            achieved = dom["flop"] / (per_call_s * dom["share"]) / 1e12
-            roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
-                    "frac": achieved / pk, "traffic": load_traffic(args.config, tokens),
-                    "kernel": dom["kernel"], "share_of_call": dom["share"],
-                    "call_TFLOP/s": nflops / per_call_s / 1e12,
-                    "peak_source": pk_source}
-        else:
-            achieved = nflops / per_call_s / 1e12
-            roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
-                    "frac": achieved / pk, "traffic": load_traffic(args.config, tokens),
-                    "kernel": kernel_label(tokens, c.rank * c.paths * (c.n_in + c.n_out)),
-                    "peak_source": pk_source}
+        pk, pk_source = tensor_peak(peaks, clocks)
+        per_kernel = time_contractions(d, [d.x], stream, device, max(3, min(args.steps, 50)))
+        dom = max(per_kernel.values(), key=lambda k: k["share"])
+        achieved = dom["flop"] / (per_call_s * dom["share"]) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s", "frac": achieved / pk,
+                "traffic": load_traffic(args.config, tokens), "kernel": dom["kernel"],
+                "share_of_call": dom["share"], "call_TFLOP/s": nflops / per_call_s / 1e12, "peak_source": pk_source}
     cpu = None
     if world == 1 and not args.no_cpu:
         import oracle
         per, nb, nf, desc = oracle_sample(synth.make_config(args.config, min(tokens, 64)), args.cpu_seconds)
         cpu = {"value": (nb / per / 1e9) if decode else (nf / per / 1e12), "unit": "GB/s" if decode else "TFLOP/s",
                "cores": oracle.num_threads(), "kind": "oracle", "sample": desc}
+    set_mb = nsets * d.set_bytes / 1e6
     out = {"metric": METRIC, "value": value, "unit": "GB/s" if decode else "TFLOP/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
-           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
-           "data": "synthetic",
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "numerics": NUMERICS, "data": "synthetic",
            "config": {"workload": workload_name(c, tokens), "tokens": tokens, "weight_sets": nsets,
-                      "l2": ("weights rotated over %.0f MB > 2x L2" % (nsets * set_bytes / 1e6)) if nsets > 1
-                      else "inputs larger than L2",
-                      "launch": "CUDA graphs of %d back-to-back calls" % per_graph,
+                      "step": "one pass over %d distinct weight copies: %d lb_linear_forward calls chained on one "
+                              "stream from one CUDA graph" % (nsets, nsets),
+                      "l2": ("weights rotated over %.0f MB > 2x L2; warm-up passes over every copy" % set_mb)
+                      if set_mb * 1e6 > 2 * L2_BYTES else
+                      ("inputs larger than L2" if io_bytes > 2 * L2_BYTES else "weights within L2 (%.0f MB)" % set_mb),
                       "parallelism": "replicas" if world > 1 else "single GPU"},
-           "us_per_call": per_call_s * 1e6, "us_per_call_isolated_cold_l2": iso_us,
+           "us_per_call": per_call_s * 1e6, "calls_timed": calls, "us_per_call_isolated_cold_l2": iso_us,
            "algorithmic_bytes_per_call": nbytes, "algorithmic_flops_per_call": nflops,
-           "roofline": roof, "per_kernel": per_kernel, "cpu_baseline": cpu, "parity": parity,
-           "clocks": clk.summary(),
+           "roofline": roof, "cpu_baseline": cpu, "parity": parity, "clocks": clocks,
            "e2e": {"value": e2e_value, "unit": "GB/s" if decode else "TFLOP/s",
-                   "h2d_bytes_per_step": 2 * tokens * c.n_in, "d2h_bytes_per_step": 2 * tokens * c.n_out,
-                   "steps": e2e_steps, "call": "lb_linear_forward_host (pinned host x and y; " + (
+                   "h2d_bytes_per_step": 2 * tokens * d.n_in * nsets, "d2h_bytes_per_step": 2 * tokens * d.n_out * nsets,
+                   "us_per_call": e2e_ms * 1e3 / calls, "calls": calls,
+                   "call": "lb_linear_forward_host from Python (pinned host x and y; " + (
                        "x gathered by a kernel in one pass, y written in place by the last kernel)" if tokens <= 128 else
                        "copied through device buffers inside the call)")},
-           "gpu_launches": 2 * args.steps,  # contraction 1 + contraction 2 per call, decode and prefill
+           "gpu_launches": 2 * calls,  # contraction 1 + contraction 2 per call, decode and prefill
            "impl": "lb"}
+    if prefill:
+        out["prefill"] = prefill
+    if block is not None:
+        out["decode_block_fused"] = block
     if dense is not None:
-        dense["speedup"] = dense["us_per_call"] / (per_call_s * 1e6)
         out["dense_baseline"] = dense
     print(json.dumps(out), flush=True)
 
@@ -725,13 +860,19 @@ def run_lb(args, world, rank, local):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["lb", "reference"], default="lb")
     ap.add_argument("--config", default="llama2_7b_q", choices=sorted(synth.CONFIGS))
     ap.add_argument("--tokens", type=int, default=0, help="default: the config's first token count")
+    ap.add_argument("--min-sets", type=int, default=1024,
+                    help="decode: weight copies per step at least (more if needed to pass 2x L2)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--e2e-steps", type=int, default=5000)
+    ap.add_argument("--prefill", default="qwen3_14b_gate,qwen3_14b_kv",
+                    help="prefill workloads measured beside the main line (comma-separated)")
+    ap.add_argument("--prefill-seconds", type=float, default=0.3)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the prefill, fused-block and dense-baseline measurements")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-parity", action="store_true")
     ap.add_argument("--block", choices=sorted(BLOCKS), default=None,
@@ -739,7 +880,7 @@ def main(argv=None):
     ap.add_argument("--fused", action="store_true",
                     help="with --block: linears that share their input run as one siblings call")
     ap.add_argument("--dense-baseline", action="store_true",
-                    help="also time a cuBLAS bf16 GEMM on the reconstructed dense weight (same tokens)")
+                    help="with --no-extras: also time a cuBLAS bf16 GEMM on this workload's dense weight")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

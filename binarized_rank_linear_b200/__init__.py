@@ -177,6 +177,28 @@ def _dtype_code(t) -> int:
     return codes[t.dtype]
 
 
+def _require(t, name: str, dtype, device: str = "cuda", contiguous: bool = False) -> None:
+    """Checks an activation tensor before its pointer crosses the C ABI: the
+    library reads the bits as the element type and layout its header states,
+    so a tensor of another dtype or with a non-unit inner stride would be read
+    as wrong data without an error."""
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D, got shape {tuple(t.shape)}")
+    if t.stride(1) != 1 and t.shape[1] > 1:
+        raise ValueError(f"{name} must have unit inner stride, got strides {t.stride()}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (rows of exactly {t.shape[1]} elements)")
+    if (device == "cuda") != bool(t.is_cuda):
+        raise ValueError(f"{name} must be in {'device' if device == 'cuda' else 'host'} memory")
+
+
+def _require_workspace(ws) -> None:
+    if not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous device tensor")
+
+
 def pack_signs(src, kind: str, ld_words: int | None = None, stream=None):
     """Pack a device factor (f32 / f16 / bf16 / int8, 2-D, unit column stride)
     with ``lb_pack_signs``.  ``kind`` is ``"U"`` (src = U [n_out, r]) or
@@ -221,6 +243,16 @@ class PackedPath:
         and a tensor's storage does not move)."""
         c = self.__dict__.get("_c")
         if c is None:
+            torch = _torch()
+            for name in ("u_bits", "vt_bits"):
+                t = getattr(self, name)
+                if t.dtype != torch.int32 or t.dim() != 2 or t.stride(1) != 1 or not t.is_cuda:
+                    raise ValueError(f"{name} must be a 2-D int32 device tensor of packed words with unit "
+                                     f"inner stride")
+            for name in ("h", "g", "l"):
+                t = getattr(self, name)
+                if t.dtype != torch.float16 or t.dim() != 1 or not t.is_contiguous() or not t.is_cuda:
+                    raise ValueError(f"{name} must be a contiguous 1-D float16 device tensor")
             c = LbPath(self.u_bits.data_ptr(), self.vt_bits.data_ptr(), self.h.data_ptr(),
                        self.g.data_ptr(), self.l.data_ptr(), self.rank, self.u_bits.shape[1],
                        self.vt_bits.shape[1])
@@ -234,13 +266,16 @@ def linear_forward(x, main: PackedPath, residual: PackedPath | None = None, y=No
     -> y bf16 [tokens, n_out].  Allocates y and the workspace with torch when
     not given."""
     torch = _torch()
+    _require(x, "x", torch.bfloat16)
     tokens, n_in = x.shape
     n_out = main.h.shape[0]
     if y is None:
         y = torch.empty((tokens, n_out), dtype=torch.bfloat16, device=x.device)
-    if workspace is None:  # a caller's workspace is checked by the library itself
+    _require(y, "y", torch.bfloat16)
+    if workspace is None:  # a caller's workspace size is checked by the library itself
         need = forward_workspace_bytes(tokens, n_in, n_out, main.rank, residual.rank if residual else 0)
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    _require_workspace(workspace)
     cm = main.as_c()
     cr = residual.as_c() if residual is not None else None
     _check(lib().lb_linear_forward(
@@ -278,13 +313,17 @@ def linear_forward_siblings(x, layers, ys=None, workspace=None, stream=None):
     given as [(main, residual or None), ...]; returns their outputs (bf16
     [tokens, n_out_j]), allocated with torch when not given."""
     torch = _torch()
+    _require(x, "x", torch.bfloat16)
     tokens, n_in = x.shape
     if ys is None:
         ys = [torch.empty((tokens, main.h.shape[0]), dtype=torch.bfloat16, device=x.device) for main, _ in layers]
+    for j, y in enumerate(ys):
+        _require(y, f"ys[{j}]", torch.bfloat16)
     arr, _keep = _projections(layers, ys)
     need = int(lib().lb_siblings_workspace_bytes(tokens, n_in, len(layers), arr))
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    _require_workspace(workspace)
     _check(lib().lb_linear_forward_siblings(
         x.data_ptr(), tokens, n_in, x.stride(0), len(layers), arr, workspace.data_ptr(),
         workspace.numel() * workspace.element_size(), _stream_handle(stream)), "lb_linear_forward_siblings")
@@ -299,8 +338,17 @@ def linear_forward_host(x_host, main: PackedPath, residual: PackedPath | None, y
     is valid once the stream is synchronised.  For 1-128 tokens on pinned
     buffers x comes in through a gather kernel and y is written to y_host by
     the last kernel (y_dev is then not touched)."""
+    torch = _torch()
+    _require(x_host, "x_host", torch.bfloat16, device="cpu", contiguous=True)
+    _require(y_host, "y_host", torch.bfloat16, device="cpu", contiguous=True)
+    _require(x_dev, "x_dev", torch.bfloat16, contiguous=True)
+    _require(y_dev, "y_dev", torch.bfloat16, contiguous=True)
+    _require_workspace(workspace)
     tokens, n_in = x_host.shape
     n_out = main.h.shape[0]
+    if tuple(y_host.shape) != (tokens, n_out) or tuple(x_dev.shape) != (tokens, n_in) \
+            or tuple(y_dev.shape) != (tokens, n_out):
+        raise ValueError("x_host / x_dev must be [tokens, n_in] and y_host / y_dev [tokens, n_out]")
     cm = main.as_c()
     cr = residual.as_c() if residual is not None else None
     _check(lib().lb_linear_forward_host(
@@ -315,10 +363,12 @@ def latent_forward(x, main: PackedPath, residual: PackedPath | None = None, z=No
     + r_residual] (the latent of both paths, main first).  Allocates z with
     torch when not given (the C call allocates nothing)."""
     torch = _torch()
+    _require(x, "x", torch.bfloat16)
     tokens, n_in = x.shape
     R = main.rank + (residual.rank if residual is not None else 0)
     if z is None:
         z = torch.empty((tokens, R), dtype=torch.float16, device=x.device)
+    _require(z, "z", torch.float16)
     cm = main.as_c()
     cr = residual.as_c() if residual is not None else None
     _check(lib().lb_latent_forward(
@@ -331,10 +381,12 @@ def expand_forward(z, main: PackedPath, residual: PackedPath | None = None, y=No
     """``lb_expand_forward``: z fp16 [tokens, r_main + r_residual] -> y bf16
     [tokens, n_out].  Allocates y with torch when not given."""
     torch = _torch()
+    _require(z, "z", torch.float16)
     tokens = z.shape[0]
     n_out = main.h.shape[0]
     if y is None:
         y = torch.empty((tokens, n_out), dtype=torch.bfloat16, device=z.device)
+    _require(y, "y", torch.bfloat16)
     cm = main.as_c()
     cr = residual.as_c() if residual is not None else None
     _check(lib().lb_expand_forward(
@@ -350,10 +402,12 @@ def linear_forward_fixed_scratch(x, main: PackedPath, residual: PackedPath | Non
     workspace.  Allocates y with torch when not given (the C call itself
     allocates nothing)."""
     torch = _torch()
+    _require(x, "x", torch.bfloat16)
     tokens, n_in = x.shape
     n_out = main.h.shape[0]
     if y is None:
         y = torch.empty((tokens, n_out), dtype=torch.bfloat16, device=x.device)
+    _require(y, "y", torch.bfloat16)
     cm = main.as_c()
     cr = residual.as_c() if residual is not None else None
     _check(lib().lb_linear_forward_fixed_scratch(

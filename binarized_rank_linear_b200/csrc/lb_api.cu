@@ -17,7 +17,7 @@ __device__ int g_lb_status = 0;
 
 namespace {
 
-constexpr int kMaxDevices = 64;
+using lb::kMaxDevices;
 constexpr int64_t kMaxDim = int64_t(1) << 20;     // n_in, n_out
 constexpr int64_t kMaxRank = 32768;
 constexpr int64_t kMaxTokens = int64_t(1) << 24;

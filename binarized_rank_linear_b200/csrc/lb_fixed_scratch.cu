@@ -28,16 +28,29 @@ namespace {
 // that the second reads).
 static __device__ __align__(256) unsigned char g_fixed_scratch[LB_FIXED_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 256;
+using lb::kMaxDevices;
 std::mutex g_mutex;
 void *g_scratch_addr[kMaxDevices];  // device address of g_fixed_scratch, per device; set once
 
 // Device address of this device's array, looked up on the first call made
-// with the device current and cached after that.
-lb_status scratch_address(void **out)
+// with the device current and cached after that.  The stream must belong to
+// the current device (the legacy default stream, NULL, always does): the
+// kernels run on the stream's device, and the address is this device's.
+lb_status scratch_address(cudaStream_t stream, void **out)
 {
     int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LB_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        (void)cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    if (stream) {
+        int sdev = -1;
+        if (cudaStreamGetDevice(stream, &sdev) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return LB_ERR_INVALID_ARGUMENT;
+        }
+        if (sdev != dev) return LB_ERR_INVALID_ARGUMENT;
+    }
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!g_scratch_addr[dev]) {
         void *p = nullptr;
@@ -66,7 +79,7 @@ extern "C" lb_status lb_linear_forward_fixed_scratch(const uint16_t *x, int64_t 
     const size_t need = lb_forward_workspace_bytes(tokens, n_in, n_out, main->rank, residual ? residual->rank : 0);
     if (need > LB_FIXED_SCRATCH_BYTES) return LB_ERR_WORKSPACE_TOO_SMALL;
     void *scratch = nullptr;
-    const lb_status st = scratch_address(&scratch);
+    const lb_status st = scratch_address(static_cast<cudaStream_t>(stream), &scratch);
     if (st != LB_OK) return st;
     // Everything else (shapes, strides, alignment, the paths) is checked by
     // lb_linear_forward before it launches anything.

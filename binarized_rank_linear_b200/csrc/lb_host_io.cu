@@ -12,21 +12,20 @@ namespace {
 constexpr int kGatherThreads = 256;
 
 // dst[i] = src[i] for i < n16 (16-byte units).  src is pinned host memory
-// reached through its device mapping; every thread issues its load before
-// the dependency wait, so the copy costs one round trip over the host link
-// and that round trip overlaps the tail of the previous work on the stream.
-// The store waits for that work (the previous call's first kernel may still
-// read dst).  The next kernel is released at entry: its weight loads overlap
-// this copy, and it waits for the copy before it reads dst.
+// reached through its device mapping.  The next kernel is released at entry,
+// so its weight loads overlap this copy (it waits for the copy before it
+// reads dst).  Both the load and the store come after the dependency wait:
+// the previous kernel on the stream may still write src (a chain of host
+// calls in which one call's y_host is the next call's x_host: the last
+// kernel of a call stores y after releasing its dependents) or read dst (the
+// previous call's first kernel reads x_dev).
 __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst,
                                                                 int64_t n16)
 {
     pdl_launch_dependents();
     const int64_t i = (int64_t)blockIdx.x * kGatherThreads + threadIdx.x;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (i < n16) v = src[i];
     pdl_wait();
-    if (i < n16) dst[i] = v;
+    if (i < n16) dst[i] = src[i];
 }
 
 }  // namespace

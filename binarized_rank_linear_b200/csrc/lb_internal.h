@@ -10,6 +10,10 @@
 
 namespace lb {
 
+// Devices the library serves per process: ordinals 0 .. kMaxDevices - 1 (its
+// per-device tables have this many entries).
+constexpr int kMaxDevices = 64;
+
 // Per-device facts the launchers need (cached by lb_api.cu).
 struct DeviceInfo {
     int device = -1;

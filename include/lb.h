@@ -304,7 +304,10 @@ LB_API lb_status lb_linear_forward_siblings(const uint16_t *x, int64_t tokens, i
  *   - the first call on each device looks up the array's device address
  *     (once; later calls reuse it).  Make that first call, with the device
  *     current, before any stream capture.  If the lookup fails the call
- *     returns LB_ERR_CUDA.
+ *     returns LB_ERR_CUDA;
+ *   - `stream` must belong to the current device (NULL, the legacy default
+ *     stream, always does): the array used is the current device's.  A
+ *     stream of another device -> LB_ERR_INVALID_ARGUMENT.
  * Nothing in the array has to start at zero: each call writes every byte it
  * later reads.  All calls on one device share the one array, so two calls
  * that could run at the same time (different streams, or different host

@@ -282,3 +282,33 @@ def test_prefill_pairs_switch_takes_only_zero_or_one(L):
         assert L.lb_set_prefill_pairs(bad) == lb.LB_ERR_INVALID_ARGUMENT
     assert L.lb_set_prefill_pairs(0) == lb.LB_OK
     assert L.lb_set_prefill_pairs(1) == lb.LB_OK
+
+
+def test_binding_rejects_wrong_dtype_or_layout_before_any_call(L):
+    """The binding checks each activation's dtype, rank and inner stride (and
+    that it lives on the device) before its pointer reaches the library: an
+    fp16 tensor or a transposed view would otherwise be read as wrong bits."""
+    import torch
+    fake = lb.PackedPath(torch.zeros((64, 1), dtype=torch.int32), torch.zeros((32, 2), dtype=torch.int32),
+                         torch.zeros(64, dtype=torch.float16), torch.zeros(64, dtype=torch.float16),
+                         torch.zeros(32, dtype=torch.float16), 32)
+    with pytest.raises(TypeError, match="bfloat16"):
+        lb.linear_forward(torch.zeros((2, 64), dtype=torch.float16), fake)
+    with pytest.raises(ValueError, match="inner stride"):
+        lb.linear_forward(torch.zeros((64, 2), dtype=torch.bfloat16).t(), fake)
+    with pytest.raises(ValueError, match="device memory"):
+        lb.linear_forward(torch.zeros((2, 64), dtype=torch.bfloat16), fake)
+    with pytest.raises(TypeError, match="float16"):
+        lb.expand_forward(torch.zeros((2, 32), dtype=torch.bfloat16), fake)
+    with pytest.raises(TypeError, match="bfloat16"):
+        lb.latent_forward(torch.zeros((2, 64), dtype=torch.float32), fake)
+    with pytest.raises(TypeError, match="bfloat16"):
+        lb.linear_forward_siblings(torch.zeros((2, 64), dtype=torch.float16), [(fake, None)])
+    with pytest.raises(TypeError, match="bfloat16"):
+        lb.linear_forward_fixed_scratch(torch.zeros((2, 64), dtype=torch.int16), fake)
+    xh = torch.zeros((2, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="inner stride"):
+        lb.linear_forward_host(torch.zeros((64, 2), dtype=torch.bfloat16).t(), fake, None,
+                               torch.zeros((2, 64), dtype=torch.bfloat16), xh, xh, torch.zeros(16, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="int32"):
+        lb.PackedPath(fake.u_bits.float(), fake.vt_bits, fake.h, fake.g, fake.l, 32).as_c()

@@ -122,3 +122,34 @@ def test_source_hash_sees_code_not_comments():
     assert bench.source_code(a) == bench.source_code(b)
     assert bench.source_code(a) != bench.source_code(c)
     assert "one" not in bench.source_code(a) and "two" not in bench.source_code(a)
+
+
+@pytest.mark.parametrize("n_in,n_out,ranks", [(256, 512, [64, 32]), (96, 64, [32])])
+def test_dense_baseline_weight_is_the_oracles(n_in, n_out, ranks):
+    """The dense comparison arm multiplies by W built with PyTorch ops
+    (dense_weight_torch); it must be the oracle's dense W of the same layer
+    (fp32 build: within fp32 rounding of the fp64 product), and its bf16 copy,
+    which the GEMM reads, within bf16 rounding."""
+    import numpy as np
+    import oracle
+    import torch
+    layer = synth.make_layer(n_in, n_out, ranks, 1, config_id=1300 + n_in)
+    P = [dict(su=p["su"], sv=p["sv"], h=oracle.f16_to_f64(p["h"]), g=oracle.f16_to_f64(p["g"]),
+              l=oracle.f16_to_f64(p["l"])) for p in layer["paths"]]
+    ref = oracle.dense_weight(P)
+    W = bench.dense_weight_torch(layer, "cpu")
+    assert tuple(W.shape) == (n_out, n_in) and W.dtype == torch.float32
+    got = W.double().numpy()
+    scale = np.abs(ref).max()
+    assert np.abs(got - ref).max() <= 1e-5 * scale
+    wb = W.to(torch.bfloat16).double().numpy()
+    assert np.all(np.abs(wb - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6 * scale)
+
+
+def test_rotation_spans_twice_l2():
+    for set_bytes in (4160, 2150400, 6_100_000, 400_000_000):
+        n = bench.rotation_size(set_bytes, min_sets=1)
+        if n * set_bytes <= (4 << 30) and n < 4096:
+            assert n * set_bytes > 2 * bench.L2_BYTES
+    assert bench.rotation_size(2150400, min_sets=1024) == 1024
+    assert bench.rotation_size(10 ** 9, min_sets=1024) == 4   # capped by 4 GB of weights

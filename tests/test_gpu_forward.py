@@ -38,16 +38,23 @@ PREFILL = [name for name, c in sorted(synth.CONFIGS.items()) if c.tokens[0] > 32
 
 
 @pytest.mark.parametrize("name", PREFILL)
-def test_prefill_configs_sampled(name):
+def test_prefill_configs_every_row(name):
+    """The Qwen3-14B linears at 8192 tokens, in the launch configuration the
+    benchmark times (CTA pairs where the tile plan takes them), checked whole:
+    every output against the fp64 oracle (about 30 s of oracle time for
+    gate/up or down on a 16-core host).  Besides the whole-matrix criteria,
+    every 128-row block must meet the relative L2 bound on its own, so a fault
+    confined to one tile of the persistent schedule cannot hide in the
+    average."""
     layer = synth.make_config(name)
     M = layer["x"].shape[0]
     y = gu.bf16_to_f64(gu.run_gpu(layer))
-    rng = np.random.default_rng(1)
-    # rows of each 128-row quarter of a 512-row pair tile (both CTAs, both halves)
-    edges = [0, 1, 127, 128, 255, 256, 383, 384, 511, 512, M - 1]
-    rows = np.unique(np.concatenate([edges, rng.choice(M, 27, replace=False)]))
-    gu.assert_close(y[rows], gu.oracle_y(layer, rows), f"{name} sampled rows")
     assert np.all(np.isfinite(y))
+    ref = gu.oracle_y(layer)
+    gu.assert_close(y, ref, f"{name} all {M} rows")
+    for r0 in range(0, M, 128):
+        d = np.linalg.norm(y[r0:r0 + 128] - ref[r0:r0 + 128]) / np.linalg.norm(ref[r0:r0 + 128])
+        assert d <= gu.REL_L2_TOL, f"{name} rows {r0}..{r0 + 127}: relative L2 {d:.3e}"
 
 
 @pytest.mark.parametrize("tokens", [1, 2, 7, 8, 9, 16, 17, 31, 32, 33, 64, 255, 256, 257])
@@ -400,3 +407,37 @@ def test_host_buffer_call_equals_device_call(tokens):
     assert lb.device_status() == lb.LB_OK
     assert np.array_equal(gu.bf16_bits(y_host), gu.bf16_bits(ref))
     gu.assert_close(gu.bf16_to_f64(y_host), gu.oracle_y(layer), f"host buffers M={tokens}")
+
+
+@pytest.mark.parametrize("tokens", [1, 3, 37])
+def test_chained_host_calls_read_the_previous_output(tokens):
+    """Host-buffer calls chained layer to layer on one stream without a sync:
+    the y_host of one call is the x_host of the next.  Each call's gather
+    kernel must read x_host only after the previous call's last kernel has
+    stored it (that kernel releases its dependents before its stores), so the
+    chain gives the bits of the same chain run through device buffers."""
+    import torch
+    n = 512
+    layer = synth.make_layer(n, n, [64, 32], tokens, config_id=883)
+    paths = gu.device_paths(layer)
+    x = gu.bf16_tensor(layer["x"])
+    ws = torch.empty(max(16, lb.forward_workspace_bytes(tokens, n, n, 64, 32)), dtype=torch.uint8, device="cuda")
+    depth = 5
+    # the reference chain: device buffers, synchronised after every call
+    refs, cur = [], x
+    for _ in range(depth):
+        cur = lb.linear_forward(cur, paths[0], paths[1], workspace=ws)
+        torch.cuda.synchronize()
+        refs.append(cur.clone())
+    hosts = [x.cpu().pin_memory()] + [torch.full((tokens, n), 3.0, dtype=torch.bfloat16).pin_memory()
+                                      for _ in range(depth)]
+    x_dev = torch.empty_like(x)
+    y_dev = torch.empty((tokens, n), dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    for d in range(depth):
+        lb.linear_forward_host(hosts[d], paths[0], paths[1], hosts[d + 1], x_dev, y_dev, ws)
+    torch.cuda.synchronize()
+    assert lb.device_status() == lb.LB_OK
+    for d in range(depth):
+        assert np.array_equal(gu.bf16_bits(hosts[d + 1]), gu.bf16_bits(refs[d])), f"layer {d}"
+    gu.assert_close(gu.bf16_to_f64(hosts[1]), gu.oracle_y(layer), f"first layer M={tokens}")

@@ -50,3 +50,23 @@ def test_refused_shapes_write_nothing():
     assert e.value.status == lb.LB_ERR_UNSUPPORTED_SHAPE
     torch.cuda.synchronize()
     assert bool((y == 3.0).all())
+
+
+def test_scratch_too_small_writes_nothing():
+    """32 tokens (inside the token limit) on two paths of rank 16384: the
+    latent needs 2 MiB, more than the fixed array holds, so the call is
+    refused on the host with LB_ERR_WORKSPACE_TOO_SMALL and y keeps its
+    canary values."""
+    import torch
+    n, r, tokens = 256, 16384, 32
+    assert lb.forward_workspace_bytes(tokens, n, n, r, r) > (1 << 20)
+    layer = synth.make_layer(n, n, [r, r], tokens, config_id=1201)
+    paths = gu.device_paths(layer)
+    x = gu.bf16_tensor(layer["x"])
+    y = torch.full((tokens, n), 3.0, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(lb.LbError) as e:
+        lb.linear_forward_fixed_scratch(x, paths[0], paths[1], y=y)
+    assert e.value.status == lb.LB_ERR_WORKSPACE_TOO_SMALL
+    torch.cuda.synchronize()
+    assert bool((y == 3.0).all())
+    assert lb.device_status() == lb.LB_OK
