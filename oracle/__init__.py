@@ -22,6 +22,9 @@ Sources (web pages about LittleBit / LittleBit-2; cited by page and section):
 Functions:
 
 * :func:`forward` - the factored pass, in C (``lb_oracle.c``), plain loops.
+* :func:`backward` - the gradients of a loss with respect to x and to every
+  path's h, g and l, given dL/dy: the chain rule through the five steps of
+  the factored pass, in C (``lb_oracle.c``), plain loops.
 * :func:`dense_weight` - ``W = sum_p diag(h) S_U diag(l) S_V^T diag(g)``, the
   same layer as one dense matrix (a numpy matmul per path).
 * :func:`pack_signs` - this oracle's own bit packer for the library's packed
@@ -93,6 +96,11 @@ def _load():
             lib.oracle_expand.argtypes = [
                 ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
                 ctypes.POINTER(_Path), ctypes.c_int, ctypes.c_void_p]
+            lib.oracle_backward.restype = ctypes.c_int
+            lib.oracle_backward.argtypes = [
+                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                ctypes.POINTER(_Path), ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                ctypes.c_void_p]
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_num_threads.argtypes = []
             _lib = lib
@@ -212,6 +220,41 @@ def expand(z: np.ndarray, paths: list[dict]) -> np.ndarray:
     if rc != 0:
         raise RuntimeError(f"oracle_expand failed ({rc})")
     return y
+
+
+def backward(x: np.ndarray, dy: np.ndarray, paths: list[dict]) -> dict:
+    """fp64 backward pass of the layer for a loss L with ``dL/dy = dy``.
+
+    The pages give the forward pass (sesamedisk.com, "What the method actually
+    computes", Proposition 1) and train through it (littlebitllm.com,
+    "Pipeline": quantization-aware training with a smooth surrogate for the
+    gradient of sign); these are the chain-rule gradients of its five steps,
+    with the signs held fixed: ``dx`` [tokens, n_in] and, per path, ``dh``
+    [n_out], ``dg`` [n_in], ``dl`` [r] (lists, path order).  ``x`` and ``dy``
+    are float64 [tokens, n_in] and [tokens, n_out]; ``paths`` as for
+    :func:`forward`."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    dy = np.ascontiguousarray(dy, dtype=np.float64)
+    P = [_as_path_arrays(p) for p in paths]
+    n_in = x.shape[1]
+    n_out = P[0]["su"].shape[0]
+    if x.ndim != 2 or dy.shape != (x.shape[0], n_out):
+        raise ValueError("x must be [tokens, n_in] and dy [tokens, n_out]")
+    for p in P:
+        if p["sv"].shape[0] != n_in or p["su"].shape[0] != n_out:
+            raise ValueError("factor shapes do not match x / each other")
+    R = sum(p["rank"] for p in P)
+    dx = np.empty_like(x)
+    dh = np.empty((len(P), n_out))
+    dg = np.empty((len(P), n_in))
+    dl = np.empty(R)
+    rc = _load().oracle_backward(x.ctypes.data, dy.ctypes.data, x.shape[0], n_in, n_out, _c_paths(P), len(P),
+                                 dx.ctypes.data, dh.ctypes.data, dg.ctypes.data, dl.ctypes.data)
+    if rc != 0:
+        raise RuntimeError(f"oracle_backward failed ({rc})")
+    offs = np.cumsum([0] + [p["rank"] for p in P])
+    return {"dx": dx, "dh": [dh[j] for j in range(len(P))], "dg": [dg[j] for j in range(len(P))],
+            "dl": [dl[offs[j]:offs[j + 1]] for j in range(len(P))]}
 
 
 def dense_weight(paths: list[dict]) -> np.ndarray:
