@@ -22,6 +22,8 @@ Printed on rank 0, one JSON line:
   clocks      SM clocks and throttle reasons sampled during the timed region
   prefill     Qwen3-14B gate/up and k/v at 8192 tokens: TFLOP/s, the dominant
               kernel's roofline against the measured bf16 peak, clocks
+  backward    Qwen3-14B gate/up at 8192 tokens: lb_linear_backward (dx, dh,
+              dg, dl) TFLOP/s against the measured bf16 peak
   decode_block_fused  a Llama-2-7B decoder block's seven linears at 1 token as
               four sibling calls, chained
   dense_baseline      Llama-2-70B gate/up at 1 token against one cuBLAS bf16
@@ -180,11 +182,11 @@ class ClockSampler:
 def tensor_peak(peaks, clocks):
     """The tensor-core denominator for a timed region: the sustained figure is
     cuBLAS bf16 with the clock settled under the power cap, so it applies when
-    the region ran power-capped too (the cap reported, or the median SM clock
-    well below its maximum); otherwise the burst figure applies."""
-    reasons = clocks.get("reasons") or []
+    the region itself ran with its SM clock held down (median below 95 % of
+    the maximum); a region whose median clock is at the maximum takes the
+    burst figure even if a power-cap reason showed up in some sample."""
     mhz, top = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
-    capped = "sw_power_cap" in reasons or (mhz is not None and top and mhz < 0.9 * top)
+    capped = mhz is not None and bool(top) and mhz < 0.95 * top
     return (peaks["bf16_sustained"], peaks["source"] + " (sustained)") if capped else \
         (peaks["bf16"], peaks["source"] + " (burst)")
 
@@ -513,6 +515,61 @@ def measure_prefill(name, args, world, local, device, peaks, tokens=None):
             "per_kernel": per_kernel, "parity": parity, "clocks": clocks, "gpu_launches": 2 * calls}
 
 
+def measure_backward(name, args, world, local, device, peaks, tokens=None):
+    """The layer's backward pass (lb_linear_backward: dx and every path's dh,
+    dg, dl) on one workload at `tokens` tokens: four tensor-core contractions,
+    2 M sum_p r_p (n_in + n_out) flops each pair, so twice the forward pass's
+    algorithmic flops.  Chained from a CUDA graph, inputs larger than L2 (x
+    and dy rotated over copies where they are not), at least
+    `--prefill-seconds` of timed calls with the clocks sampled."""
+    import torch
+    import binarized_rank_linear_b200 as lb
+    c = synth.CONFIGS[name]
+    tokens = tokens or c.tokens[-1]
+    d = DeviceLayer(synth.make_config(name, tokens), device, tokens)
+    rng = np.random.default_rng(7)
+    dy = torch.from_numpy(synth.f32_to_bf16_bits(rng.standard_normal((tokens, d.n_out), dtype=np.float32))
+                          .view(np.int16)).to(device).view(torch.bfloat16)
+    io = 2 * tokens * (d.n_in + d.n_out)
+    nx = max(1, min(4, -(-2 * L2_BYTES // io) + 1)) if io <= 2 * L2_BYTES else 1
+    xs = [(d.x, dy)] + [(d.x.clone(), dy.clone()) for _ in range(nx - 1)]
+    two = lambda s: (s[0], s[1] if len(s) > 1 else None)
+    ws = torch.empty(max(16, lb.backward_workspace_bytes(tokens, d.n_in, d.n_out, d.ranks[0],
+                                                         d.ranks[1] if len(d.ranks) > 1 else 0)),
+                     dtype=torch.uint8, device=device)
+    dx = torch.empty((tokens, d.n_in), dtype=torch.bfloat16, device=device)
+    call = lambda i: lb.linear_backward(xs[i % nx][0], xs[i % nx][1], *two(d.base), dx=dx, workspace=ws)
+    call(0)
+    torch.cuda.synchronize()
+    assert lb.device_status() == lb.LB_OK
+    g = capture(call, nx, device)
+    for _ in range(max(3, args.warmup)):
+        g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    reps = max(3, int(args.prefill_seconds / max(1e-6, e0.elapsed_time(e1) / 1e3)))
+    ms, clocks = time_graph(g, reps, stream, local, world, device)
+    assert lb.device_status() == lb.LB_OK
+    calls = reps * nx
+    per_call_s = ms / 1e3 / calls
+    flops = 2 * d.nflops
+    pk, pk_source = tensor_peak(peaks, clocks)
+    achieved = flops / per_call_s / 1e12
+    return {"workload": workload_name(c, tokens) + ", backward (dx, dh, dg, dl)", "tokens": tokens, "calls": calls,
+            "us_per_call": per_call_s * 1e6, "algorithmic_flops_per_call": flops,
+            "value": aggregate(flops / 1e12 * calls, ms / 1e3, world), "unit": "TFLOP/s",
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
+                         "frac": achieved / pk, "traffic": None, "kernel": "whole lb_linear_backward call "
+                         "(2 bit transposes, sign_gemm_kernel<3> x2, sign_gemm_kernel<4> x2, reduce_partials_kernel)",
+                         "peak_source": pk_source},
+            "clocks": clocks, "gpu_launches": 9 * calls}
+
+
 def dense_baseline(d, device, seconds, stream, local, world):
     """The layer as the dense bf16 matrix of dense_weight_torch, applied with
     one cuBLAS GEMM per call (torch.matmul): the comparison behind the pages'
@@ -790,11 +847,15 @@ def run_lb(args, world, rank, local):
     # the default run also measures prefill (the metric's TFLOP/s half), a
     # whole decoder block of fused sibling calls at batch 1, and the dense
     # baseline of the pages' kernel comparison
-    prefill = block = dense = None
+    prefill = block = dense = backward = None
     if not args.no_extras:
         prefill = {}
         for name in args.prefill.split(",") if args.prefill else []:
             prefill[name] = measure_prefill(name, args, world, local, device, peaks)
+            torch.cuda.empty_cache()
+        backward = {}
+        for name in args.backward.split(",") if args.backward else []:
+            backward[name] = measure_backward(name, args, world, local, device, peaks)
             torch.cuda.empty_cache()
         block = measure_block("llama2_7b", 1, True, args.steps, args.warmup, world, local, device, seconds=0.1)
         torch.cuda.empty_cache()
@@ -850,6 +911,8 @@ def run_lb(args, world, rank, local):
            "impl": "lb"}
     if prefill:
         out["prefill"] = prefill
+    if backward:
+        out["backward"] = backward
     if block is not None:
         out["decode_block_fused"] = block
     if dense is not None:
@@ -871,6 +934,8 @@ def main(argv=None):
     ap.add_argument("--prefill", default="qwen3_14b_gate,qwen3_14b_kv",
                     help="prefill workloads measured beside the main line (comma-separated)")
     ap.add_argument("--prefill-seconds", type=float, default=0.3)
+    ap.add_argument("--backward", default="qwen3_14b_gate",
+                    help="workloads whose backward pass is measured beside the main line (comma-separated)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the prefill, fused-block and dense-baseline measurements")
     ap.add_argument("--no-cpu", action="store_true")

@@ -112,6 +112,11 @@ def lib() -> ctypes.CDLL:
             L.lb_linear_forward_host.restype = i32
             L.lb_linear_forward_host.argtypes = [vp, i64, i64, i64, ctypes.POINTER(LbPath), ctypes.POINTER(LbPath),
                                                  vp, vp, vp, vp, sz, vp]
+            L.lb_backward_workspace_bytes.restype = sz
+            L.lb_backward_workspace_bytes.argtypes = [i64, i64, i64, i64, i64]
+            L.lb_linear_backward.restype = i32
+            L.lb_linear_backward.argtypes = [vp, vp, i64, i64, i64, i64, i64, ctypes.POINTER(LbPath),
+                                             ctypes.POINTER(LbPath), vp, i64, vp, vp, vp, vp, sz, vp]
             L.lb_device_status.restype = i32
             L.lb_device_status.argtypes = [vp, ctypes.POINTER(i32)]
             L.lb_set_prefill_pairs.restype = i32
@@ -415,6 +420,49 @@ def linear_forward_fixed_scratch(x, main: PackedPath, residual: PackedPath | Non
         ctypes.byref(cr) if cr is not None else None, y.data_ptr(), y.stride(0), _stream_handle(stream)),
         "lb_linear_forward_fixed_scratch")
     return y
+
+
+def backward_workspace_bytes(tokens: int, n_in: int, n_out: int, rank_main: int, rank_residual: int = 0) -> int:
+    return int(lib().lb_backward_workspace_bytes(tokens, n_in, n_out, rank_main, rank_residual))
+
+
+def linear_backward(x, dy, main: PackedPath, residual: PackedPath | None = None, dx=None, want_dx: bool = True,
+                    workspace=None, stream=None) -> dict:
+    """``lb_linear_backward``: the gradients of a loss with respect to the
+    layer's input and scale vectors, given ``dy`` = dL/dy (bf16 [tokens,
+    n_out]) and the forward input ``x`` (bf16 [tokens, n_in]).  Returns
+    ``{"dx": bf16 [tokens, n_in] or None, "dh": fp32 [paths, n_out], "dg":
+    fp32 [paths, n_in], "dl": fp32 [r_main + r_residual]}``; outputs and the
+    workspace are allocated with torch when not given."""
+    torch = _torch()
+    _require(x, "x", torch.bfloat16)
+    _require(dy, "dy", torch.bfloat16)
+    tokens, n_in = x.shape
+    n_out = main.h.shape[0]
+    if tuple(dy.shape) != (tokens, n_out):
+        raise ValueError(f"dy must be [{tokens}, {n_out}], got {tuple(dy.shape)}")
+    npaths = 2 if residual is not None else 1
+    if dx is None and want_dx:
+        dx = torch.empty((tokens, n_in), dtype=torch.bfloat16, device=x.device)
+    if dx is not None:
+        _require(dx, "dx", torch.bfloat16)
+    dh = torch.empty((npaths, n_out), dtype=torch.float32, device=x.device)
+    dg = torch.empty((npaths, n_in), dtype=torch.float32, device=x.device)
+    dl = torch.empty((main.rank + (residual.rank if residual is not None else 0),), dtype=torch.float32,
+                     device=x.device)
+    if workspace is None:
+        need = backward_workspace_bytes(tokens, n_in, n_out, main.rank, residual.rank if residual else 0)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    _require_workspace(workspace)
+    cm = main.as_c()
+    cr = residual.as_c() if residual is not None else None
+    _check(lib().lb_linear_backward(
+        x.data_ptr(), dy.data_ptr(), tokens, n_in, n_out, x.stride(0), dy.stride(0), ctypes.byref(cm),
+        ctypes.byref(cr) if cr is not None else None, dx.data_ptr() if dx is not None else None,
+        dx.stride(0) if dx is not None else n_in, dh.data_ptr(), dg.data_ptr(), dl.data_ptr(),
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream)),
+        "lb_linear_backward")
+    return {"dx": dx, "dh": dh, "dg": dg, "dl": dl}
 
 
 def device_status(stream=None) -> int:

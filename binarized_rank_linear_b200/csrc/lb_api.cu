@@ -484,6 +484,78 @@ lb_status lb_expand_forward(const uint16_t *z, int64_t tokens, int64_t n_out, in
     return LB_OK;
 }
 
+size_t lb_backward_workspace_bytes(int64_t tokens, int64_t n_in, int64_t n_out, int64_t rank_main,
+                                   int64_t rank_residual)
+{
+    if (tokens < 0 || n_in <= 0 || n_out <= 0 || rank_main <= 0 || rank_residual < 0) return 0;
+    if (tokens > kMaxTokens || n_in > kMaxDim || n_out > kMaxDim || rank_main > kMaxRank || rank_residual > kMaxRank)
+        return 0;
+    if (tokens == 0 || n_in % 32 != 0 || n_out % 32 != 0 || rank_main % 32 != 0 || rank_residual % 32 != 0) return 0;
+    const int ranks[2] = {(int)rank_main, (int)rank_residual};
+    return lb::backward_workspace_bytes((int)tokens, (int)n_in, (int)n_out, ranks, rank_residual > 0 ? 2 : 1);
+}
+
+lb_status lb_linear_backward(const uint16_t *x, const uint16_t *dy, int64_t tokens, int64_t n_in, int64_t n_out,
+                             int64_t ldx, int64_t lddy, const lb_path *main, const lb_path *residual, uint16_t *dx,
+                             int64_t lddx, float *dh, float *dg, float *dl, void *workspace, size_t workspace_bytes,
+                             void *stream)
+{
+    if (tokens < 0 || n_in <= 0 || n_out <= 0) return LB_ERR_INVALID_ARGUMENT;
+    if (!main || !dh || !dg || !dl) return LB_ERR_INVALID_ARGUMENT;
+    if (tokens > 0 && (!x || !dy)) return LB_ERR_INVALID_ARGUMENT;  // no tokens: x and dy are not read
+    if (ldx < n_in || lddy < n_out || (dx && lddx < n_in)) return LB_ERR_INVALID_ARGUMENT;
+    if (n_in % 32 != 0 || n_out % 32 != 0 || n_in > kMaxDim || n_out > kMaxDim || tokens > kMaxTokens)
+        return LB_ERR_UNSUPPORTED_SHAPE;
+    if (ldx % 8 != 0 || lddy % 8 != 0 || !aligned16(x) || !aligned16(dy)) return LB_ERR_MISALIGNED;  // null is aligned
+    if (dx && (lddx % 8 != 0 || !aligned16(dx))) return LB_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(dh) | reinterpret_cast<uintptr_t>(dg) | reinterpret_cast<uintptr_t>(dl)) & 3u)
+        return LB_ERR_MISALIGNED;
+    lb::BackwardArgs b{};
+    b.npaths = residual ? 2 : 1;
+    lb_status st = check_path(main, n_in, n_out, &b.path[0]);
+    if (st == LB_OK && residual) st = check_path(residual, n_in, n_out, &b.path[1]);
+    if (st != LB_OK) return st;
+    const int ranks[2] = {b.path[0].rank, b.npaths > 1 ? b.path[1].rank : 0};
+    const size_t need = tokens > 0 ? lb::backward_workspace_bytes((int)tokens, (int)n_in, (int)n_out, ranks, b.npaths) : 0;
+    if (need > 0 && !workspace) return LB_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes < need) return LB_ERR_WORKSPACE_TOO_SMALL;
+    if (workspace && !aligned16(workspace)) return LB_ERR_MISALIGNED;
+    lb::DeviceInfo dev;
+    st = device_info(&dev);
+    if (st != LB_OK) return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (tokens == 0) {
+        // no tokens: every scale gradient is an empty sum
+        const int R = ranks[0] + ranks[1];
+        if (cudaMemsetAsync(dh, 0, sizeof(float) * (size_t)b.npaths * (size_t)n_out, s) != cudaSuccess ||
+            cudaMemsetAsync(dg, 0, sizeof(float) * (size_t)b.npaths * (size_t)n_in, s) != cudaSuccess ||
+            cudaMemsetAsync(dl, 0, sizeof(float) * (size_t)R, s) != cudaSuccess) {
+            cudaGetLastError();
+            return LB_ERR_CUDA;
+        }
+        return LB_OK;
+    }
+    b.x = x;
+    b.ldx = ldx;
+    b.dy = dy;
+    b.lddy = lddy;
+    b.tokens = (int)tokens;
+    b.n_in = (int)n_in;
+    b.n_out = (int)n_out;
+    b.dx = dx;
+    b.lddx = lddx;
+    b.dh = dh;
+    b.dg = dg;
+    b.dl = dl;
+    b.workspace = workspace;
+    b.workspace_bytes = workspace_bytes;
+    if (lb::backward_launch(b, dev, s) != cudaSuccess) {
+        cudaGetLastError();
+        return LB_ERR_CUDA;
+    }
+    return LB_OK;
+}
+
 lb_status lb_device_status(void *stream, lb_status *out)
 {
     if (!out) return LB_ERR_INVALID_ARGUMENT;

@@ -1,0 +1,322 @@
+// lb_backward.cu - the backward pass of the layer: the gradients with respect
+// to x and to every path's scale vectors h, g and l, given dy = dL/dy.
+//
+// The forward pass (sesamedisk.com, "Samsung LittleBit 13B Model", section
+// "What the method actually computes", Proposition 1) per path p is
+//     t = g (.) x,  c = S_V^T t,  z = l (.) c,  e = S_U z,  y = sum_p h (.) e,
+// and quantization-aware training runs back through it (littlebitllm.com,
+// "Pipeline").  With the signs held fixed the chain rule gives, per path,
+//     a  = S_U^T (h (.) dy)            (the gradient with respect to z)
+//     dl = sum over tokens of a (.) c
+//     dt = S_V (l (.) a)               (the gradient with respect to t)
+//     dg = sum over tokens of x (.) dt,   dx = sum_p g (.) dt
+//     dh = sum over tokens of dy (.) e
+// Four tcgen05 contractions compute them (the prefill kernels' modes 3 and 4,
+// lb_prefill.cu):
+//   K1  c = S_V^T (g (.) x)          x [M x n_in] against the packed rows of V^T
+//   K2  a = S_U^T (h (.) dy)         dy [M x n_out] against the rows of U^T;
+//                                    the epilogue also forms a (.) c per
+//                                    32-token block (dl partials)
+//   K3  e_p = S_U,p (l_p (.) c_p)    c against the rows of U, l on the K side,
+//                                    one accumulator per path; the epilogue
+//                                    forms dy (.) e_p per block (dh partials)
+//                                    and stores nothing
+//   K4  dt_p = S_V,p (l_p (.) a_p)   a against the rows of V; the epilogue
+//                                    stores dx = sum_p g_p (.) dt_p (bf16) and
+//                                    forms x (.) dt_p per block (dg partials)
+// then one kernel adds each partial column over the blocks in block order, so
+// the results do not depend on timing.  K2 and K4 read the factors along the
+// other axis from the forward pass: U^T packed along n_out and V packed along
+// r, which two bit-transpose launches make from the forward's packed words
+// into the workspace, so the call takes the forward pass's lb_path as it is.
+// c and a travel between the contractions as fp16, unscaled.
+#include <algorithm>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "lb_common.cuh"
+#include "lb_internal.h"
+
+namespace lb {
+namespace {
+
+// ------------------------------------------------------------ bit transpose
+// out[col][row / 32] bit (row % 32) = in[row][col / 32] bit (col % 32), for a
+// packed matrix of `rows` x `cols` bits (both multiples of 32).  One warp per
+// column word cb and up to kRowBlocks consecutive 32-row blocks rb: for each
+// block, lane l loads row 32 rb + l's word cb, and the ballot of bit j over
+// the lanes is output row 32 cb + j's word rb, kept by lane j.  Each lane
+// then stores its consecutive output words together (one 32-byte sector).
+constexpr int kTransposeWarps = 8;
+constexpr int kRowBlocks = 8;
+
+__global__ void __launch_bounds__(32 * kTransposeWarps)
+    transpose_bits_kernel(const uint32_t *__restrict__ in, int64_t ld_in, int rows, int cols,
+                          uint32_t *__restrict__ out, int64_t ld_out)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t job = (int64_t)blockIdx.x * kTransposeWarps + (threadIdx.x >> 5);
+    const int rbs = rows >> 5, cbs = cols >> 5;
+    const int groups = (rbs + kRowBlocks - 1) / kRowBlocks;
+    if (job >= (int64_t)groups * cbs) return;  // whole warps leave together
+    const int rg = (int)(job % groups), cb = (int)(job / groups);
+    const int rb0 = rg * kRowBlocks, nrb = min(kRowBlocks, rbs - rb0);
+    uint32_t w[kRowBlocks];
+#pragma unroll
+    for (int q = 0; q < kRowBlocks; ++q)
+        w[q] = q < nrb ? __ldg(in + (int64_t)(32 * (rb0 + q) + lane) * ld_in + cb) : 0u;
+    uint32_t mine[kRowBlocks];
+#pragma unroll
+    for (int q = 0; q < kRowBlocks; ++q) {
+        mine[q] = 0u;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const uint32_t t = __ballot_sync(0xffffffffu, (w[q] >> j) & 1u);
+            if (lane == j) mine[q] = t;
+        }
+    }
+    uint32_t *dst = out + (int64_t)(32 * cb + lane) * ld_out + rb0;
+#pragma unroll
+    for (int q = 0; q < kRowBlocks; ++q)
+        if (q < nrb) dst[q] = mine[q];
+}
+
+cudaError_t transpose_bits(const uint32_t *in, int64_t ld_in, int rows, int cols, uint32_t *out, int64_t ld_out,
+                           cudaStream_t stream)
+{
+    const int64_t jobs = (int64_t)((rows / 32 + kRowBlocks - 1) / kRowBlocks) * (cols / 32);
+    const unsigned grid = (unsigned)((jobs + kTransposeWarps - 1) / kTransposeWarps);
+    transpose_bits_kernel<<<grid, 32 * kTransposeWarps, 0, stream>>>(in, ld_in, rows, cols, out, ld_out);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ partial sums
+// out[n] = sum over the 32-token blocks rb = 0 .. blocks - 1 of part[rb][n],
+// for up to kMaxSegments vectors in one launch.  A CTA takes 32 columns; its
+// kGroups warps take the blocks rb = g, g + kGroups, ... of those columns
+// (each in block order), and warp 0 adds the kGroups sums in group order:
+// a fixed order, so the result does not depend on timing.
+constexpr int kMaxSegments = 5;
+constexpr int kGroups = 8;
+struct ReduceSeg {
+    const float *part;
+    float *out;
+    int n;
+};
+struct ReduceParams {
+    ReduceSeg seg[kMaxSegments];
+    int nseg;
+    int blocks;  // 32-token blocks
+};
+
+__global__ void __launch_bounds__(32 * kGroups) reduce_partials_kernel(const __grid_constant__ ReduceParams p)
+{
+    __shared__ float sums[kGroups][32];
+    const int lane = threadIdx.x & 31, g = threadIdx.x >> 5;
+    int64_t col = (int64_t)blockIdx.x * 32 + lane;
+    const ReduceSeg *seg = nullptr;
+    for (int s = 0; s < p.nseg; ++s) {
+        if (col < p.seg[s].n) {
+            seg = &p.seg[s];
+            break;
+        }
+        col -= p.seg[s].n;
+    }
+    float acc = 0.0f;
+    if (seg != nullptr)
+        for (int rb = g; rb < p.blocks; rb += kGroups) acc += __ldg(seg->part + (int64_t)rb * seg->n + col);
+    sums[g][lane] = acc;
+    __syncthreads();
+    if (g == 0 && seg != nullptr) {
+        float t = 0.0f;
+#pragma unroll
+        for (int q = 0; q < kGroups; ++q) t += sums[q][lane];
+        seg->out[col] = t;
+    }
+}
+
+size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+// Workspace layout of one call (every piece 256-byte aligned).
+struct BwdLayout {
+    size_t ut[2], v[2];     // transposed sign words of each path
+    size_t c, a;            // fp16 [M x R]
+    size_t pl, ph[2], pg[2];  // partials
+    size_t total;
+};
+
+BwdLayout layout(int M, int n_in, int n_out, const int *ranks, int npaths)
+{
+    BwdLayout L{};
+    size_t off = 0;
+    const int R = ranks[0] + (npaths > 1 ? ranks[1] : 0);
+    const size_t RB = (size_t)((M + 31) / 32);
+    for (int q = 0; q < npaths; ++q) {
+        L.ut[q] = off;
+        off += align256((size_t)ranks[q] * (size_t)(n_out / 32) * 4);
+        L.v[q] = off;
+        off += align256((size_t)n_in * (size_t)(ranks[q] / 32) * 4);
+    }
+    L.c = off;
+    off += align256((size_t)M * R * 2);
+    L.a = off;
+    off += align256((size_t)M * R * 2);
+    L.pl = off;
+    off += align256(RB * R * 4);
+    for (int q = 0; q < npaths; ++q) {
+        L.ph[q] = off;
+        off += align256(RB * (size_t)n_out * 4);
+        L.pg[q] = off;
+        off += align256(RB * (size_t)n_in * 4);
+    }
+    L.total = off;
+    return L;
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(int tokens, int n_in, int n_out, const int *ranks, int npaths)
+{
+    return layout(tokens, n_in, n_out, ranks, npaths).total;
+}
+
+cudaError_t backward_launch(const BackwardArgs &b, const DeviceInfo &dev, cudaStream_t stream)
+{
+    const int M = b.tokens, npaths = b.npaths;
+    const int ranks[2] = {b.path[0].rank, npaths > 1 ? b.path[1].rank : 0};
+    const int r0 = ranks[0], r1 = ranks[1], R = r0 + r1;
+    const BwdLayout L = layout(M, b.n_in, b.n_out, ranks, npaths);
+    uint8_t *ws = static_cast<uint8_t *>(b.workspace);
+    uint32_t *ut[2] = {nullptr, nullptr}, *v[2] = {nullptr, nullptr};
+    cudaError_t e = cudaSuccess;
+    for (int q = 0; q < npaths && e == cudaSuccess; ++q) {
+        const PathDesc &P = b.path[q];
+        ut[q] = reinterpret_cast<uint32_t *>(ws + L.ut[q]);
+        v[q] = reinterpret_cast<uint32_t *>(ws + L.v[q]);
+        // U [n_out x r] -> U^T [r x n_out]; V^T [r x n_in] -> V [n_in x r]
+        e = transpose_bits(P.u_bits, P.u_ld, b.n_out, P.rank, ut[q], b.n_out / 32, stream);
+        if (e == cudaSuccess) e = transpose_bits(P.vt_bits, P.vt_ld, P.rank, b.n_in, v[q], P.rank / 32, stream);
+    }
+    if (e != cudaSuccess) return e;
+    uint16_t *c = reinterpret_cast<uint16_t *>(ws + L.c);
+    uint16_t *a = reinterpret_cast<uint16_t *>(ws + L.a);
+    float *pl = reinterpret_cast<float *>(ws + L.pl);
+    float *ph[2] = {reinterpret_cast<float *>(ws + L.ph[0]), npaths > 1 ? reinterpret_cast<float *>(ws + L.ph[1]) : nullptr};
+    float *pg[2] = {reinterpret_cast<float *>(ws + L.pg[0]), npaths > 1 ? reinterpret_cast<float *>(ws + L.pg[1]) : nullptr};
+    const PathDesc &P0 = b.path[0], &P1 = b.path[1];
+    const bool two = npaths > 1;
+
+    // K1: c = S_V^T (g (.) x), unscaled
+    Bwd1Args k1{};
+    k1.M = M;
+    k1.K = b.n_in;
+    k1.r0 = r0;
+    k1.r1 = r1;
+    k1.a = b.x;
+    k1.lda = b.ldx;
+    k1.bits0 = P0.vt_bits;
+    k1.ld0 = P0.vt_ld;
+    k1.s0 = P0.g;
+    if (two) {
+        k1.bits1 = P1.vt_bits;
+        k1.ld1 = P1.vt_ld;
+        k1.s1 = P1.g;
+    }
+    k1.out = c;
+    k1.ldo = R;
+    e = bwd_contraction1(k1, dev, stream);
+    if (e != cudaSuccess) return e;
+
+    // K2: a = S_U^T (h (.) dy), unscaled; dl partials sum a (.) c
+    Bwd1Args k2{};
+    k2.M = M;
+    k2.K = b.n_out;
+    k2.r0 = r0;
+    k2.r1 = r1;
+    k2.a = b.dy;
+    k2.lda = b.lddy;
+    k2.bits0 = ut[0];
+    k2.ld0 = b.n_out / 32;
+    k2.s0 = P0.h;
+    if (two) {
+        k2.bits1 = ut[1];
+        k2.ld1 = b.n_out / 32;
+        k2.s1 = P1.h;
+    }
+    k2.out = a;
+    k2.ldo = R;
+    k2.aux = c;
+    k2.ldaux = R;
+    k2.part = pl;
+    e = bwd_contraction1(k2, dev, stream);
+    if (e != cudaSuccess) return e;
+
+    // K3: e_p = S_U,p (l_p (.) c_p); dh partials sum dy (.) e_p
+    Bwd2Args k3{};
+    k3.M = M;
+    k3.N = b.n_out;
+    k3.r0 = r0;
+    k3.r1 = r1;
+    k3.a = c;
+    k3.lda = R;
+    k3.bits0 = P0.u_bits;
+    k3.ld0 = P0.u_ld;
+    k3.l0 = P0.l;
+    if (two) {
+        k3.bits1 = P1.u_bits;
+        k3.ld1 = P1.u_ld;
+        k3.l1 = P1.l;
+    }
+    k3.aux = b.dy;
+    k3.ldaux = b.lddy;
+    k3.part0 = ph[0];
+    k3.part1 = ph[1];
+    e = bwd_contraction2(k3, dev, stream);
+    if (e != cudaSuccess) return e;
+
+    // K4: dt_p = S_V,p (l_p (.) a_p); dx = sum_p g_p (.) dt_p; dg partials sum x (.) dt_p
+    Bwd2Args k4{};
+    k4.M = M;
+    k4.N = b.n_in;
+    k4.r0 = r0;
+    k4.r1 = r1;
+    k4.a = a;
+    k4.lda = R;
+    k4.bits0 = v[0];
+    k4.ld0 = r0 / 32;
+    k4.l0 = P0.l;
+    if (two) {
+        k4.bits1 = v[1];
+        k4.ld1 = r1 / 32;
+        k4.l1 = P1.l;
+    }
+    k4.aux = b.x;
+    k4.ldaux = b.ldx;
+    k4.part0 = pg[0];
+    k4.part1 = pg[1];
+    k4.out = b.dx;
+    k4.ldo = b.lddx;
+    k4.t0 = P0.g;
+    k4.t1 = two ? P1.g : nullptr;
+    e = bwd_contraction2(k4, dev, stream);
+    if (e != cudaSuccess) return e;
+
+    // the partial sums, added over the 32-token blocks in block order
+    ReduceParams rp{};
+    rp.blocks = (M + 31) / 32;
+    int total = 0;
+    auto add = [&](const float *part, float *out, int n) {
+        rp.seg[rp.nseg++] = ReduceSeg{part, out, n};
+        total += n;
+    };
+    add(pl, b.dl, R);
+    add(ph[0], b.dh, b.n_out);
+    if (two) add(ph[1], b.dh + b.n_out, b.n_out);
+    add(pg[0], b.dg, b.n_in);
+    if (two) add(pg[1], b.dg + b.n_in, b.n_in);
+    // every segment's length is a multiple of 32, so a CTA's 32 columns lie in one segment
+    reduce_partials_kernel<<<(unsigned)(total / 32), 32 * kGroups, 0, stream>>>(rp);
+    return cudaGetLastError();
+}
+
+}  // namespace lb

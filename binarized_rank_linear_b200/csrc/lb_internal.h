@@ -128,6 +128,63 @@ cudaError_t prefill_latent(const ForwardArgs &a, const DeviceInfo &dev, cudaStre
 cudaError_t prefill_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream, const uint16_t *z,
                            int64_t ldz);
 
+// ---------------------------------------------------------------- backward (lb_backward.cu, lb_prefill.cu)
+// The backward pass's two contraction shapes on the prefill kernels.
+// Contraction-1 shape: C[m, n] = sum_k A[m, k] B[n, k] with A bf16 [M x K],
+// B[n, k] = sign(row n of bits_p)[k] s_p[k] (rows n < r0 from path 0, the
+// rest from path 1), stored unscaled as fp16 [M x (r0 + r1)]; with aux (fp16
+// [M x N]) also part[m / 32][n] = sum over the 32-row block of C * aux.
+struct Bwd1Args {
+    int M, K, r0, r1;
+    const uint16_t *a;
+    int64_t lda;
+    const uint32_t *bits0, *bits1;  // packed rows along K (bits1 null: one path)
+    int64_t ld0, ld1;
+    const uint16_t *s0, *s1;  // per-K scale of each path's rows (fp16, length K)
+    uint16_t *out;
+    int64_t ldo;
+    const uint16_t *aux;
+    int64_t ldaux;
+    float *part;
+};
+cudaError_t bwd_contraction1(const Bwd1Args &b, const DeviceInfo &dev, cudaStream_t stream);
+// Contraction-2 shape: C_p[m, n] = sum over path p's columns k of
+// A[m, k] sign(row n of bits_p)[k] l_p[k], A fp16 [M x (r0 + r1)] (the paths
+// side by side); part_p[m / 32][n] = sum over the 32-row block of C_p * aux
+// (aux bf16 [M x N]); with out, also out[m, n] = sum_p t_p[n] C_p[m, n] (bf16).
+struct Bwd2Args {
+    int M, N, r0, r1;
+    const uint16_t *a;
+    int64_t lda;
+    const uint32_t *bits0, *bits1;  // packed rows n along the path's latent
+    int64_t ld0, ld1;
+    const uint16_t *l0, *l1;  // latent scale of each path
+    const uint16_t *aux;
+    int64_t ldaux;
+    float *part0, *part1;
+    uint16_t *out;  // may be null
+    int64_t ldo;
+    const uint16_t *t0, *t1;
+};
+cudaError_t bwd_contraction2(const Bwd2Args &b, const DeviceInfo &dev, cudaStream_t stream);
+
+// The whole backward pass (lb_linear_backward), already validated.
+struct BackwardArgs {
+    const uint16_t *x;
+    int64_t ldx;
+    const uint16_t *dy;
+    int64_t lddy;
+    int tokens, n_in, n_out, npaths;
+    PathDesc path[2];
+    uint16_t *dx;  // may be null
+    int64_t lddx;
+    float *dh, *dg, *dl;
+    void *workspace;
+    size_t workspace_bytes;
+};
+size_t backward_workspace_bytes(int tokens, int n_in, int n_out, const int *ranks, int npaths);
+cudaError_t backward_launch(const BackwardArgs &b, const DeviceInfo &dev, cudaStream_t stream);
+
 // Either contraction alone, the latent in caller memory: z fp16 [tokens][ldz]
 // (token-major, the paths side by side, path 0 first); any number of tokens
 // (up to 32 on the lb_mid.cu kernels, more on the prefill kernels).

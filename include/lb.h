@@ -282,6 +282,56 @@ LB_API lb_status lb_linear_forward_siblings(const uint16_t *x, int64_t tokens, i
                                      int nproj, const lb_projection *proj, void *workspace,
                                      size_t workspace_bytes, void *stream);
 
+/* ---------------------------------------------------------- backward pass
+ * lb_linear_backward: the gradients of a loss L with respect to the layer's
+ * input and to every path's scale vectors, given dy = dL/dy.  The pages train
+ * the layer by quantization-aware training through the factored pass
+ * (littlebitllm.com, "Pipeline"; trove.briskstack.com, "How it works"), whose
+ * steps are those of Proposition 1 (sesamedisk.com, "Samsung LittleBit 13B
+ * Model", "What the method actually computes").  With the signs held fixed,
+ * the chain rule through those steps gives, per path p and summed over tokens
+ * m where marked:
+ *     a_p  = sign(U_p)^T (h_p (.) dy)                (d L / d z_p)
+ *     dl_p = sum_m a_p (.) c_p,    c_p = sign(V_p)^T (g_p (.) x)
+ *     dt_p = sign(V_p) (l_p (.) a_p)                  (d L / d (g_p (.) x))
+ *     dg_p = sum_m x (.) dt_p,     dx = sum_p g_p (.) dt_p
+ *     dh_p = sum_m dy (.) e_p,     e_p = sign(U_p) (l_p (.) c_p)
+ * The gradient through sign() to the real-valued factors needs the smooth
+ * surrogate the pages name (SmoothSign) but do not define; it is not computed.
+ *   x       : device bf16 [tokens x n_in], row stride ldx (the forward input)
+ *   dy      : device bf16 [tokens x n_out], row stride lddy
+ *   main, residual : the paths exactly as for lb_linear_forward (the same
+ *             packed words; the call transposes them into the workspace)
+ *   dx      : device bf16 [tokens x n_in], row stride lddx, or NULL for none;
+ *             written, never read
+ *   dh      : device fp32 [paths x n_out]: path 0's n_out values, then path 1's
+ *   dg      : device fp32 [paths x n_in], the same order
+ *   dl      : device fp32 [r_main + r_residual]: path 0's latents first
+ *   workspace : at least lb_backward_workspace_bytes(...) bytes, 16-byte
+ *             aligned, contents on entry irrelevant; calls sharing it must be
+ *             ordered on one stream
+ * Numerics: four tensor-core contractions with fp32 accumulation: the two
+ *   over n_in and n_out in bf16 x bf16 (x and dy as given, g and h rounded
+ *   to bf16), the two over the latent in fp16 x fp16 (c_p and a_p rounded to
+ *   fp16, unscaled, so they must stay below 65504 in magnitude, else
+ *   LB_ERR_RANGE on the device status word and the results are undefined;
+ *   l exact).  Sums over tokens run in a fixed order (32-token blocks, then
+ *   the blocks in order): results are deterministic.  dx is rounded to bf16
+ *   once; dh, dg and dl are fp32.
+ * Shapes, alignment and strides as lb_linear_forward (dx like x; dh, dg, dl
+ *   4-byte aligned).  tokens == 0 sets dh, dg and dl to zero and nothing else
+ *   (x, dy and dx are then not read and may be NULL).
+ * Errors: LB_ERR_INVALID_ARGUMENT (null pointers other than dx, negative
+ *   sizes, short strides), LB_ERR_UNSUPPORTED_SHAPE, LB_ERR_MISALIGNED,
+ *   LB_ERR_WORKSPACE_TOO_SMALL, LB_ERR_NOT_SUPPORTED_DEVICE, LB_ERR_CUDA; on
+ *   an error found on the host nothing is launched and nothing is written. */
+LB_API size_t lb_backward_workspace_bytes(int64_t tokens, int64_t n_in, int64_t n_out, int64_t rank_main,
+                                          int64_t rank_residual);
+LB_API lb_status lb_linear_backward(const uint16_t *x, const uint16_t *dy, int64_t tokens, int64_t n_in,
+                                    int64_t n_out, int64_t ldx, int64_t lddy, const lb_path *main,
+                                    const lb_path *residual, uint16_t *dx, int64_t lddx, float *dh, float *dg,
+                                    float *dl, void *workspace, size_t workspace_bytes, void *stream);
+
 /* ---------------------------------------------------------- fixed scratch
  * lb_linear_forward_fixed_scratch: lb_linear_forward for 1..32 tokens with
  * no workspace argument.  The pages have no counterpart; this is a service of

@@ -312,3 +312,24 @@ def test_binding_rejects_wrong_dtype_or_layout_before_any_call(L):
                                torch.zeros((2, 64), dtype=torch.bfloat16), xh, xh, torch.zeros(16, dtype=torch.uint8))
     with pytest.raises(ValueError, match="int32"):
         lb.PackedPath(fake.u_bits.float(), fake.vt_bits, fake.h, fake.g, fake.l, 32).as_c()
+
+
+def test_backward_workspace_and_host_refusals(L):
+    """lb_backward_workspace_bytes answers on the host; lb_linear_backward
+    refuses bad arguments before it touches CUDA (no device here)."""
+    import ctypes
+    R, M, n_in, n_out = 2 * 1088, 8192, 5120, 17408
+    need = lb.backward_workspace_bytes(M, n_in, n_out, 1088, 1088)
+    # transposed signs, c and a in fp16, and fp32 partials per 32-token block
+    assert need >= 2 * 1088 * (n_in + n_out) // 8 + 2 * M * R * 2 + (M // 32) * (R + 2 * n_out + 2 * n_in) * 4
+    assert lb.backward_workspace_bytes(0, n_in, n_out, 1088, 1088) == 0
+    assert lb.backward_workspace_bytes(M, 100, n_out, 1088, 0) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    p = lb.LbPath(1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 32, 0, 0)
+    args = lambda **k: [k.get("x", fake), fake, 8, k.get("n_in", 64), 64, k.get("ldx", 64), 64, ctypes.byref(p), None,
+                        fake, 64, k.get("dh", fake), fake, fake, fake, 1 << 30, None]
+    assert L.lb_linear_backward(*args(x=None)) == lb.LB_ERR_INVALID_ARGUMENT
+    assert L.lb_linear_backward(*args(dh=None)) == lb.LB_ERR_INVALID_ARGUMENT
+    assert L.lb_linear_backward(*args(n_in=48, ldx=48)) == lb.LB_ERR_UNSUPPORTED_SHAPE
+    assert L.lb_linear_backward(*args(ldx=60)) == lb.LB_ERR_INVALID_ARGUMENT
+    assert L.lb_linear_backward(*args(x=ctypes.c_void_p((1 << 20) + 2))) == lb.LB_ERR_MISALIGNED

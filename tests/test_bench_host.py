@@ -102,13 +102,14 @@ def test_kernel_labels_follow_the_dispatch():
 
 def test_tensor_peak_follows_the_sampled_clocks():
     """The sustained (power-capped) cuBLAS figure is the denominator only when
-    the timed region itself ran capped; otherwise the burst figure is."""
+    the timed region itself ran with its clock held down; otherwise the burst
+    figure is, even if a power-cap reason appeared in some sample."""
     peaks = dict(hbm=6542.4, bf16=1651.4, bf16_sustained=1401.9, source="measured")
     at_max = {"sm_mhz": 1965.0, "sm_max_mhz": 1965, "reasons": [], "samples": 12}
     assert bench.tensor_peak(peaks, at_max) == (1651.4, "measured (burst)")
-    capped = dict(at_max, reasons=["sw_power_cap"])
-    assert bench.tensor_peak(peaks, capped) == (1401.9, "measured (sustained)")
-    slow = dict(at_max, sm_mhz=1365.0)
+    capped_at_max = dict(at_max, reasons=["sw_power_cap"])
+    assert bench.tensor_peak(peaks, capped_at_max) == (1651.4, "measured (burst)")
+    slow = dict(at_max, sm_mhz=1492.0, reasons=["sw_power_cap"])
     assert bench.tensor_peak(peaks, slow) == (1401.9, "measured (sustained)")
     assert bench.tensor_peak(peaks, {"error": "nvml unavailable"}) == (1651.4, "measured (burst)")
 
