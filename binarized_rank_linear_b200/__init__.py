@@ -119,6 +119,8 @@ def lib() -> ctypes.CDLL:
                                              ctypes.POINTER(LbPath), vp, i64, vp, vp, vp, vp, sz, vp]
             L.lb_device_status.restype = i32
             L.lb_device_status.argtypes = [vp, ctypes.POINTER(i32)]
+            L.lb_debug_inject_stall.restype = i32
+            L.lb_debug_inject_stall.argtypes = [i32, ctypes.c_uint64]
             L.lb_set_prefill_pairs.restype = i32
             L.lb_set_prefill_pairs.argtypes = [i32]
             _lib = L
@@ -471,6 +473,15 @@ def device_status(stream=None) -> int:
     out = ctypes.c_int(0)
     _check(lib().lb_device_status(_stream_handle(stream), ctypes.byref(out)), "lb_device_status")
     return int(out.value)
+
+
+def debug_inject_stall(enable: bool, wait_limit_ns: int = 2_000_000_000) -> None:
+    """``lb_debug_inject_stall`` (tests only): make the tcgen05 decode kernels
+    enqueued afterwards give up their bounded waits after ``wait_limit_ns``
+    and skip one stage-barrier arrival, so that they time out and record
+    LB_ERR_DEVICE_TIMEOUT; ``enable=False`` restores the defaults."""
+    _check(lib().lb_debug_inject_stall(1 if enable else 0, int(wait_limit_ns) if enable else 0),
+           "lb_debug_inject_stall")
 
 
 def set_prefill_pairs(enable: bool) -> None:

@@ -138,6 +138,15 @@ size_t workspace_for(int64_t tokens, int64_t n_in, int64_t n_out, const int *ran
 
 bool lb::prefill_pairs_enabled() { return g_prefill_pairs.load(std::memory_order_relaxed) != 0; }
 
+namespace {
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+std::atomic<unsigned long long> g_debug_wait_ns{kDefaultWaitNs};  // lb_debug_inject_stall
+std::atomic<int> g_debug_skip{0};
+}  // namespace
+
+unsigned long long lb::debug_wait_ns() { return g_debug_wait_ns.load(std::memory_order_relaxed); }
+int lb::debug_skip_arrival() { return g_debug_skip.load(std::memory_order_relaxed); }
+
 extern "C" {
 
 const char *lb_status_string(lb_status s)
@@ -580,6 +589,15 @@ lb_status lb_device_status(void *stream, lb_status *out)
         }
     }
     *out = static_cast<lb_status>(v);
+    return LB_OK;
+}
+
+lb_status lb_debug_inject_stall(int enable, uint64_t wait_limit_ns)
+{
+    if (enable != 0 && enable != 1) return LB_ERR_INVALID_ARGUMENT;
+    if (enable && (wait_limit_ns < 1000ull || wait_limit_ns > kDefaultWaitNs)) return LB_ERR_INVALID_ARGUMENT;
+    g_debug_wait_ns.store(enable ? wait_limit_ns : kDefaultWaitNs, std::memory_order_relaxed);
+    g_debug_skip.store(enable, std::memory_order_relaxed);
     return LB_OK;
 }
 

@@ -97,6 +97,12 @@ cudaError_t decode_prepare_device(const DeviceInfo &dev);
 size_t group_workspace_bytes(const GroupArgs &g);
 cudaError_t group_forward(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t stream);
 
+// Fault injection for tests (lb_debug_inject_stall): the limit of the
+// tcgen05 decode kernels' bounded waits (ns) and whether their first
+// producer warp skips one arrival.  Read when a launch is prepared.
+unsigned long long debug_wait_ns();
+int debug_skip_arrival();
+
 // Up to kMidMaxTokens tokens per launch pair on tcgen05 with the sign matrix
 // as the 128-row MMA operand and the tokens as N (lb_mid.cu).
 constexpr int kMidMaxTokens = 128;

@@ -93,6 +93,12 @@ struct MidParams {
 template <int NQ>  // layer slots: 1 for one layer, kMaxSiblings for a group
 struct MidGroup {
     int nlayers;
+    // Bounded waits give up after wait_ns.  skip_arrival (a fault-injection
+    // hook for tests, lb_debug_inject_stall): the first producer warp of CTA 0
+    // does not arrive on its first K-block's stage barrier, so the MMA
+    // thread's wait on it runs out and the CTA winds down.
+    unsigned long long wait_ns;
+    int skip_arrival;
     MidParams layer[NQ];  // in row (mode 1) or tile (mode 2) order
 };
 
@@ -216,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int j = 0; j < nkb; ++j) {
                 const int s = j % STAGES;
                 const uint32_t ph = (uint32_t)(j / STAGES) & 1u;
-                if (!mbar_wait(empty0 + 8 * s, ph ^ 1u) || abort_flag) {
+                if (!mbar_wait(empty0 + 8 * s, ph ^ 1u, g.wait_ns) || abort_flag) {
                     abort_flag = 1;
                     break;
                 }
@@ -226,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             if (abort_flag) {
                 for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
-                    mbar_wait(full0 + 8 * (j % STAGES), (uint32_t)(j / STAGES) & 1u);
+                    mbar_wait(full0 + 8 * (j % STAGES), (uint32_t)(j / STAGES) & 1u, g.wait_ns);
             }
         }
     } else if (warp == 1) {
@@ -236,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int j = 0; j < nkb; ++j) {
                 const int s = j % STAGES;
                 const uint32_t ph = (uint32_t)(j / STAGES) & 1u;
-                if (!mbar_wait(full0 + 8 * s, ph) || abort_flag) {
+                if (!mbar_wait(full0 + 8 * s, ph, g.wait_ns) || abort_flag) {
                     abort_flag = 1;
                     break;
                 }
@@ -250,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             umma_commit(accf);
             // every MMA issued has finished before the CTA frees tensor memory
             umma_commit(drain);
-            if (!mbar_wait(drain, 0)) abort_flag = 1;
+            if (!mbar_wait(drain, 0, g.wait_ns)) abort_flag = 1;
         }
     } else {
         // ---------------- producers: group grp expands blocks j = grp, grp + 2, ...
@@ -325,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int kb = kb0 + j;
             const int s = j % STAGES;
             const uint32_t ph = (uint32_t)(j / STAGES) & 1u;
-            bool ok = mbar_wait(empty0 + 8 * s, ph ^ 1u) && !abort_flag;
+            bool ok = mbar_wait(empty0 + 8 * s, ph ^ 1u, g.wait_ns) && !abort_flag;
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) {
                 abort_flag = 1;
@@ -375,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                                  sc[q]);
             fence_async_shared();
             __syncwarp();
-            if (lane == 0) mbar_arrive(full0 + 8 * s);
+            if (lane == 0 && !(g.skip_arrival && blockIdx.x == 0 && pw == 0 && j == 0)) mbar_arrive(full0 + 8 * s);
             // refill the slots (used above; every lane is past its reads after
             // the __syncwarp) with the group's block two ahead
             copy_block(j + 4, slot);
@@ -383,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         cp_async_wait_all();  // no copy may land after the CTA is gone
         // warps 2..5: this thread's row 32 (warp % 4) + lane of the accumulator
         if (pw < 4) {
-            bool ok = !abort_flag && mbar_wait(accf, 0);
+            bool ok = !abort_flag && mbar_wait(accf, 0, g.wait_ns);
             ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
             if (!ok) abort_flag = 1;
             tc_fence_after();
@@ -495,6 +501,8 @@ cudaError_t launch_mid(const GroupArgs &g, const DeviceInfo &dev, cudaStream_t s
 {
     MidGroup<NQ> G{};
     G.nlayers = g.nproj;
+    G.wait_ns = debug_wait_ns();
+    G.skip_arrival = debug_skip_arrival();
     int tiles = 0, nk = 0, koff = 0;
     if (MODE == 1) {
         int R = 0;

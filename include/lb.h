@@ -384,6 +384,20 @@ LB_API lb_status lb_device_status(void *stream, lb_status *out);
  * LB_ERR_INVALID_ARGUMENT unless `enable` is 0 or 1. */
 LB_API lb_status lb_set_prefill_pairs(int enable);
 
+/* Fault injection, for tests of the library's own failure handling; not
+ * for production use.  No counterpart on the pages.
+ * With enable = 1, every tcgen05 decode kernel (5..128 tokens) enqueued
+ * afterwards gives up its bounded waits after wait_limit_ns (1 us .. 2 s)
+ * instead of 2 s, and in each of them one producer warp of the first CTA
+ * skips its arrival on its first stage barrier.  The MMA thread's wait on
+ * that barrier then runs out: the kernel records LB_ERR_DEVICE_TIMEOUT on the
+ * device status word, lets its copies and MMAs finish, frees its tensor
+ * memory and returns (no trap, no hang); the outputs of such a call are
+ * undefined.  enable = 0 restores the defaults for later calls.  The setting
+ * is process-wide.  Errors: LB_ERR_INVALID_ARGUMENT for enable outside
+ * {0, 1} or a limit outside the range. */
+LB_API lb_status lb_debug_inject_stall(int enable, uint64_t wait_limit_ns);
+
 #ifdef __cplusplus
 }
 #endif

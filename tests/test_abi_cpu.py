@@ -333,3 +333,11 @@ def test_backward_workspace_and_host_refusals(L):
     assert L.lb_linear_backward(*args(n_in=48, ldx=48)) == lb.LB_ERR_UNSUPPORTED_SHAPE
     assert L.lb_linear_backward(*args(ldx=60)) == lb.LB_ERR_INVALID_ARGUMENT
     assert L.lb_linear_backward(*args(x=ctypes.c_void_p((1 << 20) + 2))) == lb.LB_ERR_MISALIGNED
+
+
+def test_fault_hook_arguments(L):
+    assert L.lb_debug_inject_stall(2, 1000000) == lb.LB_ERR_INVALID_ARGUMENT
+    assert L.lb_debug_inject_stall(1, 999) == lb.LB_ERR_INVALID_ARGUMENT
+    assert L.lb_debug_inject_stall(1, 3_000_000_000) == lb.LB_ERR_INVALID_ARGUMENT
+    assert L.lb_debug_inject_stall(1, 1_000_000) == lb.LB_OK
+    assert L.lb_debug_inject_stall(0, 0) == lb.LB_OK
