@@ -101,6 +101,10 @@ TILE_PLAN_CASES = [
     pytest.param(5000, 1056, 288, [480, 512], id="m5000-c1-pair-h2-ragged-k"),
     pytest.param(520, 288, 8192, [480, 512], id="m520-c2-pair-h2-ragged-k-mid-block-paths"),
     pytest.param(3000, 1056, 2048, [480, 512], id="m3000-pair-both-ragged-k"),
+    # few tiles of a long K in contraction 1 (the Qwen3-14B k/v shape at fewer tokens)
+    pytest.param(2048, 5120, 1024, [224, 224], id="m2048-c1-few-tiles-long-k"),
+    pytest.param(1000, 4096, 512, [128, 96], id="m1000-c1-long-k-ragged-m"),
+    pytest.param(700, 2048, 256, [32, 32], id="m700-c1-narrow-long-k"),
 ]
 
 
@@ -162,8 +166,8 @@ def test_integer_exact_is_bitwise(tokens):
 
 @pytest.mark.parametrize("n_in,n_out,ranks,tokens", [(256, 8192, [512, 512], 520), (256, 256, [512, 512], 2600),
                                                      (512, 224, [64, 32], 300), (512, 224, [64, 32], 1000),
-                                                     (288, 8192, [480, 512], 520)],
-                         ids=["c2-h2", "c1-wide", "m300", "m1000", "ragged-k"])
+                                                     (288, 8192, [480, 512], 520), (4096, 256, [128, 96], 1000)],
+                         ids=["c2-h2", "c1-wide", "m300", "m1000", "ragged-k", "c1-long-k"])
 def test_integer_exact_prefill_tiles_are_bitwise(n_in, n_out, ranks, tokens, prefill_pairs):
     """The integer-exact case on prefill shapes, on CTA pairs and on single
     CTAs.  Every value is an integer well inside fp32's exact range and z
@@ -177,7 +181,7 @@ def test_integer_exact_prefill_tiles_are_bitwise(n_in, n_out, ranks, tokens, pre
 
 
 @pytest.mark.parametrize("tokens,n_in,n_out,ranks", [(700, 256, 4096, [32, 32]), (2100, 256, 4096, [160, 160]),
-                                                     (520, 256, 8192, [512, 512])])
+                                                     (520, 256, 8192, [512, 512]), (2048, 5120, 1024, [224, 224])])
 def test_pair_and_single_cta_tiles_agree_bitwise(tokens, n_in, n_out, ranks):
     """Every output element sums the same K-steps in the same order whether
     its row sits in a single-CTA tile or in a CTA pair's, and the epilogue
@@ -441,3 +445,18 @@ def test_chained_host_calls_read_the_previous_output(tokens):
     for d in range(depth):
         assert np.array_equal(gu.bf16_bits(hosts[d + 1]), gu.bf16_bits(refs[d])), f"layer {d}"
     gu.assert_close(gu.bf16_to_f64(hosts[1]), gu.oracle_y(layer), f"first layer M={tokens}")
+
+
+def test_few_tiles_long_k_is_deterministic_and_sign_flip_invariant():
+    """The Qwen3-14B k/v shape at 2048 tokens (few output tiles, a long K):
+    repeated calls give the same bits, and so does a joint sign flip of latent
+    pairs."""
+    layer = synth.make_layer(5120, 1024, [224, 224], 2048, config_id=1600)
+    paths = gu.device_paths(layer)
+    y0 = gu.bf16_bits(gu.run_gpu(layer, paths=paths))
+    for _ in range(3):
+        assert np.array_equal(gu.bf16_bits(gu.run_gpu(layer, paths=paths)), y0)
+    flip = lambda a: (a * np.where(np.arange(a.shape[1]) % 2 == 0, -1, 1)).astype(np.int8)
+    flipped = dict(layer, paths=[dict(p, su=flip(p["su"]), sv=flip(p["sv"])) for p in layer["paths"]])
+    assert np.array_equal(gu.bf16_bits(gu.run_gpu(flipped)), y0)
+    gu.assert_close(oracle.bf16_bits_to_f64(y0), gu.oracle_y(layer), "k/v shape, 2048 tokens")
