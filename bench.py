@@ -817,9 +817,12 @@ def run_lb(args, world, rank, local):
     del flush
 
     # end to end through the C ABI with host buffers (lb_linear_forward_host):
-    # the same steps (passes over the weight copies), every call copying its x
-    # in from pinned host memory and its y back to pinned host memory inside
-    # the one call, issued eagerly from Python
+    # the same steps (passes over the weight copies), every call bringing its
+    # x in from pinned host memory and its y back to pinned host memory
+    # inside the one call.  Two ways to issue them: the calls captured once
+    # into a CUDA graph per step (as a serving loop issues its decode steps;
+    # each replay moves every call's x and y across the host link again), and
+    # eagerly from Python, one ctypes call at a time
     x_host = torch.empty_like(d.x, device="cpu").pin_memory()
     x_host.copy_(d.x.cpu())
     y_host = torch.empty((tokens, d.n_out), dtype=torch.bfloat16).pin_memory()
@@ -831,6 +834,17 @@ def run_lb(args, world, rank, local):
     for i in range(nsets):
         call_host(i)
     torch.cuda.synchronize()
+    hg = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(hg, stream=torch.cuda.Stream(device), capture_error_mode="relaxed"):
+        for i in range(nsets):
+            call_host(i)
+    for _ in range(args.warmup):
+        hg.replay()
+    torch.cuda.synchronize()
+    y_host.fill_(0)
+    e2e_ms, _ = time_graph(hg, args.steps, stream, local, world, device)
+    e2e_ok = bool(torch.equal(y_host.to(device), d.y)) if tokens <= 128 else None  # the last call's y arrived
+    del hg
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -839,7 +853,7 @@ def run_lb(args, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    eager_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
     e2e_value = aggregate(units * calls, e2e_ms / 1e3, world)
     d.sets = [d.base]
     torch.cuda.empty_cache()
@@ -848,17 +862,21 @@ def run_lb(args, world, rank, local):
     # whole decoder block of fused sibling calls at batch 1, and the dense
     # baseline of the pages' kernel comparison
     prefill = block = dense = backward = None
-    if not args.no_extras:
+    extras = set() if args.no_extras else set(args.extras.split(","))
+    if "prefill" in extras:
         prefill = {}
         for name in args.prefill.split(",") if args.prefill else []:
             prefill[name] = measure_prefill(name, args, world, local, device, peaks)
             torch.cuda.empty_cache()
+    if "backward" in extras:
         backward = {}
         for name in args.backward.split(",") if args.backward else []:
             backward[name] = measure_backward(name, args, world, local, device, peaks)
             torch.cuda.empty_cache()
+    if "block" in extras:
         block = measure_block("llama2_7b", 1, True, args.steps, args.warmup, world, local, device, seconds=0.1)
         torch.cuda.empty_cache()
+    if "dense" in extras:
         dense = dense_comparison("llama2_70b_gate", args, world, local, device)
         torch.cuda.empty_cache()
     if args.dense_baseline and dense is None:
@@ -904,9 +922,14 @@ def run_lb(args, world, rank, local):
            "e2e": {"value": e2e_value, "unit": "GB/s" if decode else "TFLOP/s",
                    "h2d_bytes_per_step": 2 * tokens * d.n_in * nsets, "d2h_bytes_per_step": 2 * tokens * d.n_out * nsets,
                    "us_per_call": e2e_ms * 1e3 / calls, "calls": calls,
-                   "call": "lb_linear_forward_host from Python (pinned host x and y; " + (
+                   "call": "lb_linear_forward_host (pinned host x and y; " + (
                        "x gathered by a kernel in one pass, y written in place by the last kernel)" if tokens <= 128 else
-                       "copied through device buffers inside the call)")},
+                       "copied through device buffers inside the call)") +
+                   ", %d calls per step captured in a CUDA graph" % nsets,
+                   "y_host_matches_device_call": e2e_ok,
+                   "eager": {"value": aggregate(units * calls, eager_ms / 1e3, world),
+                             "us_per_call": eager_ms * 1e3 / calls,
+                             "call": "the same calls issued one at a time from Python"}},
            "gpu_launches": 2 * calls,  # contraction 1 + contraction 2 per call, decode and prefill
            "impl": "lb"}
     if prefill:
@@ -936,8 +959,9 @@ def main(argv=None):
     ap.add_argument("--prefill-seconds", type=float, default=0.3)
     ap.add_argument("--backward", default="qwen3_14b_gate",
                     help="workloads whose backward pass is measured beside the main line (comma-separated)")
-    ap.add_argument("--no-extras", action="store_true",
-                    help="skip the prefill, fused-block and dense-baseline measurements")
+    ap.add_argument("--extras", default="prefill,backward,block,dense",
+                    help="measurements beside the main line: any of prefill, backward, block, dense")
+    ap.add_argument("--no-extras", action="store_true", help="none of the --extras")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-parity", action="store_true")
     ap.add_argument("--block", choices=sorted(BLOCKS), default=None,
