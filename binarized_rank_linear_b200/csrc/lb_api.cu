@@ -63,7 +63,8 @@ lb_status device_info(lb::DeviceInfo *out)
         cudaGetLastError();
         return LB_ERR_CUDA;
     }
-    if (lb::decode_prepare_device(info) != cudaSuccess || lb::prefill_prepare_device(info) != cudaSuccess) {
+    if (lb::decode_prepare_device(info) != cudaSuccess || lb::prefill_prepare_device(info) != cudaSuccess ||
+        lb::wgrad_prepare_device(info) != cudaSuccess) {
         cudaGetLastError();
         return LB_ERR_CUDA;
     }

@@ -17,10 +17,10 @@
 //   K2  a = S_U^T (h (.) dy)         dy [M x n_out] against the rows of U^T;
 //                                    the epilogue also forms a (.) c per
 //                                    32-token block (dl partials)
-//   K3  e_p = S_U,p (l_p (.) c_p)    c against the rows of U, l on the K side,
-//                                    one accumulator per path; the epilogue
-//                                    forms dy (.) e_p per block (dh partials)
-//                                    and stores nothing
+//   K3  dh_p = sum_k S_U,p l_p G     G = dy^T c, the tokens as the MMA's
+//                                    K (lb_wgrad.cu); the epilogue applies
+//                                    each row's signs and l and sums over k
+//                                    (dh partials per tile column)
 //   K4  dt_p = S_V,p (l_p (.) a_p)   a against the rows of V; the epilogue
 //                                    stores dx = sum_p g_p (.) dt_p (bf16) and
 //                                    forms x (.) dt_p per block (dg partials)
@@ -29,7 +29,8 @@
 // other axis from the forward pass: U^T packed along n_out and V packed along
 // r, which two bit-transpose launches make from the forward's packed words
 // into the workspace, so the call takes the forward pass's lb_path as it is.
-// c and a travel between the contractions as fp16, unscaled.
+// c (bf16, the type of dy, as K3 needs) and a (fp16) travel between the
+// contractions unscaled.
 #include <algorithm>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -91,7 +92,7 @@ cudaError_t transpose_bits(const uint32_t *in, int64_t ld_in, int rows, int cols
 }
 
 // ------------------------------------------------------------ partial sums
-// out[n] = sum over the 32-token blocks rb = 0 .. blocks - 1 of part[rb][n],
+// out[n] = sum over the rows rb = 0 .. blocks - 1 of part[rb][n],
 // for up to kMaxSegments vectors in one launch.  A CTA takes 32 columns; its
 // kGroups warps take the blocks rb = g, g + kGroups, ... of those columns
 // (each in block order), and warp 0 adds the kGroups sums in group order:
@@ -102,11 +103,11 @@ struct ReduceSeg {
     const float *part;
     float *out;
     int n;
+    int blocks;  // rows of partials: 32-token blocks, or K3's tile columns and token parts
 };
 struct ReduceParams {
     ReduceSeg seg[kMaxSegments];
     int nseg;
-    int blocks;  // 32-token blocks
 };
 
 __global__ void __launch_bounds__(32 * kGroups) reduce_partials_kernel(const __grid_constant__ ReduceParams p)
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(32 * kGroups) reduce_partials_kernel(const __g
     }
     float acc = 0.0f;
     if (seg != nullptr)
-        for (int rb = g; rb < p.blocks; rb += kGroups) acc += __ldg(seg->part + (int64_t)rb * seg->n + col);
+        for (int rb = g; rb < seg->blocks; rb += kGroups) acc += __ldg(seg->part + (int64_t)rb * seg->n + col);
     sums[g][lane] = acc;
     __syncthreads();
     if (g == 0 && seg != nullptr) {
@@ -163,9 +164,11 @@ BwdLayout layout(int M, int n_in, int n_out, const int *ranks, int npaths)
     off += align256((size_t)M * R * 2);
     L.pl = off;
     off += align256(RB * R * 4);
+    // K3's partial rows: at most wgrad_max_parts (at least the 32-token blocks)
+    const size_t HB = std::max(RB, (size_t)wgrad_max_parts(R, M));
     for (int q = 0; q < npaths; ++q) {
         L.ph[q] = off;
-        off += align256(RB * (size_t)n_out * 4);
+        off += align256(HB * (size_t)n_out * 4);
         L.pg[q] = off;
         off += align256(RB * (size_t)n_in * 4);
     }
@@ -224,6 +227,7 @@ cudaError_t backward_launch(const BackwardArgs &b, const DeviceInfo &dev, cudaSt
     }
     k1.out = c;
     k1.ldo = R;
+    k1.out_bf16 = 1;
     e = bwd_contraction1(k1, dev, stream);
     if (e != cudaSuccess) return e;
 
@@ -247,32 +251,34 @@ cudaError_t backward_launch(const BackwardArgs &b, const DeviceInfo &dev, cudaSt
     k2.ldo = R;
     k2.aux = c;
     k2.ldaux = R;
+    k2.aux_bf16 = 1;
     k2.part = pl;
     e = bwd_contraction1(k2, dev, stream);
     if (e != cudaSuccess) return e;
 
-    // K3: e_p = S_U,p (l_p (.) c_p); dh partials sum dy (.) e_p
-    Bwd2Args k3{};
-    k3.M = M;
-    k3.N = b.n_out;
+    // K3: dh_p[o] = sum_k sign(U_p[o, k]) l_p[k] G[o, k], G = dy^T c
+    WgradArgs k3{};
+    k3.tokens = M;
+    k3.n_out = b.n_out;
+    k3.R = R;
     k3.r0 = r0;
-    k3.r1 = r1;
-    k3.a = c;
-    k3.lda = R;
-    k3.bits0 = P0.u_bits;
-    k3.ld0 = P0.u_ld;
+    k3.dy = b.dy;
+    k3.lddy = b.lddy;
+    k3.c = c;
+    k3.ldc = R;
+    k3.u0 = P0.u_bits;
+    k3.uld0 = P0.u_ld;
     k3.l0 = P0.l;
     if (two) {
-        k3.bits1 = P1.u_bits;
-        k3.ld1 = P1.u_ld;
+        k3.u1 = P1.u_bits;
+        k3.uld1 = P1.u_ld;
         k3.l1 = P1.l;
     }
-    k3.aux = b.dy;
-    k3.ldaux = b.lddy;
     k3.part0 = ph[0];
     k3.part1 = ph[1];
-    e = bwd_contraction2(k3, dev, stream);
+    e = wgrad_dh(k3, dev, stream);
     if (e != cudaSuccess) return e;
+    const int hrows = wgrad_plan(b.n_out, R, M, dev.sm_count).rows;
 
     // K4: dt_p = S_V,p (l_p (.) a_p); dx = sum_p g_p (.) dt_p; dg partials sum x (.) dt_p
     Bwd2Args k4{};
@@ -301,19 +307,19 @@ cudaError_t backward_launch(const BackwardArgs &b, const DeviceInfo &dev, cudaSt
     e = bwd_contraction2(k4, dev, stream);
     if (e != cudaSuccess) return e;
 
-    // the partial sums, added over the 32-token blocks in block order
+    // the partial sums, each added over its rows in row order
     ReduceParams rp{};
-    rp.blocks = (M + 31) / 32;
+    const int tb = (M + 31) / 32;
     int total = 0;
-    auto add = [&](const float *part, float *out, int n) {
-        rp.seg[rp.nseg++] = ReduceSeg{part, out, n};
+    auto add = [&](const float *part, float *out, int n, int blocks) {
+        rp.seg[rp.nseg++] = ReduceSeg{part, out, n, blocks};
         total += n;
     };
-    add(pl, b.dl, R);
-    add(ph[0], b.dh, b.n_out);
-    if (two) add(ph[1], b.dh + b.n_out, b.n_out);
-    add(pg[0], b.dg, b.n_in);
-    if (two) add(pg[1], b.dg + b.n_in, b.n_in);
+    add(pl, b.dl, R, tb);
+    add(ph[0], b.dh, b.n_out, hrows);
+    if (two) add(ph[1], b.dh + b.n_out, b.n_out, hrows);
+    add(pg[0], b.dg, b.n_in, tb);
+    if (two) add(pg[1], b.dg + b.n_in, b.n_in, tb);
     // every segment's length is a multiple of 32, so a CTA's 32 columns lie in one segment
     reduce_partials_kernel<<<(unsigned)(total / 32), 32 * kGroups, 0, stream>>>(rp);
     return cudaGetLastError();

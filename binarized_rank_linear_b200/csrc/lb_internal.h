@@ -138,8 +138,9 @@ cudaError_t prefill_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStre
 // The backward pass's two contraction shapes on the prefill kernels.
 // Contraction-1 shape: C[m, n] = sum_k A[m, k] B[n, k] with A bf16 [M x K],
 // B[n, k] = sign(row n of bits_p)[k] s_p[k] (rows n < r0 from path 0, the
-// rest from path 1), stored unscaled as fp16 [M x (r0 + r1)]; with aux (fp16
-// [M x N]) also part[m / 32][n] = sum over the 32-row block of C * aux.
+// rest from path 1), stored unscaled as fp16 (or bf16: out_bf16)
+// [M x (r0 + r1)]; with aux (fp16, or bf16: aux_bf16, [M x N]) also
+// part[m / 32][n] = sum over the 32-row block of C * aux.
 struct Bwd1Args {
     int M, K, r0, r1;
     const uint16_t *a;
@@ -152,6 +153,7 @@ struct Bwd1Args {
     const uint16_t *aux;
     int64_t ldaux;
     float *part;
+    int out_bf16, aux_bf16;
 };
 cudaError_t bwd_contraction1(const Bwd1Args &b, const DeviceInfo &dev, cudaStream_t stream);
 // Contraction-2 shape: C_p[m, n] = sum over path p's columns k of
@@ -173,6 +175,30 @@ struct Bwd2Args {
     const uint16_t *t0, *t1;
 };
 cudaError_t bwd_contraction2(const Bwd2Args &b, const DeviceInfo &dev, cudaStream_t stream);
+
+// The h-gradient as a weight-gradient product (lb_wgrad.cu): for every row o
+// of the paths' U and every path p, sums over k in path p of
+// sign(U_p[o, k]) l_p[k] G[o, k] with G = dy^T c (dy bf16 [tokens x n_out],
+// c bf16 [tokens x R], the paths side by side), one partial per tile column
+// and token part: part_p[row][o], rows = WgradPlan::rows.
+struct WgradPlan {
+    int bn, ntn, nsplit, kps, rows;
+};
+WgradPlan wgrad_plan(int n_out, int R, int tokens, int sms);
+int wgrad_max_parts(int R, int tokens);  // the most partial rows any plan takes
+struct WgradArgs {
+    int tokens, n_out, R, r0;
+    const uint16_t *dy;
+    int64_t lddy;
+    const uint16_t *c;
+    int64_t ldc;
+    const uint32_t *u0, *u1;
+    int64_t uld0, uld1;
+    const uint16_t *l0, *l1;
+    float *part0, *part1;  // part1 null: one path
+};
+cudaError_t wgrad_prepare_device(const DeviceInfo &dev);
+cudaError_t wgrad_dh(const WgradArgs &w, const DeviceInfo &dev, cudaStream_t stream);
 
 // The whole backward pass (lb_linear_backward), already validated.
 struct BackwardArgs {

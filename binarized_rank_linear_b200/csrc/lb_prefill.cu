@@ -172,6 +172,7 @@ struct SignGemmParams {
     int64_t ldaux;
     float *part0, *part1;        // column-dot partials [ceil(M / 32) x N] (part1: mode 4, path 1)
     const uint16_t *t0, *t1;     // mode 4: per-column scales of the stored output (fp16, length N)
+    int out_bf16, aux_bf16;      // mode 3: store C as bf16 (else fp16); aux is bf16 (else fp16)
 };
 
 // Persistent: CTA c computes the tiles t = c, c + gridDim.x, ...
@@ -644,6 +645,19 @@ __global__ void __launch_bounds__(Shape<H, P, MODE>::kThreads, 1)
                 break;
             }
             tc_fence_after();
+            // mode 4: the column dot's operand for a chunk is loaded one chunk
+            // ahead, so its latency overlaps the previous chunk's work
+            uint4 axn[4] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
+                            make_uint4(0u, 0u, 0u, 0u)};
+            auto load_aux = [&](int nn) {
+                if (row_in) {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(
+                        static_cast<const uint16_t *>(p.aux) + (int64_t)(m0 + lane) * p.ldaux + nn);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) axn[q] = __ldg(src + q);
+                }
+            };
+            if (MODE == 4) load_aux(n0);
             for (int c32 = 0; c32 < p.bn && n0 + c32 < p.N; c32 += 32) {
                 const int nn = n0 + c32;
                 uint32_t o[16];
@@ -659,14 +673,8 @@ __global__ void __launch_bounds__(Shape<H, P, MODE>::kThreads, 1)
                     const bool two = p.r0 < p.K;
                     const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)((b + eh) * BN + c32);
                     const uint32_t red = sRed + (uint32_t)ew * S::kRedBytes;
-                    uint4 ax[4] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
-                                   make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
-                    if (row_in) {
-                        const uint4 *src = reinterpret_cast<const uint4 *>(
-                            static_cast<const uint16_t *>(p.aux) + (int64_t)(m0 + lane) * p.ldaux + nn);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) ax[q] = __ldg(src + q);
-                    }
+                    const uint4 ax[4] = {axn[0], axn[1], axn[2], axn[3]};
+                    if (c32 + 32 < p.bn && nn + 32 < p.N) load_aux(nn + 32);
                     for (int pth = 0; pth < (two ? 2 : 1); ++pth) {
                         uint32_t v[32];
                         tmem_ld32(tl + 128u * (uint32_t)pth, v);
@@ -752,9 +760,14 @@ __global__ void __launch_bounds__(Shape<H, P, MODE>::kThreads, 1)
                                      : "r"(lsm + 4u * (uint32_t)(c32 + 4 * q4)));
                         const float z0 = __uint_as_float(v[4 * q4]) * lq.x, z1 = __uint_as_float(v[4 * q4 + 1]) * lq.y;
                         const float z2 = __uint_as_float(v[4 * q4 + 2]) * lq.z, z3 = __uint_as_float(v[4 * q4 + 3]) * lq.w;
-                        overflow |= row_in && (beyond_f16(z0) | beyond_f16(z1) | beyond_f16(z2) | beyond_f16(z3));
-                        o[2 * q4] = pack_half2(z0, z1);
-                        o[2 * q4 + 1] = pack_half2(z2, z3);
+                        if (MODE == 3 && p.out_bf16) {
+                            o[2 * q4] = pack_bf162(z0, z1);
+                            o[2 * q4 + 1] = pack_bf162(z2, z3);
+                        } else {
+                            overflow |= row_in && (beyond_f16(z0) | beyond_f16(z1) | beyond_f16(z2) | beyond_f16(z3));
+                            o[2 * q4] = pack_half2(z0, z1);
+                            o[2 * q4 + 1] = pack_half2(z2, z3);
+                        }
                     }
                     if (MODE == 3 && p.aux != nullptr) {
                         // the column dot of the accumulator with aux (fp16)
@@ -770,10 +783,17 @@ __global__ void __launch_bounds__(Shape<H, P, MODE>::kThreads, 1)
                             const uint32_t aw[8] = {ax[0].x, ax[0].y, ax[0].z, ax[0].w,
                                                     ax[1].x, ax[1].y, ax[1].z, ax[1].w};
                             float pr[16];
+                            if (p.aux_bf16) {
 #pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                pr[j] = ((j & 1) ? hi_f16(aw[j >> 1]) : lo_f16(aw[j >> 1])) *
-                                        __uint_as_float(v[16 * hh + j]);
+                                for (int j = 0; j < 16; ++j)
+                                    pr[j] = ((j & 1) ? hi_bf16(aw[j >> 1]) : lo_bf16(aw[j >> 1])) *
+                                            __uint_as_float(v[16 * hh + j]);
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 16; ++j)
+                                    pr[j] = ((j & 1) ? hi_f16(aw[j >> 1]) : lo_f16(aw[j >> 1])) *
+                                            __uint_as_float(v[16 * hh + j]);
+                            }
                             const float r = column_sum16(pr, lane);
                             if (m0 < p.M && lane < 16) p.part0[(int64_t)(m0 >> 5) * p.N + nn + 16 * hh + lane] = r;
                         }
@@ -914,23 +934,27 @@ cudaError_t launch_units(const CUtensorMap &tm, const CUtensorMap &tmo, const Si
 // One contraction on a persistent grid: min(tiles, SMs) CTAs, or
 // min(tiles, resident pairs) CTA pairs.
 // A is x (modes 1 and 3, bf16) or z (modes 2 and 4, fp16), row-major with
-// stride lda.  Mode 4 runs single-CTA 128-row tiles at most 128 wide; mode 4
-// without an output (p.out null) encodes no store map.
+// stride lda.  Mode 4 runs 256-row tiles (H = 2): at most 128 wide when it
+// has two paths (an accumulator each) or stores an output, up to 256 wide
+// with one path and no output.  Mode 4 without an output (p.out null)
+// encodes no store map.
 template <int MODE>
 cudaError_t launch_sign_gemm(SignGemmParams p, const void *a, int64_t lda, const DeviceInfo &dev,
                              cudaStream_t stream)
 {
     constexpr bool C1 = MODE == 1 || MODE == 3;
     const int pairs = prefill_pairs_enabled() ? dev.pair_slots : 0;
-    const TilePlan tp = MODE == 4 ? plan_tiles(p.M, p.N, p.K, dev.sm_count, pairs, 128, 2)
+    const int max_bn4 = (p.out == nullptr && p.r0 >= p.K) ? BN : 128;
+    const TilePlan tp = MODE == 4 ? plan_tiles(p.M, p.N, p.K, dev.sm_count, pairs, max_bn4, 2)
                                   : plan_tiles(p.M, p.N, p.K, dev.sm_count, pairs);
     const int H = tp.H;
     p.bn = tp.bn;
     CUtensorMap tm, tmo;
     std::memset(&tmo, 0, sizeof(tmo));
     cudaError_t e = encode_2d(&tm, a, p.M, p.K, lda, C1, BM * H);
-    // the output: z fp16 (modes 1, 3) or y bf16 (modes 2, 4), [M x N] with stride ldo
-    if (e == cudaSuccess && p.out != nullptr) e = encode_store_2d(&tmo, p.out, p.M, p.N, p.ldo, !C1);
+    // the output: z fp16 (modes 1, 3; mode 3 bf16 on request) or y bf16 (modes 2, 4), [M x N], stride ldo
+    if (e == cudaSuccess && p.out != nullptr)
+        e = encode_store_2d(&tmo, p.out, p.M, p.N, p.ldo, !C1 || (MODE == 3 && p.out_bf16));
     if (e != cudaSuccess) return e;
     if constexpr (MODE == 4) {
         if (tp.P == 2) return launch_units<4, 2, 2>(tm, tmo, p, std::min(tp.tiles, dev.pair_slots), stream);
@@ -1092,6 +1116,8 @@ cudaError_t bwd_contraction1(const Bwd1Args &b, const DeviceInfo &dev, cudaStrea
     p.aux = b.aux;
     p.ldaux = b.ldaux;
     p.part0 = b.part;
+    p.out_bf16 = b.out_bf16;
+    p.aux_bf16 = b.aux_bf16;
     return launch_sign_gemm<3>(p, b.a, b.lda, dev, stream);
 }
 
