@@ -19,11 +19,13 @@
 // (leading byte offset) and 1024 bytes between 8-token groups (stride byte
 // offset), and an MMA of K = 16 tokens starts 2048 bytes further on.
 //
-// Persistent single-CTA tiles of 128 rows o x bn columns k, optionally split
-// over the tokens into `nsplit` parts; a unit (tile, part) leaves one partial
-// per row and path, [ntn * nsplit][n_out] per path, which the caller adds in
-// a fixed order.  Warp 0 issues the TMA loads, warp 1 the MMAs, warps 2..5
-// drain the two double-buffered accumulators.
+// Persistent tiles of 256 rows o on a CTA pair (cta_group::2: CTA r holds
+// rows 128 r .. of A and columns bn r / 2 .. of B; CTA 0 issues the MMAs),
+// or of 128 rows on single CTAs, x bn columns k, optionally split over the
+// tokens into `nsplit` parts; a unit (tile, part) leaves one partial per row
+// and path, [ntn * nsplit][n_out] per path, which the caller adds in a fixed
+// order.  Warp 0 issues the TMA loads, warp 1 the MMAs, warps 2..5 drain the
+// two double-buffered accumulators.
 #include <algorithm>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -37,15 +39,24 @@ namespace {
 
 using namespace tc;
 
-constexpr int WM = 128;                     // rows o per tile (one MMA, M = 128)
+constexpr int WM = 128;                     // rows o per CTA (M = 128; a pair's MMA: 256)
 constexpr int WBN = 256;                    // widest tile along k
 constexpr int WBK = 64;                     // tokens per K-block
 constexpr uint32_t BOX = 64 * 64 * 2;       // one TMA box: 64 MN x 64 tokens, 8 KB
-constexpr uint32_t W_A = (WM / 64) * BOX;   // 16 KB
-constexpr uint32_t W_B = (WBN / 64) * BOX;  // 32 KB
-constexpr int WSTAGES = 4;
+constexpr uint32_t W_A = (WM / 64) * BOX;   // 16 KB: this CTA's rows of A
 constexpr int kWThreads = 32 * 6;
-constexpr size_t kWSmem = 1024 + (size_t)WSTAGES * (W_A + W_B) + 256;
+// P = 1: a CTA stages all bn columns of B; P = 2: half of them (the pair's
+// MMA takes columns 0 .. bn/2 - 1 from CTA 0 and the rest from CTA 1)
+// (P = 2 leaves one stage's B bytes free after the last stage: what the
+// MMA reads from a stage then lies inside the allocation whichever half of
+// B it takes.)
+template <int P>
+struct WShape {
+    static constexpr uint32_t kB = (WBN / P / 64) * BOX;  // 32 or 16 KB
+    static constexpr uint32_t kPad = P == 2 ? kB : 0;
+    static constexpr int kStages = P == 1 ? 4 : 6;
+    static constexpr size_t kSmem = 1024 + (size_t)kStages * (W_A + kB) + kPad + 256;
+};
 
 struct WgradParams {
     int M;       // rows o (n_out)
@@ -70,15 +81,19 @@ __device__ __forceinline__ uint64_t smem_desc_mn(uint32_t addr, uint32_t lbo)
            (2ull << 61);
 }
 
+template <int P>
 __global__ void __launch_bounds__(kWThreads, 1)
     wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const WgradParams p)
 {
+    constexpr int WSTAGES = WShape<P>::kStages;
+    constexpr uint32_t W_B = WShape<P>::kB;
+    constexpr int PM = WM * P;  // rows o of a (pair's) tile
     extern __shared__ uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     const uint32_t sA = base, sB = base + WSTAGES * W_A;
-    const uint32_t bars = sB + WSTAGES * W_B;
+    const uint32_t bars = sB + WSTAGES * W_B + WShape<P>::kPad;
     // full[WSTAGES], empty[WSTAGES], acc_full[2], acc_empty[2], drain, then the tmem address
     const uint32_t full0 = bars, empty0 = bars + 8 * WSTAGES, accf0 = bars + 16 * WSTAGES;
     const uint32_t acce0 = accf0 + 16, drain = acce0 + 16;
@@ -86,12 +101,14 @@ __global__ void __launch_bounds__(kWThreads, 1)
     __shared__ int abort_shared;
     volatile int &abort_flag = abort_shared;
 
-    const int tiles_m = (p.M + WM - 1) / WM, tiles_n = (p.N + p.bn - 1) / p.bn;
+    const int rank = P == 2 ? (int)cluster_rank() : 0;
+    const int tiles_m = (p.M + PM - 1) / PM, tiles_n = (p.N + p.bn - 1) / p.bn;
     const int nk = (p.K + WBK - 1) / WBK;
     const int units = tiles_m * tiles_n * p.nsplit;
-    const int G = gridDim.x, c = blockIdx.x;
+    const int G = gridDim.x / P, c = blockIdx.x / P;  // persistent units: CTAs, or pairs
     const int my_units = c < units ? (units - c + G - 1) / G : 0;
-    // unit t: rows (t % tiles_m), then columns, then the token part
+    // unit t: columns (t % tiles_n), then rows, then the token part, so the
+    // units running at once share their rows of dy (the larger operand) in L2
     auto unit_kb = [&](int t, int &kb0, int &kb1) {
         const int sp = t / (tiles_m * tiles_n);
         kb0 = sp * p.kps;
@@ -106,28 +123,40 @@ __global__ void __launch_bounds__(kWThreads, 1)
             }
             for (int b = 0; b < 2; ++b) {
                 mbar_init(accf0 + 8 * b, 1);
-                mbar_init(acce0 + 8 * b, 4);
+                mbar_init(acce0 + 8 * b, 4 * P);  // every epilogue warp (of the pair)
             }
             mbar_init(drain, 1);
             abort_flag = 0;
             asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         }
         __syncwarp();
-        tmem_alloc(smem_u32(tmem_slot), 512);
+        if constexpr (P == 2)
+            tmem_alloc_pair(smem_u32(tmem_slot), 512);
+        else
+            tmem_alloc(smem_u32(tmem_slot), 512);
         tc_fence_before();
     }
-    __syncthreads();
+    if (P == 2)
+        cluster_sync();  // both CTAs' barriers are initialised before either arrives on the other's
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // P = 2: CTA 0's full and acc-empty barriers, as this CTA reaches them
+    const uint32_t full_lead = P == 2 ? map_shared_addr(full0, 0) : full0;
+    const uint32_t acce_lead = P == 2 ? map_shared_addr(acce0, 0) : acce0;
 
     if (warp == 0) {
         // ---------------- TMA: A (dy^T) and B (c) boxes of each K-block
         if (lane == 0) {
             int gb = 0, issued = 0;
+            // this CTA's columns of B: all bn (P = 1), or half from bn/2 rank on
+            const int bw = p.bn / P, nb = (bw + 63) / 64;
+            const uint32_t stage_bytes = (uint32_t)(WM / 64 + nb) * BOX;
             for (int i = 0; i < my_units && !abort_flag; ++i) {
                 const int t = c + i * G;
-                const int o0 = (t % tiles_m) * WM, k0 = ((t / tiles_m) % tiles_n) * p.bn;
-                const int nb = (p.bn + 63) / 64;
+                const int o0 = ((t / tiles_n) % tiles_m) * PM + rank * WM;
+                const int k0 = (t % tiles_n) * p.bn + rank * bw;
                 int kb0, kb1;
                 unit_kb(t, kb0, kb1);
                 for (int kb = kb0; kb < kb1; ++kb, ++gb) {
@@ -137,24 +166,50 @@ __global__ void __launch_bounds__(kWThreads, 1)
                         abort_flag = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(full0 + 8 * s, (uint32_t)(WM / 64 + nb) * BOX);
-                    for (int j = 0; j < WM / 64; ++j)
-                        tma_load_2d(sA + s * W_A + j * BOX, &tmA, o0 + 64 * j, kb * WBK, full0 + 8 * s);
-                    for (int j = 0; j < nb; ++j)
-                        tma_load_2d(sB + s * W_B + j * BOX, &tmB, k0 + 64 * j, kb * WBK, full0 + 8 * s);
+                    if (P == 1) {
+                        mbar_arrive_expect_tx(full0 + 8 * s, stage_bytes);
+                        for (int j = 0; j < WM / 64; ++j)
+                            tma_load_2d(sA + s * W_A + j * BOX, &tmA, o0 + 64 * j, kb * WBK, full0 + 8 * s);
+                        for (int j = 0; j < nb; ++j)
+                            tma_load_2d(sB + s * W_B + j * BOX, &tmB, k0 + 64 * j, kb * WBK, full0 + 8 * s);
+                    } else {
+                        // both CTAs' bytes complete on CTA 0's barrier, which CTA 0 arms
+                        if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * s, 2 * stage_bytes);
+                        for (int j = 0; j < WM / 64; ++j)
+                            tma_load_2d_pair(sA + s * W_A + j * BOX, &tmA, o0 + 64 * j, kb * WBK, full_lead + 8 * s);
+                        for (int j = 0; j < nb; ++j)
+                            tma_load_2d_pair(sB + s * W_B + j * BOX, &tmB, k0 + 64 * j, kb * WBK, full_lead + 8 * s);
+                    }
                     ++issued;
                 }
             }
-            if (abort_flag)
+            if (abort_flag && P == 2 && rank == 1) {
+                // this CTA cannot wait on CTA 0's barriers: give copies in
+                // flight time to land (they take microseconds)
+                const unsigned long long t0 = globaltimer();
+                while (globaltimer() - t0 < 200000ull) {
+                }
+            } else if (abort_flag) {
                 for (int q = (issued > WSTAGES ? issued - WSTAGES : 0); q < issued; ++q)
                     mbar_wait(full0 + 8 * (q % WSTAGES), (uint32_t)(q / WSTAGES) & 1u);
+            }
         }
     } else if (warp == 1) {
         // ---------------- MMA: unit i accumulates in columns 256 (i % 2) ..
-        if (lane == 0) {
-            // bf16 operands, fp32 accumulate, A and B MN-major, M = 128, N = bn
+        // P = 2: CTA 0 issues the pair's MMAs and signals both CTAs; CTA 1
+        // only waits for the last of them before it may free tensor memory.
+        if (lane == 0 && P == 2 && rank == 1) {
+            if (!mbar_wait(drain, 0)) abort_flag = 1;
+        } else if (lane == 0) {
+            // bf16 operands, fp32 accumulate, A and B MN-major, M = 128 P, N = bn
             const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
-                                   ((uint32_t)(p.bn >> 3) << 17) | ((uint32_t)(WM >> 4) << 24);
+                                   ((uint32_t)(p.bn >> 3) << 17) | ((uint32_t)(PM >> 4) << 24);
+            auto commit = [&](uint32_t bar) {
+                if constexpr (P == 2)
+                    umma_commit_pair(bar);
+                else
+                    umma_commit(bar);
+            };
             int gb = 0;
             for (int i = 0; i < my_units && !abort_flag; ++i) {
                 const int t = c + i * G;
@@ -179,14 +234,19 @@ __global__ void __launch_bounds__(kWThreads, 1)
                     for (int kk = 0; kk < WBK / 16; ++kk) {  // 16 tokens: 2048 bytes further on
                         const uint64_t ad = smem_desc_mn(sA + s * W_A + (uint32_t)kk * 2048u, BOX);
                         const uint64_t bd = smem_desc_mn(sB + s * W_B + (uint32_t)kk * 2048u, BOX);
-                        umma(acc, ad, bd, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+                        const uint32_t acc_flag = (kb != kb0 || kk != 0) ? 1u : 0u;
+                        if constexpr (P == 2)
+                            umma_pair(acc, ad, bd, idesc, acc_flag);
+                        else
+                            umma(acc, ad, bd, idesc, acc_flag);
                     }
-                    umma_commit(empty0 + 8 * s);
+                    commit(empty0 + 8 * s);
                 }
                 if (abort_flag) break;
-                umma_commit(accf0 + 8 * b);
+                commit(accf0 + 8 * b);
             }
-            umma_commit(drain);
+            // every MMA issued has finished before the CTA (and its pair) frees tensor memory
+            commit(drain);
             if (!mbar_wait(drain, 0)) abort_flag = 1;
         }
     } else {
@@ -197,8 +257,8 @@ __global__ void __launch_bounds__(kWThreads, 1)
         for (int i = 0; i < my_units; ++i) {
             const int t = c + i * G;
             const int b = i & 1, use = i >> 1;
-            const int tn = (t / tiles_m) % tiles_n, sp = t / (tiles_m * tiles_n);
-            const int o = (t % tiles_m) * WM + 32 * quad + lane;
+            const int tn = t % tiles_n, sp = t / (tiles_m * tiles_n);
+            const int o = ((t / tiles_n) % tiles_m) * PM + rank * WM + 32 * quad + lane;
             const int k0 = tn * p.bn;
             bool ok = !abort_flag && mbar_wait(accf0 + 8 * b, (uint32_t)(use & 1));
             ok = __all_sync(0xffffffffu, ok);
@@ -236,7 +296,12 @@ __global__ void __launch_bounds__(kWThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acce0 + 8 * b);
+            if (lane == 0) {
+                if (P == 2 && rank == 1)
+                    mbar_arrive_remote(acce_lead + 8 * b);
+                else
+                    mbar_arrive(acce0 + 8 * b);
+            }
             if (o < p.M) {
                 const int64_t row = (int64_t)(tn * p.nsplit + sp) * p.M + o;
                 p.part0[row] = s0;
@@ -244,25 +309,36 @@ __global__ void __launch_bounds__(kWThreads, 1)
             }
         }
     }
+    tc_fence_before();
     __syncthreads();
+    // P = 2: neither CTA leaves (or frees its half of tensor memory) while
+    // the other may still arrive on its barriers or read its shared memory
+    if (P == 2) cluster_sync();
     if (abort_flag && threadIdx.x == 0) set_status(p.status, LB_ERR_DEVICE_TIMEOUT);
     if (warp == 0) {
+        __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        if constexpr (P == 2)
+            tmem_dealloc_pair(tmem, 512);
+        else
+            tmem_dealloc(tmem, 512);
     }
 }
 
 }  // namespace
 
 // Tile width, token split and partial count of the h-gradient product for
-// n_out rows, R latent columns and `tokens` tokens on `sms` SMs.
+// n_out rows, R latent columns and `tokens` tokens on `sms` SMs.  The plan is
+// made for CTA pairs (256-row tiles, sms / 2 of them at once) and kept for
+// single CTAs, so both give the same token parts and the same sums.
 WgradPlan wgrad_plan(int n_out, int R, int tokens, int sms)
 {
     WgradPlan w{};
     const int ntn = (R + WBN - 1) / WBN;
     w.bn = ((R + ntn - 1) / ntn + 31) & ~31;
     w.ntn = (R + w.bn - 1) / w.bn;
-    const int tiles = ((n_out + WM - 1) / WM) * w.ntn;
+    const int tiles = ((n_out + 2 * WM - 1) / (2 * WM)) * w.ntn;
+    sms = std::max(1, sms / 2);
     const int nk = std::max(1, (tokens + WBK - 1) / WBK);
     // makespan in K-blocks: waves x (blocks per part + a unit's fixed cost of
     // about two K-blocks); at most wgrad_max_parts parts
@@ -292,7 +368,11 @@ int wgrad_max_parts(int R, int tokens)
 cudaError_t wgrad_prepare_device(const DeviceInfo &dev)
 {
     (void)dev;
-    return cudaFuncSetAttribute(wgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kWSmem);
+    cudaError_t e = cudaFuncSetAttribute(wgrad_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)WShape<1>::kSmem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(wgrad_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)WShape<2>::kSmem);
+    return e;
 }
 
 cudaError_t wgrad_dh(const WgradArgs &w, const DeviceInfo &dev, cudaStream_t stream)
@@ -322,9 +402,24 @@ cudaError_t wgrad_dh(const WgradArgs &w, const DeviceInfo &dev, cudaStream_t str
     p.part0 = w.part0;
     p.part1 = w.part1;
     p.status = dev.status;
+    if (prefill_pairs_enabled() && dev.pair_slots > 0) {
+        const int units = ((w.n_out + 2 * WM - 1) / (2 * WM)) * pl.ntn * pl.nsplit;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)(2 * std::min(units, dev.pair_slots)));
+        cfg.blockDim = dim3(kWThreads);
+        cfg.dynamicSmemBytes = WShape<2>::kSmem;
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, wgrad_kernel<2>, ta, tb, p);
+    }
     const int units = ((w.n_out + WM - 1) / WM) * pl.ntn * pl.nsplit;
-    const int grid = std::min(units, dev.sm_count);
-    wgrad_kernel<<<grid, kWThreads, kWSmem, stream>>>(ta, tb, p);
+    wgrad_kernel<1><<<std::min(units, dev.sm_count), kWThreads, WShape<1>::kSmem, stream>>>(ta, tb, p);
     return cudaGetLastError();
 }
 
