@@ -11,26 +11,27 @@
 //     dt = S_V (l (.) a)               (the gradient with respect to t)
 //     dg = sum over tokens of x (.) dt,   dx = sum_p g (.) dt
 //     dh = sum over tokens of dy (.) e
-// Four tcgen05 contractions compute them (the prefill kernels' modes 3 and 4,
-// lb_prefill.cu):
-//   K1  c = S_V^T (g (.) x)          x [M x n_in] against the packed rows of V^T
-//   K2  a = S_U^T (h (.) dy)         dy [M x n_out] against the rows of U^T;
-//                                    the epilogue also forms a (.) c per
-//                                    32-token block (dl partials)
-//   K3  dh_p = sum_k S_U,p l_p G     G = dy^T c, the tokens as the MMA's
-//                                    K (lb_wgrad.cu); the epilogue applies
-//                                    each row's signs and l and sums over k
-//                                    (dh partials per tile column)
-//   K4  dt_p = S_V,p (l_p (.) a_p)   a against the rows of V; the epilogue
-//                                    stores dx = sum_p g_p (.) dt_p (bf16) and
-//                                    forms x (.) dt_p per block (dg partials)
-// then one kernel adds each partial column over the blocks in block order, so
-// the results do not depend on timing.  K2 and K4 read the factors along the
+// Five tcgen05 products compute them:
+//   K1  c = S_V^T (g (.) x)            x [M x n_in] against the packed rows of
+//                                      V^T (lb_prefill.cu, mode 3); bf16
+//   K2  a_s = l (.) S_U^T (h (.) dy)   dy [M x n_out] against the rows of U^T
+//                                      (mode 3), scaled by l on the way out;
+//                                      the epilogue also forms a (.) c per
+//                                      32-token block (dl partials); bf16
+//   K3  dh_p[o] = sum_k sign(U_p[o, k]) l_p[k] (dy^T c)[o, k]
+//   K4  dg_p[i] = sum_k sign(V_p[i, k]) (x^T a_s)[i, k]
+//                                      both with the tokens as the MMA's K
+//                                      (lb_wgrad.cu): per row a sum over k in
+//                                      the epilogue (partials per tile column)
+//   K5  dx = sum_p g_p (.) S_V,p a_s,p the forward's contraction-2 shape in
+//                                      bf16 (mode 2), V packed along r
+// then one kernel adds each partial column over its rows in order, so the
+// results do not depend on timing.  K2, K4 and K5 read the factors along the
 // other axis from the forward pass: U^T packed along n_out and V packed along
 // r, which two bit-transpose launches make from the forward's packed words
 // into the workspace, so the call takes the forward pass's lb_path as it is.
-// c (bf16, the type of dy, as K3 needs) and a (fp16) travel between the
-// contractions unscaled.
+// c and a_s travel between the products in bf16, the type of x and dy that
+// K3 and K4 multiply them with.
 #include <algorithm>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -170,7 +171,7 @@ BwdLayout layout(int M, int n_in, int n_out, const int *ranks, int npaths)
         L.ph[q] = off;
         off += align256(HB * (size_t)n_out * 4);
         L.pg[q] = off;
-        off += align256(RB * (size_t)n_in * 4);
+        off += align256(HB * (size_t)n_in * 4);
     }
     L.total = off;
     return L;
@@ -231,7 +232,8 @@ cudaError_t backward_launch(const BackwardArgs &b, const DeviceInfo &dev, cudaSt
     e = bwd_contraction1(k1, dev, stream);
     if (e != cudaSuccess) return e;
 
-    // K2: a = S_U^T (h (.) dy), unscaled; dl partials sum a (.) c
+    // K2: a_s = l (.) S_U^T (h (.) dy), scaled by l on the way out; dl
+    // partials sum a (.) c from the unscaled accumulator
     Bwd1Args k2{};
     k2.M = M;
     k2.K = b.n_out;
@@ -242,13 +244,16 @@ cudaError_t backward_launch(const BackwardArgs &b, const DeviceInfo &dev, cudaSt
     k2.bits0 = ut[0];
     k2.ld0 = b.n_out / 32;
     k2.s0 = P0.h;
+    k2.l0 = P0.l;
     if (two) {
         k2.bits1 = ut[1];
         k2.ld1 = b.n_out / 32;
         k2.s1 = P1.h;
+        k2.l1 = P1.l;
     }
     k2.out = a;
     k2.ldo = R;
+    k2.out_bf16 = 1;
     k2.aux = c;
     k2.ldaux = R;
     k2.aux_bf16 = 1;
@@ -259,53 +264,71 @@ cudaError_t backward_launch(const BackwardArgs &b, const DeviceInfo &dev, cudaSt
     // K3: dh_p[o] = sum_k sign(U_p[o, k]) l_p[k] G[o, k], G = dy^T c
     WgradArgs k3{};
     k3.tokens = M;
-    k3.n_out = b.n_out;
+    k3.rows = b.n_out;
     k3.R = R;
     k3.r0 = r0;
-    k3.dy = b.dy;
-    k3.lddy = b.lddy;
-    k3.c = c;
-    k3.ldc = R;
-    k3.u0 = P0.u_bits;
-    k3.uld0 = P0.u_ld;
+    k3.a = b.dy;
+    k3.lda = b.lddy;
+    k3.b = c;
+    k3.ldb = R;
+    k3.bits0 = P0.u_bits;
+    k3.bld0 = P0.u_ld;
     k3.l0 = P0.l;
     if (two) {
-        k3.u1 = P1.u_bits;
-        k3.uld1 = P1.u_ld;
+        k3.bits1 = P1.u_bits;
+        k3.bld1 = P1.u_ld;
         k3.l1 = P1.l;
     }
     k3.part0 = ph[0];
     k3.part1 = ph[1];
-    e = wgrad_dh(k3, dev, stream);
+    e = wgrad_scale_grad(k3, dev, stream);
     if (e != cudaSuccess) return e;
-    const int hrows = wgrad_plan(b.n_out, R, M, dev.sm_count).rows;
 
-    // K4: dt_p = S_V,p (l_p (.) a_p); dx = sum_p g_p (.) dt_p; dg partials sum x (.) dt_p
-    Bwd2Args k4{};
-    k4.M = M;
-    k4.N = b.n_in;
+    // K4: dg_p[i] = sum_k sign(V_p[i, k]) H[i, k], H = x^T a_s (l already in a_s)
+    WgradArgs k4{};
+    k4.tokens = M;
+    k4.rows = b.n_in;
+    k4.R = R;
     k4.r0 = r0;
-    k4.r1 = r1;
-    k4.a = a;
-    k4.lda = R;
+    k4.a = b.x;
+    k4.lda = b.ldx;
+    k4.b = a;
+    k4.ldb = R;
     k4.bits0 = v[0];
-    k4.ld0 = r0 / 32;
-    k4.l0 = P0.l;
+    k4.bld0 = r0 / 32;
     if (two) {
         k4.bits1 = v[1];
-        k4.ld1 = r1 / 32;
-        k4.l1 = P1.l;
+        k4.bld1 = r1 / 32;
     }
-    k4.aux = b.x;
-    k4.ldaux = b.ldx;
     k4.part0 = pg[0];
     k4.part1 = pg[1];
-    k4.out = b.dx;
-    k4.ldo = b.lddx;
-    k4.t0 = P0.g;
-    k4.t1 = two ? P1.g : nullptr;
-    e = bwd_contraction2(k4, dev, stream);
+    e = wgrad_scale_grad(k4, dev, stream);
     if (e != cudaSuccess) return e;
+
+    // K5: dx = sum_p g_p (.) S_V,p a_s,p
+    if (b.dx != nullptr) {
+        BwdDxArgs k5{};
+        k5.M = M;
+        k5.n_in = b.n_in;
+        k5.r0 = r0;
+        k5.r1 = r1;
+        k5.a = a;
+        k5.lda = R;
+        k5.bits0 = v[0];
+        k5.ld0 = r0 / 32;
+        k5.g0 = P0.g;
+        if (two) {
+            k5.bits1 = v[1];
+            k5.ld1 = r1 / 32;
+            k5.g1 = P1.g;
+        }
+        k5.dx = b.dx;
+        k5.lddx = b.lddx;
+        e = bwd_dx(k5, dev, stream);
+        if (e != cudaSuccess) return e;
+    }
+    const int hrows = wgrad_plan(b.n_out, R, M, dev.sm_count).rows;
+    const int grows = wgrad_plan(b.n_in, R, M, dev.sm_count).rows;
 
     // the partial sums, each added over its rows in row order
     ReduceParams rp{};
@@ -318,8 +341,8 @@ cudaError_t backward_launch(const BackwardArgs &b, const DeviceInfo &dev, cudaSt
     add(pl, b.dl, R, tb);
     add(ph[0], b.dh, b.n_out, hrows);
     if (two) add(ph[1], b.dh + b.n_out, b.n_out, hrows);
-    add(pg[0], b.dg, b.n_in, tb);
-    if (two) add(pg[1], b.dg + b.n_in, b.n_in, tb);
+    add(pg[0], b.dg, b.n_in, grows);
+    if (two) add(pg[1], b.dg + b.n_in, b.n_in, grows);
     // every segment's length is a multiple of 32, so a CTA's 32 columns lie in one segment
     reduce_partials_kernel<<<(unsigned)(total / 32), 32 * kGroups, 0, stream>>>(rp);
     return cudaGetLastError();

@@ -135,12 +135,13 @@ cudaError_t prefill_expand(const ForwardArgs &a, const DeviceInfo &dev, cudaStre
                            int64_t ldz);
 
 // ---------------------------------------------------------------- backward (lb_backward.cu, lb_prefill.cu)
-// The backward pass's two contraction shapes on the prefill kernels.
-// Contraction-1 shape: C[m, n] = sum_k A[m, k] B[n, k] with A bf16 [M x K],
-// B[n, k] = sign(row n of bits_p)[k] s_p[k] (rows n < r0 from path 0, the
-// rest from path 1), stored unscaled as fp16 (or bf16: out_bf16)
-// [M x (r0 + r1)]; with aux (fp16, or bf16: aux_bf16, [M x N]) also
-// part[m / 32][n] = sum over the 32-row block of C * aux.
+// The backward pass's contraction-1-shaped steps on the prefill kernels:
+// C[m, n] = sum_k A[m, k] B[n, k] with A bf16 [M x K], B[n, k] =
+// sign(row n of bits_p)[k] s_p[k] (rows n < r0 from path 0, the rest from
+// path 1), stored as l (.) C (l_p per column; C itself where l is null) in
+// fp16, or bf16 with out_bf16, [M x (r0 + r1)]; with aux (fp16, or bf16 with
+// aux_bf16, [M x N]) also part[m / 32][n] = sum over the 32-row block of the
+// unscaled C * aux.
 struct Bwd1Args {
     int M, K, r0, r1;
     const uint16_t *a;
@@ -148,6 +149,7 @@ struct Bwd1Args {
     const uint32_t *bits0, *bits1;  // packed rows along K (bits1 null: one path)
     int64_t ld0, ld1;
     const uint16_t *s0, *s1;  // per-K scale of each path's rows (fp16, length K)
+    const uint16_t *l0, *l1;  // per-column scale of the stored output, or null
     uint16_t *out;
     int64_t ldo;
     const uint16_t *aux;
@@ -156,49 +158,46 @@ struct Bwd1Args {
     int out_bf16, aux_bf16;
 };
 cudaError_t bwd_contraction1(const Bwd1Args &b, const DeviceInfo &dev, cudaStream_t stream);
-// Contraction-2 shape: C_p[m, n] = sum over path p's columns k of
-// A[m, k] sign(row n of bits_p)[k] l_p[k], A fp16 [M x (r0 + r1)] (the paths
-// side by side); part_p[m / 32][n] = sum over the 32-row block of C_p * aux
-// (aux bf16 [M x N]); with out, also out[m, n] = sum_p t_p[n] C_p[m, n] (bf16).
-struct Bwd2Args {
-    int M, N, r0, r1;
-    const uint16_t *a;
-    int64_t lda;
-    const uint32_t *bits0, *bits1;  // packed rows n along the path's latent
-    int64_t ld0, ld1;
-    const uint16_t *l0, *l1;  // latent scale of each path
-    const uint16_t *aux;
-    int64_t ldaux;
-    float *part0, *part1;
-    uint16_t *out;  // may be null
-    int64_t ldo;
-    const uint16_t *t0, *t1;
-};
-cudaError_t bwd_contraction2(const Bwd2Args &b, const DeviceInfo &dev, cudaStream_t stream);
 
-// The h-gradient as a weight-gradient product (lb_wgrad.cu): for every row o
-// of the paths' U and every path p, sums over k in path p of
-// sign(U_p[o, k]) l_p[k] G[o, k] with G = dy^T c (dy bf16 [tokens x n_out],
-// c bf16 [tokens x R], the paths side by side), one partial per tile column
-// and token part: part_p[row][o], rows = WgradPlan::rows.
+// A scale gradient as a weight-gradient product (lb_wgrad.cu): for every row
+// o of a path's sign matrix S_p (packed along the latent) and every path p,
+// the sum over k in path p of sign(S_p[o, k]) l_p[k] G[o, k], G = A^T B with
+// A bf16 [tokens x rows] and B bf16 [tokens x R] (the paths side by side), the
+// tokens as the MMA's K; l_p null means 1.  dh: A = dy, B = c, S = U, l.
+// dg: A = x, B = l (.) a, S = V, no l.  One partial per tile column and
+// token part: part_p[row][o], rows = WgradPlan::rows.
 struct WgradPlan {
     int bn, ntn, nsplit, kps, rows;
 };
-WgradPlan wgrad_plan(int n_out, int R, int tokens, int sms);
+WgradPlan wgrad_plan(int rows, int R, int tokens, int sms);
 int wgrad_max_parts(int R, int tokens);  // the most partial rows any plan takes
 struct WgradArgs {
-    int tokens, n_out, R, r0;
-    const uint16_t *dy;
-    int64_t lddy;
-    const uint16_t *c;
-    int64_t ldc;
-    const uint32_t *u0, *u1;
-    int64_t uld0, uld1;
-    const uint16_t *l0, *l1;
-    float *part0, *part1;  // part1 null: one path
+    int tokens, rows, R, r0;
+    const uint16_t *a;
+    int64_t lda;
+    const uint16_t *b;
+    int64_t ldb;
+    const uint32_t *bits0, *bits1;  // packed rows o along the path's latent (bits1 null: one path)
+    int64_t bld0, bld1;
+    const uint16_t *l0, *l1;  // latent scale of each path, or null for 1
+    float *part0, *part1;     // part1 null: one path
 };
 cudaError_t wgrad_prepare_device(const DeviceInfo &dev);
-cudaError_t wgrad_dh(const WgradArgs &w, const DeviceInfo &dev, cudaStream_t stream);
+cudaError_t wgrad_scale_grad(const WgradArgs &w, const DeviceInfo &dev, cudaStream_t stream);
+// dx = sum_p g_p (.) S_V,p (l_p (.) a_p): the forward's contraction-2 shape in
+// bf16 (A = l (.) a bf16 [M x R], B rows i = +-bf16(g_p[i]) by V packed along
+// the latent), out bf16 [M x n_in].
+struct BwdDxArgs {
+    int M, n_in, r0, r1;
+    const uint16_t *a;
+    int64_t lda;
+    const uint32_t *bits0, *bits1;
+    int64_t ld0, ld1;
+    const uint16_t *g0, *g1;
+    uint16_t *dx;
+    int64_t lddx;
+};
+cudaError_t bwd_dx(const BwdDxArgs &b, const DeviceInfo &dev, cudaStream_t stream);
 
 // The whole backward pass (lb_linear_backward), already validated.
 struct BackwardArgs {

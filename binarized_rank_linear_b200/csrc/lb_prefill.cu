@@ -44,20 +44,15 @@
 // arrives on the barriers of both CTAs; the TMA loads and producer arrivals
 // of CTA 1 count on CTA 0's stage barriers.
 //
-// Two more modes serve the layer's backward pass (lb_backward.cu):
+// One more mode serves the layer's backward pass (lb_backward.cu):
 //   mode 3:  the contraction-1 shape (bf16 operands, B1 rows scaled along K)
-//            with the latent scale optional (l0 null: unit), and optionally
-//            a column dot in the epilogue: for every output column n,
-//            part0[row block][n] = sum over the block's 32 rows m of
-//            C[m, n] * aux[m, n]  (aux fp16 [M x N]);
-//   mode 4:  the contraction-2 shape (fp16 operands) with the scale on the K
-//            dimension instead of the rows (B[n, k] = sign(.)[n, k] s_p[k],
-//            s_p[k] the latent scale of the path that column k belongs to),
-//            one accumulator per path (bn <= 128: a 128-row half's two paths
-//            take 256 columns of tensor memory), and in the epilogue the
-//            column dot of each path's result with aux (bf16 [M x N]) into
-//            part0 / part1, plus optionally the bf16 store of
-//            sum_p t_p[n] C_p[m, n].
+//            with the latent scale optional (l0 null: unit), the output in
+//            fp16 or bf16, and optionally a column dot in the epilogue: for
+//            every output column n, part0[row block][n] = sum over the
+//            block's 32 rows m of C[m, n] * aux[m, n] (the unscaled C; aux
+//            fp16 or bf16 [M x N]);
+// and mode 2 takes bf16 operands on request (bf16_ops: A bf16, the row
+// scales rounded to bf16), for the backward's dx.
 // Partial sums are per 32-row block of the output, so each is written once
 // and the caller reduces them in a fixed order: the results do not depend on
 // timing.
@@ -94,12 +89,9 @@ constexpr uint32_t OUT_BYTES = 32 * 64;       // an output box: 32 rows x 32 two
 // and expands B rows bn r / 2 .. of the tile's bn, so each CTA stages and
 // expands half of B, and the MMA reads each half of B from shared memory once
 // for both SMs.  Stages are then smaller and the ring deeper.
-//
-// Mode 4 gives up one stage for a per-epilogue-warp buffer in which its
-// column dots are transposed (32 rows of 36 floats).
 template <int H, int P, int MODE>
 struct Shape {
-    static constexpr int kStages = (P == 1 ? (H == 1 ? 4 : 3) : (H == 1 ? 6 : 4)) - (MODE == 4 ? 1 : 0);
+    static constexpr int kStages = P == 1 ? (H == 1 ? 4 : 3) : (H == 1 ? 6 : 4);
     // producer groups: one B row per thread, a group per K-block in turn
     // (P = 2: a CTA's B rows take half a group's warps, so twice the groups)
     static constexpr int kGroupWarps = kRowWarps / P;
@@ -115,9 +107,8 @@ struct Shape {
     // per stage: A tile, B tile; per epilogue warp: its output boxes and the
     // tile's latent scale in fp32 (mode 1); per producer warp: two slots of g
     // rounded to bf16; per producer thread: kRing slots of sign words
-    static constexpr uint32_t kRedBytes = MODE == 4 ? 32 * 36 * 4 : 0;  // per epilogue warp
     static constexpr size_t kSmem = 1024 + (size_t)kStages * (kABytes + kBBytes) +
-                                    (size_t)kEpiWarps * (kOutBufs * OUT_BYTES + BN * 4 + kRedBytes) +
+                                    (size_t)kEpiWarps * (kOutBufs * OUT_BYTES + BN * 4) +
                                     (size_t)kProducerWarps * (2 * G_BYTES + 32 * 8 * kRing) + 256;
     static_assert(kSmem <= 232448, "shared memory per CTA");
 };
@@ -168,11 +159,11 @@ struct SignGemmParams {
     int64_t ldo;
     int *status;
     // backward modes (3, 4)
-    const void *aux;             // column-dot operand: mode 3 fp16, mode 4 bf16, [M x N], row stride ldaux
+    const void *aux;             // mode 3: column-dot operand, fp16 or bf16 [M x N], row stride ldaux
     int64_t ldaux;
-    float *part0, *part1;        // column-dot partials [ceil(M / 32) x N] (part1: mode 4, path 1)
-    const uint16_t *t0, *t1;     // mode 4: per-column scales of the stored output (fp16, length N)
+    float *part0;                // column-dot partials [ceil(M / 32) x N]
     int out_bf16, aux_bf16;      // mode 3: store C as bf16 (else fp16); aux is bf16 (else fp16)
+    int bf16_ops;                // mode 2: A and the +-scale operand in bf16 (else fp16)
 };
 
 // Persistent: CTA c computes the tiles t = c, c + gridDim.x, ...
@@ -204,8 +195,7 @@ __global__ void __launch_bounds__(Shape<H, P, MODE>::kThreads, 1)
     const uint32_t sGbf = sOut + S::kEpiWarps * S::kOutBufs * OUT_BYTES;  // mode 1, per producer warp: g in bf16, [warp][2][path][64]
     const uint32_t sLf = sGbf + kProducerWarps * 2 * G_BYTES;  // mode 1, per epilogue warp: l of the tile in fp32
     const uint32_t sRing = sLf + S::kEpiWarps * BN * 4;  // per producer thread: kRing 8-byte sign-word slots
-    const uint32_t sRed = sRing + kProducerWarps * 32 * 8 * S::kRing;  // mode 4, per epilogue warp: transpose buffer
-    const uint32_t bars = sRed + S::kEpiWarps * S::kRedBytes;
+    const uint32_t bars = sRing + kProducerWarps * 32 * 8 * S::kRing;
     // full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain, then the tmem address
     const uint32_t full0 = bars, empty0 = bars + 8 * STAGES, accf0 = bars + 16 * STAGES;
     const uint32_t acce0 = accf0 + 16, drain = acce0 + 16;
@@ -301,7 +291,7 @@ __global__ void __launch_bounds__(Shape<H, P, MODE>::kThreads, 1)
         if (lane == 0 && P == 2 && rank == 1) {
             if (!mbar_wait(drain, 0)) abort_flag = 1;
         } else if (lane == 0) {
-            const uint32_t idesc = instr_desc(C1 ? 1u : 0u, BM * P, p.bn);
+            const uint32_t idesc = instr_desc((C1 || p.bf16_ops) ? 1u : 0u, BM * P, p.bn);
             auto commit = [&](uint32_t bar) {
                 if constexpr (P == 2)
                     umma_commit_pair(bar);
@@ -334,20 +324,7 @@ __global__ void __launch_bounds__(Shape<H, P, MODE>::kThreads, 1)
                         const uint64_t ad = smem_desc(sA + s * A_BYTES + (uint32_t)h * (BM * BK * 2));
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk) {  // +32 bytes along K per step of 16
-                            if constexpr (MODE == 4) {
-                                // path p's K columns accumulate in columns 128 p .. of the
-                                // half's accumulator (bn <= 128); a path starts at column
-                                // 0 or r0 (multiples of 32: no step of 16 spans both paths)
-                                const int col = kb * BK + kk * 16;
-                                if (col >= p.K) continue;
-                                const uint32_t pth = col >= p.r0 ? 1u : 0u;
-                                const uint32_t d = acc + (uint32_t)(h * BN) + 128u * pth;
-                                const uint32_t accum = (col != 0 && col != p.r0) ? 1u : 0u;
-                                if constexpr (P == 2)
-                                    umma_pair(d, ad + 2 * kk, bd + 2 * kk, idesc, accum);
-                                else
-                                    umma(d, ad + 2 * kk, bd + 2 * kk, idesc, accum);
-                            } else if constexpr (P == 2) {
+                            if constexpr (P == 2) {
                                 umma_pair(acc + (uint32_t)(h * BN), ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
                             } else {
                                 umma(acc + (uint32_t)(h * BN), ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0);
@@ -429,18 +406,6 @@ __global__ void __launch_bounds__(Shape<H, P, MODE>::kThreads, 1)
         // (zeros outside the matrix) and, mode 1, lanes 0..15, of its g into
         // the warp's g slot `slot`: one cp.async group.
         auto copy_block = [&](const Cursor &u, int slot) {
-            if (MODE == 4 && u.gb < my_blocks && lane < 8) {
-                // lane: K columns 8 lane .. 8 lane + 7 of the block, from the
-                // scale vector of the path they belong to (paths start at
-                // multiples of 32, so 8 columns never span both)
-                const int k0 = u.kb * BK + 8 * lane;
-                const uint16_t *src = k0 < p.r0 ? p.s0 + k0 : (p.s1 != nullptr ? p.s1 + (k0 - p.r0) : nullptr);
-                const uint32_t gdst = gbfw + (uint32_t)slot * G_BYTES + (uint32_t)lane * 16;
-                if (src != nullptr && k0 < p.K)
-                    cp_async16s(gdst, src);
-                else
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(gdst), "r"(0u) : "memory");
-            }
             if (C1 && u.gb < my_blocks && lane < 16) {
                 // lane: path lane / 8, columns 8 (lane % 8) .. 8 (lane % 8) + 7 of the block
                 const int pp = lane >> 3, k0 = u.kb * BK + 8 * (lane & 7);
@@ -499,6 +464,8 @@ __global__ void __launch_bounds__(Shape<H, P, MODE>::kThreads, 1)
             const int gb = u.gb, kb = u.kb, nn = u.nn;
             if (MODE == 2 && u.i != hi) {  // first block of a tile for this group
                 hcur = u.i == hi + 1 ? hnext : fetch_h(u.i);
+                if (p.bf16_ops)  // the row's scales rounded to bf16, the operand type
+                    hcur = pack_bf162(f16_bits_to_float((uint16_t)(hcur & 0xffffu)), f16_bits_to_float((uint16_t)(hcur >> 16)));
                 hnext = fetch_h(u.i + 1);
                 hi = u.i;
             }
@@ -538,12 +505,6 @@ __global__ void __launch_bounds__(Shape<H, P, MODE>::kThreads, 1)
                 const uint8_t *gb_ = smem_raw + (gsl + (sec_row ? BK * 2 : 0) - raw);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) sc[q] = *reinterpret_cast<const uint4 *>(gb_ + 16 * q);
-            } else if (MODE == 4) {
-                // the block's 64 K scales (fp16, as the operands), copied by lanes 0..7
-                __syncwarp();
-                const uint8_t *sl = smem_raw + (gbfw + (uint32_t)slot * G_BYTES - raw);
-#pragma unroll
-                for (int q = 0; q < 8; ++q) sc[q] = *reinterpret_cast<const uint4 *>(sl + 16 * q);
             } else {
                 const uint32_t hs0 = (hcur & 0xffffu) * 0x10001u, hs1 = (hcur >> 16) * 0x10001u;
 #pragma unroll
@@ -619,19 +580,8 @@ __global__ void __launch_bounds__(Shape<H, P, MODE>::kThreads, 1)
                     asm volatile("st.shared.f32 [%0], %1;" ::"r"(lsm + 4u * (uint32_t)cc), "f"(lv) : "memory");
                 }
                 __syncwarp();
-            } else if (MODE == 4 && p.out != nullptr) {
-                // the per-column scales of the stored output, both paths
-                // (columns cc and 128 + cc of the warp's fp32 copy)
-                for (int cc = lane; cc < p.bn && n0 + cc < p.N; cc += 32) {
-                    const int nn = n0 + cc;
-                    const float a0 = f16_bits_to_float(p.t0[nn]);
-                    const float a1 = p.t1 != nullptr ? f16_bits_to_float(p.t1[nn]) : 0.0f;
-                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(lsm + 4u * (uint32_t)cc), "f"(a0) : "memory");
-                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(lsm + 4u * (uint32_t)(128 + cc)), "f"(a1) : "memory");
-                }
-                __syncwarp();
             }
-            if ((MODE == 3 || MODE == 4) && p.aux != nullptr && row_in) {
+            if (MODE == 3 && p.aux != nullptr && row_in) {
                 // the column dot's operand for this lane's row of the tile into
                 // L2 while the accumulator fills (128 bytes per prefetch)
                 const uint16_t *ar = static_cast<const uint16_t *>(p.aux) + (int64_t)(m0 + lane) * p.ldaux;
@@ -645,108 +595,9 @@ __global__ void __launch_bounds__(Shape<H, P, MODE>::kThreads, 1)
                 break;
             }
             tc_fence_after();
-            // mode 4: the column dot's operand for a chunk is loaded one chunk
-            // ahead, so its latency overlaps the previous chunk's work
-            uint4 axn[4] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
-                            make_uint4(0u, 0u, 0u, 0u)};
-            auto load_aux = [&](int nn) {
-                if (row_in) {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(
-                        static_cast<const uint16_t *>(p.aux) + (int64_t)(m0 + lane) * p.ldaux + nn);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) axn[q] = __ldg(src + q);
-                }
-            };
-            if (MODE == 4) load_aux(n0);
             for (int c32 = 0; c32 < p.bn && n0 + c32 < p.N; c32 += 32) {
                 const int nn = n0 + c32;
                 uint32_t o[16];
-                bool store = true;
-                if constexpr (MODE == 4) {
-                    // per path: the products C_p[m, n] aux[m, n] of this lane's
-                    // row go into the warp's transpose buffer (row = lane, 36
-                    // floats apart: the 16-byte stores of 8 lanes and the
-                    // column reads of 32 lanes are conflict-free), and lane l
-                    // adds column l over the 32 rows with independent loads.
-                    // Then, when it is stored, the output sum_p t_p C_p.
-                    store = p.out != nullptr;
-                    const bool two = p.r0 < p.K;
-                    const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)((b + eh) * BN + c32);
-                    const uint32_t red = sRed + (uint32_t)ew * S::kRedBytes;
-                    const uint4 ax[4] = {axn[0], axn[1], axn[2], axn[3]};
-                    if (c32 + 32 < p.bn && nn + 32 < p.N) load_aux(nn + 32);
-                    for (int pth = 0; pth < (two ? 2 : 1); ++pth) {
-                        uint32_t v[32];
-                        tmem_ld32(tl + 128u * (uint32_t)pth, v);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            // aux words 2q, 2q + 1 hold columns 4q .. 4q + 3
-                            const uint4 &aq = ax[q >> 1];
-                            const uint32_t w0 = (q & 1) ? aq.z : aq.x, w1 = (q & 1) ? aq.w : aq.y;
-                            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(red + (uint32_t)(lane * 36 + 4 * q) * 4u),
-                                         "f"(lo_bf16(w0) * __uint_as_float(v[4 * q])),
-                                         "f"(hi_bf16(w0) * __uint_as_float(v[4 * q + 1])),
-                                         "f"(lo_bf16(w1) * __uint_as_float(v[4 * q + 2])),
-                                         "f"(hi_bf16(w1) * __uint_as_float(v[4 * q + 3]))
-                                         : "memory");
-                        }
-                        __syncwarp();
-                        float acc4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-                        for (int r = 0; r < 32; ++r) {
-                            float t;
-                            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(t) : "r"(red + (uint32_t)(r * 36 + lane) * 4u) : "memory");
-                            acc4[r & 3] += t;
-                        }
-                        __syncwarp();  // every lane is past its reads before the buffer is refilled
-                        if (m0 < p.M)
-                            (pth ? p.part1 : p.part0)[(int64_t)(m0 >> 5) * p.N + nn + lane] =
-                                (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-                    }
-                    if (store && m0 < p.M) {
-                        // straight into the warp's output box, 8 columns (one
-                        // 16-byte chunk of the lane's row) at a time
-                        const uint32_t box = obox + (uint32_t)(nst % S::kOutBufs) * OUT_BYTES;
-                        const uint32_t rowa = box + (uint32_t)lane * 64;
-                        if (lane == 0) bulk_wait_read<S::kOutBufs - 1>();
-                        __syncwarp();
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            uint32_t v0[16], v1[16];
-                            tmem_ld16(tl + (uint32_t)(16 * hh), v0);
-                            if (two) tmem_ld16(tl + 128u + (uint32_t)(16 * hh), v1);
-#pragma unroll
-                            for (int ch = 0; ch < 2; ++ch) {
-                                uint32_t w4[4];
-#pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    float w[2];
-#pragma unroll
-                                    for (int e = 0; e < 2; ++e) {
-                                        const int j = 8 * ch + 2 * q + e, cj = c32 + 16 * hh + j;
-                                        float t0, t1;
-                                        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(t0) : "r"(lsm + 4u * (uint32_t)cj));
-                                        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(t1) : "r"(lsm + 4u * (uint32_t)(128 + cj)));
-                                        w[e] = t0 * __uint_as_float(v0[j]) + (two ? t1 * __uint_as_float(v1[j]) : 0.0f);
-                                    }
-                                    w4[q] = pack_bf162(w[0], w[1]);
-                                }
-                                const uint32_t chunk = (uint32_t)(2 * hh + ch);
-                                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(rowa + ((chunk ^ rsw) << 4)),
-                                             "r"(w4[0]), "r"(w4[1]), "r"(w4[2]), "r"(w4[3])
-                                             : "memory");
-                            }
-                        }
-                        fence_async_shared();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d(&tmOut, nn, m0, box);
-                            bulk_commit();
-                        }
-                        ++nst;
-                    }
-                    store = false;  // stored above (or nothing to store)
-                } else {
                 uint32_t v[32];
                 tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)((b + eh) * BN + c32), v);
                 if (C1) {
@@ -770,7 +621,7 @@ __global__ void __launch_bounds__(Shape<H, P, MODE>::kThreads, 1)
                         }
                     }
                     if (MODE == 3 && p.aux != nullptr) {
-                        // the column dot of the accumulator with aux (fp16)
+                        // the column dot of the unscaled accumulator with aux
 #pragma unroll
                         for (int hh = 0; hh < 2; ++hh) {
                             uint4 ax[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
@@ -802,8 +653,7 @@ __global__ void __launch_bounds__(Shape<H, P, MODE>::kThreads, 1)
 #pragma unroll
                     for (int q = 0; q < 16; ++q) o[q] = pack_bf162(__uint_as_float(v[2 * q]), __uint_as_float(v[2 * q + 1]));
                 }
-                }
-                if (m0 >= p.M || !store) continue;  // the warp's rows all lie past the matrix, or nothing is stored
+                if (m0 >= p.M) continue;  // the warp's rows all lie past the matrix
                 const uint32_t box = obox + (uint32_t)(nst % S::kOutBufs) * OUT_BYTES;
                 const uint32_t rowa = box + (uint32_t)lane * 64;  // this lane's row of the box
                 // the store that last used this box has finished reading it
@@ -875,20 +725,17 @@ struct TilePlan {
     int P;  // CTAs per MMA
 };
 
-// `max_bn` and `min_h` restrict the plans (mode 4: its per-path accumulators
-// need bn <= 128, and it runs 256-row tiles, whose 576 threads leave its
-// epilogue the registers it needs).
-TilePlan plan_tiles(int M, int N, int K, int sms, int pairs, int max_bn = BN, int min_h = 1)
+TilePlan plan_tiles(int M, int N, int K, int sms, int pairs)
 {
     const long nk = (K + BK - 1) / BK;
-    TilePlan best{min_h, std::min(BN, max_bn), 0, 1};
+    TilePlan best{1, BN, 0, 1};
     long best_cost = -1;
     for (int P = 1; P <= 2; ++P) {
         const int units = P == 1 ? sms : pairs;
         if (units <= 0) continue;
-        for (int H = min_h; H <= 2; ++H) {
+        for (int H = 1; H <= 2; ++H) {
             const int tm = (M + BM * H * P - 1) / (BM * H * P);
-            for (int tn = (N + max_bn - 1) / max_bn; tn <= (N + 31) / 32; ++tn) {
+            for (int tn = (N + BN - 1) / BN; tn <= (N + 31) / 32; ++tn) {
                 const int bn = ((N + tn - 1) / tn + 31) & ~31;
                 if ((N + bn - 1) / bn != tn) continue;
                 const int tiles = tm * tn, waves = (tiles + units - 1) / units;
@@ -933,42 +780,32 @@ cudaError_t launch_units(const CUtensorMap &tm, const CUtensorMap &tmo, const Si
 
 // One contraction on a persistent grid: min(tiles, SMs) CTAs, or
 // min(tiles, resident pairs) CTA pairs.
-// A is x (modes 1 and 3, bf16) or z (modes 2 and 4, fp16), row-major with
-// stride lda.  Mode 4 runs 256-row tiles (H = 2): at most 128 wide when it
-// has two paths (an accumulator each) or stores an output, up to 256 wide
-// with one path and no output.  Mode 4 without an output (p.out null)
-// encodes no store map.
+// A is x (modes 1 and 3, bf16) or z (mode 2, fp16; bf16 with bf16_ops),
+// row-major with stride lda.
 template <int MODE>
 cudaError_t launch_sign_gemm(SignGemmParams p, const void *a, int64_t lda, const DeviceInfo &dev,
                              cudaStream_t stream)
 {
     constexpr bool C1 = MODE == 1 || MODE == 3;
     const int pairs = prefill_pairs_enabled() ? dev.pair_slots : 0;
-    const int max_bn4 = (p.out == nullptr && p.r0 >= p.K) ? BN : 128;
-    const TilePlan tp = MODE == 4 ? plan_tiles(p.M, p.N, p.K, dev.sm_count, pairs, max_bn4, 2)
-                                  : plan_tiles(p.M, p.N, p.K, dev.sm_count, pairs);
+    const TilePlan tp = plan_tiles(p.M, p.N, p.K, dev.sm_count, pairs);
     const int H = tp.H;
     p.bn = tp.bn;
     CUtensorMap tm, tmo;
     std::memset(&tmo, 0, sizeof(tmo));
-    cudaError_t e = encode_2d(&tm, a, p.M, p.K, lda, C1, BM * H);
-    // the output: z fp16 (modes 1, 3; mode 3 bf16 on request) or y bf16 (modes 2, 4), [M x N], stride ldo
+    cudaError_t e = encode_2d(&tm, a, p.M, p.K, lda, C1 || p.bf16_ops, BM * H);
+    // the output: z fp16 (modes 1, 3; mode 3 bf16 on request) or y bf16 (mode 2), [M x N], stride ldo
     if (e == cudaSuccess && p.out != nullptr)
         e = encode_store_2d(&tmo, p.out, p.M, p.N, p.ldo, !C1 || (MODE == 3 && p.out_bf16));
     if (e != cudaSuccess) return e;
-    if constexpr (MODE == 4) {
-        if (tp.P == 2) return launch_units<4, 2, 2>(tm, tmo, p, std::min(tp.tiles, dev.pair_slots), stream);
-        return launch_units<4, 2, 1>(tm, tmo, p, std::min(tp.tiles, dev.sm_count), stream);
-    } else {
-        if (tp.P == 2) {
-            const int units = std::min(tp.tiles, dev.pair_slots);
-            return H == 2 ? launch_units<MODE, 2, 2>(tm, tmo, p, units, stream)
-                          : launch_units<MODE, 1, 2>(tm, tmo, p, units, stream);
-        }
-        const int units = std::min(tp.tiles, dev.sm_count);
-        return H == 2 ? launch_units<MODE, 2, 1>(tm, tmo, p, units, stream)
-                      : launch_units<MODE, 1, 1>(tm, tmo, p, units, stream);
+    if (tp.P == 2) {
+        const int units = std::min(tp.tiles, dev.pair_slots);
+        return H == 2 ? launch_units<MODE, 2, 2>(tm, tmo, p, units, stream)
+                      : launch_units<MODE, 1, 2>(tm, tmo, p, units, stream);
     }
+    const int units = std::min(tp.tiles, dev.sm_count);
+    return H == 2 ? launch_units<MODE, 2, 1>(tm, tmo, p, units, stream)
+                  : launch_units<MODE, 1, 1>(tm, tmo, p, units, stream);
 }
 
 }  // namespace
@@ -1020,8 +857,6 @@ cudaError_t prefill_prepare_device(DeviceInfo &dev)
     if (e == cudaSuccess) e = prepare_kernel<3, 2, 1>(dev);
     if (e == cudaSuccess) e = prepare_kernel<3, 1, 2>(dev);
     if (e == cudaSuccess) e = prepare_kernel<3, 2, 2>(dev);
-    if (e == cudaSuccess) e = prepare_kernel<4, 2, 1>(dev);
-    if (e == cudaSuccess) e = prepare_kernel<4, 2, 2>(dev);
     return e;
 }
 
@@ -1105,10 +940,12 @@ cudaError_t bwd_contraction1(const Bwd1Args &b, const DeviceInfo &dev, cudaStrea
     p.bits0 = b.bits0;
     p.bld0 = b.ld0;
     p.s0 = b.s0;
+    p.l0 = b.l0;
     if (b.bits1 != nullptr) {
         p.bits1 = b.bits1;
         p.bld1 = b.ld1;
         p.s1 = b.s1;
+        p.l1 = b.l1;
     }
     p.out = b.out;
     p.ldo = b.ldo;
@@ -1121,34 +958,30 @@ cudaError_t bwd_contraction1(const Bwd1Args &b, const DeviceInfo &dev, cudaStrea
     return launch_sign_gemm<3>(p, b.a, b.lda, dev, stream);
 }
 
-cudaError_t bwd_contraction2(const Bwd2Args &b, const DeviceInfo &dev, cudaStream_t stream)
+cudaError_t bwd_dx(const BwdDxArgs &b, const DeviceInfo &dev, cudaStream_t stream)
 {
     cudaError_t e = get_encoder();
     if (e != cudaSuccess) return e;
+    // contraction 2 in bf16: dx = A . B^T, B[i, k] = sign(V_p[i, k]) bf16(g_p[i])
     SignGemmParams p{};
     p.M = b.M;
-    p.N = b.N;
+    p.N = b.n_in;
     p.K = b.r0 + b.r1;
     p.r0 = b.r0;
     p.bits8 = even8(b.bits0, b.ld0) && (b.bits1 == nullptr || (b.r0 % 64 == 0 && even8(b.bits1, b.ld1)));
     p.bits0 = b.bits0;
     p.bld0 = b.ld0;
-    p.s0 = b.l0;
+    p.s0 = b.g0;
     if (b.bits1 != nullptr) {
         p.bits1 = b.bits1;
         p.bld1 = b.ld1;
-        p.s1 = b.l1;
+        p.s1 = b.g1;
     }
-    p.out = b.out;
-    p.ldo = b.ldo;
-    p.t0 = b.t0;
-    p.t1 = b.t1;
+    p.out = b.dx;
+    p.ldo = b.lddx;
     p.status = dev.status;
-    p.aux = b.aux;
-    p.ldaux = b.ldaux;
-    p.part0 = b.part0;
-    p.part1 = b.part1;
-    return launch_sign_gemm<4>(p, b.a, b.lda, dev, stream);
+    p.bf16_ops = 1;
+    return launch_sign_gemm<2>(p, b.a, b.lda, dev, stream);
 }
 
 cudaError_t prefill_forward(const ForwardArgs &a, const DeviceInfo &dev, cudaStream_t stream)

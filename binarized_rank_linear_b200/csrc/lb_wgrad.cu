@@ -1,29 +1,31 @@
-// lb_wgrad.cu - the h-gradient of the backward pass as a weight-gradient
-// product on the tensor cores.
+// lb_wgrad.cu - the scale gradients dh and dg of the backward pass as
+// weight-gradient products on the tensor cores.
 //
-// With e_p = S_U,p (l_p (.) c_p) (sesamedisk.com, "Samsung LittleBit 13B
-// Model", "What the method actually computes", Proposition 1, run backward by
-// the chain rule),
-//     dh_p[o] = sum_m dy[m, o] e_p[m, o] = sum_k sign(U_p[o, k]) l_p[k] G[o, k],
-//     G = dy^T c   ([n_out x R], the tokens m as the contraction dimension),
-// so the sum over tokens runs inside the MMA and each output row's sum over k
-// is a per-lane epilogue: no column dot across rows, and no product tile
-// stored.  G's rows o are the accumulator's lanes; its columns k run over the
+// Run backward by the chain rule, the layer's five steps (sesamedisk.com,
+// "Samsung LittleBit 13B Model", "What the method actually computes",
+// Proposition 1) give, per path p, with c = S_V^T (g (.) x) and
+// a = S_U^T (h (.) dy),
+//     dh_p[o] = sum_m dy[m, o] e_p[m, o] = sum_k sign(U_p[o, k]) l_p[k] G[o, k],   G = dy^T c,
+//     dg_p[i] = sum_m x[m, i] dt_p[m, i] = sum_k sign(V_p[i, k]) H[i, k],          H = x^T (l (.) a),
+// so the sum over tokens runs inside the MMA and each row's sum over k is a
+// per-lane epilogue: no column dot across rows, and no product tile stored.
+// The product's rows are the accumulator's lanes; its columns k run over the
 // latents of both paths (path 0 below r0).
 //
-// Both operands are MN-major: dy [tokens x n_out] and c [tokens x R] are
+// Both operands are MN-major: A [tokens x rows] and B [tokens x R] are
 // row-major with the tokens outermost, so a K-block (64 tokens) of A is 64
-// rows of 128 bytes for each 64 columns o, and the same for B along k.  TMA
-// brings them in with 128-byte swizzle, boxes of 64 (MN) x 64 (tokens); the
-// shared-memory descriptors then step 8192 bytes between 64-wide MN chunks
-// (leading byte offset) and 1024 bytes between 8-token groups (stride byte
-// offset), and an MMA of K = 16 tokens starts 2048 bytes further on.
+// rows of 128 bytes for each 64 rows of the product, and the same for B along
+// k.  TMA brings them in with 128-byte swizzle, boxes of 64 (MN) x 64
+// (tokens); the shared-memory descriptors then step 8192 bytes between
+// 64-wide MN chunks (leading byte offset) and 1024 bytes between 8-token
+// groups (stride byte offset), and an MMA of K = 16 tokens starts 2048 bytes
+// further on.
 //
 // Persistent tiles of 256 rows o on a CTA pair (cta_group::2: CTA r holds
 // rows 128 r .. of A and columns bn r / 2 .. of B; CTA 0 issues the MMAs),
 // or of 128 rows on single CTAs, x bn columns k, optionally split over the
 // tokens into `nsplit` parts; a unit (tile, part) leaves one partial per row
-// and path, [ntn * nsplit][n_out] per path, which the caller adds in a fixed
+// and path, [ntn * nsplit][rows] per path, which the caller adds in a fixed
 // order.  Warp 0 issues the TMA loads, warp 1 the MMAs, warps 2..5 drain the
 // two double-buffered accumulators.
 #include <algorithm>
@@ -59,16 +61,16 @@ struct WShape {
 };
 
 struct WgradParams {
-    int M;       // rows o (n_out)
+    int M;       // rows o of the product
     int N;       // columns k (R = r0 + r1)
     int K;       // tokens
     int bn;      // tile width along k: a multiple of 32, at most WBN
     int nsplit;  // parts of the token range per tile
     int kps;     // K-blocks per part (the last may be shorter)
     int r0;      // columns k below r0 are path 0
-    const uint32_t *u0, *u1;  // packed rows of U_p (bit j of word w: column 32 w + j negative)
+    const uint32_t *u0, *u1;  // packed rows of S_p (bit j of word w: column 32 w + j negative)
     int64_t uld0, uld1;
-    const uint16_t *l0, *l1;  // latent scales (fp16)
+    const uint16_t *l0, *l1;  // latent scales (fp16), or null for 1
     float *part0, *part1;     // [ceil(N / bn) * nsplit][M] per path
     int *status;
 };
@@ -108,7 +110,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
     const int G = gridDim.x / P, c = blockIdx.x / P;  // persistent units: CTAs, or pairs
     const int my_units = c < units ? (units - c + G - 1) / G : 0;
     // unit t: columns (t % tiles_n), then rows, then the token part, so the
-    // units running at once share their rows of dy (the larger operand) in L2
+    // units running at once share their rows of A (the larger operand) in L2
     auto unit_kb = [&](int t, int &kb0, int &kb1) {
         const int sp = t / (tiles_m * tiles_n);
         kb0 = sp * p.kps;
@@ -147,7 +149,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
     const uint32_t acce_lead = P == 2 ? map_shared_addr(acce0, 0) : acce0;
 
     if (warp == 0) {
-        // ---------------- TMA: A (dy^T) and B (c) boxes of each K-block
+        // ---------------- TMA: the A and B boxes of each K-block
         if (lane == 0) {
             int gb = 0, issued = 0;
             // this CTA's columns of B: all bn (P = 1), or half from bn/2 rank on
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(kWThreads, 1)
                 const bool sec = k >= p.r0;
                 const int kl = sec ? k - p.r0 : k;  // column within the path (a multiple of 32)
                 const uint16_t *lv = sec ? p.l1 : p.l0;
-                const float lj = f16_bits_to_float(lv[kl + lane]);
+                const float lj = lv != nullptr ? f16_bits_to_float(lv[kl + lane]) : 1.0f;
                 const uint32_t word = o < p.M ? __ldg((sec ? p.u1 + (int64_t)o * p.uld1 : p.u0 + (int64_t)o * p.uld0) + (kl >> 5))
                                               : 0u;
                 uint32_t v[32];
@@ -327,17 +329,17 @@ __global__ void __launch_bounds__(kWThreads, 1)
 
 }  // namespace
 
-// Tile width, token split and partial count of the h-gradient product for
-// n_out rows, R latent columns and `tokens` tokens on `sms` SMs.  The plan is
+// Tile width, token split and partial count of the product for `rows` rows,
+// R latent columns and `tokens` tokens on `sms` SMs.  The plan is
 // made for CTA pairs (256-row tiles, sms / 2 of them at once) and kept for
 // single CTAs, so both give the same token parts and the same sums.
-WgradPlan wgrad_plan(int n_out, int R, int tokens, int sms)
+WgradPlan wgrad_plan(int rows, int R, int tokens, int sms)
 {
     WgradPlan w{};
     const int ntn = (R + WBN - 1) / WBN;
     w.bn = ((R + ntn - 1) / ntn + 31) & ~31;
     w.ntn = (R + w.bn - 1) / w.bn;
-    const int tiles = ((n_out + 2 * WM - 1) / (2 * WM)) * w.ntn;
+    const int tiles = ((rows + 2 * WM - 1) / (2 * WM)) * w.ntn;
     sms = std::max(1, sms / 2);
     const int nk = std::max(1, (tokens + WBK - 1) / WBK);
     // makespan in K-blocks: waves x (blocks per part + a unit's fixed cost of
@@ -375,35 +377,35 @@ cudaError_t wgrad_prepare_device(const DeviceInfo &dev)
     return e;
 }
 
-cudaError_t wgrad_dh(const WgradArgs &w, const DeviceInfo &dev, cudaStream_t stream)
+cudaError_t wgrad_scale_grad(const WgradArgs &w, const DeviceInfo &dev, cudaStream_t stream)
 {
     cudaError_t e = get_encoder();
     if (e != cudaSuccess) return e;
-    const WgradPlan pl = wgrad_plan(w.n_out, w.R, w.tokens, dev.sm_count);
+    const WgradPlan pl = wgrad_plan(w.rows, w.R, w.tokens, dev.sm_count);
     CUtensorMap ta, tb;
-    // dy: [tokens x n_out], MN (n_out) contiguous; c: [tokens x R]
-    e = encode_2d(&ta, w.dy, w.tokens, w.n_out, w.lddy, true, 64);
-    if (e == cudaSuccess) e = encode_2d(&tb, w.c, w.tokens, w.R, w.ldc, true, 64);
+    // A: [tokens x rows], B: [tokens x R], both with the rows or columns contiguous
+    e = encode_2d(&ta, w.a, w.tokens, w.rows, w.lda, true, 64);
+    if (e == cudaSuccess) e = encode_2d(&tb, w.b, w.tokens, w.R, w.ldb, true, 64);
     if (e != cudaSuccess) return e;
     WgradParams p{};
-    p.M = w.n_out;
+    p.M = w.rows;
     p.N = w.R;
     p.K = w.tokens;
     p.bn = pl.bn;
     p.nsplit = pl.nsplit;
     p.kps = pl.kps;
     p.r0 = w.r0;
-    p.u0 = w.u0;
-    p.u1 = w.u1;
-    p.uld0 = w.uld0;
-    p.uld1 = w.uld1;
+    p.u0 = w.bits0;
+    p.u1 = w.bits1;
+    p.uld0 = w.bld0;
+    p.uld1 = w.bld1;
     p.l0 = w.l0;
     p.l1 = w.l1;
     p.part0 = w.part0;
     p.part1 = w.part1;
     p.status = dev.status;
     if (prefill_pairs_enabled() && dev.pair_slots > 0) {
-        const int units = ((w.n_out + 2 * WM - 1) / (2 * WM)) * pl.ntn * pl.nsplit;
+        const int units = ((w.rows + 2 * WM - 1) / (2 * WM)) * pl.ntn * pl.nsplit;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
@@ -418,7 +420,7 @@ cudaError_t wgrad_dh(const WgradArgs &w, const DeviceInfo &dev, cudaStream_t str
         cfg.numAttrs = 1;
         return cudaLaunchKernelEx(&cfg, wgrad_kernel<2>, ta, tb, p);
     }
-    const int units = ((w.n_out + WM - 1) / WM) * pl.ntn * pl.nsplit;
+    const int units = ((w.rows + WM - 1) / WM) * pl.ntn * pl.nsplit;
     wgrad_kernel<1><<<std::min(units, dev.sm_count), kWThreads, WShape<1>::kSmem, stream>>>(ta, tb, p);
     return cudaGetLastError();
 }

@@ -310,17 +310,14 @@ LB_API lb_status lb_linear_forward_siblings(const uint16_t *x, int64_t tokens, i
  *   workspace : at least lb_backward_workspace_bytes(...) bytes, 16-byte
  *             aligned, contents on entry irrelevant; calls sharing it must be
  *             ordered on one stream
- * Numerics: tensor-core contractions with fp32 accumulation.  c_p =
- *   S_V,p^T (g_p (.) x) and a_p = S_U,p^T (h_p (.) dy), over n_in and n_out,
- *   in bf16 x bf16 (x and dy as given, g and h rounded to bf16), kept
- *   unscaled: c_p in bf16, a_p in fp16 (so a_p must stay below 65504 in
- *   magnitude, else LB_ERR_RANGE on the device status word and the results
- *   are undefined).  dh from dy^T c over the tokens (bf16 x bf16); dx and dg
- *   from the contraction of a_p over the latent (fp16 x fp16, l exact).  Every
- *   sum runs in a fixed order (dl and dg: 32-token blocks, then the blocks in
- *   order; dh: the tokens inside the MMA, then tile columns and token parts
- *   in order): results are deterministic.  dx is rounded to bf16 once; dh,
- *   dg and dl are fp32.
+ * Numerics: tensor-core products with fp32 accumulation, bf16 operands.
+ *   c = S_V^T (g (.) x) and a = S_U^T (h (.) dy) (g and h rounded to bf16)
+ *   are kept in bf16, a scaled by l; dh and dg come from dy^T c and x^T a
+ *   with the tokens as the contraction, dx from a against V with g rounded
+ *   to bf16.  Every sum runs in a fixed order (dl: 32-token blocks, then the
+ *   blocks in order; dh, dg: the tokens inside the MMA, then tile columns and
+ *   token parts in order): results are deterministic.  dx is rounded to bf16
+ *   once; dh, dg and dl are fp32.
  * Shapes, alignment and strides as lb_linear_forward (dx like x; dh, dg, dl
  *   4-byte aligned).  tokens == 0 sets dh, dg and dl to zero and nothing else
  *   (x, dy and dx are then not read and may be NULL).
