@@ -565,10 +565,10 @@ def measure_backward(name, args, world, local, device, peaks, tokens=None):
             "value": aggregate(flops / 1e12 * calls, ms / 1e3, world), "unit": "TFLOP/s",
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
                          "frac": achieved / pk, "traffic": None, "kernel": "whole lb_linear_backward call "
-                         "(2 bit transposes per path, sign_gemm_kernel<3> x2, wgrad_kernel x2 (dh, dg), "
-                         "bf16 sign_gemm_kernel<2> (dx), reduce_partials_kernel)",
+                         "(transpose_bits_kernel (both factors of every path), sign_gemm_kernel<3> x2, "
+                         "wgrad_kernel x2 (dh, dg), bf16 sign_gemm_kernel<2> (dx), reduce_partials_kernel)",
                          "peak_source": pk_source},
-            "clocks": clocks, "gpu_launches": (2 * len(d.ranks) + 6) * calls}
+            "clocks": clocks, "gpu_launches": 7 * calls}
 
 
 def dense_baseline(d, device, seconds, stream, local, world):

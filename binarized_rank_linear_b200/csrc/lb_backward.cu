@@ -28,7 +28,7 @@
 // then one kernel adds each partial column over its rows in order, so the
 // results do not depend on timing.  K2, K4 and K5 read the factors along the
 // other axis from the forward pass: U^T packed along n_out and V packed along
-// r, which two bit-transpose launches make from the forward's packed words
+// r, which one bit-transpose launch makes from the forward's packed words
 // into the workspace, so the call takes the forward pass's lb_path as it is.
 // c and a_s travel between the products in bf16, the type of x and dy that
 // K3 and K4 multiply them with.
@@ -52,44 +52,60 @@ namespace {
 constexpr int kTransposeWarps = 8;
 constexpr int kRowBlocks = 8;
 
-__global__ void __launch_bounds__(32 * kTransposeWarps)
-    transpose_bits_kernel(const uint32_t *__restrict__ in, int64_t ld_in, int rows, int cols,
-                          uint32_t *__restrict__ out, int64_t ld_out)
+// Up to four transposes in one launch: matrix q takes the CTAs first_cta[q] ..
+constexpr int kMaxTransposes = 4;
+struct TransposeJob {
+    const uint32_t *in;
+    int64_t ld_in;
+    int rows, cols;
+    uint32_t *out;
+    int64_t ld_out;
+    int first_cta;
+};
+struct TransposeBatch {
+    TransposeJob job[kMaxTransposes];
+    int n;
+};
+
+__global__ void __launch_bounds__(32 * kTransposeWarps) transpose_bits_kernel(const __grid_constant__ TransposeBatch b)
 {
+    int q = 0;
+    while (q + 1 < b.n && (int)blockIdx.x >= b.job[q + 1].first_cta) ++q;
+    const TransposeJob &t = b.job[q];
     const int lane = threadIdx.x & 31;
-    const int64_t job = (int64_t)blockIdx.x * kTransposeWarps + (threadIdx.x >> 5);
-    const int rbs = rows >> 5, cbs = cols >> 5;
+    const int64_t job = (int64_t)((int)blockIdx.x - t.first_cta) * kTransposeWarps + (threadIdx.x >> 5);
+    const int rbs = t.rows >> 5, cbs = t.cols >> 5;
     const int groups = (rbs + kRowBlocks - 1) / kRowBlocks;
     if (job >= (int64_t)groups * cbs) return;  // whole warps leave together
     const int rg = (int)(job % groups), cb = (int)(job / groups);
     const int rb0 = rg * kRowBlocks, nrb = min(kRowBlocks, rbs - rb0);
     uint32_t w[kRowBlocks];
 #pragma unroll
-    for (int q = 0; q < kRowBlocks; ++q)
-        w[q] = q < nrb ? __ldg(in + (int64_t)(32 * (rb0 + q) + lane) * ld_in + cb) : 0u;
+    for (int r = 0; r < kRowBlocks; ++r)
+        w[r] = r < nrb ? __ldg(t.in + (int64_t)(32 * (rb0 + r) + lane) * t.ld_in + cb) : 0u;
     uint32_t mine[kRowBlocks];
 #pragma unroll
-    for (int q = 0; q < kRowBlocks; ++q) {
-        mine[q] = 0u;
+    for (int r = 0; r < kRowBlocks; ++r) {
+        mine[r] = 0u;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-            const uint32_t t = __ballot_sync(0xffffffffu, (w[q] >> j) & 1u);
-            if (lane == j) mine[q] = t;
+            const uint32_t v = __ballot_sync(0xffffffffu, (w[r] >> j) & 1u);
+            if (lane == j) mine[r] = v;
         }
     }
-    uint32_t *dst = out + (int64_t)(32 * cb + lane) * ld_out + rb0;
+    uint32_t *dst = t.out + (int64_t)(32 * cb + lane) * t.ld_out + rb0;
 #pragma unroll
-    for (int q = 0; q < kRowBlocks; ++q)
-        if (q < nrb) dst[q] = mine[q];
+    for (int r = 0; r < kRowBlocks; ++r)
+        if (r < nrb) dst[r] = mine[r];
 }
 
-cudaError_t transpose_bits(const uint32_t *in, int64_t ld_in, int rows, int cols, uint32_t *out, int64_t ld_out,
-                           cudaStream_t stream)
+// Adds one matrix to a batch; returns its CTA count.
+int add_transpose(TransposeBatch &b, const uint32_t *in, int64_t ld_in, int rows, int cols, uint32_t *out,
+                  int64_t ld_out, int first_cta)
 {
     const int64_t jobs = (int64_t)((rows / 32 + kRowBlocks - 1) / kRowBlocks) * (cols / 32);
-    const unsigned grid = (unsigned)((jobs + kTransposeWarps - 1) / kTransposeWarps);
-    transpose_bits_kernel<<<grid, 32 * kTransposeWarps, 0, stream>>>(in, ld_in, rows, cols, out, ld_out);
-    return cudaGetLastError();
+    b.job[b.n++] = TransposeJob{in, ld_in, rows, cols, out, ld_out, first_cta};
+    return (int)((jobs + kTransposeWarps - 1) / kTransposeWarps);
 }
 
 // ------------------------------------------------------------ partial sums
@@ -192,15 +208,18 @@ cudaError_t backward_launch(const BackwardArgs &b, const DeviceInfo &dev, cudaSt
     const BwdLayout L = layout(M, b.n_in, b.n_out, ranks, npaths);
     uint8_t *ws = static_cast<uint8_t *>(b.workspace);
     uint32_t *ut[2] = {nullptr, nullptr}, *v[2] = {nullptr, nullptr};
-    cudaError_t e = cudaSuccess;
-    for (int q = 0; q < npaths && e == cudaSuccess; ++q) {
+    TransposeBatch tr{};
+    int ctas = 0;
+    for (int q = 0; q < npaths; ++q) {
         const PathDesc &P = b.path[q];
         ut[q] = reinterpret_cast<uint32_t *>(ws + L.ut[q]);
         v[q] = reinterpret_cast<uint32_t *>(ws + L.v[q]);
         // U [n_out x r] -> U^T [r x n_out]; V^T [r x n_in] -> V [n_in x r]
-        e = transpose_bits(P.u_bits, P.u_ld, b.n_out, P.rank, ut[q], b.n_out / 32, stream);
-        if (e == cudaSuccess) e = transpose_bits(P.vt_bits, P.vt_ld, P.rank, b.n_in, v[q], P.rank / 32, stream);
+        ctas += add_transpose(tr, P.u_bits, P.u_ld, b.n_out, P.rank, ut[q], b.n_out / 32, ctas);
+        ctas += add_transpose(tr, P.vt_bits, P.vt_ld, P.rank, b.n_in, v[q], P.rank / 32, ctas);
     }
+    transpose_bits_kernel<<<(unsigned)ctas, 32 * kTransposeWarps, 0, stream>>>(tr);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     uint16_t *c = reinterpret_cast<uint16_t *>(ws + L.c);
     uint16_t *a = reinterpret_cast<uint16_t *>(ws + L.a);
