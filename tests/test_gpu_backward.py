@@ -86,6 +86,16 @@ def test_backward_model_shapes(name, tokens):
     check_against_oracle(layer, dy, run_backward(layer, dy), f"{name} M={tokens}")
 
 
+def test_backward_kv_at_full_size():
+    """Qwen3-14B k/v at its full 8192 tokens, every output against the oracle:
+    the launch plans of the benchmarked size (the weight-gradient products
+    split over 9 token parts for dh, several for dg; 64 latent tiles)."""
+    layer = synth.make_config("qwen3_14b_kv")
+    M = layer["x"].shape[0]
+    dy = draw_dy(M, layer["n_out"], 23)
+    check_against_oracle(layer, dy, run_backward(layer, dy), f"qwen3_14b_kv M={M}")
+
+
 def test_integer_exact_scale_gradients_are_bitwise():
     """Unit scales, x and dy in {-1, 0, 1}: every intermediate is a small
     integer, exact in fp16, bf16 and fp32, so dh, dg and dl match the oracle
