@@ -158,7 +158,7 @@ size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 // Workspace layout of one call (every piece 256-byte aligned).
 struct BwdLayout {
     size_t ut[2], v[2];     // transposed sign words of each path
-    size_t c, a;            // fp16 [M x R]
+    size_t c, a;            // bf16 [M x R]: c, and l (.) a
     size_t pl, ph[2], pg[2];  // partials
     size_t total;
 };
@@ -181,7 +181,7 @@ BwdLayout layout(int M, int n_in, int n_out, const int *ranks, int npaths)
     off += align256((size_t)M * R * 2);
     L.pl = off;
     off += align256(RB * R * 4);
-    // K3's partial rows: at most wgrad_max_parts (at least the 32-token blocks)
+    // dh's and dg's partial rows (K3, K4): at most wgrad_max_parts; dl's: the 32-token blocks
     const size_t HB = std::max(RB, (size_t)wgrad_max_parts(R, M));
     for (int q = 0; q < npaths; ++q) {
         L.ph[q] = off;
