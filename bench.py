@@ -85,14 +85,15 @@ def source_code(text):
     return " ".join(text.split())
 
 
-def source_hash():
-    """Hash of every kernel source's code: a traffic figure taken on other code
-    is stale (comments and layout do not count)."""
+def source_hash(files=None):
+    """Hash of the code of the kernel sources a figure depends on (every
+    source when `files` is None): a traffic figure taken on other code is
+    stale (comments and layout do not count)."""
+    names = sorted(files) if files else sorted(f for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh", ".h")))
     h = hashlib.sha256()
-    for f in sorted(os.listdir(CSRC)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(CSRC, f)) as fh:
-                h.update(f.encode() + b"\0" + source_code(fh.read()).encode())
+    for f in names:
+        with open(os.path.join(CSRC, f)) as fh:
+            h.update(f.encode() + b"\0" + source_code(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
@@ -108,16 +109,17 @@ def load_peaks():
 
 def load_traffic(config, tokens):
     """DRAM bytes from a committed ncu summary, only if it was taken on the
-    current kernel sources: per launch of the dominant kernel where the
-    roofline is that kernel's (prefill), else per call (decode, whose
-    roofline is the whole call)."""
+    current code of the sources it names (`sources`: the call's path from the
+    ABI to its kernels; all kernel sources when absent): per launch of the
+    dominant kernel where the roofline is that kernel's (prefill), else per
+    call (decode, whose roofline is the whole call)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(f"{config}/M{tokens}")
-    if not e or e.get("source_hash") != source_hash():
+    if not e or e.get("source_hash") != source_hash(e.get("sources")):
         return None
     return e.get("dram_bytes_per_launch", e.get("dram_bytes_per_call"))
 

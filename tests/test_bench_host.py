@@ -125,6 +125,16 @@ def test_source_hash_sees_code_not_comments():
     assert "one" not in bench.source_code(a) and "two" not in bench.source_code(a)
 
 
+def test_source_hash_covers_the_named_sources():
+    """A figure's hash covers the sources it names (all of them when none are
+    named), in a fixed order."""
+    names = sorted(f for f in os.listdir(bench.CSRC) if f.endswith((".cu", ".cuh", ".h")))
+    assert bench.source_hash() == bench.source_hash(names)
+    sub = ["lb_gemv.cu", "lb_common.cuh"]
+    assert bench.source_hash(sub) == bench.source_hash(list(reversed(sub)))
+    assert bench.source_hash(sub) != bench.source_hash(names)
+
+
 @pytest.mark.parametrize("n_in,n_out,ranks", [(256, 512, [64, 32]), (96, 64, [32])])
 def test_dense_baseline_weight_is_the_oracles(n_in, n_out, ranks):
     """The dense comparison arm multiplies by W built with PyTorch ops
